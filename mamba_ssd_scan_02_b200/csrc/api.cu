@@ -1,0 +1,357 @@
+// api.cu -- the C ABI of libssd.so: argument validation, workspace layout and the launch
+// sequence of each entry point.  Nothing here allocates or synchronises on the compute paths.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "plan.h"
+
+namespace ssd {
+
+// The device error word that kernels latch failures into (one per device).
+__device__ int g_device_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr long long kTargetCtas = 2 * 148;  // scan CTAs wanted in flight (2 per B200 SM)
+constexpr size_t kAlign = 256;
+
+int *device_error_ptr() {
+  static int *ptrs[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!ptrs[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int *>(p);
+  }
+  return ptrs[dev];
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+size_t elt_size(ssd_dtype_t t) { return t == SSD_F32 ? 4 : 2; }
+
+bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb) {
+  const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+  return pa < pb + nb && pb < pa + na;
+}
+
+ssd_status_t check_config(const ssd_config_t *c, bool prefill) {
+  if (!c) return SSD_ERR_INVALID_ARG;
+  if (c->batch < 1 || c->nheads < 1 || c->ngroups < 1 || c->seqlen < 0) return SSD_ERR_INVALID_ARG;
+  if (c->nheads % c->ngroups != 0) return SSD_ERR_INVALID_ARG;
+  if (c->io_dtype != SSD_F32 && c->io_dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
+  if (c->headdim != kHeadDim || c->dstate != kDState) return SSD_ERR_UNSUPPORTED;
+  if (prefill && c->chunk != 64 && c->chunk != 128 && c->chunk != 256) return SSD_ERR_UNSUPPORTED;
+  if (c->conv_width < 0 || c->conv_width > 4) return SSD_ERR_UNSUPPORTED;
+  const long long d_inner = (long long)c->nheads * c->headdim;
+  if (c->norm_groups < 0 || (c->norm_groups > 0 && d_inner % c->norm_groups != 0))
+    return SSD_ERR_INVALID_ARG;
+  if (!(c->norm_eps >= 0.f) || !(c->dt_min <= c->dt_max) || isnan(c->dt_min)) return SSD_ERR_INVALID_ARG;
+  if (c->n_segments < 0) return SSD_ERR_INVALID_ARG;
+  if (c->kernel != SSD_KERNEL_AUTO && c->kernel != SSD_KERNEL_SIMT && c->kernel != SSD_KERNEL_TENSOR)
+    return SSD_ERR_INVALID_ARG;
+  if (c->batch > 65535 || c->nheads > 65535 || c->seqlen > (1 << 21))
+    return SSD_ERR_UNSUPPORTED;  // grid limits
+  return SSD_OK;
+}
+
+// Internal sequence segments: enough (b, h, segment) CTAs to fill the GPU, each segment a
+// whole number of chunks and at least four 64-token tiles long.
+void choose_segments(const ssd_config_t *c, int *n_seg, int *seg_len) {
+  const int L = c->seqlen, Q = c->chunk;
+  int n = c->n_segments;
+  if (n == 0) {
+    const long long bh = (long long)c->batch * c->nheads;
+    n = 1;
+    if (bh < kTargetCtas && L > 4 * 64) {
+      n = (int)((kTargetCtas + bh - 1) / bh);
+      n = n < L / (4 * 64) ? n : L / (4 * 64);
+      if (n > 64) n = 64;
+      if (n < 1) n = 1;
+    }
+  }
+  if (n < 1) n = 1;
+  long long len = L > 0 ? ((long long)L + n - 1) / n : Q;
+  len = (len + Q - 1) / Q * Q;
+  *seg_len = (int)len;
+  *n_seg = L > 0 ? (int)((L + len - 1) / len) : 1;
+}
+
+struct WsLayout {
+  size_t u, dte, yf, seg_state, seg_decay, total;
+};
+
+WsLayout prefill_layout(const ssd_config_t *c) {
+  WsLayout w{};
+  int n_seg, seg_len;
+  choose_segments(c, &n_seg, &seg_len);
+  const size_t T = (size_t)c->batch * c->seqlen;
+  const size_t d_inner = (size_t)c->nheads * c->headdim;
+  const size_t conv_dim = d_inner + 2 * (size_t)c->ngroups * c->dstate;
+  size_t off = 0;
+  w.u = off;         off = round_up(off + T * conv_dim * 4, kAlign);
+  w.dte = off;       off = round_up(off + T * c->nheads * 4, kAlign);
+  w.yf = off;        if (c->norm_groups > 0) off = round_up(off + T * d_inner * 4, kAlign);
+  w.seg_state = off;
+  w.seg_decay = off;
+  if (n_seg > 1) {
+    off = round_up(off + (size_t)n_seg * c->batch * c->nheads * c->headdim * c->dstate * 4, kAlign);
+    w.seg_decay = off;
+    off = round_up(off + (size_t)n_seg * c->batch * c->nheads * 4, kAlign);
+  }
+  w.total = off;
+  return w;
+}
+
+ssd_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
+
+#define SSD_TRY(expr)                            \
+  do {                                           \
+    cudaError_t e_ = (expr);                     \
+    if (e_ != cudaSuccess) return SSD_ERR_CUDA;  \
+  } while (0)
+
+ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cudaStream_t s) {
+  ssd_status_t st = check_config(c, true);
+  if (st != SSD_OK) return st;
+  if (!a) return SSD_ERR_INVALID_ARG;
+  const int H = c->nheads, P = c->headdim, N = c->dstate, G = c->ngroups, W = c->conv_width;
+  const long long d_inner = (long long)H * P, conv_dim = d_inner + 2LL * G * N;
+  const size_t es = elt_size(c->io_dtype);
+  const bool has_tokens = c->seqlen > 0;
+  if (has_tokens) {
+    if (!a->xBC || !a->dt || !a->A || !a->D || !a->dt_bias || !a->y) return SSD_ERR_INVALID_ARG;
+    if (W > 0 && !a->conv_w) return SSD_ERR_INVALID_ARG;
+    if (c->norm_groups > 0 && !a->z) return SSD_ERR_INVALID_ARG;
+    if (a->xBC_row_stride < conv_dim || a->dt_row_stride < H || a->y_row_stride < d_inner)
+      return SSD_ERR_INVALID_ARG;
+    if (c->norm_groups > 0 && a->z_row_stride < d_inner) return SSD_ERR_INVALID_ARG;
+    if (!aligned16(a->xBC) || !aligned16(a->y) || (a->z && !aligned16(a->z)) ||
+        a->xBC_row_stride % 8 || a->y_row_stride % 8 || (a->z && a->z_row_stride % 8))
+      return SSD_ERR_ALIGNMENT;
+  }
+  if ((a->h0 && !aligned16(a->h0)) || (a->h_final && !aligned16(a->h_final)) ||
+      (a->conv_state_in && !aligned16(a->conv_state_in)) ||
+      (a->conv_state_out && !aligned16(a->conv_state_out)))
+    return SSD_ERR_ALIGNMENT;
+  const size_t cache_bytes = (size_t)c->batch * W * conv_dim * es;
+  if (a->conv_state_in && a->conv_state_out &&
+      ranges_overlap(a->conv_state_in, cache_bytes, a->conv_state_out, cache_bytes))
+    return SSD_ERR_INVALID_ARG;
+
+  PrefillPlan p{};
+  p.B = c->batch; p.L = c->seqlen; p.H = H; p.P = P; p.N = N; p.G = G; p.Q = c->chunk; p.W = W;
+  p.norm_groups = c->norm_groups; p.hpg = H / G; p.d_inner = (int)d_inner; p.conv_dim = (int)conv_dim;
+  p.eps = c->norm_eps; p.dt_min = c->dt_min; p.dt_max = c->dt_max; p.softplus = c->dt_softplus;
+  p.bf16 = c->io_dtype == SSD_BF16;
+  choose_segments(c, &p.n_seg, &p.seg_len);
+  p.xBC = a->xBC; p.xs = a->xBC_row_stride; p.dt = a->dt; p.ds = a->dt_row_stride;
+  p.z = a->z; p.zs = a->z_row_stride; p.A = a->A; p.D = a->D; p.dt_bias = a->dt_bias;
+  p.conv_w = a->conv_w; p.conv_b = a->conv_b; p.norm_w = a->norm_w; p.h0 = a->h0;
+  p.csi = a->conv_state_in; p.y = a->y; p.ys = a->y_row_stride; p.h_final = a->h_final;
+  p.cso = a->conv_state_out;
+  p.err = device_error_ptr();
+
+  if (!has_tokens) return from_cuda(traced("ssd_carry", s, [&] { return launch_carry_only(p, s); }));
+
+  const WsLayout lay = prefill_layout(c);
+  if (a->workspace_bytes < lay.total || (lay.total && !a->workspace) ||
+      (reinterpret_cast<uintptr_t>(a->workspace) % kAlign) != 0)
+    return SSD_ERR_WORKSPACE;
+  char *ws = static_cast<char *>(a->workspace);
+  p.u = reinterpret_cast<float *>(ws + lay.u);
+  p.dte = reinterpret_cast<float *>(ws + lay.dte);
+  p.yf = c->norm_groups > 0 ? reinterpret_cast<float *>(ws + lay.yf) : nullptr;
+  p.seg_state = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.seg_state) : nullptr;
+  p.seg_decay = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.seg_decay) : nullptr;
+
+  if (c->kernel == SSD_KERNEL_TENSOR) return SSD_ERR_UNSUPPORTED;
+
+  SSD_TRY(traced("ssd_dt", s, [&] { return launch_dt(p, s); }));
+  SSD_TRY(traced("ssd_conv_silu", s, [&] { return launch_conv_silu_f32(p, s); }));
+  if (p.n_seg == 1) {
+    SSD_TRY(traced("ssd_scan_simt", s, [&] { return launch_scan_simt(p, 0, s); }));
+  } else {
+    SSD_TRY(traced("ssd_scan_simt_states", s, [&] { return launch_scan_simt(p, 1, s); }));
+    SSD_TRY(traced("ssd_state_pass", s, [&] { return launch_state_pass(p, s); }));
+    SSD_TRY(traced("ssd_scan_simt", s, [&] { return launch_scan_simt(p, 2, s); }));
+  }
+  if (p.norm_groups > 0) SSD_TRY(traced("ssd_gated_norm", s, [&] { return launch_gated_norm(p, s); }));
+  SSD_TRY(traced("ssd_conv_state_out", s, [&] { return launch_conv_state_out(p, s); }));
+  return SSD_OK;
+}
+
+ssd_status_t run_decode(const ssd_config_t *c, const ssd_decode_args_t *a, cudaStream_t s) {
+  ssd_status_t st = check_config(c, false);
+  if (st != SSD_OK) return st;
+  if (!a) return SSD_ERR_INVALID_ARG;
+  const int H = c->nheads, P = c->headdim, N = c->dstate, G = c->ngroups, W = c->conv_width;
+  const long long d_inner = (long long)H * P, conv_dim = d_inner + 2LL * G * N;
+  if (!a->xBC || !a->dt || !a->A || !a->D || !a->dt_bias || !a->y || !a->state)
+    return SSD_ERR_INVALID_ARG;
+  if (W > 0 && (!a->conv_w || !a->conv_state_in || !a->conv_state_out)) return SSD_ERR_INVALID_ARG;
+  if (c->norm_groups > 0 && (!a->z || c->norm_groups % G != 0)) {
+    return !a->z ? SSD_ERR_INVALID_ARG : SSD_ERR_UNSUPPORTED;
+  }
+  if (a->xBC_row_stride < conv_dim || a->dt_row_stride < H || a->y_row_stride < d_inner ||
+      (c->norm_groups > 0 && a->z_row_stride < d_inner))
+    return SSD_ERR_INVALID_ARG;
+  if (!aligned16(a->xBC) || !aligned16(a->y) || !aligned16(a->state) || (a->z && !aligned16(a->z)) ||
+      (a->conv_state_in && !aligned16(a->conv_state_in)) ||
+      (a->conv_state_out && !aligned16(a->conv_state_out)) || a->xBC_row_stride % 8 ||
+      a->y_row_stride % 8 || (a->z && a->z_row_stride % 8))
+    return SSD_ERR_ALIGNMENT;
+  const size_t cache_bytes = (size_t)c->batch * W * conv_dim * elt_size(c->io_dtype);
+  if (W > 0 && ranges_overlap(a->conv_state_in, cache_bytes, a->conv_state_out, cache_bytes))
+    return SSD_ERR_INVALID_ARG;
+  if ((long long)(H / G) * P > 8192) return SSD_ERR_UNSUPPORTED;  // group staged in shared memory
+  DecodePlan p{};
+  p.B = c->batch; p.H = H; p.P = P; p.N = N; p.G = G; p.W = W; p.norm_groups = c->norm_groups;
+  p.hpg = H / G; p.d_inner = (int)d_inner; p.conv_dim = (int)conv_dim; p.eps = c->norm_eps;
+  p.dt_min = c->dt_min; p.dt_max = c->dt_max; p.softplus = c->dt_softplus;
+  p.bf16 = c->io_dtype == SSD_BF16;
+  p.xBC = a->xBC; p.xs = a->xBC_row_stride; p.dt = a->dt; p.ds = a->dt_row_stride; p.z = a->z;
+  p.zs = a->z_row_stride; p.A = a->A; p.D = a->D; p.dt_bias = a->dt_bias; p.conv_w = a->conv_w;
+  p.conv_b = a->conv_b; p.norm_w = a->norm_w; p.state = a->state; p.csi = a->conv_state_in;
+  p.cso = a->conv_state_out; p.y = a->y; p.ys = a->y_row_stride;
+  return from_cuda(traced("ssd_decode", s, [&] { return launch_decode(p, s); }));
+}
+
+struct MixerLayout {
+  size_t hn, zxbcdt, g, ssd, total;
+  ssd_config_t scfg;
+};
+
+MixerLayout mixer_layout(const ssd_mixer_config_t *m) {
+  MixerLayout l{};
+  l.scfg = m->ssd;
+  const size_t T = (size_t)m->ssd.batch * m->ssd.seqlen;
+  const size_t d_inner = (size_t)m->ssd.nheads * m->ssd.headdim;
+  const size_t proj = 2 * d_inner + 2 * (size_t)m->ssd.ngroups * m->ssd.dstate + m->ssd.nheads;
+  const size_t proj_pad = round_up(proj, 8);
+  size_t off = 0;
+  l.hn = off;      off = round_up(off + T * m->d_model * 2, kAlign);
+  l.zxbcdt = off;  off = round_up(off + T * proj_pad * 2, kAlign);
+  l.g = off;       off = round_up(off + T * d_inner * 2, kAlign);
+  l.ssd = off;     off = round_up(off + prefill_layout(&l.scfg).total, kAlign);
+  l.total = off;
+  return l;
+}
+
+ssd_status_t run_mixer(const ssd_mixer_config_t *m, const ssd_mixer_args_t *a, cudaStream_t s) {
+  if (!m || !a) return SSD_ERR_INVALID_ARG;
+  ssd_status_t st = check_config(&m->ssd, true);
+  if (st != SSD_OK) return st;
+  if (m->ssd.io_dtype != SSD_BF16 || m->ssd.seqlen < 1) return SSD_ERR_UNSUPPORTED;
+  if (m->d_model < 64 || m->d_model % 64 != 0) return SSD_ERR_UNSUPPORTED;
+  if (!a->hidden || !a->W_in || !a->W_out || !a->out) return SSD_ERR_INVALID_ARG;
+  if (!aligned16(a->hidden) || !aligned16(a->W_in) || !aligned16(a->W_out) || !aligned16(a->out) ||
+      (a->rms_w && !aligned16(a->rms_w)))
+    return SSD_ERR_ALIGNMENT;
+  const MixerLayout l = mixer_layout(m);
+  if (!a->workspace || a->workspace_bytes < l.total ||
+      (reinterpret_cast<uintptr_t>(a->workspace) % kAlign) != 0)
+    return SSD_ERR_WORKSPACE;
+  const int H = m->ssd.nheads, P = m->ssd.headdim, N = m->ssd.dstate, G = m->ssd.ngroups;
+  const long long d_inner = (long long)H * P, conv_dim = d_inner + 2LL * G * N;
+  const long long proj = 2 * d_inner + 2LL * G * N + H, proj_pad = (long long)round_up(proj, 8);
+  const long long T = (long long)m->ssd.batch * m->ssd.seqlen;
+  if (T > INT32_MAX) return SSD_ERR_UNSUPPORTED;
+  char *ws = static_cast<char *>(a->workspace);
+  void *hn = ws + l.hn, *zx = ws + l.zxbcdt, *g = ws + l.g;
+  SSD_TRY(traced("ssd_rmsnorm", s, [&] {
+    return launch_rmsnorm_bf16(a->hidden, a->rms_w, hn, T, m->d_model, m->rms_eps, s);
+  }));
+  SSD_TRY(traced("gemm_in_proj", s, [&] {
+    return launch_gemm_bf16_tn(hn, m->d_model, a->W_in, m->d_model, zx, proj_pad, (int)T, (int)proj,
+                               m->d_model, s);
+  }));
+  const __nv_bfloat16 *zxb = static_cast<const __nv_bfloat16 *>(zx);
+  ssd_prefill_args_t pa{};
+  pa.z = zxb;                         pa.z_row_stride = proj_pad;
+  pa.xBC = zxb + d_inner;             pa.xBC_row_stride = proj_pad;
+  pa.dt = zxb + d_inner + conv_dim;   pa.dt_row_stride = proj_pad;
+  pa.A = a->A; pa.D = a->D; pa.dt_bias = a->dt_bias; pa.conv_w = a->conv_w; pa.conv_b = a->conv_b;
+  pa.norm_w = a->norm_w; pa.h0 = a->h0; pa.conv_state_in = a->conv_state_in;
+  pa.y = g; pa.y_row_stride = d_inner; pa.h_final = a->h_final; pa.conv_state_out = a->conv_state_out;
+  pa.workspace = ws + l.ssd; pa.workspace_bytes = l.total - l.ssd;
+  st = run_prefill(&l.scfg, &pa, s);
+  if (st != SSD_OK) return st;
+  SSD_TRY(traced("gemm_out_proj", s, [&] {
+    return launch_gemm_bf16_tn(g, d_inner, a->W_out, d_inner, a->out, m->d_model, (int)T, m->d_model,
+                               (int)d_inner, s);
+  }));
+  return SSD_OK;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_bf16_tn(const void *A, long long lda, const void *Bm, long long ldb, void *C,
+                                long long ldc, int M, int N, int K, cudaStream_t s) {
+  return launch_gemm_simt_bf16_tn(A, lda, Bm, ldb, C, ldc, M, N, K, s);
+}
+
+}  // namespace ssd
+
+using namespace ssd;
+
+extern "C" {
+
+size_t ssd_workspace_size(const ssd_config_t *cfg) {
+  if (check_config(cfg, true) != SSD_OK) return 0;
+  return prefill_layout(cfg).total;
+}
+
+ssd_status_t ssd_prefill(const ssd_config_t *cfg, const ssd_prefill_args_t *args, void *stream) {
+  return run_prefill(cfg, args, static_cast<cudaStream_t>(stream));
+}
+
+ssd_status_t ssd_decode_step(const ssd_config_t *cfg, const ssd_decode_args_t *args, void *stream) {
+  return run_decode(cfg, args, static_cast<cudaStream_t>(stream));
+}
+
+size_t ssd_mixer_workspace_size(const ssd_mixer_config_t *cfg) {
+  if (!cfg || check_config(&cfg->ssd, true) != SSD_OK) return 0;
+  return mixer_layout(cfg).total;
+}
+
+ssd_status_t mamba2_mixer_forward(const ssd_mixer_config_t *cfg, const ssd_mixer_args_t *args,
+                                  void *stream) {
+  return run_mixer(cfg, args, static_cast<cudaStream_t>(stream));
+}
+
+const char *ssd_status_string(ssd_status_t s) {
+  switch (s) {
+    case SSD_OK: return "SSD_OK";
+    case SSD_ERR_INVALID_ARG: return "SSD_ERR_INVALID_ARG: missing or inconsistent argument";
+    case SSD_ERR_UNSUPPORTED: return "SSD_ERR_UNSUPPORTED: shape or option not implemented";
+    case SSD_ERR_ALIGNMENT: return "SSD_ERR_ALIGNMENT: pointer or row stride not 16-byte aligned";
+    case SSD_ERR_CUDA: return "SSD_ERR_CUDA: CUDA runtime call or launch failed";
+    case SSD_ERR_TIMEOUT: return "SSD_ERR_TIMEOUT: a bounded device-side wait gave up";
+    case SSD_ERR_DEVICE_BOUNDS: return "SSD_ERR_DEVICE_BOUNDS: device-side index check failed";
+    case SSD_ERR_WORKSPACE: return "SSD_ERR_WORKSPACE: workspace missing, misaligned or too small";
+  }
+  return "unknown ssd_status_t";
+}
+
+ssd_status_t ssd_get_device_error(void *stream) {
+  int *p = device_error_ptr();
+  if (!p) return SSD_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SSD_ERR_CUDA;
+  if (cudaMemcpy(&v, p, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return SSD_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return SSD_ERR_CUDA;
+  }
+  return static_cast<ssd_status_t>(v);
+}
+
+int ssd_version(void) { return 100; }
+
+}  // extern "C"

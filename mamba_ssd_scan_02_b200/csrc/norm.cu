@@ -1,0 +1,101 @@
+// norm.cu -- the z-gated RMSNorm applied to the scan output, and the plain RMSNorm at the
+// mixer input.  The Nemotron Nano 2 layers normalise with RMSNorm ("NVIDIA Nemotron Nano 2"
+// summary, section "Method"); in the Mamba-2 mixer the scan output is gated by SiLU(z) and
+// then normalised over groups of d_inner / norm_groups consecutive channels:
+//   g = y * silu(z);   out = g / sqrt(mean_group(g^2) + eps) * w
+#include "common.cuh"
+#include "plan.h"
+
+namespace ssd {
+namespace {
+
+constexpr int kNormThreads = 256;
+
+__device__ float block_sum(float v, float *red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x / 32, l = threadIdx.x % 32;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float t = threadIdx.x < blockDim.x / 32 ? red[threadIdx.x] : 0.f;
+  if (w == 0) {
+    t = warp_sum(t);
+    if (l == 0) red[0] = t;
+  }
+  __syncthreads();
+  return red[0];
+}
+
+// One CTA per (row, norm group).  y is fp32 [rows, d_inner] dense; z/out/w in the io dtype.
+template <typename T>
+__global__ void __launch_bounds__(kNormThreads) gated_norm_kernel(
+    const float *__restrict__ y, const T *__restrict__ z, long long zs, const T *__restrict__ w,
+    T *__restrict__ out, long long os, int d_inner, int gs, float eps, int L) {
+  __shared__ float red[32];
+  const long long row = blockIdx.x;
+  const int c0 = blockIdx.y * gs;
+  const float *yr = y + row * d_inner + c0;
+  const T *zr = z + row * zs + c0;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < gs; i += kNormThreads) {
+    const float gv = yr[i] * silu(io<T>::ld(zr + i));
+    ss += gv * gv;
+  }
+  ss = block_sum(ss, red);
+  const float r = rsqrtf(ss / gs + eps);
+  T *orow = out + row * os + c0;
+  for (int i = threadIdx.x; i < gs; i += kNormThreads) {
+    const float gv = yr[i] * silu(io<T>::ld(zr + i));
+    io<T>::st(orow + i, gv * r * (w ? io<T>::ld(w + c0 + i) : 1.f));
+  }
+}
+
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_bf16_kernel(
+    const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w,
+    __nv_bfloat16 *__restrict__ out, int width, float eps) {
+  __shared__ float red[32];
+  const long long row = blockIdx.x;
+  const __nv_bfloat16 *xr = x + row * width;
+  float ss = 0.f;
+  for (int i = threadIdx.x * 8; i < width; i += kNormThreads * 8) {
+    float v[8];
+    load8(xr + i, v);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) ss += v[k] * v[k];
+  }
+  ss = block_sum(ss, red);
+  const float r = rsqrtf(ss / width + eps);
+  for (int i = threadIdx.x * 8; i < width; i += kNormThreads * 8) {
+    float v[8], wv[8];
+    load8(xr + i, v);
+    if (w) load8(w + i, wv);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = v[k] * r * (w ? wv[k] : 1.f);
+    store8(out + row * width + i, v);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s) {
+  const int gs = p.d_inner / p.norm_groups;
+  dim3 grid((unsigned)((long long)p.B * p.L), p.norm_groups);
+  if (p.bf16)
+    gated_norm_kernel<__nv_bfloat16><<<grid, kNormThreads, 0, s>>>(
+        p.yf, (const __nv_bfloat16 *)p.z, p.zs, (const __nv_bfloat16 *)p.norm_w,
+        (__nv_bfloat16 *)p.y, p.ys, p.d_inner, gs, p.eps, p.L);
+  else
+    gated_norm_kernel<float><<<grid, kNormThreads, 0, s>>>(p.yf, (const float *)p.z, p.zs,
+                                                           (const float *)p.norm_w, (float *)p.y,
+                                                           p.ys, p.d_inner, gs, p.eps, p.L);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm_bf16(const void *x, const void *w, void *out, long long rows, int width,
+                                float eps, cudaStream_t s) {
+  rmsnorm_bf16_kernel<<<(unsigned)rows, kNormThreads, 0, s>>>(
+      (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)w, (__nv_bfloat16 *)out, width, eps);
+  return cudaGetLastError();
+}
+
+}  // namespace ssd

@@ -1,0 +1,90 @@
+// plan.h -- resolved launch parameters shared by the C-ABI layer and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "../../include/ssd.h"
+
+namespace ssd {
+
+// Everything a prefill launch needs, after validation: shapes, pointers, workspace carve-outs.
+struct PrefillPlan {
+  int B, L, H, P, N, G, Q, W, norm_groups;
+  int hpg, d_inner, conv_dim;
+  float eps, dt_min, dt_max;
+  int softplus;
+  bool bf16;
+  int n_seg, seg_len;  // internal sequence segments (1 = none)
+  // user tensors
+  const void *xBC; long long xs;
+  const void *dt;  long long ds;
+  const void *z;   long long zs;
+  const float *A, *D, *dt_bias;
+  const void *conv_w, *conv_b, *norm_w;
+  const float *h0;
+  const void *csi;
+  void *y; long long ys;
+  float *h_final;
+  void *cso;
+  // workspace
+  float *u;          // [B, L, conv_dim] conv+SiLU output (SIMT path)
+  float *dte;        // [B, L, H] effective dt
+  float *yf;         // [B, L, d_inner] pre-norm output (when norm_groups > 0)
+  float *seg_state;  // [n_seg, B, H, P, N]
+  float *seg_decay;  // [n_seg, B, H]
+  void *bc;          // [B, L, 2*G*N] bf16 conv+SiLU output of the B|C channels (tensor path)
+  int *err;          // device error word
+};
+
+struct DecodePlan {
+  int B, H, P, N, G, W, norm_groups, hpg, d_inner, conv_dim;
+  float eps, dt_min, dt_max;
+  int softplus;
+  bool bf16;
+  const void *xBC; long long xs;
+  const void *dt;  long long ds;
+  const void *z;   long long zs;
+  const float *A, *D, *dt_bias;
+  const void *conv_w, *conv_b, *norm_w;
+  float *state;
+  const void *csi;
+  void *cso;
+  void *y; long long ys;
+};
+
+// front end (frontend.cu)
+cudaError_t launch_conv_silu_f32(const PrefillPlan &p, cudaStream_t s);
+cudaError_t launch_dt(const PrefillPlan &p, cudaStream_t s);
+cudaError_t launch_conv_state_out(const PrefillPlan &p, cudaStream_t s);
+cudaError_t launch_carry_only(const PrefillPlan &p, cudaStream_t s);  // seqlen == 0
+// chunked scan on CUDA cores (scan_simt.cu); mode 0 full, 1 state-only, 2 output-only
+cudaError_t launch_scan_simt(const PrefillPlan &p, int mode, cudaStream_t s);
+// inter-segment state pass (state_pass.cu)
+cudaError_t launch_state_pass(const PrefillPlan &p, cudaStream_t s);
+// norms (norm.cu)
+cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s);
+cudaError_t launch_rmsnorm_bf16(const void *x, const void *w, void *out, long long rows, int width,
+                                float eps, cudaStream_t s);
+// decode (decode.cu)
+cudaError_t launch_decode(const DecodePlan &p, cudaStream_t s);
+// GEMM C[M,N] = A[M,K] . B[N,K]^T, bf16 in/out, fp32 accumulate
+cudaError_t launch_gemm_bf16_tn(const void *A, long long lda, const void *Bm, long long ldb, void *C,
+                                long long ldc, int M, int N, int K, cudaStream_t s);
+cudaError_t launch_gemm_simt_bf16_tn(const void *A, long long lda, const void *Bm, long long ldb,
+                                     void *C, long long ldc, int M, int N, int K, cudaStream_t s);
+
+// ---- tracing (trace.cu): event pairs around each launch while enabled ------------------
+bool trace_enabled();
+int trace_begin(cudaStream_t s);                        // -1 when tracing is off
+void trace_end(int slot, const char *name, cudaStream_t s);
+
+template <class F>
+cudaError_t traced(const char *name, cudaStream_t s, F &&launch) {
+  const int slot = trace_begin(s);
+  cudaError_t e = launch();
+  if (slot >= 0) trace_end(slot, name, s);
+  return e;
+}
+
+}  // namespace ssd

@@ -1,0 +1,50 @@
+// state_pass.cu -- inter-segment state pass of the segmented chunked scan.
+//
+// When a sequence is split into n_seg segments scanned in parallel, each segment k first
+// produces its local final state s_k (scanned from a zero state) and its total decay
+// lambda_k = exp(sum of dt*A over the segment).  The state entering segment k is then
+//   h_in[0] = h0,   h_in[k] = lambda_{k-1} h_in[k-1] + s_{k-1},
+// and the state after the last segment is lambda_{n-1} h_in[n-1] + s_{n-1} = h_final.
+// This is the same linear recurrence as the token scan, applied at segment granularity.
+// One thread per 4 state elements (float4), sequential over the segments; h_in[k]
+// overwrites s_k in place (s_k is read first).
+#include "common.cuh"
+#include "plan.h"
+
+namespace ssd {
+namespace {
+
+__global__ void state_pass_kernel(float4 *__restrict__ seg_state, const float *__restrict__ seg_decay,
+                                  const float4 *__restrict__ h0, float4 *__restrict__ h_final,
+                                  int n_seg, long long BH, int PN4) {
+  const long long n = BH * PN4;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long bh = i / PN4;
+    float4 h = h0 ? h0[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = 0; k < n_seg; ++k) {
+      float4 *slot = seg_state + (long long)k * BH * PN4 + i;
+      const float4 s = *slot;
+      *slot = h;
+      const float a = seg_decay[(long long)k * BH + bh];
+      h = make_float4(a * h.x + s.x, a * h.y + s.y, a * h.z + s.z, a * h.w + s.w);
+    }
+    if (h_final) h_final[i] = h;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_state_pass(const PrefillPlan &p, cudaStream_t s) {
+  const long long BH = (long long)p.B * p.H;
+  const int PN4 = p.P * p.N / 4;
+  const long long n = BH * PN4;
+  long long g = (n + 255) / 256;
+  if (g > 148 * 8) g = 148 * 8;
+  state_pass_kernel<<<(int)g, 256, 0, s>>>(reinterpret_cast<float4 *>(p.seg_state), p.seg_decay,
+                                           reinterpret_cast<const float4 *>(p.h0),
+                                           reinterpret_cast<float4 *>(p.h_final), p.n_seg, BH, PN4);
+  return cudaGetLastError();
+}
+
+}  // namespace ssd

@@ -116,7 +116,7 @@ class Oracle:
         L.oracle_rmsnorm.argtypes = [cll, ci, vp, ci, vp, ci, cd, vp]
         L.oracle_decode_step.restype = None
         L.oracle_decode_step.argtypes = [ctypes.POINTER(_Shape), vp, ci, vp, ci, vp, vp, vp, ci,
-                                         vp, vp, ci, vp, ci, vp, vp, ci, ci, vp]
+                                         vp, vp, ci, vp, ci, vp, vp, ci, ci, vp, ci]
 
     # ---- scalar helpers -------------------------------------------------------------------
     def silu(self, x: float) -> float:
@@ -231,7 +231,8 @@ class Oracle:
 
     # ---- decode -----------------------------------------------------------------------------
     def decode_step(self, cfg: dict, xBC_t, dt_t, A, D, dt_bias, conv_w, conv_b, conv_state_in,
-                    state: np.ndarray, z_t=None, norm_w=None, heads=None) -> dict:
+                    state: np.ndarray, z_t=None, norm_w=None, heads=None,
+                    threads: int | None = None) -> dict:
         """One token per batch row.  ``state`` [B, nh, P, N] float64 is updated in place.
         Returns y (pre-gate [B, nh, P]), out (gated norm, if norm_groups), conv_state_out."""
         Bn, H, P, N, G = cfg["batch"], cfg["nheads"], cfg["headdim"], cfg["dstate"], cfg["ngroups"]
@@ -253,7 +254,8 @@ class Oracle:
         self.lib.oracle_decode_step(ctypes.byref(shape), _p(xBC_t), _code(xBC_t), _p(dt_t),
                                     _code(dt_t), _p(A), _p(D), _p(dt_bias), _F64, _p(conv_w),
                                     _p(conv_b), _F64, _p(csi), _code(csi), _p(cso),
-                                    _p(state), lo, hi, _p(y))
+                                    _p(state), lo, hi, _p(y),
+                                    int(threads if threads else (os.cpu_count() or 1)))
         res = {"y": y, "conv_state_out": cso}
         ng = cfg.get("norm_groups", 0)
         if ng:

@@ -274,45 +274,51 @@ void oracle_decode_step(const oracle_shape_t *s, const void *xBC_t, int xdt, con
                         int ddt, const void *A, const void *D, const void *dt_bias, int pdt,
                         const void *conv_w, const void *conv_b, int cdt, const void *conv_state_in,
                         int sdt, double *conv_state_out, double *state, int h_lo, int h_hi,
-                        double *y) {
+                        double *y, int threads) {
   const int Bn = s->batch, H = s->nheads, P = s->headdim, N = s->dstate, G = s->ngroups;
   const int W = s->conv_width, hpg = H / G, d_inner = H * P, conv_dim = d_inner + 2 * G * N;
   const int nh = h_hi - h_lo;
-  double *cache = (double *)malloc(sizeof(double) * (W > 0 ? W : 1) * conv_dim);
-  double *u = (double *)malloc(sizeof(double) * conv_dim);
+  const int Wr = W > 0 ? W : 1;
+  double *cache = (double *)malloc(sizeof(double) * (size_t)Bn * Wr * conv_dim);
+  double *u = (double *)malloc(sizeof(double) * (size_t)Bn * conv_dim);
   for (int b = 0; b < Bn; ++b) {
+    double *cb = cache + (size_t)b * Wr * conv_dim, *ub = u + (size_t)b * conv_dim;
     /* shift the cache and append the new raw input */
     for (int c = 0; c < conv_dim; ++c) {
       for (int k = 0; k + 1 < W; ++k)
-        cache[k * conv_dim + c] = ld(conv_state_in, sdt, ((long long)b * W + k + 1) * conv_dim + c);
-      if (W > 0) cache[(W - 1) * conv_dim + c] = ld(xBC_t, xdt, (long long)b * conv_dim + c);
+        cb[k * conv_dim + c] = ld(conv_state_in, sdt, ((long long)b * W + k + 1) * conv_dim + c);
+      if (W > 0) cb[(W - 1) * conv_dim + c] = ld(xBC_t, xdt, (long long)b * conv_dim + c);
     }
     for (int c = 0; c < conv_dim; ++c) {
       if (W == 0) {
-        u[c] = ld(xBC_t, xdt, (long long)b * conv_dim + c);
+        ub[c] = ld(xBC_t, xdt, (long long)b * conv_dim + c);
         continue;
       }
       double acc = conv_b ? ld(conv_b, cdt, c) : 0.0;
-      for (int k = 0; k < W; ++k) acc += ld(conv_w, cdt, (long long)c * W + k) * cache[k * conv_dim + c];
-      u[c] = oracle_silu(acc);
+      for (int k = 0; k < W; ++k) acc += ld(conv_w, cdt, (long long)c * W + k) * cb[k * conv_dim + c];
+      ub[c] = oracle_silu(acc);
     }
     if (conv_state_out && W > 0)
-      memcpy(conv_state_out + (long long)b * W * conv_dim, cache, sizeof(double) * W * conv_dim);
-    for (int hi = 0; hi < nh; ++hi) {
-      const int h = h_lo + hi, g = h / hpg;
-      const double dt = oracle_dt(ld(dt_t, ddt, (long long)b * H + h), ld(dt_bias, pdt, h),
-                                  s->dt_softplus, s->dt_min, s->dt_max);
-      const double a = exp(dt * ld(A, pdt, h)), Dh = ld(D, pdt, h);
-      double *st = state + ((long long)b * nh + hi) * P * N;
-      const double *ux = u + h * P, *uB = u + d_inner + g * N, *uC = u + d_inner + G * N + g * N;
-      for (int p = 0; p < P; ++p) {
-        double acc = 0.0;
-        for (int n = 0; n < N; ++n) {
-          st[p * N + n] = a * st[p * N + n] + dt * ux[p] * uB[n];
-          acc += st[p * N + n] * uC[n];
-        }
-        y[((long long)b * nh + hi) * P + p] = acc + Dh * ux[p];
+      memcpy(conv_state_out + (long long)b * W * conv_dim, cb, sizeof(double) * W * conv_dim);
+  }
+  const long long pairs = (long long)Bn * nh;
+#pragma omp parallel for schedule(static) num_threads(threads > 0 ? threads : 1)
+  for (long long pr = 0; pr < pairs; ++pr) {
+    const int b = (int)(pr / nh), hi = (int)(pr % nh);
+    const int h = h_lo + hi, g = h / hpg;
+    const double *ub = u + (size_t)b * conv_dim;
+    const double dt = oracle_dt(ld(dt_t, ddt, (long long)b * H + h), ld(dt_bias, pdt, h),
+                                s->dt_softplus, s->dt_min, s->dt_max);
+    const double a = exp(dt * ld(A, pdt, h)), Dh = ld(D, pdt, h);
+    double *st = state + ((long long)b * nh + hi) * P * N;
+    const double *ux = ub + h * P, *uB = ub + d_inner + g * N, *uC = ub + d_inner + G * N + g * N;
+    for (int p = 0; p < P; ++p) {
+      double acc = 0.0;
+      for (int n = 0; n < N; ++n) {
+        st[p * N + n] = a * st[p * N + n] + dt * ux[p] * uB[n];
+        acc += st[p * N + n] * uC[n];
       }
+      y[((long long)b * nh + hi) * P + p] = acc + Dh * ux[p];
     }
   }
   free(cache);
