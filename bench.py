@@ -316,28 +316,37 @@ def bench_decode(args, rank, world, torch, ssd, dist, steps_total=16384, graph_s
 
 
 def cpu_baseline(target_s: float = 10.0):
-    """fp64 oracle on a bounded sample of the prefill workload (one norm group of heads,
-    a token prefix), scaled to tokens/s of the whole layer."""
+    """fp64 oracle on a bounded sample of the prefill workload (a token prefix of whole norm
+    groups of heads), scaled to tokens/s of the whole layer."""
     import oracle
     o = oracle.get()
     cfg = datagen.config(1)
     inp = datagen.make_inputs(1)
     cores = os.cpu_count() or 1
-    heads = (0, 16)
-    tok = 512
+    tok, groups, reps = 512, 1, 1
+    hpg = cfg["nheads"] // cfg["ngroups"]
     while True:
         t0 = time.time()
-        o.ssd_prefill(dict(cfg, seqlen=tok), inp["xBC"][:, :tok], inp["dt"][:, :tok], inp["A"],
-                      inp["D"], inp["dt_bias"], conv_w=inp["conv_w"], heads=heads, threads=cores)
+        for _ in range(reps):
+            o.ssd_prefill(dict(cfg, seqlen=tok), inp["xBC"][:, :tok], inp["dt"][:, :tok],
+                          inp["A"], inp["D"], inp["dt_bias"], conv_w=inp["conv_w"],
+                          heads=(0, groups * hpg), threads=cores)
         dt = time.time() - t0
-        if dt >= target_s or tok >= cfg["seqlen"]:
+        if dt >= target_s:
             break
-        tok = min(cfg["seqlen"], int(tok * max(2.0, min(8.0, target_s / max(dt, 1e-3)))))
-    frac = (heads[1] - heads[0]) / cfg["nheads"]
-    return {"value": round(tok * frac / dt, 2), "unit": "tokens/s", "cores": cores,
+        grow = max(2.0, min(8.0, target_s / max(dt, 1e-3)))
+        if tok < cfg["seqlen"]:
+            tok = min(cfg["seqlen"], int(tok * grow))
+        elif groups < cfg["ngroups"]:
+            groups = min(cfg["ngroups"], int(groups * grow))
+        else:
+            reps = int(reps * grow) + 1
+    frac = groups / cfg["ngroups"]
+    return {"value": round(reps * tok * frac / dt, 2), "unit": "tokens/s", "cores": cores,
             "kind": "oracle",
-            "sample": f"prefill_8k inputs, first {tok} tokens x heads {heads[0]}-{heads[1] - 1} "
-                      f"(1/{int(1 / frac)} of the layer), fp64, {dt:.1f} s"}
+            "sample": f"prefill_8k inputs, first {tok} tokens x heads 0-{groups * hpg - 1} "
+                      f"({groups}/{cfg['ngroups']} of the layer) x {reps} run(s), fp64, "
+                      f"{dt:.1f} s"}
 
 
 def reference_arm(args):

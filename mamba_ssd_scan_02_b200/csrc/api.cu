@@ -59,51 +59,82 @@ ssd_status_t check_config(const ssd_config_t *c, bool prefill) {
   return SSD_OK;
 }
 
-// Internal sequence segments: enough (b, h, segment) CTAs to fill the GPU, each segment a
-// whole number of chunks and at least four 64-token tiles long.
-void choose_segments(const ssd_config_t *c, int *n_seg, int *seg_len) {
-  const int L = c->seqlen, Q = c->chunk;
+// Internal sequence segments: each a whole number of `tile`-token chunks, enough
+// (b, h, segment) CTAs to fill `target` CTA slots, and at least four tiles long.
+void choose_segments(const ssd_config_t *c, int tile, long long target, int *n_seg, int *seg_len) {
+  const int L = c->seqlen;
   int n = c->n_segments;
   if (n == 0) {
     const long long bh = (long long)c->batch * c->nheads;
     n = 1;
-    if (bh < kTargetCtas && L > 4 * 64) {
-      n = (int)((kTargetCtas + bh - 1) / bh);
-      n = n < L / (4 * 64) ? n : L / (4 * 64);
+    if (bh < target && L > 4 * tile) {
+      n = (int)(target / bh);
+      n = n < L / (4 * tile) ? n : L / (4 * tile);
       if (n > 64) n = 64;
       if (n < 1) n = 1;
     }
   }
   if (n < 1) n = 1;
-  long long len = L > 0 ? ((long long)L + n - 1) / n : Q;
-  len = (len + Q - 1) / Q * Q;
+  long long len = L > 0 ? ((long long)L + n - 1) / n : tile;
+  len = (len + tile - 1) / tile * tile;
   *seg_len = (int)len;
   *n_seg = L > 0 ? (int)((L + len - 1) / len) : 1;
 }
 
+constexpr int kTcTile = 128;       // tokens per chunk of the tensor-core scan
+constexpr long long kTcTarget = 148;  // one tensor-core scan CTA per SM
+
+void simt_segments(const ssd_config_t *c, int *n, int *len) {
+  choose_segments(c, c->chunk, kTargetCtas, n, len);
+}
+void tc_segments(const ssd_config_t *c, int *n, int *len) {
+  choose_segments(c, kTcTile, kTcTarget, n, len);
+}
+
+// The two scan paths use the workspace differently; the layouts overlap (a call uses one).
 struct WsLayout {
-  size_t u, dte, yf, seg_state, seg_decay, total;
+  // CUDA-core path
+  size_t u, dte, yf, seg_state, seg_decay, simt_end;
+  // tensor-core path
+  size_t tc_bc, tc_dte, tc_cs, tc_yf, tc_seg_state, tc_seg_decay, tc_end;
+  int Lpad;
+  size_t total;
 };
 
 WsLayout prefill_layout(const ssd_config_t *c) {
   WsLayout w{};
-  int n_seg, seg_len;
-  choose_segments(c, &n_seg, &seg_len);
   const size_t T = (size_t)c->batch * c->seqlen;
   const size_t d_inner = (size_t)c->nheads * c->headdim;
   const size_t conv_dim = d_inner + 2 * (size_t)c->ngroups * c->dstate;
+  const size_t state = (size_t)c->batch * c->nheads * c->headdim * c->dstate * 4;
+  int n_seg, seg_len;
+  simt_segments(c, &n_seg, &seg_len);
   size_t off = 0;
-  w.u = off;         off = round_up(off + T * conv_dim * 4, kAlign);
-  w.dte = off;       off = round_up(off + T * c->nheads * 4, kAlign);
-  w.yf = off;        if (c->norm_groups > 0) off = round_up(off + T * d_inner * 4, kAlign);
-  w.seg_state = off;
-  w.seg_decay = off;
+  w.u = off;    off = round_up(off + T * conv_dim * 4, kAlign);
+  w.dte = off;  off = round_up(off + T * c->nheads * 4, kAlign);
+  w.yf = off;   if (c->norm_groups > 0) off = round_up(off + T * d_inner * 4, kAlign);
+  w.seg_state = w.seg_decay = off;
   if (n_seg > 1) {
-    off = round_up(off + (size_t)n_seg * c->batch * c->nheads * c->headdim * c->dstate * 4, kAlign);
+    off = round_up(off + (size_t)n_seg * state, kAlign);
     w.seg_decay = off;
     off = round_up(off + (size_t)n_seg * c->batch * c->nheads * 4, kAlign);
   }
-  w.total = off;
+  w.simt_end = off;
+  tc_segments(c, &n_seg, &seg_len);
+  w.Lpad = (int)((c->seqlen + kTcTile - 1) / kTcTile * kTcTile);
+  off = 0;
+  w.tc_bc = off;   off = round_up(off + T * 2 * c->ngroups * c->dstate * 2, kAlign);
+  w.tc_dte = off;  off = round_up(off + (size_t)c->batch * c->nheads * w.Lpad * 4, kAlign);
+  w.tc_cs = off;   off = round_up(off + (size_t)c->batch * c->nheads * w.Lpad * 4, kAlign);
+  w.tc_yf = off;   if (c->norm_groups > 0) off = round_up(off + T * d_inner * 4, kAlign);
+  w.tc_seg_state = w.tc_seg_decay = off;
+  if (n_seg > 1) {
+    off = round_up(off + (size_t)n_seg * state, kAlign);
+    w.tc_seg_decay = off;
+    off = round_up(off + (size_t)n_seg * c->batch * c->nheads * 4, kAlign);
+  }
+  w.tc_end = off;
+  w.total = w.simt_end > w.tc_end ? w.simt_end : w.tc_end;
   return w;
 }
 
@@ -148,7 +179,6 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
   p.norm_groups = c->norm_groups; p.hpg = H / G; p.d_inner = (int)d_inner; p.conv_dim = (int)conv_dim;
   p.eps = c->norm_eps; p.dt_min = c->dt_min; p.dt_max = c->dt_max; p.softplus = c->dt_softplus;
   p.bf16 = c->io_dtype == SSD_BF16;
-  choose_segments(c, &p.n_seg, &p.seg_len);
   p.xBC = a->xBC; p.xs = a->xBC_row_stride; p.dt = a->dt; p.ds = a->dt_row_stride;
   p.z = a->z; p.zs = a->z_row_stride; p.A = a->A; p.D = a->D; p.dt_bias = a->dt_bias;
   p.conv_w = a->conv_w; p.conv_b = a->conv_b; p.norm_w = a->norm_w; p.h0 = a->h0;
@@ -163,14 +193,42 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
       (reinterpret_cast<uintptr_t>(a->workspace) % kAlign) != 0)
     return SSD_ERR_WORKSPACE;
   char *ws = static_cast<char *>(a->workspace);
+
+  bool use_tc = false;
+  if (c->kernel == SSD_KERNEL_TENSOR) {
+    if (!p.bf16 || !tc_scan_available()) return SSD_ERR_UNSUPPORTED;
+    use_tc = true;
+  } else if (c->kernel == SSD_KERNEL_AUTO) {
+    use_tc = p.bf16 && tc_scan_available();
+  }
+
+  if (use_tc) {
+    tc_segments(c, &p.n_seg, &p.seg_len);
+    p.Lpad = lay.Lpad;
+    p.bc = ws + lay.tc_bc;
+    p.dte_hm = reinterpret_cast<float *>(ws + lay.tc_dte);
+    p.cs_hm = reinterpret_cast<float *>(ws + lay.tc_cs);
+    p.yf = c->norm_groups > 0 ? reinterpret_cast<float *>(ws + lay.tc_yf) : nullptr;
+    p.seg_state = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.tc_seg_state) : nullptr;
+    p.seg_decay = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.tc_seg_decay) : nullptr;
+    SSD_TRY(traced("ssd_dt_cumsum", s, [&] { return launch_dt_cumsum(p, p.dte_hm, p.cs_hm, p.Lpad, s); }));
+    SSD_TRY(traced("ssd_bc_conv", s, [&] { return launch_bc_conv_f16(p, s); }));
+    if (p.n_seg > 1) {
+      SSD_TRY(traced("ssd_scan_tc_states", s, [&] { return launch_scan_tc(p, 1, s); }));
+      SSD_TRY(traced("ssd_state_pass", s, [&] { return launch_state_pass(p, s); }));
+    }
+    SSD_TRY(traced("ssd_scan_tc", s, [&] { return launch_scan_tc(p, 0, s); }));
+    if (p.norm_groups > 0) SSD_TRY(traced("ssd_gated_norm", s, [&] { return launch_gated_norm(p, s); }));
+    SSD_TRY(traced("ssd_conv_state_out", s, [&] { return launch_conv_state_out(p, s); }));
+    return SSD_OK;
+  }
+
+  simt_segments(c, &p.n_seg, &p.seg_len);
   p.u = reinterpret_cast<float *>(ws + lay.u);
   p.dte = reinterpret_cast<float *>(ws + lay.dte);
   p.yf = c->norm_groups > 0 ? reinterpret_cast<float *>(ws + lay.yf) : nullptr;
   p.seg_state = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.seg_state) : nullptr;
   p.seg_decay = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.seg_decay) : nullptr;
-
-  if (c->kernel == SSD_KERNEL_TENSOR) return SSD_ERR_UNSUPPORTED;
-
   SSD_TRY(traced("ssd_dt", s, [&] { return launch_dt(p, s); }));
   SSD_TRY(traced("ssd_conv_silu", s, [&] { return launch_conv_silu_f32(p, s); }));
   if (p.n_seg == 1) {

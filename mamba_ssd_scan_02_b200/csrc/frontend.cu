@@ -16,14 +16,18 @@ constexpr int kConvTokens = 32;  // tokens per thread (sliding window kept in re
 
 // One thread: 8 consecutive channels x kConvTokens consecutive tokens of one batch row.
 // 16-byte vector loads along the channel dimension are coalesced across the warp.
-template <typename T, int W>
+// Channels [c_begin, c_begin + C_out) of the C-channel input are convolved; the output row
+// holds C_out channels (fp32 for the CUDA-core path, bf16 for the tensor-core path).
+template <typename T, typename OutT, int W>
 __global__ void __launch_bounds__(128) conv_silu_kernel(const T *__restrict__ xBC, long long xs,
                                                         const T *__restrict__ csi,
                                                         const T *__restrict__ w,
                                                         const T *__restrict__ bias,
-                                                        float *__restrict__ u, int L, int C) {
-  const int c8 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
-  if (c8 >= C) return;
+                                                        OutT *__restrict__ u, int L, int C,
+                                                        int c_begin, int C_out) {
+  const int o8 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (o8 >= C_out) return;
+  const int c8 = c_begin + o8;
   const int b = blockIdx.z;
   const int t0 = blockIdx.y * kConvTokens;
   const T *xrow = xBC + (long long)b * L * xs;
@@ -64,7 +68,7 @@ __global__ void __launch_bounds__(128) conv_silu_kernel(const T *__restrict__ xB
       for (int j = 1; j < W; ++j) acc += wt[W - 1 - j][i] * hist[3 - j][i];
       out[i] = silu(acc);
     }
-    store8(u + ((long long)b * L + t) * C + c8, out);
+    store8(u + ((long long)b * L + t) * C_out + o8, out);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       hist[0][i] = hist[1][i];
@@ -83,6 +87,54 @@ __global__ void dt_kernel(const T *__restrict__ dt, long long ds, const float *_
     const long long r = i / H;
     const int h = (int)(i % H);
     dte[i] = effective_dt(io<T>::ld(dt + r * ds + h), bias[h], sp, lo, hi);
+  }
+}
+
+// Effective dt and its chunk-local inclusive prefix sum of dt*A, written head-major
+// [B, H, Lpad] (Lpad = L rounded up to the 128-token chunk; padding has dt = 0 so the prefix
+// stays flat).  One CTA: 128 tokens x 32 heads of one batch row; the tile is transposed
+// through shared memory so that both the dt reads and the head-major writes are coalesced.
+template <typename T>
+__global__ void __launch_bounds__(128) dt_cumsum_kernel(const T *__restrict__ dt, long long ds,
+                                                         const float *__restrict__ bias,
+                                                         const float *__restrict__ A,
+                                                         float *__restrict__ dte,
+                                                         float *__restrict__ cs, int L, int H,
+                                                         int Lpad, int sp, float lo, float hi) {
+  __shared__ float v[128][33];
+  const int c0 = blockIdx.x * 128, h0 = blockIdx.y * 32, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  for (int i = tid; i < 128 * 32; i += 128) {
+    const int t = i / 32, hh = i % 32, tt = c0 + t, h = h0 + hh;
+    float val = 0.f;
+    if (tt < L && h < H)
+      val = effective_dt(io<T>::ld(dt + ((long long)b * L + tt) * ds + h), bias[h], sp, lo, hi);
+    v[t][hh] = val;
+  }
+  __syncthreads();
+  for (int hh = warp * 8; hh < warp * 8 + 8; ++hh) {
+    const int h = h0 + hh;
+    if (h >= H) break;
+    const float a = A[h];
+    float d[4], c[4];
+    float run = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      d[i] = v[4 * lane + i][hh];
+      run += d[i] * a;
+      c[i] = run;
+    }
+    float incl = run;  // inclusive scan of the per-lane totals
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    const float excl = incl - run;
+    const long long base = ((long long)b * H + h) * Lpad + c0 + 4 * lane;
+    *reinterpret_cast<float4 *>(dte + base) = make_float4(d[0], d[1], d[2], d[3]);
+    *reinterpret_cast<float4 *>(cs + base) =
+        make_float4(excl + c[0], excl + c[1], excl + c[2], excl + c[3]);
   }
 }
 
@@ -124,31 +176,36 @@ int grid_for(long long n, int threads) {
 
 }  // namespace
 
-template <typename T, int W>
-static void conv_launch(const PrefillPlan &p, dim3 grid, int threads, cudaStream_t s) {
-  conv_silu_kernel<T, W><<<grid, threads, 0, s>>>((const T *)p.xBC, p.xs, (const T *)p.csi,
-                                                   (const T *)p.conv_w, (const T *)p.conv_b, p.u,
-                                                   p.L, p.conv_dim);
+template <typename T, typename OutT, int W>
+static void conv_launch(const PrefillPlan &p, OutT *out, int c_begin, int C_out, cudaStream_t s) {
+  const int threads = 128;
+  dim3 grid((C_out / 8 + threads - 1) / threads, (p.L + kConvTokens - 1) / kConvTokens, p.B);
+  conv_silu_kernel<T, OutT, W><<<grid, threads, 0, s>>>((const T *)p.xBC, p.xs, (const T *)p.csi,
+                                                         (const T *)p.conv_w, (const T *)p.conv_b,
+                                                         out, p.L, p.conv_dim, c_begin, C_out);
 }
 
-template <typename T>
-static void conv_dispatch(const PrefillPlan &p, dim3 grid, int threads, cudaStream_t s) {
+template <typename T, typename OutT>
+static void conv_dispatch(const PrefillPlan &p, OutT *out, int c_begin, int C_out, cudaStream_t s) {
   switch (p.W) {
-    case 0: conv_launch<T, 0>(p, grid, threads, s); break;
-    case 1: conv_launch<T, 1>(p, grid, threads, s); break;
-    case 2: conv_launch<T, 2>(p, grid, threads, s); break;
-    case 3: conv_launch<T, 3>(p, grid, threads, s); break;
-    default: conv_launch<T, 4>(p, grid, threads, s); break;
+    case 0: conv_launch<T, OutT, 0>(p, out, c_begin, C_out, s); break;
+    case 1: conv_launch<T, OutT, 1>(p, out, c_begin, C_out, s); break;
+    case 2: conv_launch<T, OutT, 2>(p, out, c_begin, C_out, s); break;
+    case 3: conv_launch<T, OutT, 3>(p, out, c_begin, C_out, s); break;
+    default: conv_launch<T, OutT, 4>(p, out, c_begin, C_out, s); break;
   }
 }
 
 cudaError_t launch_conv_silu_f32(const PrefillPlan &p, cudaStream_t s) {
-  const int threads = 128;
-  dim3 grid((p.conv_dim / 8 + threads - 1) / threads, (p.L + kConvTokens - 1) / kConvTokens, p.B);
   if (p.bf16)
-    conv_dispatch<__nv_bfloat16>(p, grid, threads, s);
+    conv_dispatch<__nv_bfloat16, float>(p, p.u, 0, p.conv_dim, s);
   else
-    conv_dispatch<float>(p, grid, threads, s);
+    conv_dispatch<float, float>(p, p.u, 0, p.conv_dim, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bc_conv_f16(const PrefillPlan &p, cudaStream_t s) {
+  conv_dispatch<__nv_bfloat16, __half>(p, (__half *)p.bc, p.d_inner, 2 * p.G * p.N, s);
   return cudaGetLastError();
 }
 
@@ -161,6 +218,18 @@ cudaError_t launch_dt(const PrefillPlan &p, cudaStream_t s) {
   else
     dt_kernel<float><<<g, 256, 0, s>>>((const float *)p.dt, p.ds, p.dt_bias, p.dte, rows, p.H,
                                         p.softplus, p.dt_min, p.dt_max);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dt_cumsum(const PrefillPlan &p, float *dte, float *cs, int Lpad, cudaStream_t s) {
+  dim3 grid(Lpad / 128, (p.H + 31) / 32, p.B);
+  if (p.bf16)
+    dt_cumsum_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>((const __nv_bfloat16 *)p.dt, p.ds, p.dt_bias,
+                                                          p.A, dte, cs, p.L, p.H, Lpad, p.softplus,
+                                                          p.dt_min, p.dt_max);
+  else
+    dt_cumsum_kernel<float><<<grid, 128, 0, s>>>((const float *)p.dt, p.ds, p.dt_bias, p.A, dte, cs,
+                                                  p.L, p.H, Lpad, p.softplus, p.dt_min, p.dt_max);
   return cudaGetLastError();
 }
 

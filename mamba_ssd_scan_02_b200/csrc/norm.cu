@@ -50,6 +50,29 @@ __global__ void __launch_bounds__(kNormThreads) gated_norm_kernel(
   }
 }
 
+// In place on the scan output stored in the io dtype (tensor-core path).
+template <typename T>
+__global__ void __launch_bounds__(kNormThreads) gated_norm_inplace_kernel(
+    T *__restrict__ y, long long ys, const T *__restrict__ z, long long zs, const T *__restrict__ w,
+    int gs, float eps) {
+  __shared__ float red[32];
+  const long long row = blockIdx.x;
+  const int c0 = blockIdx.y * gs;
+  T *yr = y + row * ys + c0;
+  const T *zr = z + row * zs + c0;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < gs; i += kNormThreads) {
+    const float gv = io<T>::ld(yr + i) * silu(io<T>::ld(zr + i));
+    ss += gv * gv;
+  }
+  ss = block_sum(ss, red);
+  const float r = rsqrtf(ss / gs + eps);
+  for (int i = threadIdx.x; i < gs; i += kNormThreads) {
+    const float gv = io<T>::ld(yr + i) * silu(io<T>::ld(zr + i));
+    io<T>::st(yr + i, gv * r * (w ? io<T>::ld(w + c0 + i) : 1.f));
+  }
+}
+
 __global__ void __launch_bounds__(kNormThreads) rmsnorm_bf16_kernel(
     const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w,
     __nv_bfloat16 *__restrict__ out, int width, float eps) {
@@ -88,6 +111,19 @@ cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s) {
     gated_norm_kernel<float><<<grid, kNormThreads, 0, s>>>(p.yf, (const float *)p.z, p.zs,
                                                            (const float *)p.norm_w, (float *)p.y,
                                                            p.ys, p.d_inner, gs, p.eps, p.L);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gated_norm_inplace(const PrefillPlan &p, cudaStream_t s) {
+  const int gs = p.d_inner / p.norm_groups;
+  dim3 grid((unsigned)((long long)p.B * p.L), p.norm_groups);
+  if (p.bf16)
+    gated_norm_inplace_kernel<__nv_bfloat16><<<grid, kNormThreads, 0, s>>>(
+        (__nv_bfloat16 *)p.y, p.ys, (const __nv_bfloat16 *)p.z, p.zs,
+        (const __nv_bfloat16 *)p.norm_w, gs, p.eps);
+  else
+    gated_norm_inplace_kernel<float><<<grid, kNormThreads, 0, s>>>(
+        (float *)p.y, p.ys, (const float *)p.z, p.zs, (const float *)p.norm_w, gs, p.eps);
   return cudaGetLastError();
 }
 

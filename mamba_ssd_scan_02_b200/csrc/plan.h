@@ -33,7 +33,10 @@ struct PrefillPlan {
   float *yf;         // [B, L, d_inner] pre-norm output (when norm_groups > 0)
   float *seg_state;  // [n_seg, B, H, P, N]
   float *seg_decay;  // [n_seg, B, H]
-  void *bc;          // [B, L, 2*G*N] bf16 conv+SiLU output of the B|C channels (tensor path)
+  void *bc;          // [B, L, 2*G*N] fp16 conv+SiLU output of the B|C channels (tensor path)
+  float *dte_hm;     // [B, H, Lpad] effective dt, head-major (tensor path)
+  float *cs_hm;      // [B, H, Lpad] chunk-local prefix sums of dt*A (tensor path)
+  int Lpad;
   int *err;          // device error word
 };
 
@@ -58,12 +61,18 @@ cudaError_t launch_conv_silu_f32(const PrefillPlan &p, cudaStream_t s);
 cudaError_t launch_dt(const PrefillPlan &p, cudaStream_t s);
 cudaError_t launch_conv_state_out(const PrefillPlan &p, cudaStream_t s);
 cudaError_t launch_carry_only(const PrefillPlan &p, cudaStream_t s);  // seqlen == 0
+cudaError_t launch_bc_conv_f16(const PrefillPlan &p, cudaStream_t s);  // B|C channels -> p.bc (fp16)
+cudaError_t launch_dt_cumsum(const PrefillPlan &p, float *dte, float *cs, int Lpad, cudaStream_t s);
 // chunked scan on CUDA cores (scan_simt.cu); mode 0 full, 1 state-only, 2 output-only
 cudaError_t launch_scan_simt(const PrefillPlan &p, int mode, cudaStream_t s);
+// chunked scan on tcgen05 tensor cores (tc_scan.cu); mode 0 full/output, 1 state-only
+bool tc_scan_available();
+cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s);
 // inter-segment state pass (state_pass.cu)
 cudaError_t launch_state_pass(const PrefillPlan &p, cudaStream_t s);
 // norms (norm.cu)
-cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s);
+cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s);          // fp32 yf -> y
+cudaError_t launch_gated_norm_inplace(const PrefillPlan &p, cudaStream_t s);  // y (io dtype) in place
 cudaError_t launch_rmsnorm_bf16(const void *x, const void *w, void *out, long long rows, int width,
                                 float eps, cudaStream_t s);
 // decode (decode.cu)

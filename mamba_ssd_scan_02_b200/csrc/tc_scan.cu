@@ -1,0 +1,669 @@
+// tc_scan.cu -- chunked SSD scan on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// One CTA per (segment, head, batch row) walks its segment's 128-token chunks in order and
+// keeps the head's P x N = 64 x 128 state on chip.  For chunk k with cs = chunk-local prefix
+// sums of dt*A (cs_Q = cs at the last token), the Mamba-2 scan becomes four dense fp16
+// contractions with fp32 accumulation in tensor memory:
+//   MMA1  S     = C . B^T                    M=128 (t) N=128 (s) K=128 (n)   -> TMEM S[k%2]
+//   mask  S~    = S o (e^{cs_t - cs_s} dt_s [s <= t]) + D_h I   (CUDA cores; written back
+//                 into the same TMEM columns as packed fp16)
+//   MMA2  Yi    = S~ . X                     M=128 (t) N=64 (p)  K=128 (s)   (A from TMEM)
+//   MMA3  Ys    = C . h_{k-1}^T              M=128 (t) N=64 (p)  K=128 (n)
+//   MMA4  dH^T  = B^T . (w o X), w_s = e^{cs_Q - cs_s} dt_s   M=128 (n) N=64 (p) K=128 (s)
+// then y_t = Yi + e^{cs_t} Ys (the D x skip is folded into the diagonal of S~) and
+// h_k = e^{cs_Q} h_{k-1} + dH, kept in fp32 registers (an fp16 copy feeds MMA3 of chunk k+1).
+// This is the token recurrence h_t = e^{dt_t A} h_{t-1} + dt_t x_t B_t^T, y_t = h_t C_t + D x_t
+// regrouped by chunk; every exponent is a difference cs_t - cs_s <= 0 or is split at a
+// 32-token block boundary where both factors stay below e^60 (else computed directly).
+// In the last chunk of a segment w o X is applied as fp16 hi + lo parts (a second MMA4), so
+// the final state carries the rounding of B only: its largest entries come from the newest
+// tokens, whose products are not averaged over many terms.
+//
+// Warp roles (512 threads): warp 0 issues TMA loads (B and C tiles of the group, the head's
+// raw x rows with a 3-token halo, per-chunk dt and prefix sums), warp 1 allocates TMEM and
+// issues the MMAs, warps 4-7 compute the head's x channels (causal conv1d + SiLU) in place
+// into the double-buffered X tile and into w o X, warps 8-11 turn S into S~, warps 12-15
+// update the state and write y.  Per chunk the MMAs are issued as MMA4(k), MMA3(k), MMA1(k+1), MMA2(k), so the
+// mask of chunk k overlaps four MMAs and the state update overlaps two.  Hand-offs use
+// mbarriers (TMA transaction counts, tcgen05.commit, thread arrivals); every wait is bounded
+// and a timeout aborts the CTA cleanly and latches SSD_ERR_TIMEOUT.
+//
+// Operands are fp16 (the conv outputs B, C, x are O(10) in the workloads, far inside the fp16
+// range; 11 significant bits keep the chunked products within the bf16-input tolerance).
+// Shared-memory operand layouts use the 128-byte swizzle: B/C tiles are two TMA boxes of
+// 64 channels x 128 tokens (K-major for MMA1/MMA3, M-major for MMA4); X, w o X and the fp16
+// state copy are 128-byte rows (N-major B operands).
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "plan.h"
+#include "tc_ptx.cuh"
+
+// Optional timeline marks for one CTA (compiled only with -DSSD_TC_TRACE): device time of
+// each role's steps per chunk, read back by a measurement tool.
+#ifdef SSD_TC_TRACE
+__device__ unsigned long long g_tc_trace[256 * 16];
+#define TC_MARK(k, e)                                                                         \
+  do {                                                                                        \
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (k) < 256)                   \
+      g_tc_trace[(k) * 16 + (e)] = ssd::tc::globaltimer();                                    \
+  } while (0)
+extern "C" int ssd_tc_trace_read(unsigned long long *out) {
+  return cudaMemcpyFromSymbol(out, g_tc_trace, sizeof(g_tc_trace)) == cudaSuccess ? 0 : 1;
+}
+#else
+#define TC_MARK(k, e) \
+  do {                \
+  } while (0)
+#endif
+
+namespace ssd {
+namespace {
+
+using namespace tc;
+
+constexpr int QC = 128;              // tokens per chunk
+constexpr int kThreadsTC = 512;
+constexpr uint32_t kTile = 16384;    // one 128-row x 128-byte operand box
+// per-stage layout (bytes)
+constexpr uint32_t OFF_C = 0;                 // C tile: channels 0-63 | 64-127
+constexpr uint32_t OFF_B = 2 * kTile;         // B tile
+constexpr uint32_t OFF_DT = 4 * kTile;        // dt[128] fp32
+constexpr uint32_t OFF_CS = OFF_DT + 512;     // cs[128] fp32
+constexpr uint32_t kStage = 4 * kTile + 1024;  // 66560 = 65 * 1024
+// CTA layout.  X[b] first receives (by TMA) the chunk's raw bf16 x rows for times t0-3 ..
+// t0+127 (131 rows of this head's 64 channels); the conv overwrites row s with X row s.
+constexpr uint32_t kXBuf = 17 * 1024;           // 131 rows of 128 bytes, padded
+constexpr uint32_t kRawRows = QC + 3;
+constexpr uint32_t OFF_X = 2 * kStage;          // X[2]   [s][p] fp16 (raw x rows first)
+constexpr uint32_t OFF_XW = OFF_X + 2 * kXBuf;  // wX[2]  [s][p] fp16, 16 KB each
+constexpr uint32_t OFF_H = OFF_XW + 2 * kTile;  // h copy [n][p] fp16, 16 KB
+constexpr uint32_t OFF_CF = OFF_H + kTile;      // column factors, 128 fp32
+constexpr uint32_t OFF_BAR = OFF_CF + 512;
+enum {
+  BAR_FULL0, BAR_FULL1, BAR_EMPTY0, BAR_EMPTY1, BAR_SREADY0, BAR_SREADY1, BAR_STREADY0,
+  BAR_STREADY1, BAR_XREADY0, BAR_XREADY1, BAR_XFREE0, BAR_XFREE1, BAR_DHREADY, BAR_HREADY,
+  BAR_YREADY, BAR_YFREE, BAR_XLOREADY, BAR_DONE, kNumBars
+};
+constexpr uint32_t OFF_MISC = OFF_BAR + 8 * 24;   // [0] TMEM base, [1] abort flag
+constexpr uint32_t kSmemUsed = OFF_MISC + 16;
+constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;  // room to align the base to 1024 bytes
+static_assert(kNumBars <= 24, "barrier slots");
+static_assert(kSmemAlloc <= 232448, "shared memory budget");
+static_assert(OFF_X % 1024 == 0 && OFF_XW % 1024 == 0 && OFF_H % 1024 == 0, "swizzle alignment");
+static_assert(kRawRows * 128 <= kXBuf, "raw x tile fits its buffer");
+
+// TMEM columns (fp32 accumulators, 128 lanes).  After the mask, S[b] holds S~ as packed fp16
+// in its first 64 columns.
+constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_YI = 256, TM_YS = 320, TM_DH = 384, TM_COLS = 512;
+
+constexpr uint32_t IDESC_S = idesc_f16(128, 128, false, false, kFmtF16);  // C K-major, B K-major
+constexpr uint32_t IDESC_YS = idesc_f16(128, 64, false, true, kFmtF16);   // C K-major, h N-major
+constexpr uint32_t IDESC_YI = idesc_f16(128, 64, false, true, kFmtF16);   // S~ (TMEM), X N-major
+constexpr uint32_t IDESC_DH = idesc_f16(128, 64, true, true, kFmtF16);    // B M-major, wX N-major
+
+struct TcArgs {
+  int B, L, H, G, hpg, conv_dim, Lpad, W, seg_len;
+  const __nv_bfloat16 *xBC;
+  long long xs;
+  const __nv_bfloat16 *csi, *conv_w, *conv_b;
+  const float *dte, *cs, *D;
+  const float *h_init;     // initial state (per segment when h_init_seg > 0) or null = 0
+  long long h_init_seg;
+  float *h_out;            // final state destination or null
+  long long h_out_seg;
+  float *seg_decay;        // [n_seg, B, H] total decay per segment, or null
+  __nv_bfloat16 *y;        // output (no gate) ...
+  long long ys;
+  float *yf;               // ... or fp32 pre-norm output [B, L, d_inner] when a gated norm follows
+  int d_inner;
+  int *err;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ uint32_t pack_f16(float a, float b) {
+  __half2 v = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
+  __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162 *>(&u);
+  return __bfloat1622float2(v);
+}
+
+// A warpgroup-uniform bounded wait: one leader thread waits on the mbarrier, then the
+// group syncs on its named barrier and reads the (shared) abort flag.
+__device__ __forceinline__ bool wg_wait(uint32_t bar, uint32_t parity, bool leader, int nb,
+                                        volatile int *abort_flag, int *err) {
+  if (leader) mbar_wait(bar, parity, abort_flag, err);
+  named_bar(nb, 128);
+  return *abort_flag == 0;
+}
+
+// ---- MMA issue (single thread) ---------------------------------------------------------
+__device__ __forceinline__ void issue_S(uint32_t stage, uint32_t tS) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t koff = (j >> 2) * kTile + (j & 3) * 32;
+    mma_f16_ss(tS, smem_desc_sw128(stage + OFF_C + koff, 16, 1024),
+               smem_desc_sw128(stage + OFF_B + koff, 16, 1024), IDESC_S, j > 0);
+  }
+}
+__device__ __forceinline__ void issue_Ys(uint32_t stage, uint32_t hbase, uint32_t tYs) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t koff = (j >> 2) * kTile + (j & 3) * 32;
+    mma_f16_ss(tYs, smem_desc_sw128(stage + OFF_C + koff, 16, 1024),
+               smem_desc_sw128(hbase + j * 2048, 8192, 1024), IDESC_YS, j > 0);
+  }
+}
+// S~ in TMEM: 16 fp16 of K per MMA = 8 columns
+__device__ __forceinline__ void issue_Yi(uint32_t tSt, uint32_t xbase, uint32_t tYi) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    mma_f16_ts(tYi, tSt + 8 * j, smem_desc_sw128(xbase + j * 2048, 8192, 1024), IDESC_YI, j > 0);
+}
+__device__ __forceinline__ void issue_dH(uint32_t stage, uint32_t xwbase, uint32_t tDH, bool acc) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    mma_f16_ss(tDH, smem_desc_sw128(stage + OFF_B + j * 2048, kTile, 1024),
+               smem_desc_sw128(xwbase + j * 2048, 8192, 1024), IDESC_DH, (j > 0 || acc) ? 1u : 0u);
+}
+
+// Row r (128 bytes) of a 128-byte-swizzled tile: 16-byte chunk c sits at chunk c ^ (r & 7).
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return (uint32_t)row * 128u + ((uint32_t)(chunk ^ (row & 7)) << 4);
+}
+
+__device__ __forceinline__ void write_h_tile(unsigned char *smem, const float (&hr)[64], int n) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint4 v = make_uint4(pack_f16(hr[8 * c + 0], hr[8 * c + 1]), pack_f16(hr[8 * c + 2], hr[8 * c + 3]),
+                         pack_f16(hr[8 * c + 4], hr[8 * c + 5]), pack_f16(hr[8 * c + 6], hr[8 * c + 7]));
+    *reinterpret_cast<uint4 *>(smem + OFF_H + swz(n, c)) = v;
+  }
+}
+
+template <bool kStateOnly>
+__global__ void __launch_bounds__(kThreadsTC, 1)
+    ssd_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_bc,
+                       const __grid_constant__ CUtensorMap tm_x, const TcArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *smem =
+      reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z, g = h / a.hpg;
+  const int t_begin = seg * a.seg_len;
+  const int t_end = min(a.L, t_begin + a.seg_len);
+  const int nck = t_end > t_begin ? (t_end - t_begin + QC - 1) / QC : 0;
+  const int last = nck - 1;
+  const uint32_t bar0 = sb + OFF_BAR;
+#define BAR(i) (bar0 + 8u * (uint32_t)(i))
+  uint32_t *misc = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
+
+  if (tid == 0) {
+    for (int i = 0; i < kNumBars; ++i) {
+      uint32_t cnt = 1;
+      if (i == BAR_EMPTY0 || i == BAR_EMPTY1) cnt = kStateOnly ? 3 : 4;
+      mbar_init(BAR(i), cnt);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_bc);
+    prefetch_tmap(&tm_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(sb + OFF_MISC, TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int k = 0;
+      for (; k < nck; ++k) {
+        const int st = k & 1;
+        if (k >= 2 && !mbar_wait(BAR(BAR_EMPTY0 + st), ((k >> 1) - 1) & 1, abort_flag, a.err)) break;
+        if (k >= 2 && !mbar_wait(BAR(BAR_XFREE0 + st), ((k >> 1) - 1) & 1, abort_flag, a.err)) break;
+        const uint32_t sst = sb + st * kStage;
+        const int t0 = t_begin + k * QC;
+        const uint32_t full = BAR(BAR_FULL0 + st);
+        TC_MARK(k, 12);
+        mbar_arrive_expect_tx(full, (kStateOnly ? 2 * kTile : 4 * kTile) + 1024 + kRawRows * 128);
+        tma_load_3d(sb + OFF_X + st * kXBuf, &tm_x, h * 64, t0 - 3, b, full);
+        const int cB = g * 128, cC = a.G * 128 + g * 128;
+        if (!kStateOnly) {
+          tma_load_3d(sst + OFF_C, &tm_bc, cC, t0, b, full);
+          tma_load_3d(sst + OFF_C + kTile, &tm_bc, cC + 64, t0, b, full);
+        }
+        tma_load_3d(sst + OFF_B, &tm_bc, cB, t0, b, full);
+        tma_load_3d(sst + OFF_B + kTile, &tm_bc, cB + 64, t0, b, full);
+        const long long hoff = ((long long)b * a.H + h) * a.Lpad + t0;
+        bulk_load(sst + OFF_DT, a.dte + hoff, 512, full);
+        bulk_load(sst + OFF_CS, a.cs + hoff, 512, full);
+      }
+      // every load issued must land before the CTA may exit
+      int never_abort = 0;
+      for (int j = (k >= 2 ? k - 2 : 0); j < k; ++j)
+        mbar_wait(BAR(BAR_FULL0 + (j & 1)), (j >> 1) & 1, &never_abort, a.err);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t tYi = tmem + TM_YI, tYs = tmem + TM_YS, tDH = tmem + TM_DH;
+      bool ok = true;
+      if (nck > 0 && !kStateOnly) {
+        ok = mbar_wait(BAR(BAR_FULL0), 0, abort_flag, a.err);
+        if (ok) {
+          tc_fence_after();
+          issue_S(sb, tmem + TM_S0);
+          mma_commit(BAR(BAR_SREADY0));
+        }
+      }
+      for (int k = 0; ok && k < nck; ++k) {
+        const int st = k & 1;
+        const uint32_t sst = sb + st * kStage;
+        // h_{k-1} in shared memory and dH free
+        if (!(ok = mbar_wait(BAR(BAR_HREADY), k & 1, abort_flag, a.err))) break;
+        if (kStateOnly && !(ok = mbar_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, abort_flag, a.err))) break;
+        if (!(ok = mbar_wait(BAR(BAR_XREADY0 + st), (k >> 1) & 1, abort_flag, a.err))) break;
+        tc_fence_after();
+        TC_MARK(k, 8);
+        issue_dH(sst, sb + OFF_XW + st * kTile, tDH, false);
+        if (!kStateOnly) {
+          if (k > 0 && !(ok = mbar_wait(BAR(BAR_YFREE), (k - 1) & 1, abort_flag, a.err))) break;
+          tc_fence_after();
+          TC_MARK(k, 9);
+          issue_Ys(sst, sb + OFF_H, tYs);
+        }
+        if (k != last) mma_commit(BAR(BAR_DHREADY));
+        if (!kStateOnly) {
+          if (k + 1 < nck) {
+            const int s2 = (k + 1) & 1;
+            if (!(ok = mbar_wait(BAR(BAR_FULL0 + s2), ((k + 1) >> 1) & 1, abort_flag, a.err))) break;
+            tc_fence_after();
+            TC_MARK(k, 10);
+            issue_S(sb + s2 * kStage, tmem + (s2 ? TM_S1 : TM_S0));
+            mma_commit(BAR(BAR_SREADY0 + s2));
+          }
+          if (!(ok = mbar_wait(BAR(BAR_STREADY0 + st), (k >> 1) & 1, abort_flag, a.err))) break;
+          tc_fence_after();
+          TC_MARK(k, 11);
+          issue_Yi(tmem + (st ? TM_S1 : TM_S0), sb + OFF_X + st * kXBuf, tYi);
+          mma_commit(BAR(BAR_YREADY));
+        }
+        mma_commit(BAR(BAR_XFREE0 + st));
+        mma_commit(BAR(BAR_EMPTY0 + st));
+        if (k == last) {  // low part of w o X (in the other w o X slot) for the final state
+          if (!(ok = mbar_wait(BAR(BAR_XLOREADY), 0, abort_flag, a.err))) break;
+          tc_fence_after();
+          issue_dH(sst, sb + OFF_XW + (st ^ 1) * kTile, tDH, true);
+          mma_commit(BAR(BAR_DHREADY));
+        }
+      }
+      // no MMA may still be running when TMEM is released
+      mma_commit(BAR(BAR_DONE));
+      int never_abort = 0;
+      mbar_wait(BAR(BAR_DONE), 0, &never_abort, a.err);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------------------------------------------------------- conv + SiLU -> X, w o X
+    // Warp cw makes tokens 32cw..32cw+31; lane l channels 2l, 2l+1.  Raw row r of the X
+    // buffer holds time t0-3+r; token s reads rows s..s+3 (a 4-register window) and then
+    // overwrites row s with its X row.  Rows 32cw+32..+34 belong to the next warp's tokens,
+    // so every warp reads them before the group barrier that precedes all writes.
+    const int cw = warp - 4;
+    const bool leader = (tid == 128);
+    const int ch = h * 64 + 2 * lane;
+    const int W = a.W;
+    float e0[4], e1[4], bias0 = 0.f, bias1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {  // weight for the input at time t-3+j
+      const int k = j - (4 - W);
+      e0[j] = (W > 0 && k >= 0) ? __bfloat162float(a.conv_w[(long long)ch * W + k]) : 0.f;
+      e1[j] = (W > 0 && k >= 0) ? __bfloat162float(a.conv_w[(long long)(ch + 1) * W + k]) : 0.f;
+    }
+    if (W > 0 && a.conv_b) {
+      bias0 = __bfloat162float(a.conv_b[ch]);
+      bias1 = __bfloat162float(a.conv_b[ch + 1]);
+    }
+    const uint32_t lane_byte = (uint32_t)(lane & 3) << 2;
+    for (int k = 0; k < nck; ++k) {
+      const int st = k & 1;
+      const bool is_last = (k == last);
+      if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, 1, abort_flag, a.err)) break;
+      if (is_last && k >= 1 &&
+          !wg_wait(BAR(BAR_XFREE0 + (st ^ 1)), ((k - 1) >> 1) & 1, leader, 1, abort_flag, a.err))
+        break;
+      const float *cs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
+      const float *dtv = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
+      const float cs_end = cs[QC - 1];
+      const float wl = __expf(cs_end - cs[32 * cw + lane]) * dtv[32 * cw + lane];
+      unsigned char *xt = smem + OFF_X + st * kXBuf;
+      unsigned char *xwt = smem + OFF_XW + st * kTile;
+      unsigned char *xlt = smem + OFF_XW + (st ^ 1) * kTile;
+      auto raw_row = [&](int r) -> uint32_t {
+        return *reinterpret_cast<const uint32_t *>(xt + swz(r, lane >> 2) + lane_byte);
+      };
+      // window: times t-3, t-2, t-1 for the warp's first token
+      uint32_t w0 = raw_row(32 * cw), w1 = raw_row(32 * cw + 1), w2 = raw_row(32 * cw + 2);
+      const int t0 = t_begin + k * QC;
+      if (cw == 0 && t0 == 0) {  // history before the first token comes from the conv cache
+        uint32_t hist[3] = {0u, 0u, 0u};
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          const int tau = j - 3;
+          if (a.csi && W + tau >= 0)
+            hist[j] = *reinterpret_cast<const uint32_t *>(a.csi + ((long long)b * W + (W + tau)) * a.conv_dim + ch);
+        }
+        w0 = hist[0];
+        w1 = hist[1];
+        w2 = hist[2];
+      }
+      const uint32_t nb0 = raw_row(32 * cw + 32), nb1 = raw_row(32 * cw + 33), nb2 = raw_row(32 * cw + 34);
+      named_bar(1, 128);  // all boundary rows read before any row is overwritten
+      if (leader) TC_MARK(k, 0);
+#pragma unroll 1
+      for (int g = 0; g < 8; ++g) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = 4 * g + u, s_ = 32 * cw + i;
+          const int nxt = i + 3;  // window row for time t
+          uint32_t w3;
+          if (nxt < 32) w3 = raw_row(32 * cw + nxt);
+          else w3 = nxt == 32 ? nb0 : (nxt == 33 ? nb1 : nb2);
+          const float2 xm3 = unpack_bf16(w0), xm2 = unpack_bf16(w1), xm1 = unpack_bf16(w2);
+          const float2 x0 = unpack_bf16(w3);
+          float u0, u1;
+          if (W == 0) {
+            u0 = x0.x;
+            u1 = x0.y;
+          } else {
+            u0 = silu(bias0 + e0[0] * xm3.x + e0[1] * xm2.x + e0[2] * xm1.x + e0[3] * x0.x);
+            u1 = silu(bias1 + e1[0] * xm3.y + e1[1] * xm2.y + e1[2] * xm1.y + e1[3] * x0.y);
+          }
+          const float ws = __shfl_sync(0xffffffffu, wl, i);
+          const uint32_t off = swz(s_, lane >> 2) + lane_byte;
+          *reinterpret_cast<uint32_t *>(xt + off) = pack_f16(u0, u1);
+          const float v0 = u0 * ws, v1 = u1 * ws;
+          const __half2 hi = __floats2half2_rn(v0, v1);
+          *reinterpret_cast<__half2 *>(xwt + off) = hi;
+          if (is_last) {
+            const float2 hf = __half22float2(hi);
+            *reinterpret_cast<uint32_t *>(xlt + off) = pack_f16(v0 - hf.x, v1 - hf.y);
+          }
+          w0 = w1;
+          w1 = w2;
+          w2 = w3;
+        }
+      }
+      fence_proxy_async();
+      named_bar(1, 128);
+      if (leader) {
+        TC_MARK(k, 1);
+        mbar_arrive(BAR(BAR_XREADY0 + st));
+        if (is_last) mbar_arrive(BAR(BAR_XLOREADY));
+        mbar_arrive(BAR(BAR_EMPTY0 + st));
+      }
+    }
+  } else if (warp >= 8 && warp < 12) {
+    // ---------------------------------------------------------------- S -> S~ (decay mask)
+    if (!kStateOnly) {
+      const int mw = warp - 8;
+      const int t = 32 * mw + lane;
+      const bool leader = (tid == 256);
+      float *cf = reinterpret_cast<float *>(smem + OFF_CF);
+      const float Dh = a.D[h];
+      for (int k = 0; k < nck; ++k) {
+        const int st = k & 1;
+        if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, 2, abort_flag, a.err)) break;
+        if (!wg_wait(BAR(BAR_SREADY0 + st), (k >> 1) & 1, leader, 2, abort_flag, a.err)) break;
+        tc_fence_after();
+        const float *cs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
+        const float *dtv = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
+        {  // column factor of column t: e^{r_J - cs_t} dt_t with r_J = cs at the end of t's block
+          const float rJ = cs[32 * (t >> 5) + 31];
+          cf[t] = __expf(rJ - cs[t]) * dtv[t];
+        }
+        named_bar(2, 128);
+        if (leader) TC_MARK(k, 2);
+        const float cst = cs[t];
+        const uint32_t trow = tmem + (st ? TM_S1 : TM_S0) + ((uint32_t)(32 * mw) << 16);
+#pragma unroll 1
+        for (int J = 0; J < 4; ++J) {
+          uint32_t pk[16];
+          if (J <= mw) {
+            float v[32];
+            tmem_ld32(trow + 32 * J, v);
+            tmem_ld_wait();
+            const float rJ = cs[32 * J + 31];
+            const bool direct = (cs[32 * J] - rJ) > 60.f;  // block too steep to factor
+            const float rf = direct ? 0.f : __expf(cst - rJ);
+            const float4 *cf4 = reinterpret_cast<const float4 *>(cf + 32 * J);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 c4 = cf4[q];
+              const float cq[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int c = 4 * q + e, s = 32 * J + c;
+                float val = direct ? v[c] * __expf(cst - cs[s]) * dtv[s] : v[c] * rf * cq[e];
+                if (J == mw) {  // diagonal block: causal mask and the D x skip
+                  if (s > t) val = 0.f;
+                  if (s == t) val += Dh;
+                }
+                v[c] = val;
+              }
+            }
+#pragma unroll
+            for (int c = 0; c < 16; ++c) pk[c] = pack_f16(v[2 * c], v[2 * c + 1]);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) pk[c] = 0u;
+          }
+          // S~ columns 32J..32J+31 -> packed TMEM columns 16J..16J+15 (already read)
+          tmem_st16(trow + 16 * J, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        named_bar(2, 128);
+        if (leader) {
+          TC_MARK(k, 3);
+          mbar_arrive(BAR(BAR_STREADY0 + st));
+          mbar_arrive(BAR(BAR_EMPTY0 + st));
+        }
+      }
+    }
+  } else if (warp >= 12) {
+    // ---------------------------------------------------------------- state update + output
+    const int ew = warp - 12;
+    const int n = 32 * ew + lane;  // TMEM lane: state row n, output row t = n
+    const bool leader = (tid == 384);
+    const uint32_t lane_off = (uint32_t)(32 * ew) << 16;
+    const long long bh = (long long)b * a.H + h;
+    float hr[64];
+    {
+      const float *hin = a.h_init ? a.h_init + seg * a.h_init_seg + bh * 8192 : nullptr;
+#pragma unroll
+      for (int p = 0; p < 64; ++p) hr[p] = hin ? hin[p * 128 + n] : 0.f;
+    }
+    write_h_tile(smem, hr, n);
+    fence_proxy_async();
+    named_bar(3, 128);
+    if (leader) mbar_arrive(BAR(BAR_HREADY));
+    float decay_sum = 0.f;
+    for (int k = 0; k < nck; ++k) {
+      const int st = k & 1;
+      if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, 3, abort_flag, a.err)) break;
+      const float *cs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
+      const float cs_end = cs[QC - 1];
+      const float et = __expf(cs[n]);
+      decay_sum += cs_end;
+      const float ak = __expf(cs_end);
+      if (!wg_wait(BAR(BAR_DHREADY), k & 1, leader, 3, abort_flag, a.err)) break;
+      tc_fence_after();
+      if (leader) TC_MARK(k, 4);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float v[32];
+        tmem_ld32(tmem + TM_DH + 32 * half + lane_off, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) hr[32 * half + i] = ak * hr[32 * half + i] + v[i];
+      }
+      if (k != last) {
+        write_h_tile(smem, hr, n);
+        fence_proxy_async();
+      }
+      tc_fence_before();
+      named_bar(3, 128);
+      if (leader) {
+        TC_MARK(k, 5);
+        mbar_arrive(BAR(BAR_HREADY));
+      }
+      if (!kStateOnly) {
+        if (!wg_wait(BAR(BAR_YREADY), k & 1, leader, 3, abort_flag, a.err)) break;
+        tc_fence_after();
+        if (leader) TC_MARK(k, 6);
+        const int tok = t_begin + k * QC + n;
+        const long long row = (long long)b * a.L + tok;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float yi[16], ysv[16];
+          tmem_ld16(tmem + TM_YI + 16 * q + lane_off, yi);
+          tmem_ld16(tmem + TM_YS + 16 * q + lane_off, ysv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) yi[i] += et * ysv[i];
+          if (tok < t_end) {
+            if (a.yf) {
+              float4 *dst = reinterpret_cast<float4 *>(a.yf + row * a.d_inner + h * 64 + 16 * q);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) dst[i] = make_float4(yi[4 * i], yi[4 * i + 1], yi[4 * i + 2], yi[4 * i + 3]);
+            } else {
+              uint4 *dst = reinterpret_cast<uint4 *>(a.y + row * a.ys + h * 64 + 16 * q);
+              dst[0] = make_uint4(pack_bf16(yi[0], yi[1]), pack_bf16(yi[2], yi[3]),
+                                  pack_bf16(yi[4], yi[5]), pack_bf16(yi[6], yi[7]));
+              dst[1] = make_uint4(pack_bf16(yi[8], yi[9]), pack_bf16(yi[10], yi[11]),
+                                  pack_bf16(yi[12], yi[13]), pack_bf16(yi[14], yi[15]));
+            }
+          }
+        }
+        tc_fence_before();
+        named_bar(3, 128);
+        if (leader) {
+          TC_MARK(k, 7);
+          mbar_arrive(BAR(BAR_YFREE));
+        }
+      }
+      if (leader) mbar_arrive(BAR(BAR_EMPTY0 + st));
+    }
+    if (*abort_flag == 0) {
+      float *hout = a.h_out ? a.h_out + seg * a.h_out_seg + bh * 8192 : nullptr;
+      if (hout) {
+#pragma unroll
+        for (int p = 0; p < 64; ++p) hout[p * 128 + n] = hr[p];
+      }
+      if (a.seg_decay && n == 0) a.seg_decay[(long long)seg * a.B * a.H + bh] = __expf(decay_sum);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TM_COLS);
+  }
+#undef BAR
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+bool tc_scan_available() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return false;
+  return major == 10 && minor == 0 && encode_fn() != nullptr;
+}
+
+// mode 0: full scan of each segment from h_init (h0 or the inter-segment states) writing y;
+// mode 1: state-only pass (zero initial state) writing per-segment states and decays.
+cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
+  auto enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap tm;
+  const cuuint64_t C2 = 2ull * p.G * p.N;
+  cuuint64_t dims[3] = {C2, (cuuint64_t)p.L, (cuuint64_t)p.B};
+  cuuint64_t strides[2] = {C2 * 2, C2 * 2 * (cuuint64_t)p.L};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, p.bc, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  // raw x rows of one head: box of 64 channels x (128 + 3) tokens of the bf16 input
+  CUtensorMap tmx;
+  cuuint64_t xdims[3] = {(cuuint64_t)p.conv_dim, (cuuint64_t)p.L, (cuuint64_t)p.B};
+  cuuint64_t xstrides[2] = {(cuuint64_t)p.xs * 2, (cuuint64_t)p.xs * 2 * (cuuint64_t)p.L};
+  cuuint32_t xbox[3] = {64, kRawRows, 1};
+  r = enc(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(p.xBC), xdims, xstrides, xbox,
+          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  TcArgs a{};
+  a.B = p.B; a.L = p.L; a.H = p.H; a.G = p.G; a.hpg = p.hpg; a.conv_dim = p.conv_dim;
+  a.Lpad = p.Lpad; a.W = p.W; a.seg_len = p.seg_len;
+  a.xBC = (const __nv_bfloat16 *)p.xBC; a.xs = p.xs; a.csi = (const __nv_bfloat16 *)p.csi;
+  a.conv_w = (const __nv_bfloat16 *)p.conv_w; a.conv_b = (const __nv_bfloat16 *)p.conv_b;
+  a.dte = p.dte_hm; a.cs = p.cs_hm; a.D = p.D;
+  a.y = (__nv_bfloat16 *)p.y; a.ys = p.ys; a.err = p.err;
+  a.yf = p.norm_groups > 0 ? p.yf : nullptr;
+  a.d_inner = p.d_inner;
+  const long long seg_stride = (long long)p.B * p.H * p.P * p.N;
+  dim3 grid(p.n_seg, p.H, p.B);
+  cudaError_t e;
+  if (mode == 1) {
+    a.h_init = nullptr; a.h_init_seg = 0;
+    a.h_out = p.seg_state; a.h_out_seg = seg_stride; a.seg_decay = p.seg_decay;
+    e = set_smem_attr(ssd_scan_tc_kernel<true>, kSmemAlloc, s);
+    if (e != cudaSuccess) return e;
+    ssd_scan_tc_kernel<true><<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, a);
+  } else {
+    if (p.n_seg > 1) {
+      a.h_init = p.seg_state; a.h_init_seg = seg_stride; a.h_out = nullptr;
+    } else {
+      a.h_init = p.h0; a.h_init_seg = 0; a.h_out = p.h_final;
+    }
+    a.h_out_seg = 0; a.seg_decay = nullptr;
+    e = set_smem_attr(ssd_scan_tc_kernel<false>, kSmemAlloc, s);
+    if (e != cudaSuccess) return e;
+    ssd_scan_tc_kernel<false><<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace ssd

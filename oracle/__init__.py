@@ -97,6 +97,8 @@ class Oracle:
             compile_oracle(lib_path)
         self.lib = ctypes.CDLL(lib_path)
         L = self.lib
+        L.oracle_round_bf16.restype = ctypes.c_double
+        L.oracle_round_bf16.argtypes = [ctypes.c_double]
         L.oracle_silu.restype = ctypes.c_double
         L.oracle_silu.argtypes = [ctypes.c_double]
         L.oracle_softplus.restype = ctypes.c_double
@@ -119,6 +121,14 @@ class Oracle:
                                          vp, vp, ci, vp, ci, vp, vp, ci, ci, vp, ci]
 
     # ---- scalar helpers -------------------------------------------------------------------
+    def round_bf16(self, x: float) -> float:
+        return self.lib.oracle_round_bf16(float(x))
+
+    def round_bf16_array(self, a: np.ndarray) -> np.ndarray:
+        """Elementwise nearest-bf16 rounding (ties to even) of a float64 array."""
+        f = np.vectorize(self.lib.oracle_round_bf16, otypes=[np.float64])
+        return f(np.asarray(a, np.float64))
+
     def silu(self, x: float) -> float:
         return self.lib.oracle_silu(float(x))
 
@@ -269,12 +279,18 @@ class Oracle:
 
     # ---- full mixer layer ---------------------------------------------------------------------
     def mixer_forward(self, cfg: dict, hidden, rms_w, W_in, W_out, A, D, dt_bias, conv_w, conv_b,
-                      norm_w, rows=None, tokens=None, threads=None) -> np.ndarray:
+                      norm_w, rows=None, tokens=None, threads=None,
+                      bf16_activations: bool = True) -> np.ndarray:
         """RMSNorm -> in_proj -> (z | xBC | dt) -> conv/SiLU + scan + gated RMSNorm -> out_proj.
 
         hidden [B, L, d_model]; W_in [2*d_inner + 2GN + H, d_model]; W_out [d_model, d_inner].
         ``rows`` selects batch rows and ``tokens`` a causal prefix length (both exact, because
         rows are independent and the layer is causal).  Returns out [len(rows), tokens, d_model].
+
+        The layer runs in bf16 ("bfloat16 precision", Nemotron Nano 2 abstract): with
+        ``bf16_activations`` the three activation tensors the layer materialises between its
+        steps (RMSNorm output, in_proj output, gated-norm output) are rounded to bf16; all
+        arithmetic is fp64 otherwise.
         """
         Bn, L, H, P, N, G = (cfg["batch"], cfg["seqlen"], cfg["nheads"], cfg["headdim"],
                              cfg["dstate"], cfg["ngroups"])
@@ -283,8 +299,9 @@ class Oracle:
         d_model = cfg["d_model"]
         d_inner = H * P
         hid = np.ascontiguousarray(hidden[rows][:, :T])
-        hn = self.rmsnorm(hid.reshape(-1, d_model), rms_w, eps=cfg.get("rms_eps", 1e-5))
-        zxbcdt = hn @ to_f64(W_in).T  # library matmul in fp64
+        rnd = self._round_bf16_fast if bf16_activations else (lambda v: v)
+        hn = rnd(self.rmsnorm(hid.reshape(-1, d_model), rms_w, eps=cfg.get("rms_eps", 1e-5)))
+        zxbcdt = rnd(hn @ to_f64(W_in).T)  # library matmul in fp64
         zxbcdt = zxbcdt.reshape(len(rows), T, -1)
         conv_dim = d_inner + 2 * G * N
         z = np.ascontiguousarray(zxbcdt[..., :d_inner])
@@ -293,8 +310,16 @@ class Oracle:
         c2 = dict(cfg, batch=len(rows), seqlen=T)
         r = self.ssd_prefill(c2, xBC, dt, A, D, dt_bias, conv_w=conv_w, conv_b=conv_b, z=z,
                              norm_w=norm_w, threads=threads)
-        g = r["out"].reshape(-1, d_inner)
+        g = rnd(r["out"].reshape(-1, d_inner))
         return (g @ to_f64(W_out).T).reshape(len(rows), T, d_model)
+
+    @staticmethod
+    def _round_bf16_fast(a: np.ndarray) -> np.ndarray:
+        """Vectorised nearest-bf16 rounding, ties to even, from float64 (same definition as
+        oracle_round_bf16: keep 8 significant bits of the binary mantissa)."""
+        a = np.asarray(a, np.float64)
+        m, e = np.frexp(a)
+        return np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)
 
 
 def quadratic_form(x, Bm, Cm, dt, A, D, h0=None) -> np.ndarray:

@@ -63,6 +63,16 @@ static double ld(const void *p, int dtype, long long i) {
   return (double)f;
 }
 
+/* Round to the nearest bf16 value (8 significant bits), ties to even, computed directly from
+ * the double (no intermediate float rounding).  Used only where the layer materialises a
+ * bf16 activation tensor. */
+double oracle_round_bf16(double x) {
+  if (x == 0.0 || !isfinite(x)) return x;
+  int e;
+  const double m = frexp(x, &e); /* x = m * 2^e, 0.5 <= |m| < 1 */
+  return ldexp(nearbyint(ldexp(m, 8)), e - 8);
+}
+
 /* SiLU(x) = x * sigmoid(x) = x / (1 + e^{-x}). */
 double oracle_silu(double x) { return x / (1.0 + exp(-x)); }
 

@@ -23,11 +23,26 @@ def rel_err(got, want) -> float:
     return float(np.max(np.abs(got - want))) / max(rms, 1e-300)
 
 
-def assert_close(got, want, tol, what):
+# unit roundoff of the stored output: round-to-nearest into bf16 moves a value by at most
+# 2^-8 of its magnitude (8 significant bits), fp32 by 2^-24
+UNIT_ROUNDOFF = {"bf16": 2.0 ** -8, "f32": 2.0 ** -24}
+
+
+def assert_close(got, want, tol, what, out_dtype="f32", both_rounded=False):
+    """max|got - want| <= tol * RMS(want), applied on top of the rounding of the output into
+    its storage dtype: |got - want| <= tol * RMS(want) + u * |want| elementwise (u = 2^-8 for
+    bf16 outputs).  When `want` is itself a stored GPU result (two roundings), the allowance
+    is 2u: the two values may round to neighbouring representable numbers.  Returns the plain
+    max|err|/RMS."""
     got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
     assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    rms = max(float(np.sqrt(np.mean(want * want))), 1e-300)
+    excess = np.abs(got - want) - (2 if both_rounded else 1) * UNIT_ROUNDOFF[out_dtype] * np.abs(want)
+    r_ex = float(np.max(excess)) / rms
     r = rel_err(got, want)
-    assert r <= tol, f"{what}: max|err|/RMS = {r:.3e} > {tol:.1e}"
+    assert r_ex <= tol, (f"{what}: max(|err| - u|ref|)/RMS = {r_ex:.3e} > {tol:.1e} "
+                         f"(plain max|err|/RMS = {r:.3e})")
     return r
 
 

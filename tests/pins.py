@@ -367,7 +367,8 @@ def pin_mixer_composition(o, seed=11):
     nw = r.uniform(0.5, 1.5, d)
     W_out = np.zeros((proj, d))
     W_out[:d] = np.eye(d)
-    out = o.mixer_forward(cfg, hid, None, np.eye(proj), W_out, A, D, bias, cw, None, nw)
+    out = o.mixer_forward(cfg, hid, None, np.eye(proj), W_out, A, D, bias, cw, None, nw,
+                          bf16_activations=False)
     hn = o.rmsnorm(hid.reshape(-1, proj), None).reshape(B, L, proj)
     ref = o.ssd_prefill(cfg, np.ascontiguousarray(hn[..., d:2 * d + 2 * G * N]),
                         np.ascontiguousarray(hn[..., 2 * d + 2 * G * N:]), A, D, bias, conv_w=cw,
@@ -377,10 +378,29 @@ def pin_mixer_composition(o, seed=11):
     return ok, f"rel err {e:.2e}"
 
 
+def pin_bf16_rounding(o, seed=12):
+    """Nearest-bf16 rounding: representable values are fixed points, ties go to the even
+    mantissa, and on float32 inputs it agrees with the integer round-half-even of the bit
+    pattern (an independent formulation); the vectorised form agrees with the scalar one."""
+    from mamba_ssd_scan_02_b200 import datagen
+    r = _rng(seed)
+    cases = [(1.0, 1.0), (1.0 + 2 ** -8, 1.0), (1.0 + 3 * 2 ** -8, 1.0 + 2 ** -6),
+             (-(1.0 + 2 ** -7), -(1.0 + 2 ** -7)), (1.0 + 2 ** -8 + 2 ** -30, 1.0 + 2 ** -7),
+             (3.0e-3, float(datagen.bf16_value(datagen.bf16_bits(np.float32([3.0e-3])))[0])),
+             (0.0, 0.0)]
+    ok = all(o.round_bf16(x) == want for x, want in cases)
+    x32 = (r.standard_normal(2000) * 10.0 ** r.uniform(-6, 6, 2000)).astype(np.float32)
+    via_bits = datagen.bf16_value(datagen.bf16_bits(x32)).astype(np.float64)
+    ok = ok and np.array_equal(o.round_bf16_array(x32.astype(np.float64)), via_bits)
+    x64 = r.standard_normal(500) * 3.0
+    ok = ok and np.array_equal(o._round_bf16_fast(x64), o.round_bf16_array(x64))
+    return bool(ok), ""
+
+
 ALL_PINS = [pin_activation_identities, pin_quadratic_form, pin_quadratic_with_conv,
             pin_prefix_sum, pin_zero_dt, pin_geometric, pin_chunk_invariance, pin_split_carry,
             pin_decode_equals_prefill, pin_conv_impulse, pin_norm_invariants, pin_linearity,
-            pin_mixer_composition]
+            pin_mixer_composition, pin_bf16_rounding]
 
 # planted mistakes in ssd_oracle.c (ORACLE_MUTANT values)
 MUTANTS = {1: "D*x term dropped", 2: "sign of A flipped", 3: "output read before the update",

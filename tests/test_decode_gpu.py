@@ -30,7 +30,7 @@ def _run_steps(oracle, cfg, steps, seed=3):
     cache2 = torch.empty_like(cache)
     ost = inp["h0"].astype(np.float64)
     ocache = inp["conv_state_in"]
-    p = {k: dev(inp[k]) for k in ("A", "D", "dt_bias", "conv_w", "conv_b", "norm_w")}
+    p = {k: dev(inp.get(k)) for k in ("A", "D", "dt_bias", "conv_w", "conv_b", "norm_w")}
     worst = 0.0
     for t in range(steps):
         xt = np.ascontiguousarray(inp["xBC"][:, t]); dtt = np.ascontiguousarray(inp["dt"][:, t])
@@ -38,10 +38,11 @@ def _run_steps(oracle, cfg, steps, seed=3):
         y = ssd.decode_step(cfg, dev(xt), dev(dtt), p["A"], p["D"], p["dt_bias"], p["conv_w"],
                             p["conv_b"], state, cache, cache2, dev(zt), p["norm_w"])
         r = oracle.decode_step(cfg, xt, dtt, inp["A"], inp["D"], inp["dt_bias"], inp["conv_w"],
-                               inp["conv_b"], ocache, ost, z_t=zt, norm_w=inp["norm_w"])
+                               inp["conv_b"], ocache, ost, z_t=zt, norm_w=inp.get("norm_w"))
         want = r["out"] if cfg["norm_groups"] else r["y"].reshape(Bn, -1)
         tol = TOL_BF16 if bf else TOL_F32
-        worst = max(worst, assert_close(y.float().cpu().numpy(), want, tol, f"step {t} y"))
+        worst = max(worst, assert_close(y.float().cpu().numpy(), want, tol, f"step {t} y",
+                                        out_dtype=cfg["dtype"]))
         # the carried cache is the oracle's shifted cache, bit for bit
         ocache = np.ascontiguousarray(np.concatenate([ocache[:, 1:], xt[:, None]], axis=1))
         assert np.array_equal(host(cache2), ocache), f"conv cache, step {t}"
@@ -82,7 +83,8 @@ def test_decode_equals_prefill(cuda_lib):
                             dev(np.ascontiguousarray(inp["z"][:, t])), p["norm_w"])
         cache, cache2 = cache2, cache
         ref = yfull[:, t].float().cpu().numpy()
-        assert_close(y.float().cpu().numpy(), ref, TOL_BF16, f"decode step {j}")
+        assert_close(y.float().cpu().numpy(), ref, TOL_BF16, f"decode step {j}", out_dtype="bf16",
+                     both_rounded=True)
     assert_close(host(state), host(hfull), TOL_BF16, "state")
     assert torch.equal(cache, cfull)
 
@@ -129,7 +131,8 @@ def test_decode_16k_steps_full_size(cuda_lib, oracle):
                                norm_w=norm_w)
         oc_b = np.ascontiguousarray(np.concatenate([oc_b[:, 1:], pool["xBC"][i][:, None]], axis=1))
         assert np.array_equal(host(gc), oc_b), f"conv cache, step {s}"
-        assert_close(y.float().cpu().numpy(), r["out"], TOL_BF16, f"all rows, step {s}")
+        assert_close(y.float().cpu().numpy(), r["out"], TOL_BF16, f"all rows, step {s}",
+                     out_dtype="bf16")
     assert_close(host(gst), ost_b, TOL_BF16, "state after 64 steps (all rows)")
     del gst, gc, gc2
 
@@ -151,6 +154,7 @@ def test_decode_16k_steps_full_size(cuda_lib, oracle):
         ocache = np.ascontiguousarray(
             np.concatenate([ocache[:, 1:], pool["xBC"][i][rows][:, None]], axis=1))
         if s % 1024 == 1023:
-            assert_close(y.float().cpu().numpy()[rows], r["out"], TOL_BF16, f"rows 0/63, step {s}")
+            assert_close(y.float().cpu().numpy()[rows], r["out"], TOL_BF16, f"rows 0/63, step {s}",
+                         out_dtype="bf16")
     assert_close(host(state)[rows], ost, TOL_BF16, "state after 16384 steps")
     assert np.array_equal(host(cache)[rows], ocache)

@@ -26,7 +26,7 @@ def test_mixer_small(cuda_lib, oracle):
                norm_groups=2)
     inp = datagen.make_inputs(4, cfg)
     out = _mixer(cfg, inp)
-    assert_close(out.float().cpu().numpy(), _oracle(oracle, cfg, inp), TOL_BF16, "mixer small")
+    assert_close(out.float().cpu().numpy(), _oracle(oracle, cfg, inp), TOL_BF16, "mixer small", out_dtype="bf16")
 
 
 def test_mixer_odd_tokens_and_width(cuda_lib, oracle):
@@ -34,7 +34,7 @@ def test_mixer_odd_tokens_and_width(cuda_lib, oracle):
                norm_groups=2)
     inp = datagen.make_inputs(4, cfg)
     out = _mixer(cfg, inp)
-    assert_close(out.float().cpu().numpy(), _oracle(oracle, cfg, inp), TOL_BF16, "mixer odd")
+    assert_close(out.float().cpu().numpy(), _oracle(oracle, cfg, inp), TOL_BF16, "mixer odd", out_dtype="bf16")
 
 
 def test_mixer_12b_width_full_size(cuda_lib, oracle):
@@ -45,4 +45,4 @@ def test_mixer_12b_width_full_size(cuda_lib, oracle):
     out = _mixer(cfg, inp)
     got = out[[0, 7], :1024].float().cpu().numpy()
     want = _oracle(oracle, cfg, inp, rows=[0, 7], tokens=1024)
-    assert_close(got, want, TOL_BF16, "mixer 12B width")
+    assert_close(got, want, TOL_BF16, "mixer 12B width", out_dtype="bf16")
