@@ -18,7 +18,7 @@ constexpr int kConvTokens = 32;  // tokens per thread (sliding window kept in re
 // 16-byte vector loads along the channel dimension are coalesced across the warp.
 // Channels [c_begin, c_begin + C_out) of the C-channel input are convolved; the output row
 // holds C_out channels (fp32 for the CUDA-core path, bf16 for the tensor-core path).
-template <typename T, typename OutT, int W>
+template <typename T, typename OutT, int W, int TPT>
 __global__ void __launch_bounds__(128) conv_silu_kernel(const T *__restrict__ xBC, long long xs,
                                                         const T *__restrict__ csi,
                                                         const T *__restrict__ w,
@@ -29,7 +29,7 @@ __global__ void __launch_bounds__(128) conv_silu_kernel(const T *__restrict__ xB
   if (o8 >= C_out) return;
   const int c8 = c_begin + o8;
   const int b = blockIdx.z;
-  const int t0 = blockIdx.y * kConvTokens;
+  const int t0 = blockIdx.y * TPT;
   const T *xrow = xBC + (long long)b * L * xs;
   float wt[4][8], bs[8];
 #pragma unroll
@@ -52,28 +52,38 @@ __global__ void __launch_bounds__(128) conv_silu_kernel(const T *__restrict__ xB
       for (int i = 0; i < 8; ++i) hist[j][i] = 0.f;
     }
   }
-  const int t1 = min(L, t0 + kConvTokens);
-  for (int t = t0; t < t1; ++t) {
-    float cur[8], out[8];
-    load8(xrow + (long long)t * xs + c8, cur);
+  const int t1 = min(L, t0 + TPT);
+  // groups of 4 tokens: the 4 row loads are issued before any of them is used
+  for (int tg = t0; tg < t1; tg += 4) {
+    float cur[4][8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (W == 0) {
-        out[i] = cur[i];
-        continue;
-      }
-      // tap k multiplies time t-(W-1)+k: k = W-1 is cur, k = W-1-j is hist[3-j]
-      float acc = bs[i] + wt[W > 0 ? W - 1 : 0][i] * cur[i];
-#pragma unroll
-      for (int j = 1; j < W; ++j) acc += wt[W - 1 - j][i] * hist[3 - j][i];
-      out[i] = silu(acc);
+    for (int j = 0; j < 4; ++j) {
+      if (tg + j < t1) load8(xrow + (long long)(tg + j) * xs + c8, cur[j]);
     }
-    store8(u + ((long long)b * L + t) * C_out + o8, out);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      hist[0][i] = hist[1][i];
-      hist[1][i] = hist[2][i];
-      hist[2][i] = cur[i];
+    for (int j = 0; j < 4; ++j) {
+      const int t = tg + j;
+      if (t >= t1) break;
+      float out[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (W == 0) {
+          out[i] = cur[j][i];
+          continue;
+        }
+        // tap k multiplies time t-(W-1)+k: k = W-1 is cur, k = W-1-m is hist[3-m]
+        float acc = bs[i] + wt[W > 0 ? W - 1 : 0][i] * cur[j][i];
+#pragma unroll
+        for (int m = 1; m < W; ++m) acc += wt[W - 1 - m][i] * hist[3 - m][i];
+        out[i] = silu(acc);
+      }
+      store8(u + ((long long)b * L + t) * C_out + o8, out);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        hist[0][i] = hist[1][i];
+        hist[1][i] = hist[2][i];
+        hist[2][i] = cur[j][i];
+      }
     }
   }
 }
@@ -92,8 +102,9 @@ __global__ void dt_kernel(const T *__restrict__ dt, long long ds, const float *_
 
 // Effective dt and its chunk-local inclusive prefix sum of dt*A, written head-major
 // [B, H, Lpad] (Lpad = L rounded up to the 128-token chunk; padding has dt = 0 so the prefix
-// stays flat).  One CTA: 128 tokens x 32 heads of one batch row; the tile is transposed
-// through shared memory so that both the dt reads and the head-major writes are coalesced.
+// stays flat).  One CTA: one 128-token chunk x 8 heads of one batch row.  Thread t reads the
+// 8 heads of token t (16 bytes for bf16 when H % 8 == 0, else element by element), the tile
+// is transposed through shared memory, and each warp scans two heads.
 template <typename T>
 __global__ void __launch_bounds__(128) dt_cumsum_kernel(const T *__restrict__ dt, long long ds,
                                                          const float *__restrict__ bias,
@@ -101,26 +112,34 @@ __global__ void __launch_bounds__(128) dt_cumsum_kernel(const T *__restrict__ dt
                                                          float *__restrict__ dte,
                                                          float *__restrict__ cs, int L, int H,
                                                          int Lpad, int sp, float lo, float hi) {
-  __shared__ float v[128][33];
-  const int c0 = blockIdx.x * 128, h0 = blockIdx.y * 32, b = blockIdx.z;
+  __shared__ float v[128][9];
+  const int c0 = blockIdx.x * 128, h0 = blockIdx.y * 8, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  for (int i = tid; i < 128 * 32; i += 128) {
-    const int t = i / 32, hh = i % 32, tt = c0 + t, h = h0 + hh;
-    float val = 0.f;
-    if (tt < L && h < H)
-      val = effective_dt(io<T>::ld(dt + ((long long)b * L + tt) * ds + h), bias[h], sp, lo, hi);
-    v[t][hh] = val;
+  {
+    const int tt = c0 + tid;
+    float raw[8];
+    const T *row = dt + ((long long)b * L + tt) * ds + h0;
+    if (tt < L && sizeof(T) == 2 && (H % 8) == 0 && (ds % 8) == 0) {
+      load8(reinterpret_cast<const __nv_bfloat16 *>(row), raw);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) raw[j] = (tt < L && h0 + j < H) ? io<T>::ld(row + j) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      v[tid][j] = (tt < L && h0 + j < H) ? effective_dt(raw[j], bias[h0 + j], sp, lo, hi) : 0.f;
   }
   __syncthreads();
-  for (int hh = warp * 8; hh < warp * 8 + 8; ++hh) {
-    const int h = h0 + hh;
+#pragma unroll
+  for (int jj = 0; jj < 2; ++jj) {
+    const int j = 2 * warp + jj, h = h0 + j;
     if (h >= H) break;
     const float a = A[h];
     float d[4], c[4];
     float run = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      d[i] = v[4 * lane + i][hh];
+      d[i] = v[4 * lane + i][j];
       run += d[i] * a;
       c[i] = run;
     }
@@ -176,13 +195,22 @@ int grid_for(long long n, int threads) {
 
 }  // namespace
 
+// Many channels (the CUDA-core path converts every channel): 32 tokens per thread; few
+// channels (B|C only): 8 tokens per thread, for enough threads to hide the load latency.
 template <typename T, typename OutT, int W>
 static void conv_launch(const PrefillPlan &p, OutT *out, int c_begin, int C_out, cudaStream_t s) {
   const int threads = 128;
-  dim3 grid((C_out / 8 + threads - 1) / threads, (p.L + kConvTokens - 1) / kConvTokens, p.B);
-  conv_silu_kernel<T, OutT, W><<<grid, threads, 0, s>>>((const T *)p.xBC, p.xs, (const T *)p.csi,
-                                                         (const T *)p.conv_w, (const T *)p.conv_b,
-                                                         out, p.L, p.conv_dim, c_begin, C_out);
+  if (C_out >= 4096) {
+    dim3 grid((C_out / 8 + threads - 1) / threads, (p.L + kConvTokens - 1) / kConvTokens, p.B);
+    conv_silu_kernel<T, OutT, W, kConvTokens><<<grid, threads, 0, s>>>(
+        (const T *)p.xBC, p.xs, (const T *)p.csi, (const T *)p.conv_w, (const T *)p.conv_b, out, p.L,
+        p.conv_dim, c_begin, C_out);
+  } else {
+    dim3 grid((C_out / 8 + threads - 1) / threads, (p.L + 7) / 8, p.B);
+    conv_silu_kernel<T, OutT, W, 8><<<grid, threads, 0, s>>>(
+        (const T *)p.xBC, p.xs, (const T *)p.csi, (const T *)p.conv_w, (const T *)p.conv_b, out, p.L,
+        p.conv_dim, c_begin, C_out);
+  }
 }
 
 template <typename T, typename OutT>
@@ -222,7 +250,7 @@ cudaError_t launch_dt(const PrefillPlan &p, cudaStream_t s) {
 }
 
 cudaError_t launch_dt_cumsum(const PrefillPlan &p, float *dte, float *cs, int Lpad, cudaStream_t s) {
-  dim3 grid(Lpad / 128, (p.H + 31) / 32, p.B);
+  dim3 grid(Lpad / 128, (p.H + 7) / 8, p.B);
   if (p.bf16)
     dt_cumsum_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>((const __nv_bfloat16 *)p.dt, p.ds, p.dt_bias,
                                                           p.A, dte, cs, p.L, p.H, Lpad, p.softplus,

@@ -11,7 +11,7 @@
 //   MMA3  Ys    = C . h_{k-1}^T              M=128 (t) N=64 (p)  K=128 (n)
 //   MMA4  dH^T  = B^T . (w o X), w_s = e^{cs_Q - cs_s} dt_s   M=128 (n) N=64 (p) K=128 (s)
 // then y_t = Yi + e^{cs_t} Ys (the D x skip is folded into the diagonal of S~) and
-// h_k = e^{cs_Q} h_{k-1} + dH, kept in fp32 registers (an fp16 copy feeds MMA3 of chunk k+1).
+// h_k = e^{cs_Q} h_{k-1} + dH, kept in fp32 in TMEM (an fp16 copy feeds MMA3 of chunk k+1).
 // This is the token recurrence h_t = e^{dt_t A} h_{t-1} + dt_t x_t B_t^T, y_t = h_t C_t + D x_t
 // regrouped by chunk; every exponent is a difference cs_t - cs_s <= 0 or is split at a
 // 32-token block boundary where both factors stay below e^60 (else computed directly).
@@ -19,11 +19,11 @@
 // the final state carries the rounding of B only: its largest entries come from the newest
 // tokens, whose products are not averaged over many terms.
 //
-// Warp roles (512 threads): warp 0 issues TMA loads (B and C tiles of the group, the head's
+// Warp roles (640 threads): warp 0 issues TMA loads (B and C tiles of the group, the head's
 // raw x rows with a 3-token halo, per-chunk dt and prefix sums), warp 1 allocates TMEM and
-// issues the MMAs, warps 4-7 compute the head's x channels (causal conv1d + SiLU) in place
-// into the double-buffered X tile and into w o X, warps 8-11 turn S into S~, warps 12-15
-// update the state and write y.  Per chunk the MMAs are issued as MMA4(k), MMA3(k), MMA1(k+1), MMA2(k), so the
+// issues the MMAs, warps 4-11 compute the head's x channels (causal conv1d + SiLU) in place
+// into the double-buffered X tile and into w o X, warps 12-15 turn S into S~, warps 16-19
+// update the state (kept in fp32 in TMEM) and write y.  Per chunk the MMAs are issued as MMA4(k), MMA3(k), MMA1(k+1), MMA2(k), so the
 // mask of chunk k overlaps four MMAs and the state update overlaps two.  Hand-offs use
 // mbarriers (TMA transaction counts, tcgen05.commit, thread arrivals); every wait is bounded
 // and a timeout aborts the CTA cleanly and latches SSD_ERR_TIMEOUT.
@@ -63,7 +63,9 @@ namespace {
 using namespace tc;
 
 constexpr int QC = 128;              // tokens per chunk
-constexpr int kThreadsTC = 512;
+constexpr int kThreadsTC = 640;       // 20 warps
+constexpr int kConvWarps = 8;          // warps 4..11
+constexpr int kTokPerConvWarp = QC / kConvWarps;  // 16
 constexpr uint32_t kTile = 16384;    // one 128-row x 128-byte operand box
 // per-stage layout (bytes)
 constexpr uint32_t OFF_C = 0;                 // C tile: channels 0-63 | 64-127
@@ -71,31 +73,37 @@ constexpr uint32_t OFF_B = 2 * kTile;         // B tile
 constexpr uint32_t OFF_DT = 4 * kTile;        // dt[128] fp32
 constexpr uint32_t OFF_CS = OFF_DT + 512;     // cs[128] fp32
 constexpr uint32_t kStage = 4 * kTile + 1024;  // 66560 = 65 * 1024
-// CTA layout.  X[b] first receives (by TMA) the chunk's raw bf16 x rows for times t0-3 ..
-// t0+127 (131 rows of this head's 64 channels); the conv overwrites row s with X row s.
+// CTA layout.  X[b] (three buffers, chunk k uses b = k % 3) first receives by TMA the chunk's
+// raw bf16 x rows for times t0-3 .. t0+127 (131 rows of this head's 64 channels); the conv
+// overwrites row s with X row s.  w o X has a single buffer (MMA4 reads it right away).
+constexpr int kXBufs = 3;
 constexpr uint32_t kXBuf = 17 * 1024;           // 131 rows of 128 bytes, padded
 constexpr uint32_t kRawRows = QC + 3;
-constexpr uint32_t OFF_X = 2 * kStage;          // X[2]   [s][p] fp16 (raw x rows first)
-constexpr uint32_t OFF_XW = OFF_X + 2 * kXBuf;  // wX[2]  [s][p] fp16, 16 KB each
-constexpr uint32_t OFF_H = OFF_XW + 2 * kTile;  // h copy [n][p] fp16, 16 KB
-constexpr uint32_t OFF_CF = OFF_H + kTile;      // column factors, 128 fp32
-constexpr uint32_t OFF_BAR = OFF_CF + 512;
+constexpr uint32_t OFF_X = 2 * kStage;              // X[3]  [s][p] fp16 (raw x rows first)
+constexpr uint32_t OFF_XW = OFF_X + kXBufs * kXBuf;  // w o X [s][p] fp16, 16 KB
+constexpr uint32_t OFF_H = OFF_XW + kTile;          // h copy [n][p] fp16, 16 KB
+constexpr uint32_t OFF_CF = OFF_H + kTile;          // column factors, 128 fp32
+constexpr uint32_t OFF_CSM = OFF_CF + 512;          // the mask's copies of cs and dt
+constexpr uint32_t OFF_DTM = OFF_CSM + 512;
+constexpr uint32_t OFF_BAR = OFF_DTM + 512;
 enum {
-  BAR_FULL0, BAR_FULL1, BAR_EMPTY0, BAR_EMPTY1, BAR_SREADY0, BAR_SREADY1, BAR_STREADY0,
-  BAR_STREADY1, BAR_XREADY0, BAR_XREADY1, BAR_XFREE0, BAR_XFREE1, BAR_DHREADY, BAR_HREADY,
-  BAR_YREADY, BAR_YFREE, BAR_XLOREADY, BAR_DONE, kNumBars
+  BAR_FULL0, BAR_FULL1, BAR_EMPTY0, BAR_EMPTY1, BAR_FULLX0, BAR_FULLX1, BAR_FULLX2, BAR_XFREE0,
+  BAR_XFREE1, BAR_XFREE2, BAR_SREADY0, BAR_SREADY1, BAR_STREADY0, BAR_STREADY1, BAR_XREADY,
+  BAR_XWFREE, BAR_DHREADY, BAR_HREADY, BAR_YREADY, BAR_YFREE, BAR_XLOREADY, BAR_DONE, kNumBars
 };
-constexpr uint32_t OFF_MISC = OFF_BAR + 8 * 24;   // [0] TMEM base, [1] abort flag
+constexpr uint32_t OFF_MISC = OFF_BAR + 8 * 32;   // [0] TMEM base, [1] abort flag
 constexpr uint32_t kSmemUsed = OFF_MISC + 16;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;  // room to align the base to 1024 bytes
-static_assert(kNumBars <= 24, "barrier slots");
+static_assert(kNumBars <= 32, "barrier slots");
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
-static_assert(OFF_X % 1024 == 0 && OFF_XW % 1024 == 0 && OFF_H % 1024 == 0, "swizzle alignment");
+static_assert(OFF_X % 1024 == 0 && kXBuf % 1024 == 0 && OFF_XW % 1024 == 0 && OFF_H % 1024 == 0,
+              "swizzle alignment");
 static_assert(kRawRows * 128 <= kXBuf, "raw x tile fits its buffer");
 
 // TMEM columns (fp32 accumulators, 128 lanes).  After the mask, S[b] holds S~ as packed fp16
 // in its first 64 columns.
-constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_YI = 256, TM_YS = 320, TM_DH = 384, TM_COLS = 512;
+constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_YI = 256, TM_YS = 320, TM_DH = 384, TM_H = 448,
+                   TM_COLS = 512;  // TM_H: the fp32 state h^T (row n, column p)
 
 constexpr uint32_t IDESC_S = idesc_f16(128, 128, false, false, kFmtF16);  // C K-major, B K-major
 constexpr uint32_t IDESC_YS = idesc_f16(128, 64, false, true, kFmtF16);   // C K-major, h N-major
@@ -136,15 +144,15 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
 // A warpgroup-uniform bounded wait: one leader thread waits on the mbarrier, then the
 // group syncs on its named barrier and reads the (shared) abort flag.
 __device__ __forceinline__ bool wg_wait(uint32_t bar, uint32_t parity, bool leader, int nb,
-                                        volatile int *abort_flag, int *err) {
+                                        volatile int *abort_flag, int *err, int nthreads = 128) {
   if (leader) mbar_wait(bar, parity, abort_flag, err);
-  named_bar(nb, 128);
+  named_bar(nb, nthreads);
   return *abort_flag == 0;
 }
 
 // ---- MMA issue (single thread) ---------------------------------------------------------
 __device__ __forceinline__ void issue_S(uint32_t stage, uint32_t tS) {
-#pragma unroll
+#pragma unroll 1
   for (int j = 0; j < 8; ++j) {
     const uint32_t koff = (j >> 2) * kTile + (j & 3) * 32;
     mma_f16_ss(tS, smem_desc_sw128(stage + OFF_C + koff, 16, 1024),
@@ -152,7 +160,7 @@ __device__ __forceinline__ void issue_S(uint32_t stage, uint32_t tS) {
   }
 }
 __device__ __forceinline__ void issue_Ys(uint32_t stage, uint32_t hbase, uint32_t tYs) {
-#pragma unroll
+#pragma unroll 1
   for (int j = 0; j < 8; ++j) {
     const uint32_t koff = (j >> 2) * kTile + (j & 3) * 32;
     mma_f16_ss(tYs, smem_desc_sw128(stage + OFF_C + koff, 16, 1024),
@@ -161,12 +169,12 @@ __device__ __forceinline__ void issue_Ys(uint32_t stage, uint32_t hbase, uint32_
 }
 // S~ in TMEM: 16 fp16 of K per MMA = 8 columns
 __device__ __forceinline__ void issue_Yi(uint32_t tSt, uint32_t xbase, uint32_t tYi) {
-#pragma unroll
+#pragma unroll 1
   for (int j = 0; j < 8; ++j)
     mma_f16_ts(tYi, tSt + 8 * j, smem_desc_sw128(xbase + j * 2048, 8192, 1024), IDESC_YI, j > 0);
 }
 __device__ __forceinline__ void issue_dH(uint32_t stage, uint32_t xwbase, uint32_t tDH, bool acc) {
-#pragma unroll
+#pragma unroll 1
   for (int j = 0; j < 8; ++j)
     mma_f16_ss(tDH, smem_desc_sw128(stage + OFF_B + j * 2048, kTile, 1024),
                smem_desc_sw128(xwbase + j * 2048, 8192, 1024), IDESC_DH, (j > 0 || acc) ? 1u : 0u);
@@ -177,12 +185,13 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return (uint32_t)row * 128u + ((uint32_t)(chunk ^ (row & 7)) << 4);
 }
 
-__device__ __forceinline__ void write_h_tile(unsigned char *smem, const float (&hr)[64], int n) {
+// fp16 copy of state columns p = 32*half .. 32*half+31 of row n into the h tile
+__device__ __forceinline__ void write_h_tile(unsigned char *smem, const float (&hr)[32], int n, int half) {
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
+  for (int c = 0; c < 4; ++c) {
     uint4 v = make_uint4(pack_f16(hr[8 * c + 0], hr[8 * c + 1]), pack_f16(hr[8 * c + 2], hr[8 * c + 3]),
                          pack_f16(hr[8 * c + 4], hr[8 * c + 5]), pack_f16(hr[8 * c + 6], hr[8 * c + 7]));
-    *reinterpret_cast<uint4 *>(smem + OFF_H + swz(n, c)) = v;
+    *reinterpret_cast<uint4 *>(smem + OFF_H + swz(n, 4 * half + c)) = v;
   }
 }
 
@@ -230,18 +239,22 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
+    // Raw x rows of chunk k go to X[k % 3] once MMA2 of chunk k-3 has released it; the B/C
+    // tiles, dt and prefix sums go to stage k % 2 once chunk k-2's consumers released it.
     if (lane == 0) {
-      int k = 0;
+      int k = 0, nx = 0, nbc = 0;
       for (; k < nck; ++k) {
-        const int st = k & 1;
-        if (k >= 2 && !mbar_wait(BAR(BAR_EMPTY0 + st), ((k >> 1) - 1) & 1, abort_flag, a.err)) break;
-        if (k >= 2 && !mbar_wait(BAR(BAR_XFREE0 + st), ((k >> 1) - 1) & 1, abort_flag, a.err)) break;
-        const uint32_t sst = sb + st * kStage;
+        const int xb = k % kXBufs, st = k & 1;
         const int t0 = t_begin + k * QC;
+        if (k >= kXBufs && !mbar_wait(BAR(BAR_XFREE0 + xb), (k / kXBufs - 1) & 1, abort_flag, a.err)) break;
+        mbar_arrive_expect_tx(BAR(BAR_FULLX0 + xb), kRawRows * 128);
+        tma_load_3d(sb + OFF_X + xb * kXBuf, &tm_x, h * 64, t0 - 3, b, BAR(BAR_FULLX0 + xb));
+        ++nx;
+        if (k >= 2 && !mbar_wait(BAR(BAR_EMPTY0 + st), ((k >> 1) - 1) & 1, abort_flag, a.err)) break;
+        const uint32_t sst = sb + st * kStage;
         const uint32_t full = BAR(BAR_FULL0 + st);
         TC_MARK(k, 12);
-        mbar_arrive_expect_tx(full, (kStateOnly ? 2 * kTile : 4 * kTile) + 1024 + kRawRows * 128);
-        tma_load_3d(sb + OFF_X + st * kXBuf, &tm_x, h * 64, t0 - 3, b, full);
+        mbar_arrive_expect_tx(full, (kStateOnly ? 2 * kTile : 4 * kTile) + 1024);
         const int cB = g * 128, cC = a.G * 128 + g * 128;
         if (!kStateOnly) {
           tma_load_3d(sst + OFF_C, &tm_bc, cC, t0, b, full);
@@ -252,10 +265,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const long long hoff = ((long long)b * a.H + h) * a.Lpad + t0;
         bulk_load(sst + OFF_DT, a.dte + hoff, 512, full);
         bulk_load(sst + OFF_CS, a.cs + hoff, 512, full);
+        ++nbc;
       }
       // every load issued must land before the CTA may exit
       int never_abort = 0;
-      for (int j = (k >= 2 ? k - 2 : 0); j < k; ++j)
+      for (int j = (nx >= kXBufs ? nx - kXBufs : 0); j < nx; ++j)
+        mbar_wait(BAR(BAR_FULLX0 + j % kXBufs), (j / kXBufs) & 1, &never_abort, a.err);
+      for (int j = (nbc >= 2 ? nbc - 2 : 0); j < nbc; ++j)
         mbar_wait(BAR(BAR_FULL0 + (j & 1)), (j >> 1) & 1, &never_abort, a.err);
     }
   } else if (warp == 1) {
@@ -272,21 +288,23 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
       }
       for (int k = 0; ok && k < nck; ++k) {
-        const int st = k & 1;
+        const int st = k & 1, xb = k % kXBufs;
         const uint32_t sst = sb + st * kStage;
         // h_{k-1} in shared memory and dH free
         if (!(ok = mbar_wait(BAR(BAR_HREADY), k & 1, abort_flag, a.err))) break;
         if (kStateOnly && !(ok = mbar_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, abort_flag, a.err))) break;
-        if (!(ok = mbar_wait(BAR(BAR_XREADY0 + st), (k >> 1) & 1, abort_flag, a.err))) break;
+        if (!(ok = mbar_wait(BAR(BAR_XREADY), k & 1, abort_flag, a.err))) break;
         tc_fence_after();
         TC_MARK(k, 8);
-        issue_dH(sst, sb + OFF_XW + st * kTile, tDH, false);
+        issue_dH(sst, sb + OFF_XW, tDH, false);
+        mma_commit(BAR(BAR_XWFREE));
         if (!kStateOnly) {
           if (k > 0 && !(ok = mbar_wait(BAR(BAR_YFREE), (k - 1) & 1, abort_flag, a.err))) break;
           tc_fence_after();
           TC_MARK(k, 9);
           issue_Ys(sst, sb + OFF_H, tYs);
         }
+        mma_commit(BAR(BAR_EMPTY0 + st));  // MMA1/MMA3/MMA4 of chunk k done with the B/C tiles
         if (k != last) mma_commit(BAR(BAR_DHREADY));
         if (!kStateOnly) {
           if (k + 1 < nck) {
@@ -300,15 +318,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           if (!(ok = mbar_wait(BAR(BAR_STREADY0 + st), (k >> 1) & 1, abort_flag, a.err))) break;
           tc_fence_after();
           TC_MARK(k, 11);
-          issue_Yi(tmem + (st ? TM_S1 : TM_S0), sb + OFF_X + st * kXBuf, tYi);
+          issue_Yi(tmem + (st ? TM_S1 : TM_S0), sb + OFF_X + xb * kXBuf, tYi);
           mma_commit(BAR(BAR_YREADY));
         }
-        mma_commit(BAR(BAR_XFREE0 + st));
-        mma_commit(BAR(BAR_EMPTY0 + st));
-        if (k == last) {  // low part of w o X (in the other w o X slot) for the final state
+        mma_commit(BAR(BAR_XFREE0 + xb));
+        if (k == last) {  // low part of w o X (in the spare X buffer) for the final state
           if (!(ok = mbar_wait(BAR(BAR_XLOREADY), 0, abort_flag, a.err))) break;
           tc_fence_after();
-          issue_dH(sst, sb + OFF_XW + (st ^ 1) * kTile, tDH, true);
+          issue_dH(sst, sb + OFF_X + ((k + 1) % kXBufs) * kXBuf, tDH, true);
           mma_commit(BAR(BAR_DHREADY));
         }
       }
@@ -317,14 +334,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       int never_abort = 0;
       mbar_wait(BAR(BAR_DONE), 0, &never_abort, a.err);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 4 && warp < 4 + kConvWarps) {
     // ---------------------------------------------------------------- conv + SiLU -> X, w o X
-    // Warp cw makes tokens 32cw..32cw+31; lane l channels 2l, 2l+1.  Raw row r of the X
-    // buffer holds time t0-3+r; token s reads rows s..s+3 (a 4-register window) and then
-    // overwrites row s with its X row.  Rows 32cw+32..+34 belong to the next warp's tokens,
+    // Warp cw makes tokens 16cw..16cw+15; lane l channels 2l, 2l+1.  Raw row r of the X
+    // buffer holds time t0-3+r; token s reads rows s..s+3 (a register window) and then
+    // overwrites row s with its X row.  Rows 16cw+16..+18 belong to the next warp's tokens,
     // so every warp reads them before the group barrier that precedes all writes.
     const int cw = warp - 4;
-    const bool leader = (tid == 128);
+    const bool leader = (tid == 5 * 32);  // leaders sit on different SM sub-partitions
     const int ch = h * 64 + 2 * lane;
     const int W = a.W;
     float e0[4], e1[4], bias0 = 0.f, bias1 = 0.f;
@@ -338,26 +355,31 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       bias0 = __bfloat162float(a.conv_b[ch]);
       bias1 = __bfloat162float(a.conv_b[ch + 1]);
     }
-    const uint32_t lane_byte = (uint32_t)(lane & 3) << 2;
+    // byte offset of this lane's 4 bytes within a swizzled row r, by r mod 8
+    uint32_t loff[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) loff[u] = ((uint32_t)((lane >> 2) ^ u) << 4) + ((uint32_t)(lane & 3) << 2);
+    const int tok0 = kTokPerConvWarp * cw;  // multiple of 8
     for (int k = 0; k < nck; ++k) {
-      const int st = k & 1;
+      const int st = k & 1, xb = k % kXBufs, lb = (k + 1) % kXBufs;
       const bool is_last = (k == last);
-      if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, 1, abort_flag, a.err)) break;
-      if (is_last && k >= 1 &&
-          !wg_wait(BAR(BAR_XFREE0 + (st ^ 1)), ((k - 1) >> 1) & 1, leader, 1, abort_flag, a.err))
+      if (!wg_wait(BAR(BAR_FULLX0 + xb), (k / kXBufs) & 1, leader, 1, abort_flag, a.err, 256)) break;
+      if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, 1, abort_flag, a.err, 256)) break;
+      if (k >= 1 && !wg_wait(BAR(BAR_XWFREE), (k - 1) & 1, leader, 1, abort_flag, a.err, 256)) break;
+      // the low part of w o X goes to X[(k+1) % 3], last used by chunk k-2
+      if (is_last && k >= 2 &&
+          !wg_wait(BAR(BAR_XFREE0 + lb), ((k - 2) / kXBufs) & 1, leader, 1, abort_flag, a.err, 256))
         break;
       const float *cs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
       const float *dtv = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
       const float cs_end = cs[QC - 1];
-      const float wl = __expf(cs_end - cs[32 * cw + lane]) * dtv[32 * cw + lane];
-      unsigned char *xt = smem + OFF_X + st * kXBuf;
-      unsigned char *xwt = smem + OFF_XW + st * kTile;
-      unsigned char *xlt = smem + OFF_XW + (st ^ 1) * kTile;
-      auto raw_row = [&](int r) -> uint32_t {
-        return *reinterpret_cast<const uint32_t *>(xt + swz(r, lane >> 2) + lane_byte);
-      };
-      // window: times t-3, t-2, t-1 for the warp's first token
-      uint32_t w0 = raw_row(32 * cw), w1 = raw_row(32 * cw + 1), w2 = raw_row(32 * cw + 2);
+      const float wl = lane < kTokPerConvWarp ? __expf(cs_end - cs[tok0 + lane]) * dtv[tok0 + lane] : 0.f;
+      unsigned char *xt = smem + OFF_X + xb * kXBuf + tok0 * 128;   // row tok0
+      unsigned char *xwt = smem + OFF_XW + tok0 * 128;
+      unsigned char *xlt = smem + OFF_X + lb * kXBuf + tok0 * 128;
+      // rows tok0 + r for r = 0..18 (tok0 is a multiple of 8, so row mod 8 = r mod 8)
+#define RAW(r) (*reinterpret_cast<const uint32_t *>(xt + (r) * 128 + loff[(r) & 7]))
+      uint32_t r0 = RAW(0), r1 = RAW(1), r2 = RAW(2);
       const int t0 = t_begin + k * QC;
       if (cw == 0 && t0 == 0) {  // history before the first token comes from the conv cache
         uint32_t hist[3] = {0u, 0u, 0u};
@@ -367,24 +389,32 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           if (a.csi && W + tau >= 0)
             hist[j] = *reinterpret_cast<const uint32_t *>(a.csi + ((long long)b * W + (W + tau)) * a.conv_dim + ch);
         }
-        w0 = hist[0];
-        w1 = hist[1];
-        w2 = hist[2];
+        r0 = hist[0];
+        r1 = hist[1];
+        r2 = hist[2];
       }
-      const uint32_t nb0 = raw_row(32 * cw + 32), nb1 = raw_row(32 * cw + 33), nb2 = raw_row(32 * cw + 34);
-      named_bar(1, 128);  // all boundary rows read before any row is overwritten
-      if (leader) TC_MARK(k, 0);
+      const uint32_t nb0 = RAW(16), nb1 = RAW(17), nb2 = RAW(18);
+      named_bar(1, 256);  // all boundary rows read before any row is overwritten
+      if (leader) {
+        TC_MARK(k, 0);
+        mbar_arrive(BAR(BAR_EMPTY0 + st));  // dt and prefix sums already read
+      }
+      float2 xm3 = unpack_bf16(r0), xm2 = unpack_bf16(r1), xm1 = unpack_bf16(r2);
 #pragma unroll 1
-      for (int g = 0; g < 8; ++g) {
+      for (int g = 0; g < 2; ++g) {
+        float2 xn[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = 4 * g + u, s_ = 32 * cw + i;
-          const int nxt = i + 3;  // window row for time t
+        for (int u = 0; u < 8; ++u) {
+          const int nxt = 8 * g + u + 3;  // row of time t for token 8g+u
           uint32_t w3;
-          if (nxt < 32) w3 = raw_row(32 * cw + nxt);
-          else w3 = nxt == 32 ? nb0 : (nxt == 33 ? nb1 : nb2);
-          const float2 xm3 = unpack_bf16(w0), xm2 = unpack_bf16(w1), xm1 = unpack_bf16(w2);
-          const float2 x0 = unpack_bf16(w3);
+          if (nxt < 16) w3 = RAW(nxt);
+          else w3 = nxt == 16 ? nb0 : (nxt == 17 ? nb1 : nb2);
+          xn[u] = unpack_bf16(w3);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = 8 * g + u;
+          const float2 x0 = xn[u];
           float u0, u1;
           if (W == 0) {
             u0 = x0.x;
@@ -394,7 +424,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             u1 = silu(bias1 + e1[0] * xm3.y + e1[1] * xm2.y + e1[2] * xm1.y + e1[3] * x0.y);
           }
           const float ws = __shfl_sync(0xffffffffu, wl, i);
-          const uint32_t off = swz(s_, lane >> 2) + lane_byte;
+          const uint32_t off = i * 128 + loff[u];
           *reinterpret_cast<uint32_t *>(xt + off) = pack_f16(u0, u1);
           const float v0 = u0 * ws, v1 = u1 * ws;
           const __half2 hi = __floats2half2_rn(v0, v1);
@@ -403,26 +433,26 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             const float2 hf = __half22float2(hi);
             *reinterpret_cast<uint32_t *>(xlt + off) = pack_f16(v0 - hf.x, v1 - hf.y);
           }
-          w0 = w1;
-          w1 = w2;
-          w2 = w3;
+          xm3 = xm2;
+          xm2 = xm1;
+          xm1 = x0;
         }
       }
+#undef RAW
       fence_proxy_async();
-      named_bar(1, 128);
+      named_bar(1, 256);
       if (leader) {
         TC_MARK(k, 1);
-        mbar_arrive(BAR(BAR_XREADY0 + st));
+        mbar_arrive(BAR(BAR_XREADY));
         if (is_last) mbar_arrive(BAR(BAR_XLOREADY));
-        mbar_arrive(BAR(BAR_EMPTY0 + st));
       }
     }
-  } else if (warp >= 8 && warp < 12) {
+  } else if (warp >= 12 && warp < 16) {
     // ---------------------------------------------------------------- S -> S~ (decay mask)
     if (!kStateOnly) {
-      const int mw = warp - 8;
+      const int mw = warp - 12;
       const int t = 32 * mw + lane;
-      const bool leader = (tid == 256);
+      const bool leader = (tid == 14 * 32);
       float *cf = reinterpret_cast<float *>(smem + OFF_CF);
       const float Dh = a.D[h];
       for (int k = 0; k < nck; ++k) {
@@ -430,13 +460,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, 2, abort_flag, a.err)) break;
         if (!wg_wait(BAR(BAR_SREADY0 + st), (k >> 1) & 1, leader, 2, abort_flag, a.err)) break;
         tc_fence_after();
-        const float *cs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
-        const float *dtv = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
-        {  // column factor of column t: e^{r_J - cs_t} dt_t with r_J = cs at the end of t's block
-          const float rJ = cs[32 * (t >> 5) + 31];
-          cf[t] = __expf(rJ - cs[t]) * dtv[t];
+        float *cs = reinterpret_cast<float *>(smem + OFF_CSM);
+        float *dtv = reinterpret_cast<float *>(smem + OFF_DTM);
+        {  // private copies (the stage is released at once); column factor of column t:
+           // e^{r_J - cs_t} dt_t with r_J = cs at the end of t's block
+          const float *scs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
+          const float *sdt = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
+          const float rJ = scs[32 * (t >> 5) + 31];
+          cs[t] = scs[t];
+          dtv[t] = sdt[t];
+          cf[t] = __expf(rJ - scs[t]) * sdt[t];
         }
         named_bar(2, 128);
+        if (leader) mbar_arrive(BAR(BAR_EMPTY0 + st));
         if (leader) TC_MARK(k, 2);
         const float cst = cs[t];
         const uint32_t trow = tmem + (st ? TM_S1 : TM_S0) + ((uint32_t)(32 * mw) << 16);
@@ -481,25 +517,34 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (leader) {
           TC_MARK(k, 3);
           mbar_arrive(BAR(BAR_STREADY0 + st));
-          mbar_arrive(BAR(BAR_EMPTY0 + st));
         }
       }
     }
-  } else if (warp >= 12) {
+  } else if (warp >= 16) {
     // ---------------------------------------------------------------- state update + output
-    const int ew = warp - 12;
+    const int ew = warp - 16;
     const int n = 32 * ew + lane;  // TMEM lane: state row n, output row t = n
-    const bool leader = (tid == 384);
+    const bool leader = (tid == 19 * 32);
     const uint32_t lane_off = (uint32_t)(32 * ew) << 16;
     const long long bh = (long long)b * a.H + h;
-    float hr[64];
-    {
+    {  // initial state -> TMEM (fp32) and the fp16 copy
       const float *hin = a.h_init ? a.h_init + seg * a.h_init_seg + bh * 8192 : nullptr;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        float hr[32];
+        uint32_t hu[32];
 #pragma unroll
-      for (int p = 0; p < 64; ++p) hr[p] = hin ? hin[p * 128 + n] : 0.f;
+        for (int i = 0; i < 32; ++i) {
+          hr[i] = hin ? hin[(32 * half + i) * 128 + n] : 0.f;
+          hu[i] = __float_as_uint(hr[i]);
+        }
+        tmem_st32(tmem + TM_H + 32 * half + lane_off, hu);
+        write_h_tile(smem, hr, n, half);
+      }
+      tmem_st_wait();
     }
-    write_h_tile(smem, hr, n);
     fence_proxy_async();
+    tc_fence_before();
     named_bar(3, 128);
     if (leader) mbar_arrive(BAR(BAR_HREADY));
     float decay_sum = 0.f;
@@ -513,19 +558,27 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const float ak = __expf(cs_end);
       if (!wg_wait(BAR(BAR_DHREADY), k & 1, leader, 3, abort_flag, a.err)) break;
       tc_fence_after();
-      if (leader) TC_MARK(k, 4);
-#pragma unroll
+      if (leader) {
+        TC_MARK(k, 4);
+        mbar_arrive(BAR(BAR_EMPTY0 + st));  // prefix sums already read by the group
+      }
+#pragma unroll 1
       for (int half = 0; half < 2; ++half) {
-        float v[32];
-        tmem_ld32(tmem + TM_DH + 32 * half + lane_off, v);
+        float dh[32], hr[32];
+        tmem_ld32(tmem + TM_DH + 32 * half + lane_off, dh);
+        tmem_ld32(tmem + TM_H + 32 * half + lane_off, hr);
         tmem_ld_wait();
+        uint32_t hu[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) hr[32 * half + i] = ak * hr[32 * half + i] + v[i];
+        for (int i = 0; i < 32; ++i) {
+          hr[i] = ak * hr[i] + dh[i];
+          hu[i] = __float_as_uint(hr[i]);
+        }
+        tmem_st32(tmem + TM_H + 32 * half + lane_off, hu);
+        if (k != last) write_h_tile(smem, hr, n, half);
       }
-      if (k != last) {
-        write_h_tile(smem, hr, n);
-        fence_proxy_async();
-      }
+      tmem_st_wait();
+      if (k != last) fence_proxy_async();
       tc_fence_before();
       named_bar(3, 128);
       if (leader) {
@@ -538,25 +591,25 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (leader) TC_MARK(k, 6);
         const int tok = t_begin + k * QC + n;
         const long long row = (long long)b * a.L + tok;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float yi[16], ysv[16];
-          tmem_ld16(tmem + TM_YI + 16 * q + lane_off, yi);
-          tmem_ld16(tmem + TM_YS + 16 * q + lane_off, ysv);
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          float yi[32], ysv[32];
+          tmem_ld32(tmem + TM_YI + 32 * half + lane_off, yi);
+          tmem_ld32(tmem + TM_YS + 32 * half + lane_off, ysv);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) yi[i] += et * ysv[i];
+          for (int i = 0; i < 32; ++i) yi[i] += et * ysv[i];
           if (tok < t_end) {
             if (a.yf) {
-              float4 *dst = reinterpret_cast<float4 *>(a.yf + row * a.d_inner + h * 64 + 16 * q);
+              float4 *dst = reinterpret_cast<float4 *>(a.yf + row * a.d_inner + h * 64 + 32 * half);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) dst[i] = make_float4(yi[4 * i], yi[4 * i + 1], yi[4 * i + 2], yi[4 * i + 3]);
+              for (int i = 0; i < 8; ++i) dst[i] = make_float4(yi[4 * i], yi[4 * i + 1], yi[4 * i + 2], yi[4 * i + 3]);
             } else {
-              uint4 *dst = reinterpret_cast<uint4 *>(a.y + row * a.ys + h * 64 + 16 * q);
-              dst[0] = make_uint4(pack_bf16(yi[0], yi[1]), pack_bf16(yi[2], yi[3]),
-                                  pack_bf16(yi[4], yi[5]), pack_bf16(yi[6], yi[7]));
-              dst[1] = make_uint4(pack_bf16(yi[8], yi[9]), pack_bf16(yi[10], yi[11]),
-                                  pack_bf16(yi[12], yi[13]), pack_bf16(yi[14], yi[15]));
+              uint4 *dst = reinterpret_cast<uint4 *>(a.y + row * a.ys + h * 64 + 32 * half);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(pack_bf16(yi[8 * i], yi[8 * i + 1]), pack_bf16(yi[8 * i + 2], yi[8 * i + 3]),
+                                    pack_bf16(yi[8 * i + 4], yi[8 * i + 5]), pack_bf16(yi[8 * i + 6], yi[8 * i + 7]));
             }
           }
         }
@@ -567,13 +620,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           mbar_arrive(BAR(BAR_YFREE));
         }
       }
-      if (leader) mbar_arrive(BAR(BAR_EMPTY0 + st));
     }
     if (*abort_flag == 0) {
       float *hout = a.h_out ? a.h_out + seg * a.h_out_seg + bh * 8192 : nullptr;
       if (hout) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          float hr[32];
+          tmem_ld32(tmem + TM_H + 32 * half + lane_off, hr);
+          tmem_ld_wait();
 #pragma unroll
-        for (int p = 0; p < 64; ++p) hout[p * 128 + n] = hr[p];
+          for (int i = 0; i < 32; ++i) hout[(32 * half + i) * 128 + n] = hr[i];
+        }
       }
       if (a.seg_decay && n == 0) a.seg_decay[(long long)seg * a.B * a.H + bh] = __expf(decay_sum);
     }
