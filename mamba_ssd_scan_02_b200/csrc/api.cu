@@ -348,8 +348,13 @@ ssd_status_t run_mixer(const ssd_mixer_config_t *m, const ssd_mixer_args_t *a, c
 
 }  // namespace
 
+// Tensor-core GEMM on sm_100 when the operands satisfy TMA's alignment rules, else CUDA cores.
 cudaError_t launch_gemm_bf16_tn(const void *A, long long lda, const void *Bm, long long ldb, void *C,
                                 long long ldc, int M, int N, int K, cudaStream_t s) {
+  const bool aligned = aligned16(A) && aligned16(Bm) && aligned16(C) && lda % 8 == 0 && ldb % 8 == 0 &&
+                       ldc % 8 == 0;
+  if (aligned && tc_scan_available())
+    return launch_gemm_tc_bf16_tn(A, lda, Bm, ldb, C, ldc, M, N, K, device_error_ptr(), s);
   return launch_gemm_simt_bf16_tn(A, lda, Bm, ldb, C, ldc, M, N, K, s);
 }
 

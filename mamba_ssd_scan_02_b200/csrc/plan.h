@@ -80,6 +80,8 @@ cudaError_t launch_decode(const DecodePlan &p, cudaStream_t s);
 // GEMM C[M,N] = A[M,K] . B[N,K]^T, bf16 in/out, fp32 accumulate
 cudaError_t launch_gemm_bf16_tn(const void *A, long long lda, const void *Bm, long long ldb, void *C,
                                 long long ldc, int M, int N, int K, cudaStream_t s);
+cudaError_t launch_gemm_tc_bf16_tn(const void *A, long long lda, const void *Bm, long long ldb, void *C,
+                                   long long ldc, int M, int N, int K, int *err, cudaStream_t s);
 cudaError_t launch_gemm_simt_bf16_tn(const void *A, long long lda, const void *Bm, long long ldb,
                                      void *C, long long ldc, int M, int N, int K, cudaStream_t s);
 
