@@ -166,6 +166,25 @@ ssd_status_t mamba2_mixer_forward(const ssd_mixer_config_t *cfg, const ssd_mixer
 /* Human-readable name of a status code (static storage). */
 const char *ssd_status_string(ssd_status_t status);
 
+/* Size of the fixed device scratch that ssd_prefill_noalloc uses (64 MiB per device). */
+#define SSD_NOALLOC_WORKSPACE_BYTES (64ull << 20)
+
+/* ssd_prefill for callers that must not allocate device memory themselves (their device memory
+ * belongs to a framework allocator or a fixed pool, or they cannot afford the device-wide
+ * synchronisation a cudaMalloc may cause).  Inputs and outputs are passed exactly as for
+ * ssd_prefill; args->workspace and args->workspace_bytes are ignored.  Scratch comes from one
+ * array of SSD_NOALLOC_WORKSPACE_BYTES that the library reserves on every device it is loaded
+ * on and keeps until the process exits; the call itself allocates and frees nothing.
+ *  - Returns SSD_ERR_WORKSPACE when ssd_workspace_size(cfg) exceeds that size: about 1,400
+ *    tokens of a 128-head, 8-group layer in one call, more for smaller layers.
+ *  - The first call on a device looks up the array's device address; make that first call
+ *    before starting any stream capture.
+ *  - All calls share the array: calls whose kernels may run at the same time (different
+ *    streams without ordering, several host threads) race and must be ordered by the caller.
+ *    Nothing needs clearing between calls.
+ * This entry point is a property of this library; the paper has no counterpart to it. */
+ssd_status_t ssd_prefill_noalloc(const ssd_config_t *cfg, const ssd_prefill_args_t *args, void *stream);
+
 /* Waits for `stream`, then returns and clears the status latched by kernels on this device
  * (SSD_OK, SSD_ERR_TIMEOUT or SSD_ERR_DEVICE_BOUNDS). */
 ssd_status_t ssd_get_device_error(void *stream);

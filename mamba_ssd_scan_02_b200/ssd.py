@@ -77,7 +77,8 @@ class TraceRecord(ctypes.Structure):
 
 EXPORTS = ("ssd_workspace_size", "ssd_prefill", "ssd_decode_step", "ssd_mixer_workspace_size",
            "mamba2_mixer_forward", "ssd_status_string", "ssd_get_device_error", "ssd_version",
-           "ssd_trace_enable", "ssd_trace_read")
+           "ssd_trace_enable", "ssd_trace_read", "ssd_prefill_noalloc")
+NOALLOC_WORKSPACE_BYTES = 64 << 20
 
 _lib = None
 
@@ -110,6 +111,8 @@ def load(path: str = LIB_PATH):
     lib.ssd_get_device_error.argtypes = [vp]
     lib.ssd_version.restype = c_int
     lib.ssd_version.argtypes = []
+    lib.ssd_prefill_noalloc.restype = c_int
+    lib.ssd_prefill_noalloc.argtypes = [ctypes.POINTER(SsdConfig), ctypes.POINTER(PrefillArgs), vp]
     lib.ssd_trace_enable.restype = c_int
     lib.ssd_trace_enable.argtypes = [c_int]
     lib.ssd_trace_read.restype = c_int
@@ -223,6 +226,37 @@ def prefill(cfg: dict, xBC, dt, A, D, dt_bias, conv_w=None, conv_b=None, z=None,
         h_final=_ptr(h_final), conv_state_out=_ptr(conv_state_out), workspace=_ptr(workspace),
         workspace_bytes=workspace.numel())
     _check(lib.ssd_prefill(ctypes.byref(c), ctypes.byref(a), _stream(stream)), "ssd_prefill")
+    return y, h_final, conv_state_out
+
+
+def prefill_noalloc(cfg: dict, xBC, dt, A, D, dt_bias, conv_w=None, conv_b=None, z=None, norm_w=None,
+                    h0=None, conv_state_in=None, *, y=None, h_final=None, conv_state_out=None,
+                    stream=None, kernel: int | None = None):
+    """ssd_prefill_noalloc: the same computation as prefill() with the library's fixed device
+    scratch instead of a caller workspace (for callers that must not allocate device memory).
+    Outputs that are not passed are allocated here by torch; the C call allocates nothing."""
+    import torch
+    lib = load()
+    Bn, L = xBC.shape[0], xBC.shape[1]
+    c = make_config(cfg, seqlen=L, kernel=kernel)
+    H, P, N, G, W = c.nheads, c.headdim, c.dstate, c.ngroups, c.conv_width
+    d_inner, conv_dim = H * P, H * P + 2 * G * N
+    dev = xBC.device
+    if y is None:
+        y = torch.empty((Bn, L, d_inner), dtype=io_dtype(cfg), device=dev)
+    if h_final is None:
+        h_final = torch.empty((Bn, H, P, N), dtype=torch.float32, device=dev)
+    if conv_state_out is None and W > 0:
+        conv_state_out = torch.empty((Bn, W, conv_dim), dtype=io_dtype(cfg), device=dev)
+    a = PrefillArgs(
+        xBC=_ptr(xBC), xBC_row_stride=_row_stride(xBC), dt=_ptr(dt), dt_row_stride=_row_stride(dt),
+        z=_ptr(z), z_row_stride=_row_stride(z) if z is not None else 0, A=_ptr(A), D=_ptr(D),
+        dt_bias=_ptr(dt_bias), conv_w=_ptr(conv_w), conv_b=_ptr(conv_b), norm_w=_ptr(norm_w),
+        h0=_ptr(h0), conv_state_in=_ptr(conv_state_in), y=_ptr(y), y_row_stride=_row_stride(y),
+        h_final=_ptr(h_final), conv_state_out=_ptr(conv_state_out), workspace=None,
+        workspace_bytes=0)
+    _check(lib.ssd_prefill_noalloc(ctypes.byref(c), ctypes.byref(a), _stream(stream)),
+           "ssd_prefill_noalloc")
     return y, h_final, conv_state_out
 
 
