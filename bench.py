@@ -10,8 +10,14 @@ events on the launching stream.  The same line carries:
   - "roofline": the dominant kernel's algorithmic GB/s against the measured HBM copy peak;
   - "e2e": the same metric with host (pinned) inputs copied in and outputs copied back
     inside the timed region;
+  - "clocks": nvidia-smi SM clocks and throttle reasons sampled during the timed region
+    (extended by one second of the same step when the region is shorter than that);
   - "decode": the 16384-step decode workload (B64 H128, fp32 state of 256 MiB), state-update
     GB/s with the steps replayed from CUDA graphs;
+  - "long_context": 131072 tokens in 4 segments of 32768 with state and conv-cache carry,
+    chunk 256, gated RMSNorm;
+  - "mixer": the whole mixer layer at the 12B width (d_model 5120, 160 heads, B8 L8192),
+    tensor-core roofline of its dominant GEMM;
   - "cpu_baseline": the fp64 oracle timed on a bounded sample of the prefill workload.
 Multi-GPU (torchrun): one process per GPU, each an independent replica (weak scaling), time
 = max over ranks.  --impl reference times the fp64 CPU oracle on the same metric.
@@ -19,11 +25,13 @@ Multi-GPU (torchrun): one process per GPU, each an independent replica (weak sca
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 import numpy as np
@@ -35,7 +43,12 @@ from mamba_ssd_scan_02_b200 import datagen  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "SSD prefill tokens/s/layer"
+HEADLINE_CONFIG = {"workload": "prefill_8k", "batch": 1, "seqlen": 8192, "nheads": 128,
+                   "headdim": 64, "dstate": 128, "ngroups": 8, "chunk": 128, "conv_width": 4,
+                   "state_dtype": "f32", "l2": "flushed between timed steps (256 MiB write)"}
 
 
 def peaks():
@@ -47,22 +60,53 @@ def peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel's sources are still
+    the ones that were captured (else None)."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)[f"{kernel}@{workload}"]
+    except (OSError, ValueError, KeyError):
+        return None
+    h = hashlib.sha256()
+    for rel in rec["sources"]:
+        try:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
+        except OSError:
+            return None
+    return rec["bytes_per_launch"] if h.hexdigest() == rec["sources_sha256"] else None
+
+
 # ---------------------------------------------------------------------------------------------
-# algorithmic byte counts (each required input once, each output once, state in/out once)
-def prefill_bytes(cfg) -> int:
+# algorithmic byte counts (each required input once, each output once, state in/out once,
+# parameters once)
+def scan_bytes(cfg, state_in=False) -> int:
+    """Tensors the scan itself must move: x, B, C, dt in, y out, final (and initial) state."""
     Bn, L, H, P, N, G = (cfg["batch"], cfg["seqlen"], cfg["nheads"], cfg["headdim"], cfg["dstate"],
                          cfg["ngroups"])
     e = 2 if cfg["dtype"] == "bf16" else 4
-    cd = datagen.conv_dim(cfg)
-    d_inner = H * P
-    b = Bn * L * (cd + H) * e          # xBC + dt
-    b += Bn * L * d_inner * e          # y
-    if cfg.get("norm_groups"):
-        b += Bn * L * d_inner * e      # z
-    b += Bn * H * P * N * 4            # final state out
-    b += cd * cfg["conv_width"] * e + 3 * H * 4  # parameters
-    b += Bn * cfg["conv_width"] * cd * e  # conv cache out
+    b = Bn * L * (H * P + 2 * G * N + H) * e + Bn * L * H * P * e
+    b += Bn * H * P * N * 4 * (2 if state_in else 1)
     return b
+
+
+def prefill_bytes(cfg, state_in=False) -> int:
+    """The whole prefill call: scan_bytes plus z (gated norm), conv cache, parameters."""
+    Bn, L, H, P = cfg["batch"], cfg["seqlen"], cfg["nheads"], cfg["headdim"]
+    e = 2 if cfg["dtype"] == "bf16" else 4
+    cd, W = datagen.conv_dim(cfg), cfg["conv_width"]
+    b = scan_bytes(cfg, state_in)
+    if cfg.get("norm_groups"):
+        b += Bn * L * H * P * e + H * P * e        # z, norm weight
+    b += cd * W * e + 3 * H * 4                    # conv weight, A, D, dt_bias
+    b += Bn * W * cd * e * (2 if state_in else 1)  # conv cache out (and in)
+    return b
+
+
+def gated_norm_bytes(cfg) -> int:
+    Bn, L, d = cfg["batch"], cfg["seqlen"], cfg["nheads"] * cfg["headdim"]
+    return 3 * Bn * L * d * 2 + d * 2              # y in, z in, out (bf16), weight
 
 
 def decode_bytes(cfg) -> int:
@@ -78,72 +122,178 @@ def decode_bytes(cfg) -> int:
     return b
 
 
+def mixer_flops(cfg) -> dict:
+    T = cfg["batch"] * cfg["seqlen"]
+    H, P, N, G, Q = cfg["nheads"], cfg["headdim"], cfg["dstate"], cfg["ngroups"], 128
+    d_inner, dm = H * P, cfg["d_model"]
+    proj = 2 * d_inner + 2 * G * N + H
+    ssd = T * (H * (2 * Q * P + 4 * N * P) + G * 2 * Q * N)
+    return {"in_proj": 2 * T * proj * dm, "out_proj": 2 * T * dm * d_inner, "ssd": ssd}
+
+
 # ---------------------------------------------------------------------------------------------
 class ClockSampler:
-    """nvidia-smi clock/throttle sampling during the timed region."""
+    """nvidia-smi clock/throttle sampling every 100 ms in a reader thread; each sample is
+    stamped with the host's monotonic clock when it arrives."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, index: int):
-        self.index = index
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
         self.proc = None
+        self.samples = []
+        self.lock = threading.Lock()
 
-    def __enter__(self):
+    def start(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.QUERY}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return self
+        threading.Thread(target=self._read, daemon=True).start()
+        t0 = time.monotonic()
+        while time.monotonic() - t0 < 10 and not self.samples and self.proc.poll() is None:
+            time.sleep(0.05)
         return self
 
-    def __exit__(self, *exc):
-        self.lines = []
-        if self.proc:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
-
-    def summary(self):
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+    def _read(self):
+        for ln in self.proc.stdout:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
             try:
-                sm.append(float(f[1]))
-                smax = float(f[2])
+                s = (time.monotonic(), float(f[1]), float(f[2]),
+                     {n for n, v in zip(self.NAMES, f[5:9]) if v.lower() == "active"})
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+            with self.lock:
+                self.samples.append(s)
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float, window: str):
+        with self.lock:
+            sel = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "window": window}
+        reasons = set().union(*(s[3] for s in sel))
+        return {"sm_mhz": statistics.median(s[1] for s in sel), "sm_max_mhz": sel[-1][2],
+                "reasons": sorted(reasons), "samples": len(sel), "window": window}
+
+
+def smi_gpu_id(torch, dev: int) -> str:
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except (AttributeError, RuntimeError):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        return vis.split(",")[dev] if vis else str(dev)
+
+
+class Ctx:
+    """What every workload needs: torch, the binding, the process group, the clock sampler."""
+
+    def __init__(self, args, torch, ssd, dist, rank, world, clk):
+        self.args, self.torch, self.ssd, self.dist = args, torch, ssd, dist
+        self.rank, self.world, self.clk = rank, world, clk
+        self.dev = torch.device("cuda")
+        self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=self.dev)
+
+    def max_over_ranks(self, v: float) -> float:
+        if not self.dist:
+            return v
+        t = self.torch.tensor([v], dtype=self.torch.float64, device=self.dev)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def timed(self, step, steps, flush=True, trace=True):
+        """Times `steps` calls of step() with CUDA events on the current stream (barrier and
+        synchronize on both sides), then keeps the GPU on the same step for one more second
+        when the timed region was shorter, so that the clock sampler sees it under load.
+        Returns (total ms, max over ranks), the traced kernel records, and the clocks."""
+        torch = self.torch
+        stream = torch.cuda.current_stream()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        if trace:
+            self.ssd.trace_enable(True)
+            self.ssd.trace_read()
+        if self.dist:
+            self.dist.barrier()
+        torch.cuda.synchronize()
+        t0 = time.monotonic()
+        for i in range(steps):
+            if flush:
+                self.flush.fill_(float(i))  # evict the previous step's data from L2
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        t1 = time.monotonic()
+        recs = []
+        if trace:
+            self.ssd.trace_enable(False)
+            recs = self.ssd.trace_read()
+        window = "timed region"
+        if t1 - t0 < 1.0:
+            while time.monotonic() - t1 < 1.0:
+                for _ in range(4):
+                    if flush:
+                        self.flush.fill_(0.0)
+                    step()
+                torch.cuda.synchronize()
+            window = "timed region + 1 s of the same step right after it"
+        t2 = time.monotonic()
+        if self.dist:
+            self.dist.barrier()
+        ms = self.max_over_ranks(float(sum(a.elapsed_time(b) for a, b in ev)))
+        return ms, recs, self.clk.summary(t0, t2, window)
+
+
+def kernel_table(recs):
+    per = {}
+    for name, ms in recs:
+        per.setdefault(name, []).append(ms)
+    total = sum(sum(v) for v in per.values()) or 1.0
+    table = {k: {"launches": len(v), "mean_ms": round(statistics.mean(v), 5),
+                 "share": round(sum(v) / total, 4)} for k, v in per.items()}
+    dom = max(per, key=lambda k: sum(per[k])) if per else None
+    return per, table, dom
+
+
+def hbm_roofline(kernel, ms, algo_bytes, workload):
+    pk, src = peaks()
+    ach = algo_bytes / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(ach / pk["hbm_gbs"], 4),
+            "traffic": recorded_traffic(kernel, workload), "kernel": kernel,
+            "kernel_ms": round(ms, 5), "algorithmic_bytes": algo_bytes,
+            "peak_source": f"{src} HBM copy (burst)"}
 
 
 # ---------------------------------------------------------------------------------------------
-def bench_prefill(args, rank, world, torch, ssd, dist):
+def bench_prefill(c: Ctx):
+    torch, ssd, args = c.torch, c.ssd, c.args
     cfg = datagen.config(1)
     inp = datagen.make_inputs(1)
-    dev = torch.device("cuda")
     d = {k: ssd.to_device(v) for k, v in inp.items() if isinstance(v, np.ndarray)}
     Bn, L, H, P, N = cfg["batch"], cfg["seqlen"], cfg["nheads"], cfg["headdim"], cfg["dstate"]
-    y = torch.empty((Bn, L, H * P), dtype=torch.bfloat16, device=dev)
-    hf = torch.empty((Bn, H, P, N), dtype=torch.float32, device=dev)
-    cso = torch.empty((Bn, 4, datagen.conv_dim(cfg)), dtype=torch.bfloat16, device=dev)
-    ws = ssd.alloc_workspace(ssd.workspace_size(cfg), dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream()
+    y = torch.empty((Bn, L, H * P), dtype=torch.bfloat16, device=c.dev)
+    hf = torch.empty((Bn, H, P, N), dtype=torch.float32, device=c.dev)
+    cso = torch.empty((Bn, 4, datagen.conv_dim(cfg)), dtype=torch.bfloat16, device=c.dev)
+    ws = ssd.alloc_workspace(ssd.workspace_size(cfg), c.dev)
 
     def step():
         ssd.prefill(cfg, d["xBC"], d["dt"], d["A"], d["D"], d["dt_bias"], d["conv_w"], None, None,
@@ -151,53 +301,18 @@ def bench_prefill(args, rank, world, torch, ssd, dist):
 
     for _ in range(args.warmup):
         step()
-    torch.cuda.synchronize()
-    ssd.trace_enable(True)
-    ssd.trace_read()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        for i in range(args.steps):
-            flush.fill_(float(i))            # evict the previous step's data from L2
-            starts[i].record(stream)
-            step()
-            ends[i].record(stream)
-        torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    ssd.trace_enable(False)
-    recs = ssd.trace_read()
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = float(sum(step_ms))
-    if dist:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    # dominant kernel: largest total traced time
-    per = {}
-    for name, ms in recs:
-        per.setdefault(name, []).append(ms)
-    dom = max(per, key=lambda k: sum(per[k]))
-    dom_ms = statistics.mean(per[dom])
-    pk, pk_src = peaks()
-    algo = prefill_bytes(cfg)
-    achieved = algo / (dom_ms * 1e-3) / 1e9
+    total_ms, recs, clocks = c.timed(step, args.steps)
+    per, table, dom = kernel_table(recs)
     tokens = Bn * L
     res = {
-        "value": world * tokens * args.steps / (total_ms * 1e-3),
+        "value": c.world * tokens * args.steps / (total_ms * 1e-3),
         "ms_per_step": total_ms / args.steps,
         "gpu_launches": len(recs),
-        "clocks": clk.summary(),
-        "kernels": {k: {"launches": len(v), "mean_ms": round(statistics.mean(v), 5),
-                        "share": round(sum(v) / sum(sum(x) for x in per.values()), 4)}
-                    for k, v in per.items()},
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
-                     "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
-                     "kernel": dom, "kernel_ms": round(dom_ms, 5), "algorithmic_bytes": algo,
-                     "peak_source": pk_src},
+        "clocks": clocks,
+        "kernels": table,
+        # ssd_scan_tc moves every tensor of scan_bytes (x, B|C, dt in; y, state out)
+        "roofline": hbm_roofline(dom, statistics.mean(per[dom]), scan_bytes(cfg), "prefill_8k"),
+        "path_bytes_per_step": prefill_bytes(cfg),
     }
     # end to end: pinned host inputs in, results out, inside the timed region
     hx = torch.empty(d["xBC"].shape, dtype=torch.bfloat16, pin_memory=True)
@@ -217,43 +332,32 @@ def bench_prefill(args, rank, world, torch, ssd, dist):
         hy.copy_(y, non_blocking=True)
         hh.copy_(hf, non_blocking=True)
 
-    for _ in range(2):
+    for _ in range(max(2, args.warmup)):
         e2e_step()
-    torch.cuda.synchronize()
-    e2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.fill_(float(i))
-        e2[i][0].record(stream)
-        e2e_step()
-        e2[i][1].record(stream)
-    torch.cuda.synchronize()
-    e_ms = sum(a.elapsed_time(b) for a, b in e2)
-    if dist:
-        t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
-    res["e2e"] = {"value": world * tokens * args.steps / (e_ms * 1e-3), "unit": "tokens/s",
+    e_ms, _, _ = c.timed(e2e_step, args.steps, trace=False)
+    res["e2e"] = {"value": c.world * tokens * args.steps / (e_ms * 1e-3), "unit": "tokens/s",
                   "h2d_bytes_per_step": hx.numel() * 2 + hdt.numel() * 2,
                   "d2h_bytes_per_step": hy.numel() * 2 + hh.numel() * 4}
     return res
 
 
-def bench_decode(args, rank, world, torch, ssd, dist, steps_total=16384, graph_steps=256):
+def bench_decode(c: Ctx, steps_total=16384, graph_steps=256):
+    torch, ssd = c.torch, c.ssd
     cfg = datagen.config(2)
-    Bn, H, P, N = cfg["batch"], cfg["nheads"], cfg["headdim"], cfg["dstate"]
-    dev = torch.device("cuda")
+    Bn, H, P = cfg["batch"], cfg["nheads"], cfg["headdim"]
     pcfg = dict(cfg, seqlen=cfg["prefill_len"], norm_groups=0)
     pin = datagen.make_inputs(2, pcfg)
     dp = {k: ssd.to_device(pin[k]) for k in ("A", "D", "dt_bias", "conv_w")}
     _, state, cache = ssd.prefill(pcfg, ssd.to_device(pin["xBC"]), ssd.to_device(pin["dt"]),
                                   dp["A"], dp["D"], dp["dt_bias"], dp["conv_w"])
     del pin
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()  # the 8192-token prefill at batch 64 used ~20 GB; give it back
     pool = {k: ssd.to_device(v) for k, v in datagen.decode_pool(cfg).items()}
     npool = pool["xBC"].shape[0]
-    norm_w = torch.ones(H * P, dtype=torch.bfloat16, device=dev)
+    norm_w = torch.ones(H * P, dtype=torch.bfloat16, device=c.dev)
     caches = [cache, torch.empty_like(cache)]
-    y = torch.empty((Bn, H * P), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((Bn, H * P), dtype=torch.bfloat16, device=c.dev)
 
     def run(n, offset=0):
         for s in range(n):
@@ -285,34 +389,105 @@ def bench_decode(args, rank, world, torch, ssd, dist, steps_total=16384, graph_s
         g.replay()
     torch.cuda.synchronize()
     reps = max(1, steps_total // graph_steps)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    a.record()
-    for _ in range(reps):
-        g.replay()
-    b.record()
-    torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+
+    def replay_all():
+        for _ in range(reps):
+            g.replay()
+
+    # the 256 MiB state stream exceeds L2 by itself: no flush needed
+    ms, _, clocks = c.timed(replay_all, 1, flush=False, trace=False)
     del g
     nsteps = reps * graph_steps
     per_step_ms = ms / nsteps
     algo = decode_bytes(cfg)
-    pk, pk_src = peaks()
-    gbs = world * algo / (per_step_ms * 1e-3) / 1e9
-    kach = algo / (kms * 1e-3) / 1e9
+    gbs = c.world * algo / (per_step_ms * 1e-3) / 1e9
     return {"metric": "decode state-update GB/s", "value": round(gbs, 1), "unit": "GB/s",
-            "steps": nsteps, "ms_per_step": round(per_step_ms, 5),
-            "tokens_per_s": round(world * Bn / (per_step_ms * 1e-3), 1),
-            "algorithmic_bytes_per_step": algo, "graph_steps": graph_steps,
-            "roofline": {"bound": "hbm", "achieved": round(kach, 1), "peak": pk["hbm_gbs"],
-                         "unit": "GB/s", "frac": round(kach / pk["hbm_gbs"], 4), "traffic": None,
-                         "kernel": "ssd_decode", "kernel_ms": round(kms, 5), "peak_source": pk_src}}
+            "workload": "decode_16k", "steps": nsteps, "ms_per_step": round(per_step_ms, 5),
+            "tokens_per_s": round(c.world * Bn / (per_step_ms * 1e-3), 1),
+            "algorithmic_bytes_per_step": algo, "graph_steps": graph_steps, "clocks": clocks,
+            "roofline": hbm_roofline("ssd_decode", kms, algo, "decode_16k")}
+
+
+def bench_long_context(c: Ctx):
+    """131072 tokens as 4 prefill calls of 32768 tokens; each call's final state and conv
+    cache are the next call's initial state and cache (chunk 256, gated RMSNorm)."""
+    torch, ssd, args = c.torch, c.ssd, c.args
+    cfg = datagen.config(3)
+    inp = datagen.make_inputs(3)
+    d = {k: ssd.to_device(v) for k, v in inp.items() if isinstance(v, np.ndarray)}
+    del inp
+    Bn, L, H, P, N = cfg["batch"], cfg["seqlen"], cfg["nheads"], cfg["headdim"], cfg["dstate"]
+    nseg = cfg["segments"]
+    Ls = L // nseg
+    scfg = dict(cfg, seqlen=Ls)
+    cd = datagen.conv_dim(cfg)
+    y = torch.empty((Bn, L, H * P), dtype=torch.bfloat16, device=c.dev)
+    states = [torch.empty((Bn, H, P, N), dtype=torch.float32, device=c.dev) for _ in range(2)]
+    caches = [torch.empty((Bn, 4, cd), dtype=torch.bfloat16, device=c.dev) for _ in range(2)]
+    ws = ssd.alloc_workspace(ssd.workspace_size(scfg), c.dev)
+
+    def step():
+        for s in range(nseg):
+            sl = slice(s * Ls, (s + 1) * Ls)
+            ssd.prefill(scfg, d["xBC"][:, sl], d["dt"][:, sl], d["A"], d["D"], d["dt_bias"],
+                        d["conv_w"], None, d["z"][:, sl], d["norm_w"],
+                        states[(s + 1) % 2] if s else None, caches[(s + 1) % 2] if s else None,
+                        y=y[:, sl], h_final=states[s % 2], conv_state_out=caches[s % 2],
+                        workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    # the 2.7 GB of xBC per step exceed L2 many times over: no flush needed
+    total_ms, recs, clocks = c.timed(step, args.steps, flush=False)
+    per, table, dom = kernel_table(recs)
+    algo = scan_bytes(scfg, state_in=True) if dom.startswith("ssd_scan") else gated_norm_bytes(scfg)
+    return {"metric": METRIC, "workload": "long_context_128k",
+            "value": round(c.world * Bn * L * args.steps / (total_ms * 1e-3), 1),
+            "unit": "tokens/s", "ms_per_step": round(total_ms / args.steps, 4),
+            "segments": nseg, "segment_len": Ls, "chunk": cfg["chunk"],
+            "path_bytes_per_step": nseg * prefill_bytes(scfg, state_in=True),
+            "gpu_launches": len(recs), "kernels": table, "clocks": clocks,
+            "l2": "not flushed (inputs 2.7 GB per step)",
+            "roofline": hbm_roofline(dom, statistics.mean(per[dom]), algo, "long_context_128k")}
+
+
+def bench_mixer(c: Ctx):
+    """mamba2_mixer_forward at the 12B width: B8 L8192 d_model 5120, 160 heads."""
+    torch, ssd, args = c.torch, c.ssd, c.args
+    cfg = dict(datagen.config(4), batch=args.mixer_batch)
+    inp = datagen.make_inputs(4, cfg)
+    d = {k: ssd.to_device(v) for k, v in inp.items() if isinstance(v, np.ndarray)}
+    del inp
+    Bn, L = cfg["batch"], cfg["seqlen"]
+    out = torch.empty((Bn, L, cfg["d_model"]), dtype=torch.bfloat16, device=c.dev)
+    ws = ssd.alloc_workspace(ssd.mixer_workspace_size(cfg), c.dev)
+
+    def step():
+        ssd.mixer_forward(cfg, d["hidden"], d["rms_w"], d["W_in"], d["W_out"], d["A"], d["D"],
+                          d["dt_bias"], d["conv_w"], None, d["norm_w"], out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    total_ms, recs, clocks = c.timed(step, args.steps, flush=False)
+    per, table, dom = kernel_table(recs)
+    fl = mixer_flops(cfg)
+    pk, src = peaks()
+    gemm_ms = statistics.mean(per["gemm_in_proj"])
+    ach = fl["in_proj"] / (gemm_ms * 1e-3) / 1e12
+    step_ms = total_ms / args.steps
+    return {"metric": "mixer layer tokens/s", "workload": "mixer_12b", "batch": Bn,
+            "value": round(c.world * Bn * L * args.steps / (total_ms * 1e-3), 1),
+            "unit": "tokens/s", "ms_per_step": round(step_ms, 4),
+            "layer_tflops": round(sum(fl.values()) / (step_ms * 1e-3) / 1e12, 1),
+            "flops_per_step": fl, "gpu_launches": len(recs), "kernels": table, "clocks": clocks,
+            "l2": "not flushed (hidden 671 MB per step)",
+            "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(ach / pk["bf16_tflops"], 4),
+                         "traffic": recorded_traffic("gemm_tc_kernel", "mixer_12b_in_proj"),
+                         "kernel": "gemm_in_proj (gemm_tc_kernel)", "kernel_ms": round(gemm_ms, 4),
+                         "algorithmic_flops": fl["in_proj"],
+                         "peak_source": f"{src} cuBLAS bf16 (burst)"},
+            "dominant_kernel": dom}
 
 
 def cpu_baseline(target_s: float = 10.0):
@@ -371,12 +546,11 @@ def reference_arm(args):
     val = tok * frac * args.steps / el
     sample = f"per step: first {tok} tokens x heads 0-15 (1/8 of the layer) of prefill_8k, fp64"
     print(json.dumps({
-        "impl": "reference", "metric": "SSD prefill tokens/s/layer", "value": round(val, 2),
+        "impl": "reference", "metric": METRIC, "value": round(val, 2),
         "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "prefill_8k", "batch": 1, "seqlen": 8192, "nheads": 128,
-                   "headdim": 64, "dstate": 128, "ngroups": 8, "chunk": 128},
+        "config": dict(HEADLINE_CONFIG, parallelism=f"replicas x{args.gpus}"),
         "cpu_baseline": {"value": round(val, 2), "unit": "tokens/s", "cores": cores,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(val, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -389,7 +563,12 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--quick", action="store_true", help="skip the decode and CPU-baseline legs")
+    ap.add_argument("--quick", action="store_true",
+                    help="headline prefill only (no decode, long-context, mixer or CPU legs)")
+    ap.add_argument("--workload", choices=["all", "prefill", "decode", "long_context", "mixer"],
+                    default="all", help="run one workload alone (for profiling); prints its object")
+    ap.add_argument("--mixer-batch", type=int, default=8,
+                    help="batch of the mixer workload (smaller only for profiling captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -410,27 +589,50 @@ def main():
         import torch.distributed as tdist
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = tdist
-    res = bench_prefill(args, rank, world, torch, ssd, dist)
-    dec = None if args.quick else bench_decode(args, rank, world, torch, ssd, dist)
-    status = ssd.get_device_error()
+    clk = ClockSampler(smi_gpu_id(torch, local_rank)).start()
+    c = Ctx(args, torch, ssd, dist, rank, world, clk)
+    if args.workload != "all":
+        fn = {"prefill": bench_prefill, "decode": bench_decode, "long_context": bench_long_context,
+              "mixer": bench_mixer}[args.workload]
+        try:
+            r = fn(c)
+            r["device_status"] = ssd.get_device_error()
+        finally:
+            clk.stop()
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"workload": args.workload, "result": r}))
+        return
+    try:
+        res = bench_prefill(c)
+        dec = lng = mix = None
+        if not args.quick:
+            dec = bench_decode(c)
+            torch.cuda.empty_cache()
+            lng = bench_long_context(c)
+            torch.cuda.empty_cache()
+            mix = bench_mixer(c)
+        status = ssd.get_device_error()
+    finally:
+        clk.stop()
     if dist:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return
-    cpu = None if args.quick else cpu_baseline()
+    cpu = None if (args.quick or world > 1) else cpu_baseline()
     line = {
-        "metric": "SSD prefill tokens/s/layer", "value": round(res["value"], 1), "unit": "tokens/s",
+        "metric": METRIC, "value": round(res["value"], 1), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(res["ms_per_step"], 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "prefill_8k", "batch": 1, "seqlen": 8192, "nheads": 128,
-                   "headdim": 64, "dstate": 128, "ngroups": 8, "chunk": 128, "conv_width": 4,
-                   "state_dtype": "f32", "l2": "flushed between timed steps (256 MiB write)",
-                   "parallelism": f"replicas x{world}"},
+        "config": dict(HEADLINE_CONFIG, parallelism=f"replicas x{world}"),
         "roofline": res["roofline"], "e2e": res["e2e"], "gpu_launches": res["gpu_launches"],
-        "clocks": res["clocks"], "kernels": res["kernels"], "decode": dec, "cpu_baseline": cpu,
-        "device_status": status,
+        "clocks": res["clocks"], "kernels": res["kernels"],
+        "path_bytes_per_step": res["path_bytes_per_step"], "decode": dec, "long_context": lng,
+        "mixer": mix, "cpu_baseline": cpu, "device_status": status,
     }
     print(json.dumps(line))
 
