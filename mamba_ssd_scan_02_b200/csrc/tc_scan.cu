@@ -21,12 +21,13 @@
 //
 // Warp roles (640 threads): warp 0 issues TMA loads (B and C tiles of the group, the head's
 // raw x rows with a 3-token halo, per-chunk dt and prefix sums), warp 1 allocates TMEM and
-// issues the MMAs, warps 4-11 compute the head's x channels (causal conv1d + SiLU) in place
-// into the double-buffered X tile and into w o X, warps 12-15 turn S into S~, warps 16-19
-// update the state (kept in fp32 in TMEM) and write y.  Per chunk the MMAs are issued as MMA4(k), MMA3(k), MMA1(k+1), MMA2(k), so the
-// mask of chunk k overlaps four MMAs and the state update overlaps two.  Hand-offs use
-// mbarriers (TMA transaction counts, tcgen05.commit, thread arrivals); every wait is bounded
-// and a timeout aborts the CTA cleanly and latches SSD_ERR_TIMEOUT.
+// issues each MMA group as soon as its inputs are ready, warps 2-4, 6-8, 10-11 compute the x
+// channels (causal conv1d + SiLU) in place into X and into w o X, warps 12-15 turn S into S~,
+// warps 16-19 update the state (kept in fp32 in TMEM), refresh its fp16 copy and write y.
+// X, w o X, S (with Yi in its upper half), Ys and the B/C stages are double-buffered, so each
+// role can run a chunk ahead of the next.  Hand-offs use mbarriers (TMA transaction counts,
+// tcgen05.commit, thread arrivals); every wait is bounded and a timeout aborts the CTA
+// cleanly and latches SSD_ERR_TIMEOUT.
 //
 // Operands are fp16 (the conv outputs B, C, x are O(10) in the workloads, far inside the fp16
 // range; 11 significant bits keep the chunked products within the bf16-input tolerance).
@@ -34,6 +35,8 @@
 // 64 channels x 128 tokens (K-major for MMA1/MMA3, M-major for MMA4); X, w o X and the fp16
 // state copy are 128-byte rows (N-major B operands).
 #include <cudaTypedefs.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "plan.h"
@@ -64,7 +67,7 @@ using namespace tc;
 
 constexpr int QC = 128;              // tokens per chunk
 constexpr int kThreadsTC = 640;       // 20 warps
-constexpr int kConvWarps = 8;          // warps 4..11
+constexpr int kConvWarps = 8;          // see conv_index()
 constexpr int kTokPerConvWarp = QC / kConvWarps;  // 16
 constexpr uint32_t kTile = 16384;    // one 128-row x 128-byte operand box
 // per-stage layout (bytes)
@@ -73,23 +76,39 @@ constexpr uint32_t OFF_B = 2 * kTile;         // B tile
 constexpr uint32_t OFF_DT = 4 * kTile;        // dt[128] fp32
 constexpr uint32_t OFF_CS = OFF_DT + 512;     // cs[128] fp32
 constexpr uint32_t kStage = 4 * kTile + 1024;  // 66560 = 65 * 1024
-// CTA layout.  X[b] (three buffers, chunk k uses b = k % 3) first receives by TMA the chunk's
+// CTA layout.  X[b] (two buffers, chunk k uses b = k % 2) first receives by TMA the chunk's
 // raw bf16 x rows for times t0-3 .. t0+127 (131 rows of this head's 64 channels); the conv
-// overwrites row s with X row s.  w o X has a single buffer (MMA4 reads it right away).
-constexpr int kXBufs = 3;
+// overwrites row s with X row s.  w o X is double-buffered the same way.
+constexpr int kXBufs = 2;
 constexpr uint32_t kXBuf = 17 * 1024;           // 131 rows of 128 bytes, padded
 constexpr uint32_t kRawRows = QC + 3;
-constexpr uint32_t OFF_X = 2 * kStage;              // X[3]  [s][p] fp16 (raw x rows first)
-constexpr uint32_t OFF_XW = OFF_X + kXBufs * kXBuf;  // w o X [s][p] fp16, 16 KB
-constexpr uint32_t OFF_H = OFF_XW + kTile;          // h copy [n][p] fp16, 16 KB
+constexpr uint32_t OFF_X = 2 * kStage;              // X[2]  [s][p] fp16 (raw x rows first)
+constexpr uint32_t OFF_XW = OFF_X + kXBufs * kXBuf;  // w o X [2][s][p] fp16, 16 KB each
+constexpr uint32_t OFF_H = OFF_XW + 2 * kTile;      // h copy [n][p] fp16, 16 KB
 constexpr uint32_t OFF_CF = OFF_H + kTile;          // column factors, 128 fp32
 constexpr uint32_t OFF_CSM = OFF_CF + 512;          // the mask's copies of cs and dt
 constexpr uint32_t OFF_DTM = OFF_CSM + 512;
 constexpr uint32_t OFF_BAR = OFF_DTM + 512;
+// Barriers.  Every event that can recur before its consumer has observed the previous
+// occurrence has one barrier per buffer, so that a parity test never sees two phases at once.
 enum {
-  BAR_FULL0, BAR_FULL1, BAR_EMPTY0, BAR_EMPTY1, BAR_FULLX0, BAR_FULLX1, BAR_FULLX2, BAR_XFREE0,
-  BAR_XFREE1, BAR_XFREE2, BAR_SREADY0, BAR_SREADY1, BAR_STREADY0, BAR_STREADY1, BAR_XREADY,
-  BAR_XWFREE, BAR_DHREADY, BAR_HREADY, BAR_YREADY, BAR_YFREE, BAR_XLOREADY, BAR_DONE, kNumBars
+  BAR_FULL0, BAR_FULL1,        // stage k % 2 loaded (TMA)
+  BAR_EMPTY0, BAR_EMPTY1,      // stage k % 2 released (conv, mask, state warps + MMA commit)
+  BAR_FULLX0, BAR_FULLX1,      // raw x of chunk k in X[k % 2] (TMA)
+  BAR_XFREE0, BAR_XFREE1,      // X[k % 2] read by MMA2 of chunk k
+  BAR_SREADY0, BAR_SREADY1,    // S of chunk k in TMEM (MMA1)
+  BAR_STREADY0, BAR_STREADY1,  // S~ of chunk k in TMEM (mask warps)
+  BAR_XREADY0, BAR_XREADY1,    // X and w o X of chunk k written (conv warps)
+  BAR_XWFREE0, BAR_XWFREE1,    // w o X[k % 2] read by MMA4 of chunk k
+  BAR_DHREADY,                 // dH of chunk k in TMEM (MMA4)
+  BAR_DHFREE,                  // dH of chunk k read by the state warps
+  BAR_HTFREE,                  // h tile (h_{k-1}) read by MMA3 of chunk k
+  BAR_HREADY,                  // h tile holds h_k (state warps)
+  BAR_YREADY0, BAR_YREADY1,    // Yi and Ys of chunk k in TMEM (MMA2 commit)
+  BAR_YFREE0, BAR_YFREE1,      // Yi and Ys of chunk k read by the output warps
+  BAR_XLOREADY,                // low part of w o X of the last chunk written
+  BAR_DONE,
+  kNumBars
 };
 constexpr uint32_t OFF_MISC = OFF_BAR + 8 * 32;   // [0] TMEM base, [1] abort flag
 constexpr uint32_t kSmemUsed = OFF_MISC + 16;
@@ -100,10 +119,12 @@ static_assert(OFF_X % 1024 == 0 && kXBuf % 1024 == 0 && OFF_XW % 1024 == 0 && OF
               "swizzle alignment");
 static_assert(kRawRows * 128 <= kXBuf, "raw x tile fits its buffer");
 
-// TMEM columns (fp32 accumulators, 128 lanes).  After the mask, S[b] holds S~ as packed fp16
-// in its first 64 columns.
-constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_YI = 256, TM_YS = 320, TM_DH = 384, TM_H = 448,
+// TMEM columns (fp32 accumulators, 128 lanes).  S[b] (chunk k uses b = k % 2) first holds S;
+// the mask rewrites it as packed fp16 S~ in columns 0-63, and MMA2 then accumulates Yi into
+// columns 64-127 (whose S values the mask has read).  Ys is double-buffered likewise.
+constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_YS0 = 256, TM_YS1 = 320, TM_DH = 384, TM_H = 448,
                    TM_COLS = 512;  // TM_H: the fp32 state h^T (row n, column p)
+constexpr uint32_t TM_YI_OFF = 64;  // Yi within S[b]
 
 constexpr uint32_t IDESC_S = idesc_f16(128, 128, false, false, kFmtF16);  // C K-major, B K-major
 constexpr uint32_t IDESC_YS = idesc_f16(128, 64, false, true, kFmtF16);   // C K-major, h N-major
@@ -151,33 +172,57 @@ __device__ __forceinline__ bool wg_wait(uint32_t bar, uint32_t parity, bool lead
 }
 
 // ---- MMA issue (single thread) ---------------------------------------------------------
+// The issuing thread shares its SM sub-partition with busy warps, so each group costs it as
+// few instructions as possible: fully unrolled, with the shared-memory descriptors built once
+// and advanced by adding to their start-address field (bits 0-13, in 16-byte units; every
+// operand lies below 256 KB, so the add never carries out of the low word).
+__device__ __forceinline__ uint64_t desc_adv(uint64_t d, uint32_t bytes) {
+  const uint32_t lo = static_cast<uint32_t>(d) + (bytes >> 4);
+  return (d & 0xFFFFFFFF00000000ull) | lo;
+}
+// K step j of a K-major 128-row operand stored as two 64-column boxes: 32 bytes per step
+// within a box, the second box after four steps.
+__device__ __forceinline__ constexpr uint32_t kmajor_step(int j) { return (j >> 2) * kTile + (j & 3) * 32; }
+
 __device__ __forceinline__ void issue_S(uint32_t stage, uint32_t tS) {
-#pragma unroll 1
-  for (int j = 0; j < 8; ++j) {
-    const uint32_t koff = (j >> 2) * kTile + (j & 3) * 32;
-    mma_f16_ss(tS, smem_desc_sw128(stage + OFF_C + koff, 16, 1024),
-               smem_desc_sw128(stage + OFF_B + koff, 16, 1024), IDESC_S, j > 0);
-  }
+  const uint64_t a0 = smem_desc_sw128(stage + OFF_C, 16, 1024), b0 = smem_desc_sw128(stage + OFF_B, 16, 1024);
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    mma_f16_ss(tS, desc_adv(a0, kmajor_step(j)), desc_adv(b0, kmajor_step(j)), IDESC_S, j > 0);
 }
 __device__ __forceinline__ void issue_Ys(uint32_t stage, uint32_t hbase, uint32_t tYs) {
-#pragma unroll 1
-  for (int j = 0; j < 8; ++j) {
-    const uint32_t koff = (j >> 2) * kTile + (j & 3) * 32;
-    mma_f16_ss(tYs, smem_desc_sw128(stage + OFF_C + koff, 16, 1024),
-               smem_desc_sw128(hbase + j * 2048, 8192, 1024), IDESC_YS, j > 0);
-  }
+  const uint64_t a0 = smem_desc_sw128(stage + OFF_C, 16, 1024), b0 = smem_desc_sw128(hbase, 8192, 1024);
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    mma_f16_ss(tYs, desc_adv(a0, kmajor_step(j)), desc_adv(b0, j * 2048), IDESC_YS, j > 0);
 }
 // S~ in TMEM: 16 fp16 of K per MMA = 8 columns
 __device__ __forceinline__ void issue_Yi(uint32_t tSt, uint32_t xbase, uint32_t tYi) {
-#pragma unroll 1
-  for (int j = 0; j < 8; ++j)
-    mma_f16_ts(tYi, tSt + 8 * j, smem_desc_sw128(xbase + j * 2048, 8192, 1024), IDESC_YI, j > 0);
+  const uint64_t b0 = smem_desc_sw128(xbase, 8192, 1024);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) mma_f16_ts(tYi, tSt + 8 * j, desc_adv(b0, j * 2048), IDESC_YI, j > 0);
 }
 __device__ __forceinline__ void issue_dH(uint32_t stage, uint32_t xwbase, uint32_t tDH, bool acc) {
-#pragma unroll 1
+  const uint64_t a0 = smem_desc_sw128(stage + OFF_B, kTile, 1024), b0 = smem_desc_sw128(xwbase, 8192, 1024);
+#pragma unroll
   for (int j = 0; j < 8; ++j)
-    mma_f16_ss(tDH, smem_desc_sw128(stage + OFF_B + j * 2048, kTile, 1024),
-               smem_desc_sw128(xwbase + j * 2048, 8192, 1024), IDESC_DH, (j > 0 || acc) ? 1u : 0u);
+    mma_f16_ss(tDH, desc_adv(a0, j * 2048), desc_adv(b0, j * 2048), IDESC_DH, (j > 0 || acc) ? 1u : 0u);
+}
+
+// Conv warps: 2, 3, 4, 6, 7, 8, 10, 11 -- none on the sub-partition of warp 1 (warps 1, 5, 9,
+// ...), whose single MMA-issuing thread would otherwise be starved of issue slots.
+__device__ __forceinline__ int conv_index(int warp) {
+  switch (warp) {
+    case 2: return 0;
+    case 3: return 1;
+    case 4: return 2;
+    case 6: return 3;
+    case 7: return 4;
+    case 8: return 5;
+    case 10: return 6;
+    case 11: return 7;
+    default: return -1;
+  }
 }
 
 // Row r (128 bytes) of a 128-byte-swizzled tile: 16-byte chunk c sits at chunk c ^ (r & 7).
@@ -217,7 +262,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   if (tid == 0) {
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t cnt = 1;
-      if (i == BAR_EMPTY0 || i == BAR_EMPTY1) cnt = kStateOnly ? 3 : 4;
+      if (i == BAR_EMPTY0 || i == BAR_EMPTY1) cnt = kStateOnly ? 3 : 4;  // + mask warps
       mbar_init(BAR(i), cnt);
     }
     *abort_flag = 0;
@@ -239,14 +284,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    // Raw x rows of chunk k go to X[k % 3] once MMA2 of chunk k-3 has released it; the B/C
+    // Raw x rows of chunk k go to X[k % 2] once MMA2 of chunk k-2 has released it; the B/C
     // tiles, dt and prefix sums go to stage k % 2 once chunk k-2's consumers released it.
     if (lane == 0) {
       int k = 0, nx = 0, nbc = 0;
       for (; k < nck; ++k) {
-        const int xb = k % kXBufs, st = k & 1;
+        const int xb = k & 1, st = k & 1;
         const int t0 = t_begin + k * QC;
-        if (k >= kXBufs && !mbar_wait(BAR(BAR_XFREE0 + xb), (k / kXBufs - 1) & 1, abort_flag, a.err)) break;
+        if (k >= 2 && !mbar_wait(BAR(BAR_XFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err)) break;
         mbar_arrive_expect_tx(BAR(BAR_FULLX0 + xb), kRawRows * 128);
         tma_load_3d(sb + OFF_X + xb * kXBuf, &tm_x, h * 64, t0 - 3, b, BAR(BAR_FULLX0 + xb));
         ++nx;
@@ -269,64 +314,94 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       // every load issued must land before the CTA may exit
       int never_abort = 0;
-      for (int j = (nx >= kXBufs ? nx - kXBufs : 0); j < nx; ++j)
-        mbar_wait(BAR(BAR_FULLX0 + j % kXBufs), (j / kXBufs) & 1, &never_abort, a.err);
+      for (int j = (nx >= 2 ? nx - 2 : 0); j < nx; ++j)
+        mbar_wait(BAR(BAR_FULLX0 + (j & 1)), (j >> 1) & 1, &never_abort, a.err);
       for (int j = (nbc >= 2 ? nbc - 2 : 0); j < nbc; ++j)
         mbar_wait(BAR(BAR_FULL0 + (j & 1)), (j >> 1) & 1, &never_abort, a.err);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
+    // Issues each chunk's four MMA groups as soon as their inputs are ready, whatever the
+    // order, so that no group waits behind another one that is still blocked:
+    //   MMA1 S(j)   stage j loaded; S[j % 2] free (MMA2 of chunk j-2 issued, its output read)
+    //   MMA4 dH(j)  X(j) and w o X(j) written; dH of chunk j-1 read by the state warps
+    //   MMA3 Ys(j)  after MMA1(j); h_{j-1} in the h tile
+    //   MMA2 Yi(j)  after MMA3(j) and MMA4(j); S~(j) written by the mask warps
+    // A commit after each group signals its consumers; stage j is released by a commit after
+    // the last of MMA1/MMA3/MMA4 of chunk j.  Polling sleeps briefly when nothing is ready and
+    // gives up (abort + SSD_ERR_TIMEOUT) after ~2 s without progress.
     if (lane == 0) {
-      const uint32_t tYi = tmem + TM_YI, tYs = tmem + TM_YS, tDH = tmem + TM_DH;
+      int nS = kStateOnly ? nck : 0, nD = 0, nYs = kStateOnly ? nck : 0, nYi = kStateOnly ? nck : 0;
+      auto stage_done = [&](int j) {  // all readers of stage j issued?
+        return nD > j && (kStateOnly || (nS > j && nYs > j));
+      };
+      uint64_t t_prog = globaltimer();
       bool ok = true;
-      if (nck > 0 && !kStateOnly) {
-        ok = mbar_wait(BAR(BAR_FULL0), 0, abort_flag, a.err);
-        if (ok) {
+      while (ok && (nD < nck || nYi < nck)) {
+        bool prog = false;
+        if (nYi < nck && nYi < nYs && nYi < nD && mbar_test(BAR(BAR_STREADY0 + (nYi & 1)), (nYi >> 1) & 1)) {
+          const int j = nYi;
           tc_fence_after();
-          issue_S(sb, tmem + TM_S0);
-          mma_commit(BAR(BAR_SREADY0));
+          TC_MARK(j, 11);
+          const uint32_t tS = tmem + ((j & 1) ? TM_S1 : TM_S0);
+          issue_Yi(tS, sb + OFF_X + (j & 1) * kXBuf, tS + TM_YI_OFF);
+          mma_commit(BAR(BAR_YREADY0 + (j & 1)));
+          mma_commit(BAR(BAR_XFREE0 + (j & 1)));
+          ++nYi;
+          prog = true;
         }
-      }
-      for (int k = 0; ok && k < nck; ++k) {
-        const int st = k & 1, xb = k % kXBufs;
-        const uint32_t sst = sb + st * kStage;
-        // h_{k-1} in shared memory and dH free
-        if (!(ok = mbar_wait(BAR(BAR_HREADY), k & 1, abort_flag, a.err))) break;
-        if (kStateOnly && !(ok = mbar_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, abort_flag, a.err))) break;
-        if (!(ok = mbar_wait(BAR(BAR_XREADY), k & 1, abort_flag, a.err))) break;
-        tc_fence_after();
-        TC_MARK(k, 8);
-        issue_dH(sst, sb + OFF_XW, tDH, false);
-        mma_commit(BAR(BAR_XWFREE));
-        if (!kStateOnly) {
-          if (k > 0 && !(ok = mbar_wait(BAR(BAR_YFREE), (k - 1) & 1, abort_flag, a.err))) break;
+        if (nYs < nck && nYs < nS && mbar_test(BAR(BAR_HREADY), nYs & 1)) {
+          const int j = nYs;
           tc_fence_after();
-          TC_MARK(k, 9);
-          issue_Ys(sst, sb + OFF_H, tYs);
+          TC_MARK(j, 9);
+          issue_Ys(sb + (j & 1) * kStage, sb + OFF_H, tmem + ((j & 1) ? TM_YS1 : TM_YS0));
+          mma_commit(BAR(BAR_HTFREE));
+          ++nYs;
+          if (stage_done(j)) mma_commit(BAR(BAR_EMPTY0 + (j & 1)));
+          prog = true;
         }
-        mma_commit(BAR(BAR_EMPTY0 + st));  // MMA1/MMA3/MMA4 of chunk k done with the B/C tiles
-        if (k != last) mma_commit(BAR(BAR_DHREADY));
-        if (!kStateOnly) {
-          if (k + 1 < nck) {
-            const int s2 = (k + 1) & 1;
-            if (!(ok = mbar_wait(BAR(BAR_FULL0 + s2), ((k + 1) >> 1) & 1, abort_flag, a.err))) break;
-            tc_fence_after();
-            TC_MARK(k, 10);
-            issue_S(sb + s2 * kStage, tmem + (s2 ? TM_S1 : TM_S0));
-            mma_commit(BAR(BAR_SREADY0 + s2));
-          }
-          if (!(ok = mbar_wait(BAR(BAR_STREADY0 + st), (k >> 1) & 1, abort_flag, a.err))) break;
+        if (nD < nck && (kStateOnly || nD < nS) &&
+            mbar_test(BAR(BAR_XREADY0 + (nD & 1)), (nD >> 1) & 1) &&
+            (nD == 0 || mbar_test(BAR(BAR_DHFREE), (nD - 1) & 1)) &&
+            (nD != last || mbar_test(BAR(BAR_XLOREADY), 0)) &&
+            (!kStateOnly || mbar_test(BAR(BAR_FULL0 + (nD & 1)), (nD >> 1) & 1))) {
+          const int j = nD;
           tc_fence_after();
-          TC_MARK(k, 11);
-          issue_Yi(tmem + (st ? TM_S1 : TM_S0), sb + OFF_X + xb * kXBuf, tYi);
-          mma_commit(BAR(BAR_YREADY));
-        }
-        mma_commit(BAR(BAR_XFREE0 + xb));
-        if (k == last) {  // low part of w o X (in the spare X buffer) for the final state
-          if (!(ok = mbar_wait(BAR(BAR_XLOREADY), 0, abort_flag, a.err))) break;
-          tc_fence_after();
-          issue_dH(sst, sb + OFF_X + ((k + 1) % kXBufs) * kXBuf, tDH, true);
+          TC_MARK(j, 8);
+          const uint32_t sst = sb + (j & 1) * kStage;
+          issue_dH(sst, sb + OFF_XW + (j & 1) * kTile, tmem + TM_DH, false);
+          // last chunk: the low part of w o X (in the other w o X buffer) for the final state
+          if (j == last) issue_dH(sst, sb + OFF_XW + ((j + 1) & 1) * kTile, tmem + TM_DH, true);
+          mma_commit(BAR(BAR_XWFREE0 + (j & 1)));
           mma_commit(BAR(BAR_DHREADY));
+          if (kStateOnly) mma_commit(BAR(BAR_XFREE0 + (j & 1)));
+          ++nD;
+          if (stage_done(j)) mma_commit(BAR(BAR_EMPTY0 + (j & 1)));
+          prog = true;
+        }
+        if (nS < nck && nS <= nYi + 1 && mbar_test(BAR(BAR_FULL0 + (nS & 1)), (nS >> 1) & 1) &&
+            (nS < 2 || mbar_test(BAR(BAR_YFREE0 + (nS & 1)), ((nS >> 1) - 1) & 1))) {
+          const int j = nS;
+          tc_fence_after();
+          TC_MARK(j, 10);
+          issue_S(sb + (j & 1) * kStage, tmem + ((j & 1) ? TM_S1 : TM_S0));
+          mma_commit(BAR(BAR_SREADY0 + (j & 1)));
+          ++nS;
+          if (stage_done(j)) mma_commit(BAR(BAR_EMPTY0 + (j & 1)));
+          prog = true;
+        }
+        if (prog) {
+          t_prog = globaltimer();
+        } else {
+          if (*abort_flag) {
+            ok = false;
+          } else if (globaltimer() - t_prog > 2000000000ull) {
+            *abort_flag = 1;
+            if (a.err) atomicCAS(a.err, 0, (int)SSD_ERR_TIMEOUT);
+            ok = false;
+          } else {
+            __nanosleep(20);
+          }
         }
       }
       // no MMA may still be running when TMEM is released
@@ -334,49 +409,62 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       int never_abort = 0;
       mbar_wait(BAR(BAR_DONE), 0, &never_abort, a.err);
     }
-  } else if (warp >= 4 && warp < 4 + kConvWarps) {
+  } else if (conv_index(warp) >= 0) {
     // ---------------------------------------------------------------- conv + SiLU -> X, w o X
     // Warp cw makes tokens 16cw..16cw+15; lane l channels 2l, 2l+1.  Raw row r of the X
     // buffer holds time t0-3+r; token s reads rows s..s+3 (a register window) and then
     // overwrites row s with its X row.  Rows 16cw+16..+18 belong to the next warp's tokens,
     // so every warp reads them before the group barrier that precedes all writes.
-    const int cw = warp - 4;
-    const bool leader = (tid == 5 * 32);  // leaders sit on different SM sub-partitions
+    // SiLU(u) = u * sigmoid(u) = h + h * tanh(h) with h = u / 2.  The conv accumulates h
+    // directly (halved weights) in fp16 pairs -- the precision of the MMA operand it feeds,
+    // 11 significant bits -- and one half2 tanh serves both channels.  The last chunk of a
+    // segment, whose newest tokens dominate the final state, uses fp32 and the exact SiLU.
+    const int cw = conv_index(warp);
+    const bool leader = (tid == 2 * 32);  // leaders sit on different SM sub-partitions
     const int ch = h * 64 + 2 * lane;
     const int W = a.W;
-    float e0[4], e1[4], bias0 = 0.f, bias1 = 0.f;
+    float2 ew[4], bias2 = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {  // weight for the input at time t-3+j
+    for (int j = 0; j < 4; ++j) {  // half the weight for the input at time t-3+j
       const int k = j - (4 - W);
-      e0[j] = (W > 0 && k >= 0) ? __bfloat162float(a.conv_w[(long long)ch * W + k]) : 0.f;
-      e1[j] = (W > 0 && k >= 0) ? __bfloat162float(a.conv_w[(long long)(ch + 1) * W + k]) : 0.f;
+      ew[j].x = (W > 0 && k >= 0) ? 0.5f * __bfloat162float(a.conv_w[(long long)ch * W + k]) : 0.f;
+      ew[j].y = (W > 0 && k >= 0) ? 0.5f * __bfloat162float(a.conv_w[(long long)(ch + 1) * W + k]) : 0.f;
     }
     if (W > 0 && a.conv_b) {
-      bias0 = __bfloat162float(a.conv_b[ch]);
-      bias1 = __bfloat162float(a.conv_b[ch + 1]);
+      bias2.x = 0.5f * __bfloat162float(a.conv_b[ch]);
+      bias2.y = 0.5f * __bfloat162float(a.conv_b[ch + 1]);
     }
+    __half2 hw[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) hw[j] = __float22half2_rn(ew[j]);
+    const __half2 hbias = __float22half2_rn(bias2);
     // byte offset of this lane's 4 bytes within a swizzled row r, by r mod 8
     uint32_t loff[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) loff[u] = ((uint32_t)((lane >> 2) ^ u) << 4) + ((uint32_t)(lane & 3) << 2);
     const int tok0 = kTokPerConvWarp * cw;  // multiple of 8
     for (int k = 0; k < nck; ++k) {
-      const int st = k & 1, xb = k % kXBufs, lb = (k + 1) % kXBufs;
+      const int st = k & 1, xb = k & 1, lb = (k + 1) & 1;
       const bool is_last = (k == last);
-      if (!wg_wait(BAR(BAR_FULLX0 + xb), (k / kXBufs) & 1, leader, 1, abort_flag, a.err, 256)) break;
+      if (!wg_wait(BAR(BAR_FULLX0 + xb), (k >> 1) & 1, leader, 1, abort_flag, a.err, 256)) break;
+      if (leader) TC_MARK(k, 13);
       if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, 1, abort_flag, a.err, 256)) break;
-      if (k >= 1 && !wg_wait(BAR(BAR_XWFREE), (k - 1) & 1, leader, 1, abort_flag, a.err, 256)) break;
-      // the low part of w o X goes to X[(k+1) % 3], last used by chunk k-2
-      if (is_last && k >= 2 &&
-          !wg_wait(BAR(BAR_XFREE0 + lb), ((k - 2) / kXBufs) & 1, leader, 1, abort_flag, a.err, 256))
+      if (leader) TC_MARK(k, 14);
+      // w o X[k % 2] was last read by MMA4 of chunk k-2
+      if (k >= 2 && !wg_wait(BAR(BAR_XWFREE0 + xb), ((k >> 1) - 1) & 1, leader, 1, abort_flag, a.err, 256))
+        break;
+      // the low part of w o X goes to the other w o X buffer, last read by MMA4 of chunk k-1
+      if (is_last && k >= 1 &&
+          !wg_wait(BAR(BAR_XWFREE0 + lb), ((k - 1) >> 1) & 1, leader, 1, abort_flag, a.err, 256))
         break;
       const float *cs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
       const float *dtv = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
       const float cs_end = cs[QC - 1];
       const float wl = lane < kTokPerConvWarp ? __expf(cs_end - cs[tok0 + lane]) * dtv[tok0 + lane] : 0.f;
+      const uint32_t wl2 = pack_f16(wl, wl);
       unsigned char *xt = smem + OFF_X + xb * kXBuf + tok0 * 128;   // row tok0
-      unsigned char *xwt = smem + OFF_XW + tok0 * 128;
-      unsigned char *xlt = smem + OFF_X + lb * kXBuf + tok0 * 128;
+      unsigned char *xwt = smem + OFF_XW + xb * kTile + tok0 * 128;
+      unsigned char *xlt = smem + OFF_XW + lb * kTile + tok0 * 128;
       // rows tok0 + r for r = 0..18 (tok0 is a multiple of 8, so row mod 8 = r mod 8)
 #define RAW(r) (*reinterpret_cast<const uint32_t *>(xt + (r) * 128 + loff[(r) & 7]))
       uint32_t r0 = RAW(0), r1 = RAW(1), r2 = RAW(2);
@@ -399,51 +487,98 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         TC_MARK(k, 0);
         mbar_arrive(BAR(BAR_EMPTY0 + st));  // dt and prefix sums already read
       }
-      float2 xm3 = unpack_bf16(r0), xm2 = unpack_bf16(r1), xm1 = unpack_bf16(r2);
+      // The token loop is compiled twice: the common chunks, and the last chunk of a segment.
+      auto tokens = [&](auto last_tag) {
+        constexpr bool kLast = decltype(last_tag)::value;
+        if constexpr (!kLast) {
+          __half2 xm3 = __float22half2_rn(unpack_bf16(r0)), xm2 = __float22half2_rn(unpack_bf16(r1)),
+                  xm1 = __float22half2_rn(unpack_bf16(r2));
 #pragma unroll 1
-      for (int g = 0; g < 2; ++g) {
-        float2 xn[8];
+          for (int g = 0; g < 2; ++g) {
+            __half2 xn[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int nxt = 8 * g + u + 3;  // row of time t for token 8g+u
-          uint32_t w3;
-          if (nxt < 16) w3 = RAW(nxt);
-          else w3 = nxt == 16 ? nb0 : (nxt == 17 ? nb1 : nb2);
-          xn[u] = unpack_bf16(w3);
-        }
+            for (int u = 0; u < 8; ++u) {
+              const int nxt = 8 * g + u + 3;  // row of time t for token 8g+u
+              uint32_t w3;
+              if (nxt < 16) w3 = RAW(nxt);
+              else w3 = nxt == 16 ? nb0 : (nxt == 17 ? nb1 : nb2);
+              xn[u] = __float22half2_rn(unpack_bf16(w3));
+            }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int i = 8 * g + u;
-          const float2 x0 = xn[u];
-          float u0, u1;
-          if (W == 0) {
-            u0 = x0.x;
-            u1 = x0.y;
-          } else {
-            u0 = silu(bias0 + e0[0] * xm3.x + e0[1] * xm2.x + e0[2] * xm1.x + e0[3] * x0.x);
-            u1 = silu(bias1 + e1[0] * xm3.y + e1[1] * xm2.y + e1[2] * xm1.y + e1[3] * x0.y);
+            for (int u = 0; u < 8; ++u) {
+              const int i = 8 * g + u;
+              const __half2 x0 = xn[u];
+              __half2 xo = x0;
+              if (W != 0) {
+                __half2 acc = __hfma2(hw[0], xm3, hbias);
+                acc = __hfma2(hw[1], xm2, acc);
+                acc = __hfma2(hw[2], xm1, acc);
+                acc = __hfma2(hw[3], x0, acc);
+                xo = __hfma2(acc, h2tanh_approx(acc), acc);
+              }
+              const uint32_t off = i * 128 + loff[u];
+              *reinterpret_cast<__half2 *>(xt + off) = xo;
+              const uint32_t w2 = __shfl_sync(0xffffffffu, wl2, i);
+              *reinterpret_cast<__half2 *>(xwt + off) = __hmul2(xo, *reinterpret_cast<const __half2 *>(&w2));
+              xm3 = xm2;
+              xm2 = xm1;
+              xm1 = x0;
+            }
           }
-          const float ws = __shfl_sync(0xffffffffu, wl, i);
-          const uint32_t off = i * 128 + loff[u];
-          *reinterpret_cast<uint32_t *>(xt + off) = pack_f16(u0, u1);
-          const float v0 = u0 * ws, v1 = u1 * ws;
-          const __half2 hi = __floats2half2_rn(v0, v1);
-          *reinterpret_cast<__half2 *>(xwt + off) = hi;
-          if (is_last) {
-            const float2 hf = __half22float2(hi);
-            *reinterpret_cast<uint32_t *>(xlt + off) = pack_f16(v0 - hf.x, v1 - hf.y);
-          }
-          xm3 = xm2;
-          xm2 = xm1;
-          xm1 = x0;
+          return;
         }
-      }
+        float2 xm3 = unpack_bf16(r0), xm2 = unpack_bf16(r1), xm1 = unpack_bf16(r2);
+#pragma unroll 1
+        for (int g = 0; g < 2; ++g) {
+          float2 xn[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int nxt = 8 * g + u + 3;  // row of time t for token 8g+u
+            uint32_t w3;
+            if (nxt < 16) w3 = RAW(nxt);
+            else w3 = nxt == 16 ? nb0 : (nxt == 17 ? nb1 : nb2);
+            xn[u] = unpack_bf16(w3);
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int i = 8 * g + u;
+            const float2 x0 = xn[u];
+            float2 acc = x0;
+            if (W != 0) {
+              acc = __ffma2_rn(ew[0], xm3, bias2);
+              acc = __ffma2_rn(ew[1], xm2, acc);
+              acc = __ffma2_rn(ew[2], xm1, acc);
+              acc = __ffma2_rn(ew[3], x0, acc);
+            }
+            const uint32_t off = i * 128 + loff[u];
+            {
+              // The final state's chunk: its newest tokens dominate the final state, so X
+              // comes from the fp32 SiLU and w o X is stored as the fp16 hi + lo parts of the
+              // fp32 product.
+              const float u0 = W != 0 ? silu(2.f * acc.x) : acc.x;
+              const float u1 = W != 0 ? silu(2.f * acc.y) : acc.y;
+              const float ws = __shfl_sync(0xffffffffu, wl, i);
+              const float2 v = make_float2(u0 * ws, u1 * ws);
+              const __half2 hi = __float22half2_rn(v);
+              const float2 hf = __half22float2(hi);
+              *reinterpret_cast<uint32_t *>(xt + off) = pack_f16(u0, u1);
+              *reinterpret_cast<__half2 *>(xwt + off) = hi;
+              *reinterpret_cast<uint32_t *>(xlt + off) = pack_f16(v.x - hf.x, v.y - hf.y);
+            }
+            xm3 = xm2;
+            xm2 = xm1;
+            xm1 = x0;
+          }
+        }
+      };
+      if (is_last) tokens(std::true_type{});
+      else tokens(std::false_type{});
 #undef RAW
       fence_proxy_async();
       named_bar(1, 256);
       if (leader) {
         TC_MARK(k, 1);
-        mbar_arrive(BAR(BAR_XREADY));
+        mbar_arrive(BAR(BAR_XREADY0 + xb));
         if (is_last) mbar_arrive(BAR(BAR_XLOREADY));
       }
     }
@@ -476,40 +611,81 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (leader) TC_MARK(k, 2);
         const float cst = cs[t];
         const uint32_t trow = tmem + (st ? TM_S1 : TM_S0) + ((uint32_t)(32 * mw) << 16);
+        // Blocks of 32 columns in increasing J: S~ columns 32J..32J+31 go to the packed TMEM
+        // columns 16J..16J+15, which only hold S columns of blocks already read.
+        // Blocks J < mw lie wholly below the diagonal: S~ = S * rf * cf (a block whose cs
+        // span is too steep to factor takes the direct exponential instead).
 #pragma unroll 1
-        for (int J = 0; J < 4; ++J) {
+        for (int J = 0; J < mw; ++J) {
           uint32_t pk[16];
-          if (J <= mw) {
-            float v[32];
-            tmem_ld32(trow + 32 * J, v);
-            tmem_ld_wait();
-            const float rJ = cs[32 * J + 31];
-            const bool direct = (cs[32 * J] - rJ) > 60.f;  // block too steep to factor
-            const float rf = direct ? 0.f : __expf(cst - rJ);
+          float v[32];
+          tmem_ld32(trow + 32 * J, v);
+          tmem_ld_wait();
+          const float rJ = cs[32 * J + 31];
+          if (cs[32 * J] - rJ > 60.f) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v[c] *= __expf(cst - cs[32 * J + c]) * dtv[32 * J + c];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) pk[c] = pack_f16(v[2 * c], v[2 * c + 1]);
+          } else {
+            const float rf = __expf(cst - rJ);
+            const float2 rf2 = make_float2(rf, rf);
             const float4 *cf4 = reinterpret_cast<const float4 *>(cf + 32 * J);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               const float4 c4 = cf4[q];
-              const float cq[4] = {c4.x, c4.y, c4.z, c4.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int c = 4 * q + e, s = 32 * J + c;
-                float val = direct ? v[c] * __expf(cst - cs[s]) * dtv[s] : v[c] * rf * cq[e];
-                if (J == mw) {  // diagonal block: causal mask and the D x skip
-                  if (s > t) val = 0.f;
-                  if (s == t) val += Dh;
-                }
-                v[c] = val;
-              }
+              const float2 lo = __fmul2_rn(__fmul2_rn(make_float2(v[4 * q], v[4 * q + 1]), rf2),
+                                           make_float2(c4.x, c4.y));
+              const float2 hi = __fmul2_rn(__fmul2_rn(make_float2(v[4 * q + 2], v[4 * q + 3]), rf2),
+                                           make_float2(c4.z, c4.w));
+              pk[2 * q] = pack_f16(lo.x, lo.y);
+              pk[2 * q + 1] = pack_f16(hi.x, hi.y);
             }
-#pragma unroll
-            for (int c = 0; c < 16; ++c) pk[c] = pack_f16(v[2 * c], v[2 * c + 1]);
-          } else {
-#pragma unroll
-            for (int c = 0; c < 16; ++c) pk[c] = 0u;
           }
-          // S~ columns 32J..32J+31 -> packed TMEM columns 16J..16J+15 (already read)
           tmem_st16(trow + 16 * J, pk);
+        }
+        {  // diagonal block J = mw: causal mask (column c <= row lane) and the D x skip
+          const int J = mw;
+          uint32_t pk[16];
+          float v[32];
+          tmem_ld32(trow + 32 * J, v);
+          tmem_ld_wait();
+          const float rJ = cs[32 * J + 31];
+          if (cs[32 * J] - rJ > 60.f) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v[c] *= __expf(fminf(cst - cs[32 * J + c], 0.f)) * dtv[32 * J + c];
+          } else {
+            const float rf = __expf(cst - rJ);
+            const float2 rf2 = make_float2(rf, rf);
+            const float4 *cf4 = reinterpret_cast<const float4 *>(cf + 32 * J);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 c4 = cf4[q];
+              const float2 lo = __fmul2_rn(__fmul2_rn(make_float2(v[4 * q], v[4 * q + 1]), rf2),
+                                           make_float2(c4.x, c4.y));
+              const float2 hi = __fmul2_rn(__fmul2_rn(make_float2(v[4 * q + 2], v[4 * q + 3]), rf2),
+                                           make_float2(c4.z, c4.w));
+              v[4 * q] = lo.x;
+              v[4 * q + 1] = lo.y;
+              v[4 * q + 2] = hi.x;
+              v[4 * q + 3] = hi.y;
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float val = c <= lane ? v[c] : 0.f;
+            v[c] = c == lane ? val + Dh : val;
+          }
+#pragma unroll
+          for (int c = 0; c < 16; ++c) pk[c] = pack_f16(v[2 * c], v[2 * c + 1]);
+          tmem_st16(trow + 16 * J, pk);
+        }
+        {  // blocks J > mw lie above the diagonal: zeros
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) pk[c] = 0u;
+#pragma unroll 1
+          for (int J = mw + 1; J < 4; ++J) tmem_st16(trow + 16 * J, pk);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -556,12 +732,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const float et = __expf(cs[n]);
       decay_sum += cs_end;
       const float ak = __expf(cs_end);
+      named_bar(3, 128);  // every thread has read the prefix sums
+      if (leader) mbar_arrive(BAR(BAR_EMPTY0 + st));
       if (!wg_wait(BAR(BAR_DHREADY), k & 1, leader, 3, abort_flag, a.err)) break;
       tc_fence_after();
-      if (leader) {
-        TC_MARK(k, 4);
-        mbar_arrive(BAR(BAR_EMPTY0 + st));  // prefix sums already read by the group
-      }
+      if (leader) TC_MARK(k, 4);
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
         float dh[32], hr[32];
@@ -570,23 +745,40 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         tmem_ld_wait();
         uint32_t hu[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          hr[i] = ak * hr[i] + dh[i];
-          hu[i] = __float_as_uint(hr[i]);
+        for (int i = 0; i < 32; i += 2) {
+          const float2 r = __ffma2_rn(make_float2(ak, ak), make_float2(hr[i], hr[i + 1]),
+                                      make_float2(dh[i], dh[i + 1]));
+          hr[i] = r.x;
+          hr[i + 1] = r.y;
+          hu[i] = __float_as_uint(r.x);
+          hu[i + 1] = __float_as_uint(r.y);
         }
         tmem_st32(tmem + TM_H + 32 * half + lane_off, hu);
-        if (k != last) write_h_tile(smem, hr, n, half);
       }
       tmem_st_wait();
-      if (k != last) fence_proxy_async();
       tc_fence_before();
       named_bar(3, 128);
-      if (leader) {
-        TC_MARK(k, 5);
-        mbar_arrive(BAR(BAR_HREADY));
+      if (leader) mbar_arrive(BAR(BAR_DHFREE));  // dH read: MMA4 of chunk k+1 may overwrite it
+      if (!kStateOnly && k != last) {
+        // fp16 copy of h_k for MMA3 of chunk k+1, once MMA3 of chunk k has read h_{k-1}
+        if (!wg_wait(BAR(BAR_HTFREE), k & 1, leader, 3, abort_flag, a.err)) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          float hr[32];
+          tmem_ld32(tmem + TM_H + 32 * half + lane_off, hr);
+          tmem_ld_wait();
+          write_h_tile(smem, hr, n, half);
+        }
+        fence_proxy_async();
+        named_bar(3, 128);
+        if (leader) {
+          TC_MARK(k, 5);
+          mbar_arrive(BAR(BAR_HREADY));
+        }
       }
       if (!kStateOnly) {
-        if (!wg_wait(BAR(BAR_YREADY), k & 1, leader, 3, abort_flag, a.err)) break;
+        if (!wg_wait(BAR(BAR_YREADY0 + st), (k >> 1) & 1, leader, 3, abort_flag, a.err)) break;
         tc_fence_after();
         if (leader) TC_MARK(k, 6);
         const int tok = t_begin + k * QC + n;
@@ -594,11 +786,16 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
           float yi[32], ysv[32];
-          tmem_ld32(tmem + TM_YI + 32 * half + lane_off, yi);
-          tmem_ld32(tmem + TM_YS + 32 * half + lane_off, ysv);
+          tmem_ld32(tmem + (st ? TM_S1 : TM_S0) + TM_YI_OFF + 32 * half + lane_off, yi);
+          tmem_ld32(tmem + (st ? TM_YS1 : TM_YS0) + 32 * half + lane_off, ysv);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) yi[i] += et * ysv[i];
+          for (int i = 0; i < 32; i += 2) {
+            const float2 r = __ffma2_rn(make_float2(et, et), make_float2(ysv[i], ysv[i + 1]),
+                                        make_float2(yi[i], yi[i + 1]));
+            yi[i] = r.x;
+            yi[i + 1] = r.y;
+          }
           if (tok < t_end) {
             if (a.yf) {
               float4 *dst = reinterpret_cast<float4 *>(a.yf + row * a.d_inner + h * 64 + 32 * half);
@@ -617,7 +814,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         named_bar(3, 128);
         if (leader) {
           TC_MARK(k, 7);
-          mbar_arrive(BAR(BAR_YFREE));
+          mbar_arrive(BAR(BAR_YFREE0 + st));
         }
       }
     }
