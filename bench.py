@@ -48,7 +48,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 METRIC = "SSD prefill tokens/s/layer"
 HEADLINE_CONFIG = {"workload": "prefill_8k", "batch": 1, "seqlen": 8192, "nheads": 128,
                    "headdim": 64, "dstate": 128, "ngroups": 8, "chunk": 128, "conv_width": 4,
-                   "state_dtype": "f32", "l2": "flushed between timed steps (256 MiB write)"}
+                   "state_dtype": "f32",
+                   "l2": "flushed between timed steps: 256 MiB written, then a second 256 MiB "
+                         "buffer read, so the step starts with no dirty lines in L2"}
 
 
 def peaks():
@@ -132,6 +134,22 @@ def mixer_flops(cfg) -> dict:
 
 
 # ---------------------------------------------------------------------------------------------
+# multi-GPU accounting: every rank runs an independent replica of the workload (weak scaling)
+def max_over_ranks(torch, dist, value: float, device) -> float:
+    """The job's time is the slowest rank's: all-reduce MAX (identity on one process)."""
+    if not dist:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job rate: the units all ranks processed over the (max-over-ranks) time."""
+    return world * units_per_rank * steps / (total_ms * 1e-3)
+
+
+# ---------------------------------------------------------------------------------------------
 class ClockSampler:
     """nvidia-smi clock/throttle sampling every 100 ms in a reader thread; each sample is
     stamped with the host's monotonic clock when it arrives."""
@@ -210,13 +228,16 @@ class Ctx:
         self.rank, self.world, self.clk = rank, world, clk
         self.dev = torch.device("cuda")
         self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=self.dev)
+        self.flush_rd = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=self.dev)
+
+    def flush_l2(self, i: int):
+        """Evicts the previous step's data from L2: a write of a buffer larger than L2, then a
+        read of a second one, which writes back the dirty lines outside the timed region."""
+        self.flush.fill_(float(i))
+        self.flush_rd.sum()
 
     def max_over_ranks(self, v: float) -> float:
-        if not self.dist:
-            return v
-        t = self.torch.tensor([v], dtype=self.torch.float64, device=self.dev)
-        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks(self.torch, self.dist, v, self.dev)
 
     def timed(self, step, steps, flush=True, trace=True):
         """Times `steps` calls of step() with CUDA events on the current stream (barrier and
@@ -236,7 +257,7 @@ class Ctx:
         t0 = time.monotonic()
         for i in range(steps):
             if flush:
-                self.flush.fill_(float(i))  # evict the previous step's data from L2
+                self.flush_l2(i)
             ev[i][0].record(stream)
             step()
             ev[i][1].record(stream)
@@ -251,7 +272,7 @@ class Ctx:
             while time.monotonic() - t1 < 1.0:
                 for _ in range(4):
                     if flush:
-                        self.flush.fill_(0.0)
+                        self.flush_l2(0)
                     step()
                 torch.cuda.synchronize()
             window = "timed region + 1 s of the same step right after it"
@@ -305,7 +326,7 @@ def bench_prefill(c: Ctx):
     per, table, dom = kernel_table(recs)
     tokens = Bn * L
     res = {
-        "value": c.world * tokens * args.steps / (total_ms * 1e-3),
+        "value": job_throughput(tokens, c.world, args.steps, total_ms),
         "ms_per_step": total_ms / args.steps,
         "gpu_launches": len(recs),
         "clocks": clocks,
@@ -335,7 +356,7 @@ def bench_prefill(c: Ctx):
     for _ in range(max(2, args.warmup)):
         e2e_step()
     e_ms, _, _ = c.timed(e2e_step, args.steps, trace=False)
-    res["e2e"] = {"value": c.world * tokens * args.steps / (e_ms * 1e-3), "unit": "tokens/s",
+    res["e2e"] = {"value": job_throughput(tokens, c.world, args.steps, e_ms), "unit": "tokens/s",
                   "h2d_bytes_per_step": hx.numel() * 2 + hdt.numel() * 2,
                   "d2h_bytes_per_step": hy.numel() * 2 + hh.numel() * 4}
     return res
@@ -442,7 +463,7 @@ def bench_long_context(c: Ctx):
     per, table, dom = kernel_table(recs)
     algo = scan_bytes(scfg, state_in=True) if dom.startswith("ssd_scan") else gated_norm_bytes(scfg)
     return {"metric": METRIC, "workload": "long_context_128k",
-            "value": round(c.world * Bn * L * args.steps / (total_ms * 1e-3), 1),
+            "value": round(job_throughput(Bn * L, c.world, args.steps, total_ms), 1),
             "unit": "tokens/s", "ms_per_step": round(total_ms / args.steps, 4),
             "segments": nseg, "segment_len": Ls, "chunk": cfg["chunk"],
             "path_bytes_per_step": nseg * prefill_bytes(scfg, state_in=True),
@@ -476,7 +497,7 @@ def bench_mixer(c: Ctx):
     ach = fl["in_proj"] / (gemm_ms * 1e-3) / 1e12
     step_ms = total_ms / args.steps
     return {"metric": "mixer layer tokens/s", "workload": "mixer_12b", "batch": Bn,
-            "value": round(c.world * Bn * L * args.steps / (total_ms * 1e-3), 1),
+            "value": round(job_throughput(Bn * L, c.world, args.steps, total_ms), 1),
             "unit": "tokens/s", "ms_per_step": round(step_ms, 4),
             "layer_tflops": round(sum(fl.values()) / (step_ms * 1e-3) / 1e12, 1),
             "flops_per_step": fl, "gpu_launches": len(recs), "kernels": table, "clocks": clocks,

@@ -232,8 +232,114 @@ cudaError_t launch_conv_silu_f32(const PrefillPlan &p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// Conv + SiLU of the B and C channels into fp16 (the tensor-core scan's operand buffer).
+// A streaming kernel: one thread owns 8 channels (one 16-byte load per row) over kBcTok
+// tokens, keeps rows as packed bf16 and loads 8 rows ahead, so that each SM has tens of
+// kilobytes of loads in flight.  The 3 rows before the first token come from the row
+// above (or the conv cache / zeros at t < 0).
+constexpr int kBcTok = 16;
+constexpr int kBcThreads = 256;
+
+__device__ __forceinline__ void unpack8(const uint4 &r, float (&v)[8]) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+template <int W>
+__global__ void __launch_bounds__(kBcThreads) bc_conv_kernel(const __nv_bfloat16 *__restrict__ xBC, long long xs,
+                                                             const __nv_bfloat16 *__restrict__ csi,
+                                                             const __nv_bfloat16 *__restrict__ w,
+                                                             const __nv_bfloat16 *__restrict__ bias,
+                                                             __half *__restrict__ out, int L, int conv_dim,
+                                                             int c_begin, int C_out) {
+  const int o8 = (blockIdx.x * kBcThreads + threadIdx.x) * 8;
+  if (o8 >= C_out) return;
+  const int c8 = c_begin + o8;
+  const int b = blockIdx.z;
+  const int t0 = blockIdx.y * kBcTok;
+  const int t1 = min(L, t0 + kBcTok);
+  const __nv_bfloat16 *xrow = xBC + (long long)b * L * xs + c8;
+  float wt[4][8], bs[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    bs[i] = bias ? __bfloat162float(bias[c8 + i]) : 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) wt[k][i] = (k < W) ? __bfloat162float(w[(long long)(c8 + i) * W + k]) : 0.f;
+  }
+  uint4 hist[3];  // raw rows of times t-3, t-2, t-1
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    const int tau = t0 - 3 + j;
+    if (W > 0 && tau >= 0) {
+      hist[j] = *reinterpret_cast<const uint4 *>(xrow + (long long)tau * xs);
+    } else if (csi && W > 0 && W + tau >= 0) {
+      hist[j] = *reinterpret_cast<const uint4 *>(csi + ((long long)b * W + (W + tau)) * conv_dim + c8);
+    } else {
+      hist[j] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+#pragma unroll 1
+  for (int tg = t0; tg < t1; tg += 8) {
+    uint4 cur[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      cur[j] = tg + j < t1 ? __ldcs(reinterpret_cast<const uint4 *>(xrow + (long long)(tg + j) * xs))
+                           : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int t = tg + j;
+      if (t >= t1) break;
+      float x[4][8];  // times t-3 .. t
+      unpack8(hist[0], x[0]);
+      unpack8(hist[1], x[1]);
+      unpack8(hist[2], x[2]);
+      unpack8(cur[j], x[3]);
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        float r[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float acc = bs[i + e];
+          // tap k multiplies time t-(W-1)+k, i.e. x[4-W+k]
+#pragma unroll
+          for (int k = 0; k < W; ++k) acc = fmaf(wt[k][i + e], x[4 - W + k][i + e], acc);
+          r[e] = W > 0 ? silu(acc) : x[3][i + e];
+        }
+        const __half2 hv = __floats2half2_rn(r[0], r[1]);
+        o[i / 2] = *reinterpret_cast<const uint32_t *>(&hv);
+      }
+      *reinterpret_cast<uint4 *>(out + ((long long)b * L + t) * C_out + o8) = make_uint4(o[0], o[1], o[2], o[3]);
+      hist[0] = hist[1];
+      hist[1] = hist[2];
+      hist[2] = cur[j];
+    }
+  }
+}
+
 cudaError_t launch_bc_conv_f16(const PrefillPlan &p, cudaStream_t s) {
-  conv_dispatch<__nv_bfloat16, __half>(p, (__half *)p.bc, p.d_inner, 2 * p.G * p.N, s);
+  const int C_out = 2 * p.G * p.N;
+  if (C_out % 8 || p.xs % 8 || p.conv_dim % 8) {  // 16-byte rows needed; else the generic kernel
+    conv_dispatch<__nv_bfloat16, __half>(p, (__half *)p.bc, p.d_inner, C_out, s);
+    return cudaGetLastError();
+  }
+  dim3 grid((C_out / 8 + kBcThreads - 1) / kBcThreads, (p.L + kBcTok - 1) / kBcTok, p.B);
+  const auto *x = (const __nv_bfloat16 *)p.xBC;
+  const auto *csi = (const __nv_bfloat16 *)p.csi;
+  const auto *w = (const __nv_bfloat16 *)p.conv_w;
+  const auto *bb = (const __nv_bfloat16 *)p.conv_b;
+  __half *o = (__half *)p.bc;
+  switch (p.W) {
+    case 0: bc_conv_kernel<0><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
+    case 1: bc_conv_kernel<1><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
+    case 2: bc_conv_kernel<2><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
+    case 3: bc_conv_kernel<3><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
+    default: bc_conv_kernel<4><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
+  }
   return cudaGetLastError();
 }
 

@@ -336,6 +336,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         return nD > j && (kStateOnly || (nS > j && nYs > j));
       };
       uint64_t t_prog = globaltimer();
+      uint32_t nap = 32;  // sleep between polls: doubles up to 256 ns while nothing is ready
       bool ok = true;
       while (ok && (nD < nck || nYi < nck)) {
         bool prog = false;
@@ -392,6 +393,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         if (prog) {
           t_prog = globaltimer();
+          nap = 32;
         } else {
           if (*abort_flag) {
             ok = false;
@@ -400,7 +402,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             if (a.err) atomicCAS(a.err, 0, (int)SSD_ERR_TIMEOUT);
             ok = false;
           } else {
-            __nanosleep(20);
+            __nanosleep(nap);
+            nap = nap < 256 ? 2 * nap : 256;
           }
         }
       }
