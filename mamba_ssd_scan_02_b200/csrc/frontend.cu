@@ -6,6 +6,8 @@
 // inputs before the first token come from the incoming cache (row W-1 = the newest).  This is
 // the Mamba-2 short convolution of window 4 in the Nemotron Nano 2 layers ("NVIDIA Nemotron
 // Nano 2" summary, section "Method").
+#include <type_traits>
+
 #include "common.cuh"
 #include "plan.h"
 
@@ -233,20 +235,28 @@ cudaError_t launch_conv_silu_f32(const PrefillPlan &p, cudaStream_t s) {
 }
 
 // Conv + SiLU of the B and C channels into fp16 (the tensor-core scan's operand buffer).
-// A streaming kernel: one thread owns 8 channels (one 16-byte load per row) over kBcTok
-// tokens, keeps rows as packed bf16 and loads 8 rows ahead, so that each SM has tens of
-// kilobytes of loads in flight.  The 3 rows before the first token come from the row
-// above (or the conv cache / zeros at t < 0).
+// A streaming kernel: one thread owns 4 channels (one 8-byte load per row) over kBcTok
+// tokens with the 4-row window kept in fp32 registers, and loads 8 rows ahead; few registers
+// per thread keep several blocks per SM and tens of kilobytes of loads in flight.  The 3 rows
+// before the first token come from the rows above (or the conv cache / zeros at t < 0).
 constexpr int kBcTok = 16;
 constexpr int kBcThreads = 256;
 
-__device__ __forceinline__ void unpack8(const uint4 &r, float (&v)[8]) {
-  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    v[2 * i] = __uint_as_float(w[i] << 16);
-    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
+// SiLU(u) = u sigmoid(u) = h + h tanh(h) with h = u / 2, using the hardware tanh
+// approximation (one special-function op instead of an exponential and a reciprocal).  Its
+// error is of the order of the fp16 rounding that the result receives anyway.
+__device__ __forceinline__ float silu_tanh(float u) {
+  const float h = 0.5f * u;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+  return fmaf(h, t, h);
+}
+
+__device__ __forceinline__ void unpack4(const uint2 &r, float (&v)[4]) {
+  v[0] = __uint_as_float(r.x << 16);
+  v[1] = __uint_as_float(r.x & 0xFFFF0000u);
+  v[2] = __uint_as_float(r.y << 16);
+  v[3] = __uint_as_float(r.y & 0xFFFF0000u);
 }
 
 template <int W>
@@ -256,78 +266,89 @@ __global__ void __launch_bounds__(kBcThreads) bc_conv_kernel(const __nv_bfloat16
                                                              const __nv_bfloat16 *__restrict__ bias,
                                                              __half *__restrict__ out, int L, int conv_dim,
                                                              int c_begin, int C_out) {
-  const int o8 = (blockIdx.x * kBcThreads + threadIdx.x) * 8;
-  if (o8 >= C_out) return;
-  const int c8 = c_begin + o8;
+  const int o4 = (blockIdx.x * kBcThreads + threadIdx.x) * 4;
+  if (o4 >= C_out) return;
+  const int c4 = c_begin + o4;
   const int b = blockIdx.z;
   const int t0 = blockIdx.y * kBcTok;
   const int t1 = min(L, t0 + kBcTok);
-  const __nv_bfloat16 *xrow = xBC + (long long)b * L * xs + c8;
-  float wt[4][8], bs[8];
+  const __nv_bfloat16 *xrow = xBC + (long long)b * L * xs + c4;
+  float wt[4][4], bs[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    bs[i] = bias ? __bfloat162float(bias[c8 + i]) : 0.f;
+  for (int i = 0; i < 4; ++i) {
+    bs[i] = bias ? __bfloat162float(bias[c4 + i]) : 0.f;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) wt[k][i] = (k < W) ? __bfloat162float(w[(long long)(c8 + i) * W + k]) : 0.f;
+    for (int k = 0; k < 4; ++k) wt[k][i] = (k < W) ? __bfloat162float(w[(long long)(c4 + i) * W + k]) : 0.f;
   }
-  uint4 hist[3];  // raw rows of times t-3, t-2, t-1
+  float x3[4], x2[4], x1[4];  // times t-3, t-2, t-1
+  {
+    uint2 hist[3];
 #pragma unroll
-  for (int j = 0; j < 3; ++j) {
-    const int tau = t0 - 3 + j;
-    if (W > 0 && tau >= 0) {
-      hist[j] = *reinterpret_cast<const uint4 *>(xrow + (long long)tau * xs);
-    } else if (csi && W > 0 && W + tau >= 0) {
-      hist[j] = *reinterpret_cast<const uint4 *>(csi + ((long long)b * W + (W + tau)) * conv_dim + c8);
-    } else {
-      hist[j] = make_uint4(0u, 0u, 0u, 0u);
+    for (int j = 0; j < 3; ++j) {
+      const int tau = t0 - 3 + j;
+      if (W > 0 && tau >= 0) {
+        hist[j] = *reinterpret_cast<const uint2 *>(xrow + (long long)tau * xs);
+      } else if (csi && W > 0 && W + tau >= 0) {
+        hist[j] = *reinterpret_cast<const uint2 *>(csi + ((long long)b * W + (W + tau)) * conv_dim + c4);
+      } else {
+        hist[j] = make_uint2(0u, 0u);
+      }
     }
+    unpack4(hist[0], x3);
+    unpack4(hist[1], x2);
+    unpack4(hist[2], x1);
   }
-#pragma unroll 1
-  for (int tg = t0; tg < t1; tg += 8) {
-    uint4 cur[8];
+  // Rows in groups of 8; the common full tile runs without per-row bounds checks.
+  auto group = [&](int tg, auto full_tag) {
+    constexpr bool kFull = decltype(full_tag)::value;
+    uint2 cur[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      cur[j] = tg + j < t1 ? __ldcs(reinterpret_cast<const uint4 *>(xrow + (long long)(tg + j) * xs))
-                           : make_uint4(0u, 0u, 0u, 0u);
+      cur[j] = (kFull || tg + j < t1) ? __ldcs(reinterpret_cast<const uint2 *>(xrow + (long long)(tg + j) * xs))
+                                      : make_uint2(0u, 0u);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int t = tg + j;
-      if (t >= t1) break;
-      float x[4][8];  // times t-3 .. t
-      unpack8(hist[0], x[0]);
-      unpack8(hist[1], x[1]);
-      unpack8(hist[2], x[2]);
-      unpack8(cur[j], x[3]);
-      uint32_t o[4];
+      if (!kFull && t >= t1) break;
+      float x0[4], r[4];
+      unpack4(cur[j], x0);
 #pragma unroll
-      for (int i = 0; i < 8; i += 2) {
-        float r[2];
+      for (int i = 0; i < 4; ++i) {
+        if (W == 0) {
+          r[i] = x0[i];
+        } else {
+          // tap k multiplies time t-(W-1)+k
+          const float xs4[4] = {x3[i], x2[i], x1[i], x0[i]};
+          float acc = bs[i];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          float acc = bs[i + e];
-          // tap k multiplies time t-(W-1)+k, i.e. x[4-W+k]
-#pragma unroll
-          for (int k = 0; k < W; ++k) acc = fmaf(wt[k][i + e], x[4 - W + k][i + e], acc);
-          r[e] = W > 0 ? silu(acc) : x[3][i + e];
+          for (int k = 0; k < W; ++k) acc = fmaf(wt[k][i], xs4[4 - W + k], acc);
+          r[i] = silu_tanh(acc);
         }
-        const __half2 hv = __floats2half2_rn(r[0], r[1]);
-        o[i / 2] = *reinterpret_cast<const uint32_t *>(&hv);
+        x3[i] = x2[i];
+        x2[i] = x1[i];
+        x1[i] = x0[i];
       }
-      *reinterpret_cast<uint4 *>(out + ((long long)b * L + t) * C_out + o8) = make_uint4(o[0], o[1], o[2], o[3]);
-      hist[0] = hist[1];
-      hist[1] = hist[2];
-      hist[2] = cur[j];
+      const __half2 h01 = __floats2half2_rn(r[0], r[1]), h23 = __floats2half2_rn(r[2], r[3]);
+      *reinterpret_cast<uint2 *>(out + ((long long)b * L + t) * C_out + o4) =
+          make_uint2(*reinterpret_cast<const uint32_t *>(&h01), *reinterpret_cast<const uint32_t *>(&h23));
     }
+  };
+  if (t1 - t0 == kBcTok) {
+    group(t0, std::true_type{});
+    group(t0 + 8, std::true_type{});
+  } else {
+#pragma unroll 1
+    for (int tg = t0; tg < t1; tg += 8) group(tg, std::false_type{});
   }
 }
 
 cudaError_t launch_bc_conv_f16(const PrefillPlan &p, cudaStream_t s) {
   const int C_out = 2 * p.G * p.N;
-  if (C_out % 8 || p.xs % 8 || p.conv_dim % 8) {  // 16-byte rows needed; else the generic kernel
+  if (C_out % 4 || p.xs % 4 || p.conv_dim % 4 || p.d_inner % 4) {  // 8-byte accesses; else the generic kernel
     conv_dispatch<__nv_bfloat16, __half>(p, (__half *)p.bc, p.d_inner, C_out, s);
     return cudaGetLastError();
   }
-  dim3 grid((C_out / 8 + kBcThreads - 1) / kBcThreads, (p.L + kBcTok - 1) / kBcTok, p.B);
+  dim3 grid((C_out / 4 + kBcThreads - 1) / kBcThreads, (p.L + kBcTok - 1) / kBcTok, p.B);
   const auto *x = (const __nv_bfloat16 *)p.xBC;
   const auto *csi = (const __nv_bfloat16 *)p.csi;
   const auto *w = (const __nv_bfloat16 *)p.conv_w;

@@ -3,6 +3,8 @@
 // summary, section "Method"); in the Mamba-2 mixer the scan output is gated by SiLU(z) and
 // then normalised over groups of d_inner / norm_groups consecutive channels:
 //   g = y * silu(z);   out = g / sqrt(mean_group(g^2) + eps) * w
+#include <stdint.h>
+
 #include "common.cuh"
 #include "plan.h"
 
@@ -100,10 +102,50 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_bf16_kernel(
 
 }  // namespace
 
+// The same for bf16 tensors in one pass: a CTA of gs / 8 threads per (row, norm group), each
+// thread holding 8 consecutive channels in registers (16-byte loads and stores).
+__global__ void __launch_bounds__(1024) gated_norm_v8_kernel(
+    const float *__restrict__ y, const __nv_bfloat16 *__restrict__ z, long long zs,
+    const __nv_bfloat16 *__restrict__ w, __nv_bfloat16 *__restrict__ out, long long os, int d_inner,
+    int gs, float eps) {
+  __shared__ float red[32];
+  const long long row = blockIdx.x;
+  const int c = blockIdx.y * gs + 8 * threadIdx.x;
+  const float4 ya = __ldcs(reinterpret_cast<const float4 *>(y + row * d_inner + c));
+  const float4 yb = __ldcs(reinterpret_cast<const float4 *>(y + row * d_inner + c + 4));
+  float zv[8], g[8];
+  load8(z + row * zs + c, zv);
+  const float yv[8] = {ya.x, ya.y, ya.z, ya.w, yb.x, yb.y, yb.z, yb.w};
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    g[i] = yv[i] * silu(zv[i]);
+    ss = fmaf(g[i], g[i], ss);
+  }
+  ss = block_sum(ss, red);
+  const float r = rsqrtf(ss / gs + eps);
+  float wv[8];
+  if (w) {
+    load8(w + c, wv);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) wv[i] = 1.f;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) g[i] *= r * wv[i];
+  store8(out + row * os + c, g);
+}
+
 cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s) {
   const int gs = p.d_inner / p.norm_groups;
   dim3 grid((unsigned)((long long)p.B * p.L), p.norm_groups);
-  if (p.bf16)
+  const bool v8 = p.bf16 && gs % 256 == 0 && gs / 8 <= 1024 &&  // whole warps of 8 channels
+                  (reinterpret_cast<uintptr_t>(p.norm_w) & 15u) == 0;
+  if (v8)
+    gated_norm_v8_kernel<<<grid, gs / 8, 0, s>>>(p.yf, (const __nv_bfloat16 *)p.z, p.zs,
+                                                 (const __nv_bfloat16 *)p.norm_w, (__nv_bfloat16 *)p.y,
+                                                 p.ys, p.d_inner, gs, p.eps);
+  else if (p.bf16)
     gated_norm_kernel<__nv_bfloat16><<<grid, kNormThreads, 0, s>>>(
         p.yf, (const __nv_bfloat16 *)p.z, p.zs, (const __nv_bfloat16 *)p.norm_w,
         (__nv_bfloat16 *)p.y, p.ys, p.d_inner, gs, p.eps, p.L);
