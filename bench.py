@@ -243,14 +243,13 @@ class Ctx:
         """Times `steps` calls of step() with CUDA events on the current stream (barrier and
         synchronize on both sides), then keeps the GPU on the same step for one more second
         when the timed region was shorter, so that the clock sampler sees it under load.
+        With `trace`, a second pass of the same steps records each library launch with CUDA
+        events (for the per-kernel breakdown); the timed pass itself runs untraced.
         Returns (total ms, max over ranks), the traced kernel records, and the clocks."""
         torch = self.torch
         stream = torch.cuda.current_stream()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(steps)]
-        if trace:
-            self.ssd.trace_enable(True)
-            self.ssd.trace_read()
         if self.dist:
             self.dist.barrier()
         torch.cuda.synchronize()
@@ -263,10 +262,6 @@ class Ctx:
             ev[i][1].record(stream)
         torch.cuda.synchronize()
         t1 = time.monotonic()
-        recs = []
-        if trace:
-            self.ssd.trace_enable(False)
-            recs = self.ssd.trace_read()
         window = "timed region"
         if t1 - t0 < 1.0:
             while time.monotonic() - t1 < 1.0:
@@ -280,6 +275,17 @@ class Ctx:
         if self.dist:
             self.dist.barrier()
         ms = self.max_over_ranks(float(sum(a.elapsed_time(b) for a, b in ev)))
+        recs = []
+        if trace:
+            self.ssd.trace_enable(True)
+            self.ssd.trace_read()
+            for i in range(steps):
+                if flush:
+                    self.flush_l2(i)
+                step()
+            torch.cuda.synchronize()
+            self.ssd.trace_enable(False)
+            recs = self.ssd.trace_read()
         return ms, recs, self.clk.summary(t0, t2, window)
 
 

@@ -211,15 +211,26 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
     p.yf = c->norm_groups > 0 ? reinterpret_cast<float *>(ws + lay.tc_yf) : nullptr;
     p.seg_state = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.tc_seg_state) : nullptr;
     p.seg_decay = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.tc_seg_decay) : nullptr;
-    SSD_TRY(traced("ssd_dt_cumsum", s, [&] { return launch_dt_cumsum(p, p.dte_hm, p.cs_hm, p.Lpad, s); }));
-    SSD_TRY(traced("ssd_bc_conv", s, [&] { return launch_bc_conv_f16(p, s); }));
+    // The outgoing conv cache may be written before the scan unless it overlaps an input
+    // that later kernels read.
+    const size_t x_span = ((size_t)c->batch * c->seqlen - 1) * (size_t)a->xBC_row_stride * es + (size_t)conv_dim * es;
+    const size_t z_span = a->z ? ((size_t)c->batch * c->seqlen - 1) * (size_t)a->z_row_stride * es + (size_t)d_inner * es : 0;
+    const bool fused = front_tc_fusable(p);
+    const bool cso_early = fused && !(a->conv_state_out && (ranges_overlap(a->conv_state_out, cache_bytes, a->xBC, x_span) ||
+                                                            (a->z && ranges_overlap(a->conv_state_out, cache_bytes, a->z, z_span))));
+    if (fused) {
+      SSD_TRY(traced("ssd_front", s, [&] { return launch_front_tc(p, cso_early, s); }));
+    } else {
+      SSD_TRY(traced("ssd_dt_cumsum", s, [&] { return launch_dt_cumsum(p, p.dte_hm, p.cs_hm, p.Lpad, s); }));
+      SSD_TRY(traced("ssd_bc_conv", s, [&] { return launch_bc_conv_f16(p, s); }));
+    }
     if (p.n_seg > 1) {
       SSD_TRY(traced("ssd_scan_tc_states", s, [&] { return launch_scan_tc(p, 1, s); }));
       SSD_TRY(traced("ssd_state_pass", s, [&] { return launch_state_pass(p, s); }));
     }
     SSD_TRY(traced("ssd_scan_tc", s, [&] { return launch_scan_tc(p, 0, s); }));
     if (p.norm_groups > 0) SSD_TRY(traced("ssd_gated_norm", s, [&] { return launch_gated_norm(p, s); }));
-    SSD_TRY(traced("ssd_conv_state_out", s, [&] { return launch_conv_state_out(p, s); }));
+    if (!cso_early) SSD_TRY(traced("ssd_conv_state_out", s, [&] { return launch_conv_state_out(p, s); }));
     return SSD_OK;
   }
 

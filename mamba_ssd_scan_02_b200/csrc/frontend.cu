@@ -6,6 +6,7 @@
 // inputs before the first token come from the incoming cache (row W-1 = the newest).  This is
 // the Mamba-2 short convolution of window 4 in the Nemotron Nano 2 layers ("NVIDIA Nemotron
 // Nano 2" summary, section "Method").
+#include <algorithm>
 #include <type_traits>
 
 #include "common.cuh"
@@ -107,17 +108,17 @@ __global__ void dt_kernel(const T *__restrict__ dt, long long ds, const float *_
 // stays flat).  One CTA: one 128-token chunk x 8 heads of one batch row.  Thread t reads the
 // 8 heads of token t (16 bytes for bf16 when H % 8 == 0, else element by element), the tile
 // is transposed through shared memory, and each warp scans two heads.
+// The tile body: 128 threads (tid 0..127) and a 128 x 9 shared tile; every thread of the
+// CTA must call it (it synchronises the CTA once), an inactive tile skips the work.
 template <typename T>
-__global__ void __launch_bounds__(128) dt_cumsum_kernel(const T *__restrict__ dt, long long ds,
-                                                         const float *__restrict__ bias,
-                                                         const float *__restrict__ A,
-                                                         float *__restrict__ dte,
-                                                         float *__restrict__ cs, int L, int H,
-                                                         int Lpad, int sp, float lo, float hi) {
-  __shared__ float v[128][9];
-  const int c0 = blockIdx.x * 128, h0 = blockIdx.y * 8, b = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  {
+__device__ __forceinline__ void dt_cumsum_tile(const T *__restrict__ dt, long long ds,
+                                               const float *__restrict__ bias,
+                                               const float *__restrict__ A, float *__restrict__ dte,
+                                               float *__restrict__ cs, int L, int H, int Lpad, int sp,
+                                               float lo, float hi, int c0, int h0, int b, int tid,
+                                               float (*v)[9], bool active) {
+  const int warp = tid / 32, lane = tid % 32;
+  if (active) {
     const int tt = c0 + tid;
     float raw[8];
     const T *row = dt + ((long long)b * L + tt) * ds + h0;
@@ -132,6 +133,7 @@ __global__ void __launch_bounds__(128) dt_cumsum_kernel(const T *__restrict__ dt
       v[tid][j] = (tt < L && h0 + j < H) ? effective_dt(raw[j], bias[h0 + j], sp, lo, hi) : 0.f;
   }
   __syncthreads();
+  if (!active) return;
 #pragma unroll
   for (int jj = 0; jj < 2; ++jj) {
     const int j = 2 * warp + jj, h = h0 + j;
@@ -159,17 +161,29 @@ __global__ void __launch_bounds__(128) dt_cumsum_kernel(const T *__restrict__ dt
   }
 }
 
+template <typename T>
+__global__ void __launch_bounds__(128) dt_cumsum_kernel(const T *__restrict__ dt, long long ds,
+                                                         const float *__restrict__ bias,
+                                                         const float *__restrict__ A,
+                                                         float *__restrict__ dte,
+                                                         float *__restrict__ cs, int L, int H,
+                                                         int Lpad, int sp, float lo, float hi) {
+  __shared__ float v[128][9];
+  dt_cumsum_tile<T>(dt, ds, bias, A, dte, cs, L, H, Lpad, sp, lo, hi, blockIdx.x * 128, blockIdx.y * 8,
+                    blockIdx.z, threadIdx.x, v, true);
+}
+
 // conv_state_out[b, k, :] = raw input of time L-W+k (from the incoming cache when negative).
 // Copies 16-byte words without conversion, so the carried cache is bit-exact.
 template <int ELT>
-__global__ void conv_state_out_kernel(const char *__restrict__ xBC, long long xs_bytes,
-                                      const char *__restrict__ csi, char *__restrict__ cso, int B,
-                                      int L, int W, int C) {
+__device__ __forceinline__ void conv_state_out_range(const char *__restrict__ xBC, long long xs_bytes,
+                                                     const char *__restrict__ csi, char *__restrict__ cso,
+                                                     int B, int L, int W, int C, long long i0,
+                                                     long long stride) {
   const long long row_bytes = (long long)C * ELT;
   const long long vec_per_row = row_bytes / 16;
   const long long n = (long long)B * W * vec_per_row;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
-       i += (long long)gridDim.x * blockDim.x) {
+  for (long long i = i0; i < n; i += stride) {
     const long long v = i % vec_per_row;
     const int k = (int)((i / vec_per_row) % W);
     const int b = (int)(i / (vec_per_row * W));
@@ -181,6 +195,15 @@ __global__ void conv_state_out_kernel(const char *__restrict__ xBC, long long xs
       val = *reinterpret_cast<const uint4 *>(csi + ((long long)b * W + (W + tau)) * row_bytes + v * 16);
     *reinterpret_cast<uint4 *>(cso + ((long long)b * W + k) * row_bytes + v * 16) = val;
   }
+}
+
+template <int ELT>
+__global__ void conv_state_out_kernel(const char *__restrict__ xBC, long long xs_bytes,
+                                      const char *__restrict__ csi, char *__restrict__ cso, int B,
+                                      int L, int W, int C) {
+  conv_state_out_range<ELT>(xBC, xs_bytes, csi, cso, B, L, W, C,
+                            blockIdx.x * (long long)blockDim.x + threadIdx.x,
+                            (long long)gridDim.x * blockDim.x);
 }
 
 // seqlen == 0: the state passes through unchanged and so does the conv cache.
@@ -260,17 +283,17 @@ __device__ __forceinline__ void unpack4(const uint2 &r, float (&v)[4]) {
 }
 
 template <int W>
-__global__ void __launch_bounds__(kBcThreads) bc_conv_kernel(const __nv_bfloat16 *__restrict__ xBC, long long xs,
-                                                             const __nv_bfloat16 *__restrict__ csi,
-                                                             const __nv_bfloat16 *__restrict__ w,
-                                                             const __nv_bfloat16 *__restrict__ bias,
-                                                             __half *__restrict__ out, int L, int conv_dim,
-                                                             int c_begin, int C_out) {
-  const int o4 = (blockIdx.x * kBcThreads + threadIdx.x) * 4;
+__device__ __forceinline__ void bc_conv_tile(const __nv_bfloat16 *__restrict__ xBC, long long xs,
+                                             const __nv_bfloat16 *__restrict__ csi,
+                                             const __nv_bfloat16 *__restrict__ w,
+                                             const __nv_bfloat16 *__restrict__ bias,
+                                             __half *__restrict__ out, int L, int conv_dim, int c_begin,
+                                             int C_out, int bx, int by, int bz) {
+  const int o4 = (bx * kBcThreads + threadIdx.x) * 4;
   if (o4 >= C_out) return;
   const int c4 = c_begin + o4;
-  const int b = blockIdx.z;
-  const int t0 = blockIdx.y * kBcTok;
+  const int b = bz;
+  const int t0 = by * kBcTok;
   const int t1 = min(L, t0 + kBcTok);
   const __nv_bfloat16 *xrow = xBC + (long long)b * L * xs + c4;
   float wt[4][4], bs[4];
@@ -342,6 +365,56 @@ __global__ void __launch_bounds__(kBcThreads) bc_conv_kernel(const __nv_bfloat16
   }
 }
 
+template <int W>
+__global__ void __launch_bounds__(kBcThreads) bc_conv_kernel(const __nv_bfloat16 *__restrict__ xBC, long long xs,
+                                                             const __nv_bfloat16 *__restrict__ csi,
+                                                             const __nv_bfloat16 *__restrict__ w,
+                                                             const __nv_bfloat16 *__restrict__ bias,
+                                                             __half *__restrict__ out, int L, int conv_dim,
+                                                             int c_begin, int C_out) {
+  bc_conv_tile<W>(xBC, xs, csi, w, bias, out, L, conv_dim, c_begin, C_out, blockIdx.x, blockIdx.y, blockIdx.z);
+}
+
+// The tensor-core path's front end in one launch: dt + chunk prefix sums, the outgoing conv
+// cache and the B/C conv, each CTA taking one role by its index (the latency-bound dt and
+// cache CTAs first, so that they overlap the streaming B/C conv).
+struct FrontArgs {
+  const __nv_bfloat16 *xBC, *dt, *csi, *conv_w, *conv_b;
+  long long xs, ds;
+  const float *dt_bias, *A;
+  float *dte, *cs;
+  __half *bc;
+  __nv_bfloat16 *cso;
+  int B, L, H, Lpad, conv_dim, d_inner, C_out, W, sp;
+  float lo, hi;
+  int n_dt, dt_tiles, dt_nch, dt_nhg, n_cso, gx, gy;
+};
+
+template <int W>
+__global__ void __launch_bounds__(kBcThreads) front_tc_kernel(const FrontArgs f) {
+  __shared__ float v[2][128][9];
+  int j = blockIdx.x;
+  if (j < f.n_dt) {  // two 128-thread dt tiles per CTA
+    const int half = threadIdx.x >> 7, q = 2 * j + half;
+    const bool active = q < f.dt_tiles;
+    const int qq = active ? q : 0;
+    const int cx = qq % f.dt_nch, hy = (qq / f.dt_nch) % f.dt_nhg, b = qq / (f.dt_nch * f.dt_nhg);
+    dt_cumsum_tile<__nv_bfloat16>(f.dt, f.ds, f.dt_bias, f.A, f.dte, f.cs, f.L, f.H, f.Lpad, f.sp, f.lo,
+                                  f.hi, cx * 128, hy * 8, b, threadIdx.x & 127, v[half], active);
+    return;
+  }
+  j -= f.n_dt;
+  if (j < f.n_cso) {
+    conv_state_out_range<2>((const char *)f.xBC, f.xs * 2, (const char *)f.csi, (char *)f.cso, f.B, f.L,
+                            f.W, f.conv_dim, j * (long long)kBcThreads + threadIdx.x,
+                            (long long)f.n_cso * kBcThreads);
+    return;
+  }
+  j -= f.n_cso;
+  bc_conv_tile<W>(f.xBC, f.xs, f.csi, f.conv_w, f.conv_b, f.bc, f.L, f.conv_dim, f.d_inner, f.C_out,
+                  j % f.gx, (j / f.gx) % f.gy, j / (f.gx * f.gy));
+}
+
 cudaError_t launch_bc_conv_f16(const PrefillPlan &p, cudaStream_t s) {
   const int C_out = 2 * p.G * p.N;
   if (C_out % 4 || p.xs % 4 || p.conv_dim % 4 || p.d_inner % 4) {  // 8-byte accesses; else the generic kernel
@@ -360,6 +433,36 @@ cudaError_t launch_bc_conv_f16(const PrefillPlan &p, cudaStream_t s) {
     case 2: bc_conv_kernel<2><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
     case 3: bc_conv_kernel<3><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
     default: bc_conv_kernel<4><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
+  }
+  return cudaGetLastError();
+}
+
+// False when the shapes need the separate front-end kernels (unaligned 8-byte B/C accesses).
+bool front_tc_fusable(const PrefillPlan &p) {
+  return p.bf16 && (2 * p.G * p.N) % 4 == 0 && p.xs % 4 == 0 && p.conv_dim % 4 == 0 && p.d_inner % 4 == 0 &&
+         p.H % 8 == 0 && p.ds % 8 == 0;
+}
+
+cudaError_t launch_front_tc(const PrefillPlan &p, bool with_cso, cudaStream_t s) {
+  FrontArgs f{};
+  f.xBC = (const __nv_bfloat16 *)p.xBC; f.dt = (const __nv_bfloat16 *)p.dt;
+  f.csi = (const __nv_bfloat16 *)p.csi; f.conv_w = (const __nv_bfloat16 *)p.conv_w;
+  f.conv_b = (const __nv_bfloat16 *)p.conv_b; f.xs = p.xs; f.ds = p.ds; f.dt_bias = p.dt_bias; f.A = p.A;
+  f.dte = p.dte_hm; f.cs = p.cs_hm; f.bc = (__half *)p.bc; f.cso = (__nv_bfloat16 *)p.cso;
+  f.B = p.B; f.L = p.L; f.H = p.H; f.Lpad = p.Lpad; f.conv_dim = p.conv_dim; f.d_inner = p.d_inner;
+  f.C_out = 2 * p.G * p.N; f.W = p.W; f.sp = p.softplus; f.lo = p.dt_min; f.hi = p.dt_max;
+  f.dt_nch = p.Lpad / 128; f.dt_nhg = (p.H + 7) / 8; f.dt_tiles = f.dt_nch * f.dt_nhg * p.B;
+  f.n_dt = (f.dt_tiles + 1) / 2;
+  const long long ncso = (with_cso && p.cso && p.W > 0) ? (long long)p.B * p.W * ((long long)p.conv_dim * 2 / 16) : 0;
+  f.n_cso = ncso ? (int)std::min<long long>((ncso + kBcThreads - 1) / kBcThreads, 64) : 0;
+  f.gx = (f.C_out / 4 + kBcThreads - 1) / kBcThreads; f.gy = (p.L + kBcTok - 1) / kBcTok;
+  const long long blocks = (long long)f.n_dt + f.n_cso + (long long)f.gx * f.gy * p.B;
+  switch (p.W) {
+    case 0: front_tc_kernel<0><<<(unsigned)blocks, kBcThreads, 0, s>>>(f); break;
+    case 1: front_tc_kernel<1><<<(unsigned)blocks, kBcThreads, 0, s>>>(f); break;
+    case 2: front_tc_kernel<2><<<(unsigned)blocks, kBcThreads, 0, s>>>(f); break;
+    case 3: front_tc_kernel<3><<<(unsigned)blocks, kBcThreads, 0, s>>>(f); break;
+    default: front_tc_kernel<4><<<(unsigned)blocks, kBcThreads, 0, s>>>(f); break;
   }
   return cudaGetLastError();
 }

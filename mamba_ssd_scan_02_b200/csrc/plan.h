@@ -61,7 +61,10 @@ cudaError_t launch_conv_silu_f32(const PrefillPlan &p, cudaStream_t s);
 cudaError_t launch_dt(const PrefillPlan &p, cudaStream_t s);
 cudaError_t launch_conv_state_out(const PrefillPlan &p, cudaStream_t s);
 cudaError_t launch_carry_only(const PrefillPlan &p, cudaStream_t s);  // seqlen == 0
-cudaError_t launch_bc_conv_f16(const PrefillPlan &p, cudaStream_t s);  // B|C channels -> p.bc (fp16)
+cudaError_t launch_bc_conv_f16(const PrefillPlan &p, cudaStream_t s);
+// dt + prefix sums, B/C conv and (if with_cso) the outgoing conv cache in one launch
+bool front_tc_fusable(const PrefillPlan &p);
+cudaError_t launch_front_tc(const PrefillPlan &p, bool with_cso, cudaStream_t s);  // B|C channels -> p.bc (fp16)
 cudaError_t launch_dt_cumsum(const PrefillPlan &p, float *dte, float *cs, int Lpad, cudaStream_t s);
 // chunked scan on CUDA cores (scan_simt.cu); mode 0 full, 1 state-only, 2 output-only
 cudaError_t launch_scan_simt(const PrefillPlan &p, int mode, cudaStream_t s);
