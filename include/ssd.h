@@ -85,6 +85,8 @@ typedef struct {
   int n_segments;   /* 0 = library choice; else split each sequence into this many segments
                        scanned in parallel and joined by the inter-segment state pass */
   ssd_kernel_t kernel;
+  int norm_before_gate; /* 0: out = rmsnorm(y * silu(z)) * w (gate first, the default);
+                           1: out = rmsnorm(y) * w * silu(z) (normalise first) */
 } ssd_config_t;
 
 typedef struct {

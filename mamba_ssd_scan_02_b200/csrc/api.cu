@@ -52,6 +52,7 @@ ssd_status_t check_config(const ssd_config_t *c, bool prefill) {
     return SSD_ERR_INVALID_ARG;
   if (!(c->norm_eps >= 0.f) || !(c->dt_min <= c->dt_max) || isnan(c->dt_min)) return SSD_ERR_INVALID_ARG;
   if (c->n_segments < 0) return SSD_ERR_INVALID_ARG;
+  if (c->norm_before_gate != 0 && c->norm_before_gate != 1) return SSD_ERR_INVALID_ARG;
   if (c->kernel != SSD_KERNEL_AUTO && c->kernel != SSD_KERNEL_SIMT && c->kernel != SSD_KERNEL_TENSOR)
     return SSD_ERR_INVALID_ARG;
   if (c->batch > 65535 || c->nheads > 65535 || c->seqlen > (1 << 21))
@@ -177,6 +178,7 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
   PrefillPlan p{};
   p.B = c->batch; p.L = c->seqlen; p.H = H; p.P = P; p.N = N; p.G = G; p.Q = c->chunk; p.W = W;
   p.norm_groups = c->norm_groups; p.hpg = H / G; p.d_inner = (int)d_inner; p.conv_dim = (int)conv_dim;
+  p.nbg = c->norm_before_gate;
   p.eps = c->norm_eps; p.dt_min = c->dt_min; p.dt_max = c->dt_max; p.softplus = c->dt_softplus;
   p.bf16 = c->io_dtype == SSD_BF16;
   p.xBC = a->xBC; p.xs = a->xBC_row_stride; p.dt = a->dt; p.ds = a->dt_row_stride;
@@ -281,6 +283,7 @@ ssd_status_t run_decode(const ssd_config_t *c, const ssd_decode_args_t *a, cudaS
   DecodePlan p{};
   p.B = c->batch; p.H = H; p.P = P; p.N = N; p.G = G; p.W = W; p.norm_groups = c->norm_groups;
   p.hpg = H / G; p.d_inner = (int)d_inner; p.conv_dim = (int)conv_dim; p.eps = c->norm_eps;
+  p.nbg = c->norm_before_gate;
   p.dt_min = c->dt_min; p.dt_max = c->dt_max; p.softplus = c->dt_softplus;
   p.bf16 = c->io_dtype == SSD_BF16;
   p.xBC = a->xBC; p.xs = a->xBC_row_stride; p.dt = a->dt; p.ds = a->dt_row_stride; p.z = a->z;

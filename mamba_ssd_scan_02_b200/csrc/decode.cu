@@ -140,8 +140,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodePlan p) {
   const T *zr = reinterpret_cast<const T *>(p.z) + (long long)b * p.zs + g * nx;
   const int sub = p.norm_groups / p.G;  // norm groups inside this SSM group
   const int gs = nx / sub;
-  for (int i = tid; i < nx; i += kDecThreads) ys[i] *= silu(io<T>::ld(zr + i));
-  __syncthreads();
+  if (!p.nbg) {  // gate first (the default); else normalise y first and gate below
+    for (int i = tid; i < nx; i += kDecThreads) ys[i] *= silu(io<T>::ld(zr + i));
+    __syncthreads();
+  }
   for (int k = 0; k < sub; ++k) {
     float ss = 0.f;
     for (int i = tid; i < gs; i += kDecThreads) ss += ys[k * gs + i] * ys[k * gs + i];
@@ -159,7 +161,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodePlan p) {
     const T *wr = reinterpret_cast<const T *>(p.norm_w);
     for (int i = tid; i < gs; i += kDecThreads) {
       const int c = k * gs + i;
-      io<T>::st(yout + c, ys[c] * r * (wr ? io<T>::ld(wr + g * nx + c) : 1.f));
+      const float gate = p.nbg ? silu(io<T>::ld(zr + c)) : 1.f;
+      io<T>::st(yout + c, ys[c] * r * (wr ? io<T>::ld(wr + g * nx + c) : 1.f) * gate);
     }
   }
 }

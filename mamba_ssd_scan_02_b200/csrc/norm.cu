@@ -3,6 +3,8 @@
 // summary, section "Method"); in the Mamba-2 mixer the scan output is gated by SiLU(z) and
 // then normalised over groups of d_inner / norm_groups consecutive channels:
 //   g = y * silu(z);   out = g / sqrt(mean_group(g^2) + eps) * w
+// or, normalising before the gate (the norm_before_gate variant):
+//   out = y / sqrt(mean_group(y^2) + eps) * w * silu(z)
 #include <stdint.h>
 
 #include "common.cuh"
@@ -32,7 +34,7 @@ __device__ float block_sum(float v, float *red) {
 template <typename T>
 __global__ void __launch_bounds__(kNormThreads) gated_norm_kernel(
     const float *__restrict__ y, const T *__restrict__ z, long long zs, const T *__restrict__ w,
-    T *__restrict__ out, long long os, int d_inner, int gs, float eps, int L) {
+    T *__restrict__ out, long long os, int d_inner, int gs, float eps, int L, int nbg) {
   __shared__ float red[32];
   const long long row = blockIdx.x;
   const int c0 = blockIdx.y * gs;
@@ -40,38 +42,16 @@ __global__ void __launch_bounds__(kNormThreads) gated_norm_kernel(
   const T *zr = z + row * zs + c0;
   float ss = 0.f;
   for (int i = threadIdx.x; i < gs; i += kNormThreads) {
-    const float gv = yr[i] * silu(io<T>::ld(zr + i));
+    const float gv = nbg ? yr[i] : yr[i] * silu(io<T>::ld(zr + i));
     ss += gv * gv;
   }
   ss = block_sum(ss, red);
   const float r = rsqrtf(ss / gs + eps);
   T *orow = out + row * os + c0;
   for (int i = threadIdx.x; i < gs; i += kNormThreads) {
-    const float gv = yr[i] * silu(io<T>::ld(zr + i));
-    io<T>::st(orow + i, gv * r * (w ? io<T>::ld(w + c0 + i) : 1.f));
-  }
-}
-
-// In place on the scan output stored in the io dtype (tensor-core path).
-template <typename T>
-__global__ void __launch_bounds__(kNormThreads) gated_norm_inplace_kernel(
-    T *__restrict__ y, long long ys, const T *__restrict__ z, long long zs, const T *__restrict__ w,
-    int gs, float eps) {
-  __shared__ float red[32];
-  const long long row = blockIdx.x;
-  const int c0 = blockIdx.y * gs;
-  T *yr = y + row * ys + c0;
-  const T *zr = z + row * zs + c0;
-  float ss = 0.f;
-  for (int i = threadIdx.x; i < gs; i += kNormThreads) {
-    const float gv = io<T>::ld(yr + i) * silu(io<T>::ld(zr + i));
-    ss += gv * gv;
-  }
-  ss = block_sum(ss, red);
-  const float r = rsqrtf(ss / gs + eps);
-  for (int i = threadIdx.x; i < gs; i += kNormThreads) {
-    const float gv = io<T>::ld(yr + i) * silu(io<T>::ld(zr + i));
-    io<T>::st(yr + i, gv * r * (w ? io<T>::ld(w + c0 + i) : 1.f));
+    const float sz = silu(io<T>::ld(zr + i));
+    const float gv = nbg ? yr[i] : yr[i] * sz;
+    io<T>::st(orow + i, gv * r * (w ? io<T>::ld(w + c0 + i) : 1.f) * (nbg ? sz : 1.f));
   }
 }
 
@@ -107,7 +87,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_bf16_kernel(
 __global__ void __launch_bounds__(1024) gated_norm_v8_kernel(
     const float *__restrict__ y, const __nv_bfloat16 *__restrict__ z, long long zs,
     const __nv_bfloat16 *__restrict__ w, __nv_bfloat16 *__restrict__ out, long long os, int d_inner,
-    int gs, float eps) {
+    int gs, float eps, int nbg) {
   __shared__ float red[32];
   const long long row = blockIdx.x;
   const int c = blockIdx.y * gs + 8 * threadIdx.x;
@@ -119,7 +99,8 @@ __global__ void __launch_bounds__(1024) gated_norm_v8_kernel(
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    g[i] = yv[i] * silu(zv[i]);
+    zv[i] = silu(zv[i]);
+    g[i] = nbg ? yv[i] : yv[i] * zv[i];
     ss = fmaf(g[i], g[i], ss);
   }
   ss = block_sum(ss, red);
@@ -132,7 +113,7 @@ __global__ void __launch_bounds__(1024) gated_norm_v8_kernel(
     for (int i = 0; i < 8; ++i) wv[i] = 1.f;
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) g[i] *= r * wv[i];
+  for (int i = 0; i < 8; ++i) g[i] *= r * wv[i] * (nbg ? zv[i] : 1.f);
   store8(out + row * os + c, g);
 }
 
@@ -144,30 +125,18 @@ cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s) {
   if (v8)
     gated_norm_v8_kernel<<<grid, gs / 8, 0, s>>>(p.yf, (const __nv_bfloat16 *)p.z, p.zs,
                                                  (const __nv_bfloat16 *)p.norm_w, (__nv_bfloat16 *)p.y,
-                                                 p.ys, p.d_inner, gs, p.eps);
+                                                 p.ys, p.d_inner, gs, p.eps, p.nbg);
   else if (p.bf16)
     gated_norm_kernel<__nv_bfloat16><<<grid, kNormThreads, 0, s>>>(
         p.yf, (const __nv_bfloat16 *)p.z, p.zs, (const __nv_bfloat16 *)p.norm_w,
-        (__nv_bfloat16 *)p.y, p.ys, p.d_inner, gs, p.eps, p.L);
+        (__nv_bfloat16 *)p.y, p.ys, p.d_inner, gs, p.eps, p.L, p.nbg);
   else
     gated_norm_kernel<float><<<grid, kNormThreads, 0, s>>>(p.yf, (const float *)p.z, p.zs,
                                                            (const float *)p.norm_w, (float *)p.y,
-                                                           p.ys, p.d_inner, gs, p.eps, p.L);
+                                                           p.ys, p.d_inner, gs, p.eps, p.L, p.nbg);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gated_norm_inplace(const PrefillPlan &p, cudaStream_t s) {
-  const int gs = p.d_inner / p.norm_groups;
-  dim3 grid((unsigned)((long long)p.B * p.L), p.norm_groups);
-  if (p.bf16)
-    gated_norm_inplace_kernel<__nv_bfloat16><<<grid, kNormThreads, 0, s>>>(
-        (__nv_bfloat16 *)p.y, p.ys, (const __nv_bfloat16 *)p.z, p.zs,
-        (const __nv_bfloat16 *)p.norm_w, gs, p.eps);
-  else
-    gated_norm_inplace_kernel<float><<<grid, kNormThreads, 0, s>>>(
-        (float *)p.y, p.ys, (const float *)p.z, p.zs, (const float *)p.norm_w, gs, p.eps);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_rmsnorm_bf16(const void *x, const void *w, void *out, long long rows, int width,
                                 float eps, cudaStream_t s) {

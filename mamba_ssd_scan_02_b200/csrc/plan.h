@@ -11,6 +11,7 @@ namespace ssd {
 // Everything a prefill launch needs, after validation: shapes, pointers, workspace carve-outs.
 struct PrefillPlan {
   int B, L, H, P, N, G, Q, W, norm_groups;
+  int nbg;           // 1: normalise before gating (out = rmsnorm(y) * w * silu(z))
   int hpg, d_inner, conv_dim;
   float eps, dt_min, dt_max;
   int softplus;
@@ -42,6 +43,7 @@ struct PrefillPlan {
 
 struct DecodePlan {
   int B, H, P, N, G, W, norm_groups, hpg, d_inner, conv_dim;
+  int nbg;           // 1: normalise before gating
   float eps, dt_min, dt_max;
   int softplus;
   bool bf16;
@@ -75,7 +77,6 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s);
 cudaError_t launch_state_pass(const PrefillPlan &p, cudaStream_t s);
 // norms (norm.cu)
 cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s);          // fp32 yf -> y
-cudaError_t launch_gated_norm_inplace(const PrefillPlan &p, cudaStream_t s);  // y (io dtype) in place
 cudaError_t launch_rmsnorm_bf16(const void *x, const void *w, void *out, long long rows, int width,
                                 float eps, cudaStream_t s);
 // decode (decode.cu)

@@ -42,7 +42,7 @@ class SsdConfig(ctypes.Structure):
                 ("dstate", c_int), ("ngroups", c_int), ("chunk", c_int), ("conv_width", c_int),
                 ("norm_groups", c_int), ("norm_eps", c_float), ("dt_min", c_float),
                 ("dt_max", c_float), ("dt_softplus", c_int), ("io_dtype", c_int),
-                ("n_segments", c_int), ("kernel", c_int)]
+                ("n_segments", c_int), ("kernel", c_int), ("norm_before_gate", c_int)]
 
 
 class PrefillArgs(ctypes.Structure):
@@ -134,7 +134,8 @@ def make_config(cfg: dict, seqlen: int | None = None, kernel: int | None = None)
         dt_softplus=int(cfg.get("dt_softplus", True)),
         io_dtype=SSD_BF16 if dtype == "bf16" else SSD_F32,
         n_segments=cfg.get("n_segments", 0),
-        kernel=cfg.get("kernel", KERNEL_AUTO) if kernel is None else kernel)
+        kernel=cfg.get("kernel", KERNEL_AUTO) if kernel is None else kernel,
+        norm_before_gate=int(cfg.get("norm_before_gate", False)))
 
 
 def _ptr(t):

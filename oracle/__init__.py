@@ -113,7 +113,7 @@ class Oracle:
         L.oracle_ssd_prefill.argtypes = [ctypes.POINTER(_Shape), vp, ci, cll, vp, ci, cll, vp, vp,
                                          vp, ci, vp, vp, ci, vp, ci, vp, ci, ci, ci, vp, vp, ci]
         L.oracle_gated_rmsnorm.restype = None
-        L.oracle_gated_rmsnorm.argtypes = [cll, ci, ci, vp, vp, ci, cll, vp, ci, cd, vp]
+        L.oracle_gated_rmsnorm.argtypes = [cll, ci, ci, vp, vp, ci, cll, vp, ci, cd, ci, vp]
         L.oracle_rmsnorm.restype = None
         L.oracle_rmsnorm.argtypes = [cll, ci, vp, ci, vp, ci, cd, vp]
         L.oracle_decode_step.restype = None
@@ -205,7 +205,8 @@ class Oracle:
                 y.reshape(Bn * L, nh * P), None if z is None else
                 np.ascontiguousarray(zz).reshape(Bn * L, nh * P),
                 None if norm_w is None else np.ascontiguousarray(norm_w)[lo * P:hi * P],
-                ngroups=nh * P // gs, eps=cfg.get("norm_eps", 1e-5)).reshape(Bn, L, nh * P)
+                ngroups=nh * P // gs, eps=cfg.get("norm_eps", 1e-5),
+                norm_before_gate=cfg.get("norm_before_gate", False)).reshape(Bn, L, nh * P)
         if lo == 0 and W > 0:
             raw = xBC.reshape(Bn, L, -1)[:, :, :conv_dim]
             res["conv_state_out"] = self.conv_state_after(raw, conv_state_in, W)
@@ -219,7 +220,8 @@ class Oracle:
         return np.ascontiguousarray(np.concatenate([hist.astype(raw.dtype), raw], axis=1)[:, -W:])
 
     # ---- norms ------------------------------------------------------------------------------
-    def gated_rmsnorm(self, y: np.ndarray, z, w, ngroups: int, eps: float = 1e-5) -> np.ndarray:
+    def gated_rmsnorm(self, y: np.ndarray, z, w, ngroups: int, eps: float = 1e-5,
+                      norm_before_gate: bool = False) -> np.ndarray:
         y = np.ascontiguousarray(y, dtype=np.float64)
         T, Dn = y.shape
         z = None if z is None else np.ascontiguousarray(z)
@@ -227,7 +229,7 @@ class Oracle:
         out = np.empty_like(y)
         self.lib.oracle_gated_rmsnorm(T, Dn, ngroups, _p(y), _p(z), _code(z) if z is not None else 0,
                                       Dn, _p(w), _code(w) if w is not None else 0, float(eps),
-                                      _p(out))
+                                      int(bool(norm_before_gate)), _p(out))
         return out
 
     def rmsnorm(self, x: np.ndarray, w, eps: float = 1e-5) -> np.ndarray:
@@ -274,7 +276,8 @@ class Oracle:
             res["out"] = self.gated_rmsnorm(
                 y.reshape(Bn, nh * P), zz,
                 None if norm_w is None else np.ascontiguousarray(norm_w)[lo * P:hi * P],
-                ngroups=nh * P // gs, eps=cfg.get("norm_eps", 1e-5))
+                ngroups=nh * P // gs, eps=cfg.get("norm_eps", 1e-5),
+                norm_before_gate=cfg.get("norm_before_gate", False))
         return res
 
     # ---- full mixer layer ---------------------------------------------------------------------

@@ -229,12 +229,16 @@ void oracle_ssd_prefill(const oracle_shape_t *s, const void *xBC, int xdt, long 
 
 /*
  * z-gated RMSNorm over rows of width Dn split into ngroups groups of Dn/ngroups
- * consecutive channels: g = y * silu(z); out = g / sqrt(mean(g^2) + eps) * w.
- * y, out: fp64 [T, Dn]; z [T, Dn] with row stride z_stride (NULL = no gate,
- * g = y); w [Dn] (NULL = ones).
+ * consecutive channels.  Gate first (norm_before_gate = 0):
+ *   g = y * silu(z);  out = g / sqrt(mean(g^2) + eps) * w.
+ * Normalise first (norm_before_gate = 1):
+ *   out = y / sqrt(mean(y^2) + eps) * w * silu(z).
+ * y, out: fp64 [T, Dn]; z [T, Dn] with row stride z_stride (NULL = no gate); w [Dn]
+ * (NULL = ones).
  */
 void oracle_gated_rmsnorm(long long T, int Dn, int ngroups, const double *y, const void *z, int zdt,
-                          long long z_stride, const void *w, int wdt, double eps, double *out) {
+                          long long z_stride, const void *w, int wdt, double eps, int norm_before_gate,
+                          double *out) {
   const int gs = Dn / ngroups;
   double *g = (double *)malloc(sizeof(double) * gs);
   for (long long t = 0; t < T; ++t)
@@ -243,13 +247,14 @@ void oracle_gated_rmsnorm(long long T, int Dn, int ngroups, const double *y, con
       for (int i = 0; i < gs; ++i) {
         const int c = k * gs + i;
         const double gate = z ? oracle_silu(ld(z, zdt, t * z_stride + c)) : 1.0;
-        g[i] = y[t * Dn + c] * gate;
+        g[i] = norm_before_gate ? y[t * Dn + c] : y[t * Dn + c] * gate;
         ss += g[i] * g[i];
       }
       const double r = 1.0 / sqrt(ss / gs + eps);
       for (int i = 0; i < gs; ++i) {
         const int c = k * gs + i;
-        out[t * Dn + c] = g[i] * r * (w ? ld(w, wdt, c) : 1.0);
+        const double gate = (norm_before_gate && z) ? oracle_silu(ld(z, zdt, t * z_stride + c)) : 1.0;
+        out[t * Dn + c] = g[i] * r * (w ? ld(w, wdt, c) : 1.0) * gate;
       }
     }
   free(g);

