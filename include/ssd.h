@@ -152,6 +152,20 @@ size_t ssd_workspace_size(const ssd_config_t *cfg);
  * call's h_final and conv_state_out, gives the same result as one call (up to rounding). */
 ssd_status_t ssd_prefill(const ssd_config_t *cfg, const ssd_prefill_args_t *args, void *stream);
 
+/* Variable-length batch: nseq sequences packed back to back along the token axis, each with
+ * its own initial state and conv cache (the state is reset at every sequence boundary).
+ *  cu_seqlens: HOST array of nseq + 1 non-decreasing offsets, cu_seqlens[0] = 0; sequence i
+ *    is packed tokens [cu_seqlens[i], cu_seqlens[i+1]) (an empty sequence copies its carries).
+ *  cfg: batch = 1 and seqlen = cu_seqlens[nseq] (all tokens); the token tensors of args
+ *    (xBC, dt, z, y) are the packed [seqlen, ...] rows; h0 / h_final are [nseq, H, P, N] and
+ *    conv_state_in / conv_state_out [nseq, W, conv_dim] (NULL as in ssd_prefill).
+ *  workspace: at least ssd_varlen_workspace_size(cfg, cu_seqlens, nseq) bytes.
+ * Runs the prefill of each sequence in turn on `stream`; returns the first error (argument
+ * errors, including inconsistent offsets, as SSD_ERR_INVALID_ARG). */
+size_t ssd_varlen_workspace_size(const ssd_config_t *cfg, const int *cu_seqlens, int nseq);
+ssd_status_t ssd_prefill_varlen(const ssd_config_t *cfg, const ssd_prefill_args_t *args,
+                                const int *cu_seqlens, int nseq, void *stream);
+
 /* One token per batch row: conv-cache shift + conv + SiLU, softplus dt, the state update
  * h = exp(dt A) h + dt x B^T (fp32 state in place), y = h C + D x, optional gated RMSNorm.
  * cfg->seqlen and cfg->chunk are ignored.  norm_groups must be 0 or a multiple of ngroups. */

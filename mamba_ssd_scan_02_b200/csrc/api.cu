@@ -391,6 +391,59 @@ ssd_status_t ssd_decode_step(const ssd_config_t *cfg, const ssd_decode_args_t *a
   return run_decode(cfg, args, static_cast<cudaStream_t>(stream));
 }
 
+// Variable-length batch: each packed sequence is one batch-1 prefill on the same stream,
+// its token tensors addressed at the sequence's first row and its carries at its index.
+static bool varlen_ok(const ssd_config_t *cfg, const int *cu, int nseq) {
+  if (!cfg || !cu || nseq < 1 || cfg->batch != 1 || cu[0] != 0 || cu[nseq] != cfg->seqlen) return false;
+  for (int i = 0; i < nseq; ++i)
+    if (cu[i + 1] < cu[i]) return false;
+  return true;
+}
+
+size_t ssd_varlen_workspace_size(const ssd_config_t *cfg, const int *cu_seqlens, int nseq) {
+  if (!varlen_ok(cfg, cu_seqlens, nseq) || check_config(cfg, true) != SSD_OK) return 0;
+  size_t ws = 0;
+  for (int i = 0; i < nseq; ++i) {
+    ssd_config_t c = *cfg;
+    c.seqlen = cu_seqlens[i + 1] - cu_seqlens[i];
+    const size_t w = prefill_layout(&c).total;
+    ws = w > ws ? w : ws;
+  }
+  return ws;
+}
+
+ssd_status_t ssd_prefill_varlen(const ssd_config_t *cfg, const ssd_prefill_args_t *args,
+                                const int *cu_seqlens, int nseq, void *stream) {
+  if (!args || !varlen_ok(cfg, cu_seqlens, nseq)) return SSD_ERR_INVALID_ARG;
+  ssd_status_t st = check_config(cfg, true);
+  if (st != SSD_OK) return st;
+  const size_t es = cfg->io_dtype == SSD_F32 ? 4 : 2;
+  const long long d_inner = (long long)cfg->nheads * cfg->headdim;
+  const long long conv_dim = d_inner + 2LL * cfg->ngroups * cfg->dstate;
+  const long long state = (long long)cfg->nheads * cfg->headdim * cfg->dstate;
+  const long long cache = (long long)cfg->conv_width * conv_dim;
+  for (int i = 0; i < nseq; ++i) {
+    ssd_config_t c = *cfg;
+    const long long t0 = cu_seqlens[i];
+    c.seqlen = cu_seqlens[i + 1] - cu_seqlens[i];
+    ssd_prefill_args_t a = *args;
+    auto at = [](const void *p, long long bytes) -> const char * {
+      return p ? static_cast<const char *>(p) + bytes : nullptr;
+    };
+    a.xBC = at(args->xBC, t0 * args->xBC_row_stride * es);
+    a.dt = at(args->dt, t0 * args->dt_row_stride * es);
+    a.z = at(args->z, t0 * args->z_row_stride * es);
+    a.y = const_cast<char *>(at(args->y, t0 * args->y_row_stride * es));
+    a.h0 = reinterpret_cast<const float *>(at(args->h0, i * state * 4));
+    a.h_final = reinterpret_cast<float *>(const_cast<char *>(at(args->h_final, i * state * 4)));
+    a.conv_state_in = at(args->conv_state_in, i * cache * es);
+    a.conv_state_out = const_cast<char *>(at(args->conv_state_out, i * cache * es));
+    st = run_prefill(&c, &a, static_cast<cudaStream_t>(stream));
+    if (st != SSD_OK) return st;
+  }
+  return SSD_OK;
+}
+
 size_t ssd_mixer_workspace_size(const ssd_mixer_config_t *cfg) {
   if (!cfg || check_config(&cfg->ssd, true) != SSD_OK) return 0;
   return mixer_layout(cfg).total;

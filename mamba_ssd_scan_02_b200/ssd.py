@@ -77,7 +77,8 @@ class TraceRecord(ctypes.Structure):
 
 EXPORTS = ("ssd_workspace_size", "ssd_prefill", "ssd_decode_step", "ssd_mixer_workspace_size",
            "mamba2_mixer_forward", "ssd_status_string", "ssd_get_device_error", "ssd_version",
-           "ssd_trace_enable", "ssd_trace_read", "ssd_prefill_noalloc")
+           "ssd_trace_enable", "ssd_trace_read", "ssd_prefill_noalloc", "ssd_varlen_workspace_size",
+           "ssd_prefill_varlen")
 NOALLOC_WORKSPACE_BYTES = 64 << 20
 
 _lib = None
@@ -111,6 +112,11 @@ def load(path: str = LIB_PATH):
     lib.ssd_get_device_error.argtypes = [vp]
     lib.ssd_version.restype = c_int
     lib.ssd_version.argtypes = []
+    lib.ssd_varlen_workspace_size.restype = ctypes.c_size_t
+    lib.ssd_varlen_workspace_size.argtypes = [ctypes.POINTER(SsdConfig), ctypes.POINTER(c_int), c_int]
+    lib.ssd_prefill_varlen.restype = c_int
+    lib.ssd_prefill_varlen.argtypes = [ctypes.POINTER(SsdConfig), ctypes.POINTER(PrefillArgs),
+                                       ctypes.POINTER(c_int), c_int, vp]
     lib.ssd_prefill_noalloc.restype = c_int
     lib.ssd_prefill_noalloc.argtypes = [ctypes.POINTER(SsdConfig), ctypes.POINTER(PrefillArgs), vp]
     lib.ssd_trace_enable.restype = c_int
@@ -259,6 +265,36 @@ def prefill_noalloc(cfg: dict, xBC, dt, A, D, dt_bias, conv_w=None, conv_b=None,
     _check(lib.ssd_prefill_noalloc(ctypes.byref(c), ctypes.byref(a), _stream(stream)),
            "ssd_prefill_noalloc")
     return y, h_final, conv_state_out
+
+
+def prefill_varlen(cfg: dict, cu_seqlens, xBC, dt, A, D, dt_bias, conv_w=None, conv_b=None, z=None,
+                   norm_w=None, h0=None, conv_state_in=None, *, stream=None, kernel: int | None = None):
+    """ssd_prefill_varlen: packed sequences xBC [T, conv_dim] (T = cu_seqlens[-1]) with
+    per-sequence carries [nseq, ...]; returns (y [T, d_inner], h_final [nseq, H, P, N],
+    conv_state_out [nseq, W, conv_dim] or None)."""
+    import torch
+    lib = load()
+    cu = [int(v) for v in cu_seqlens]
+    nseq, T = len(cu) - 1, cu[-1]
+    c = make_config(dict(cfg, batch=1), seqlen=T, kernel=kernel)
+    H, P, N, G, W = c.nheads, c.headdim, c.dstate, c.ngroups, c.conv_width
+    d_inner, conv_dim = H * P, H * P + 2 * G * N
+    dev = xBC.device
+    y = torch.empty((T, d_inner), dtype=io_dtype(cfg), device=dev)
+    h_final = torch.empty((nseq, H, P, N), dtype=torch.float32, device=dev)
+    cso = torch.empty((nseq, W, conv_dim), dtype=io_dtype(cfg), device=dev) if W > 0 else None
+    cu_arr = (c_int * (nseq + 1))(*cu)
+    workspace = alloc_workspace(lib.ssd_varlen_workspace_size(ctypes.byref(c), cu_arr, nseq), dev)
+    a = PrefillArgs(
+        xBC=_ptr(xBC), xBC_row_stride=xBC.stride(-2), dt=_ptr(dt), dt_row_stride=dt.stride(-2),
+        z=_ptr(z), z_row_stride=z.stride(-2) if z is not None else 0, A=_ptr(A), D=_ptr(D),
+        dt_bias=_ptr(dt_bias), conv_w=_ptr(conv_w), conv_b=_ptr(conv_b), norm_w=_ptr(norm_w),
+        h0=_ptr(h0), conv_state_in=_ptr(conv_state_in), y=_ptr(y), y_row_stride=d_inner,
+        h_final=_ptr(h_final), conv_state_out=_ptr(cso), workspace=_ptr(workspace),
+        workspace_bytes=workspace.numel())
+    _check(lib.ssd_prefill_varlen(ctypes.byref(c), ctypes.byref(a), cu_arr, nseq, _stream(stream)),
+           "ssd_prefill_varlen")
+    return y, h_final, cso
 
 
 def decode_step(cfg: dict, xBC_t, dt_t, A, D, dt_bias, conv_w, conv_b, state, conv_state_in,

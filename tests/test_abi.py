@@ -129,3 +129,20 @@ def test_mixer_rejects_bad_args(lib):
     assert lib.mamba2_mixer_forward(ctypes.byref(m), ctypes.byref(a), None) == 2  # bf16 only
     assert lib.ssd_mixer_workspace_size(ctypes.byref(ssd.MixerConfig(ssd=_cfg(), d_model=512))) > 0
     assert not math.isnan(m.rms_eps)
+
+
+def test_varlen_rejects_inconsistent_offsets(lib):
+    """Checked on the host before anything is launched (no GPU needed)."""
+    import ctypes
+    from mamba_ssd_scan_02_b200 import ssd
+    from mamba_ssd_scan_02_b200 import datagen
+    cfg = dict(datagen.config(1), batch=1, seqlen=10)
+    c = ssd.make_config(cfg)
+    a = ssd.PrefillArgs()
+    for cu in ([0, 6, 4, 10], [1, 5, 10], [0, 5, 9]):  # decreasing / not from 0 / wrong total
+        arr = (ctypes.c_int * len(cu))(*cu)
+        assert lib.ssd_prefill_varlen(ctypes.byref(c), ctypes.byref(a), arr, len(cu) - 1, None) == 1
+        assert lib.ssd_varlen_workspace_size(ctypes.byref(c), arr, len(cu) - 1) == 0
+    c2 = ssd.make_config(dict(cfg, batch=2))
+    arr = (ctypes.c_int * 3)(0, 4, 10)
+    assert lib.ssd_prefill_varlen(ctypes.byref(c2), ctypes.byref(a), arr, 2, None) == 1
