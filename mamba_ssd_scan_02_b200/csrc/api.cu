@@ -231,6 +231,7 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
       SSD_TRY(traced("ssd_state_pass", s, [&] { return launch_state_pass(p, s); }));
     }
     SSD_TRY(traced("ssd_scan_tc", s, [&] { return launch_scan_tc(p, 0, s); }));
+    SSD_TRY(traced("ssd_state_tail", s, [&] { return launch_state_tail(p, 2, s); }));
     if (p.norm_groups > 0) SSD_TRY(traced("ssd_gated_norm", s, [&] { return launch_gated_norm(p, s); }));
     if (!cso_early) SSD_TRY(traced("ssd_conv_state_out", s, [&] { return launch_conv_state_out(p, s); }));
     return SSD_OK;

@@ -75,6 +75,8 @@ bool tc_scan_available();
 cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s);
 // inter-segment state pass (state_pass.cu)
 cudaError_t launch_state_pass(const PrefillPlan &p, cudaStream_t s);
+// fp32 recomputation of the final state's last tail_chunks chunks (tensor-core path)
+cudaError_t launch_state_tail(const PrefillPlan &p, int tail_chunks, cudaStream_t s);
 // norms (norm.cu)
 cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s);          // fp32 yf -> y
 cudaError_t launch_rmsnorm_bf16(const void *x, const void *w, void *out, long long rows, int width,

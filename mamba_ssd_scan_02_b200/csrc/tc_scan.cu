@@ -66,6 +66,7 @@ namespace {
 using namespace tc;
 
 constexpr int QC = 128;              // tokens per chunk
+constexpr int kTailChunks = 2;       // chunks of the final state recomputed in fp32
 constexpr int kThreadsTC = 640;       // 20 warps
 constexpr int kConvWarps = 8;          // see conv_index()
 constexpr int kTokPerConvWarp = QC / kConvWarps;  // 16
@@ -141,6 +142,8 @@ struct TcArgs {
   long long h_init_seg;
   float *h_out;            // final state destination or null
   long long h_out_seg;
+  int tail_chunks;         // > 0: instead of the final state, the last segment writes the state
+                           // before its last tail_chunks chunks (an fp32 pass finishes it)
   float *seg_decay;        // [n_seg, B, H] total decay per segment, or null
   __nv_bfloat16 *y;        // output (no gate) ...
   long long ys;
@@ -706,6 +709,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     const bool leader = (tid == 19 * 32);
     const uint32_t lane_off = (uint32_t)(32 * ew) << 16;
     const long long bh = (long long)b * a.H + h;
+    float *hout = a.h_out ? a.h_out + seg * a.h_out_seg + bh * 8192 : nullptr;
+    // tail mode: only the last segment writes, the state entering its last tail_chunks chunks
+    const bool tail = a.tail_chunks > 0 && seg == (int)gridDim.x - 1 && hout != nullptr;
+    const int tail_k = nck - 1 - a.tail_chunks;  // state after this chunk (-1: the initial state)
     {  // initial state -> TMEM (fp32) and the fp16 copy
       const float *hin = a.h_init ? a.h_init + seg * a.h_init_seg + bh * 8192 : nullptr;
 #pragma unroll 1
@@ -719,6 +726,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         tmem_st32(tmem + TM_H + 32 * half + lane_off, hu);
         write_h_tile(smem, hr, n, half);
+        if (tail && tail_k < 0) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) hout[(32 * half + i) * 128 + n] = hr[i];
+        }
       }
       tmem_st_wait();
     }
@@ -762,6 +773,17 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       tc_fence_before();
       named_bar(3, 128);
       if (leader) mbar_arrive(BAR(BAR_DHFREE));  // dH read: MMA4 of chunk k+1 may overwrite it
+      if (tail && k == tail_k) {  // the state entering the tail, in fp32
+        tc_fence_after();
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          float hr[32];
+          tmem_ld32(tmem + TM_H + 32 * half + lane_off, hr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) hout[(32 * half + i) * 128 + n] = hr[i];
+        }
+      }
       if (!kStateOnly && k != last) {
         // fp16 copy of h_k for MMA3 of chunk k+1, once MMA3 of chunk k has read h_{k-1}
         if (!wg_wait(BAR(BAR_HTFREE), k & 1, leader, 3, abort_flag, a.err)) break;
@@ -822,8 +844,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
     }
     if (*abort_flag == 0) {
-      float *hout = a.h_out ? a.h_out + seg * a.h_out_seg + bh * 8192 : nullptr;
-      if (hout) {
+      if (hout && a.tail_chunks == 0) {
         tc_fence_after();
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
@@ -913,11 +934,13 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
     ssd_scan_tc_kernel<true><<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, a);
   } else {
     if (p.n_seg > 1) {
-      a.h_init = p.seg_state; a.h_init_seg = seg_stride; a.h_out = nullptr;
+      a.h_init = p.seg_state; a.h_init_seg = seg_stride;
     } else {
-      a.h_init = p.h0; a.h_init_seg = 0; a.h_out = p.h_final;
+      a.h_init = p.h0; a.h_init_seg = 0;
     }
-    a.h_out_seg = 0; a.seg_decay = nullptr;
+    // the last segment leaves the state before its last two chunks; launch_state_tail
+    // recomputes those chunks in fp32
+    a.h_out = p.h_final; a.h_out_seg = 0; a.seg_decay = nullptr; a.tail_chunks = kTailChunks;
     e = set_smem_attr(ssd_scan_tc_kernel<false>, kSmemAlloc, s);
     if (e != cudaSuccess) return e;
     ssd_scan_tc_kernel<false><<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, a);

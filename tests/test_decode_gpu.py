@@ -158,3 +158,8 @@ def test_decode_16k_steps_full_size(cuda_lib, oracle):
                          out_dtype="bf16")
     assert_close(host(state)[rows], ost, TOL_BF16, "state after 16384 steps")
     assert np.array_equal(host(cache)[rows], ocache)
+
+
+@pytest.mark.parametrize("W", [2, 3])
+def test_decode_narrow_conv_windows(cuda_lib, oracle, W):
+    _run_steps(oracle, _decode_cfg(conv_width=W), steps=4)

@@ -184,3 +184,11 @@ def test_long_context_split_equals_unsplit(cuda_lib, oracle):
         assert_close(ysplit[:, :, lo * P:hi * P], ref["out"], TOL_BF16, f"cfg3 split y group {g}",
                      out_dtype="bf16")
         assert_close(host(h)[:, lo:hi], ref["h_final"], TOL_BF16, f"cfg3 h_final group {g}")
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("W", [0, 1, 2, 3])
+def test_narrow_conv_windows(cuda_lib, oracle, kernel, W):
+    """Conv windows below 4 (0 = no conv and no activation), with cache and gated norm."""
+    cfg = small_cfg(conv_width=W, seqlen=261)
+    _check(oracle, cfg, make_case(cfg, seed_idx=7), kernel, tag=f"W{W}")
