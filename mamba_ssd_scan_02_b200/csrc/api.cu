@@ -97,7 +97,7 @@ struct WsLayout {
   // CUDA-core path
   size_t u, dte, yf, seg_state, seg_decay, simt_end;
   // tensor-core path
-  size_t tc_bc, tc_dte, tc_cs, tc_yf, tc_seg_state, tc_seg_decay, tc_end;
+  size_t tc_bc, tc_dte, tc_cs, tc_yf, tc_seg_state, tc_seg_decay, tc_dh, tc_end;
   int Lpad;
   size_t total;
 };
@@ -134,6 +134,7 @@ WsLayout prefill_layout(const ssd_config_t *c) {
     w.tc_seg_decay = off;
     off = round_up(off + (size_t)n_seg * c->batch * c->nheads * 4, kAlign);
   }
+  w.tc_dh = off;   off = round_up(off + state + (size_t)c->batch * c->nheads * 4, kAlign);
   w.tc_end = off;
   w.total = w.simt_end > w.tc_end ? w.simt_end : w.tc_end;
   return w;
@@ -146,6 +147,36 @@ ssd_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_E
     cudaError_t e_ = (expr);                     \
     if (e_ != cudaSuccess) return SSD_ERR_CUDA;  \
   } while (0)
+
+// Per host thread and device: a side stream and two events that run the fp32 tail pass beside
+// the output scan (made on first use and kept for the life of the process).  Per thread, so
+// that a fork is always joined before the same objects are recorded again.
+struct SideStream {
+  cudaStream_t s;
+  cudaEvent_t fork, join;
+};
+cudaError_t side_stream(SideStream **out) {
+  constexpr int kMaxDev = 64;
+  thread_local SideStream tls[kMaxDev] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  SideStream &ss = tls[dev];
+  if (!ss.s) {
+    SideStream n{};
+    if ((e = cudaStreamCreateWithFlags(&n.s, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming)) != cudaSuccess) {
+      if (n.fork) cudaEventDestroy(n.fork);
+      cudaStreamDestroy(n.s);
+      return e;
+    }
+    ss = n;
+  }
+  *out = &ss;
+  return cudaSuccess;
+}
 
 ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cudaStream_t s) {
   ssd_status_t st = check_config(c, true);
@@ -213,6 +244,8 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
     p.yf = c->norm_groups > 0 ? reinterpret_cast<float *>(ws + lay.tc_yf) : nullptr;
     p.seg_state = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.tc_seg_state) : nullptr;
     p.seg_decay = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.tc_seg_decay) : nullptr;
+    p.tail_dh = p.h_final ? reinterpret_cast<float *>(ws + lay.tc_dh) : nullptr;
+    p.tail_dec = p.h_final ? p.tail_dh + (size_t)c->batch * c->nheads * c->headdim * c->dstate : nullptr;
     // The outgoing conv cache may be written before the scan unless it overlaps an input
     // that later kernels read.
     const size_t x_span = ((size_t)c->batch * c->seqlen - 1) * (size_t)a->xBC_row_stride * es + (size_t)conv_dim * es;
@@ -226,12 +259,25 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
       SSD_TRY(traced("ssd_dt_cumsum", s, [&] { return launch_dt_cumsum(p, p.dte_hm, p.cs_hm, p.Lpad, s); }));
       SSD_TRY(traced("ssd_bc_conv", s, [&] { return launch_bc_conv_f16(p, s); }));
     }
+    // the fp32 tail needs only the front end's outputs: it runs on a side stream, on the SMs
+    // the scan leaves free, and is joined before the fold
+    SideStream *side = nullptr;
+    if (p.tail_dh) {
+      SSD_TRY(side_stream(&side));
+      SSD_TRY(cudaEventRecord(side->fork, s));
+      SSD_TRY(cudaStreamWaitEvent(side->s, side->fork, 0));
+      SSD_TRY(traced("ssd_state_tail", side->s, [&] { return launch_state_tail(p, side->s); }));
+      SSD_TRY(cudaEventRecord(side->join, side->s));
+    }
     if (p.n_seg > 1) {
       SSD_TRY(traced("ssd_scan_tc_states", s, [&] { return launch_scan_tc(p, 1, s); }));
       SSD_TRY(traced("ssd_state_pass", s, [&] { return launch_state_pass(p, s); }));
     }
     SSD_TRY(traced("ssd_scan_tc", s, [&] { return launch_scan_tc(p, 0, s); }));
-    SSD_TRY(traced("ssd_state_tail", s, [&] { return launch_state_tail(p, 2, s); }));
+    if (side) {
+      SSD_TRY(cudaStreamWaitEvent(s, side->join, 0));
+      SSD_TRY(traced("ssd_tail_fold", s, [&] { return launch_tail_fold(p, s); }));
+    }
     if (p.norm_groups > 0) SSD_TRY(traced("ssd_gated_norm", s, [&] { return launch_gated_norm(p, s); }));
     if (!cso_early) SSD_TRY(traced("ssd_conv_state_out", s, [&] { return launch_conv_state_out(p, s); }));
     return SSD_OK;

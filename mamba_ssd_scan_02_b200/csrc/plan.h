@@ -37,6 +37,9 @@ struct PrefillPlan {
   void *bc;          // [B, L, 2*G*N] fp16 conv+SiLU output of the B|C channels (tensor path)
   float *dte_hm;     // [B, H, Lpad] effective dt, head-major (tensor path)
   float *cs_hm;      // [B, H, Lpad] chunk-local prefix sums of dt*A (tensor path)
+  float *tail_dh;    // [B, H, P, N] fp32 contribution of the final state's last chunks, from a
+                     // zero state (tensor path; null when no final state is written)
+  float *tail_dec;   // [B, H] decay over those chunks
   int Lpad;
   int *err;          // device error word
 };
@@ -75,8 +78,13 @@ bool tc_scan_available();
 cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s);
 // inter-segment state pass (state_pass.cu)
 cudaError_t launch_state_pass(const PrefillPlan &p, cudaStream_t s);
-// fp32 recomputation of the final state's last tail_chunks chunks (tensor-core path)
-cudaError_t launch_state_tail(const PrefillPlan &p, int tail_chunks, cudaStream_t s);
+// fp32 recomputation of the final state's last kTailChunks chunks (tensor-core path): what
+// those chunks add to a zero state, into p.tail_dh / p.tail_dec.  It runs on a side stream
+// beside the output scan, which leaves the state entering those chunks in h_final; the fold
+// then sets h_final = tail_dec * h_final + tail_dh.
+constexpr int kTailChunks = 2;
+cudaError_t launch_state_tail(const PrefillPlan &p, cudaStream_t s);
+cudaError_t launch_tail_fold(const PrefillPlan &p, cudaStream_t s);
 // norms (norm.cu)
 cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s);          // fp32 yf -> y
 cudaError_t launch_rmsnorm_bf16(const void *x, const void *w, void *out, long long rows, int width,

@@ -66,7 +66,6 @@ namespace {
 using namespace tc;
 
 constexpr int QC = 128;              // tokens per chunk
-constexpr int kTailChunks = 2;       // chunks of the final state recomputed in fp32
 constexpr int kThreadsTC = 640;       // 20 warps
 constexpr int kConvWarps = 8;          // see conv_index()
 constexpr int kTokPerConvWarp = QC / kConvWarps;  // 16
@@ -938,9 +937,10 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
     } else {
       a.h_init = p.h0; a.h_init_seg = 0;
     }
-    // the last segment leaves the state before its last two chunks; launch_state_tail
-    // recomputes those chunks in fp32
-    a.h_out = p.h_final; a.h_out_seg = 0; a.seg_decay = nullptr; a.tail_chunks = kTailChunks;
+    // the last segment leaves the state before its last kTailChunks chunks; the fp32 tail pass
+    // adds what those chunks contribute
+    a.h_out = p.h_final; a.h_out_seg = 0; a.seg_decay = nullptr;
+    a.tail_chunks = p.tail_dh ? kTailChunks : 0;
     e = set_smem_attr(ssd_scan_tc_kernel<false>, kSmemAlloc, s);
     if (e != cudaSuccess) return e;
     ssd_scan_tc_kernel<false><<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, a);

@@ -192,3 +192,46 @@ def test_narrow_conv_windows(cuda_lib, oracle, kernel, W):
     """Conv windows below 4 (0 = no conv and no activation), with cache and gated norm."""
     cfg = small_cfg(conv_width=W, seqlen=261)
     _check(oracle, cfg, make_case(cfg, seed_idx=7), kernel, tag=f"W{W}")
+
+
+def test_tc_prefill_graph_capture_and_reuse(cuda_lib):
+    """The tensor-core prefill runs its fp32 final-state pass on a side stream forked from the
+    caller's stream and joined before the fold.  Captured into a CUDA graph, the fork and join
+    land in the graph, so replays reproduce the eager outputs bit for bit; and back-to-back
+    calls with different inputs (the side stream and its events reused) each match their own
+    single eager call."""
+    import torch
+    from mamba_ssd_scan_02_b200 import ssd
+    cfg = small_cfg(seqlen=333)
+    names = ["xBC", "dt", "A", "D", "dt_bias", "conv_w", "conv_b", "z", "norm_w", "h0", "conv_state_in"]
+    cases = [make_case(cfg, seed_idx=s) for s in (11, 12)]
+    devs = [[(None if c.get(k) is None else ssd.to_device(c[k])) for k in names] for c in cases]
+    torch.cuda.synchronize()
+    eager = []
+    for d in devs:
+        y, hf, cso = ssd.prefill(cfg, *d, kernel=2)
+        torch.cuda.synchronize()
+        eager.append((y.clone(), hf.clone(), cso.clone()))
+    # back to back on one stream, no synchronisation in between
+    outs = [ssd.prefill(cfg, *d, kernel=2) for d in devs for _ in range(2)]
+    torch.cuda.synchronize()
+    for i, (y, hf, cso) in enumerate(outs):
+        ye, he, ce = eager[i // 2]
+        assert torch.equal(y, ye) and torch.equal(hf, he) and torch.equal(cso, ce), f"call {i}"
+    # graph capture on a side stream, then replays
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        ssd.prefill(cfg, *devs[0], kernel=2)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        yg, hg, cg = ssd.prefill(cfg, *devs[0], kernel=2)
+    for _ in range(3):
+        hg.zero_()
+        yg.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        ye, he, ce = eager[0]
+        assert torch.equal(yg, ye) and torch.equal(hg, he) and torch.equal(cg, ce)
