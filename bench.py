@@ -289,14 +289,27 @@ class Ctx:
         return ms, recs, self.clk.summary(t0, t2, window)
 
 
+# Kernels that the library runs on its side stream, concurrently with the stream's own work:
+# their time is not on the step's critical path, so they take no share and are never the
+# dominant kernel.
+OVERLAPPED = {"ssd_state_tail": "side stream, concurrent with ssd_scan_tc"}
+
+
 def kernel_table(recs):
     per = {}
     for name, ms in recs:
         per.setdefault(name, []).append(ms)
-    total = sum(sum(v) for v in per.values()) or 1.0
-    table = {k: {"launches": len(v), "mean_ms": round(statistics.mean(v), 5),
-                 "share": round(sum(v) / total, 4)} for k, v in per.items()}
-    dom = max(per, key=lambda k: sum(per[k])) if per else None
+    serial = {k: v for k, v in per.items() if k not in OVERLAPPED}
+    total = sum(sum(v) for v in serial.values()) or 1.0
+    table = {}
+    for k, v in per.items():
+        row = {"launches": len(v), "mean_ms": round(statistics.mean(v), 5)}
+        if k in OVERLAPPED:
+            row.update(share=None, overlapped=OVERLAPPED[k])
+        else:
+            row["share"] = round(sum(v) / total, 4)
+        table[k] = row
+    dom = max(serial, key=lambda k: sum(serial[k])) if serial else None
     return per, table, dom
 
 

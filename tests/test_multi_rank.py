@@ -64,3 +64,16 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_kernel_table_keeps_side_stream_kernels_off_the_critical_path():
+    """A kernel the library runs on its side stream (concurrently with the scan) is listed but
+    takes no share of the step and is never the dominant kernel, even when its own traced
+    time is the largest."""
+    import bench
+    recs = [("ssd_front", 0.03), ("ssd_state_tail", 0.5), ("ssd_scan_tc", 0.2), ("ssd_tail_fold", 0.01)] * 2
+    per, table, dom = bench.kernel_table(recs)
+    assert dom == "ssd_scan_tc"
+    assert table["ssd_state_tail"]["share"] is None and "overlapped" in table["ssd_state_tail"]
+    assert table["ssd_scan_tc"]["share"] == pytest.approx(0.2 / 0.24, abs=1e-4)
+    assert sum(r["share"] for r in table.values() if r["share"] is not None) == pytest.approx(1.0, abs=1e-3)
