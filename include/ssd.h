@@ -26,8 +26,14 @@
  *
  * Conventions for every call:
  *  - All pointers are DEVICE pointers owned by the caller.  The library never
- *    allocates, frees or synchronises on these paths; it enqueues kernels on
- *    `stream` (a cudaStream_t, NULL = legacy default stream) and returns.
+ *    allocates device memory, frees or synchronises on these paths; it enqueues
+ *    kernels on `stream` (a cudaStream_t, NULL = legacy default stream) and
+ *    returns.  The tensor-core prefill runs its fp32 final-state pass on a
+ *    library side stream, forked from `stream` after the front end and joined
+ *    back into it within the same call, so every effect of the call is ordered
+ *    on `stream` (stream capture included).  That side stream and its two
+ *    events are created by the first such call on each host thread and device
+ *    and kept for the life of the process.
  *  - Argument errors are reported synchronously before anything is launched.
  *    Launch failures come back as SSD_ERR_CUDA.  Errors raised inside kernels
  *    (a bounded wait that gave up) are latched in a device word read by
