@@ -16,8 +16,10 @@
 // regrouped by chunk; every exponent is a difference cs_t - cs_s <= 0 or is split at a
 // 32-token block boundary where both factors stay below e^60 (else computed directly).
 // In the last chunk of a segment w o X is applied as fp16 hi + lo parts (a second MMA4), so
-// the final state carries the rounding of B only: its largest entries come from the newest
-// tokens, whose products are not averaged over many terms.
+// a segment's final state carries the rounding of B only: its largest entries come from the
+// newest tokens, whose products are not averaged over many terms.  The sequence's own final
+// state goes further: in tail mode the output pass leaves the state entering the last two
+// chunks, and a separate fp32 pass (state_tail.cu) adds those chunks' contribution.
 //
 // Warp roles (640 threads): warp 0 issues TMA loads (B and C tiles of the group, the head's
 // raw x rows with a 3-token halo, per-chunk dt and prefix sums), warp 1 allocates TMEM and
