@@ -1,5 +1,6 @@
 // api.cu -- the C ABI of libssd.so: argument validation, workspace layout and the launch
-// sequence of each entry point.  Nothing here allocates or synchronises on the compute paths.
+// sequence of each entry point.  Nothing here allocates device memory or synchronises on the
+// compute paths.
 #include <math.h>
 #include <stdint.h>
 #include <string.h>
@@ -156,12 +157,11 @@ struct SideStream {
   cudaEvent_t fork, join;
 };
 cudaError_t side_stream(SideStream **out) {
-  constexpr int kMaxDev = 64;
-  thread_local SideStream tls[kMaxDev] = {};
+  thread_local SideStream tls[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   SideStream &ss = tls[dev];
   if (!ss.s) {
     SideStream n{};
@@ -177,6 +177,23 @@ cudaError_t side_stream(SideStream **out) {
   *out = &ss;
   return cudaSuccess;
 }
+
+// Once the side stream has been forked from the caller's stream, joins it back on every exit
+// (an early error return included): the caller's stream, or a graph being captured from it,
+// never ends the call with work of this call still outstanding on the side stream.
+struct SideJoin {
+  SideStream *side = nullptr;
+  cudaStream_t s = nullptr;
+  bool forked = false;
+  cudaError_t join() {
+    if (!forked) return cudaSuccess;
+    forked = false;
+    cudaError_t e = cudaEventRecord(side->join, side->s);
+    if (e != cudaSuccess) return e;
+    return cudaStreamWaitEvent(s, side->join, 0);
+  }
+  ~SideJoin() { join(); }
+};
 
 ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cudaStream_t s) {
   ssd_status_t st = check_config(c, true);
@@ -261,21 +278,22 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
     }
     // the fp32 tail needs only the front end's outputs: it runs on a side stream, on the SMs
     // the scan leaves free, and is joined before the fold
-    SideStream *side = nullptr;
+    SideJoin side;
     if (p.tail_dh) {
-      SSD_TRY(side_stream(&side));
-      SSD_TRY(cudaEventRecord(side->fork, s));
-      SSD_TRY(cudaStreamWaitEvent(side->s, side->fork, 0));
-      SSD_TRY(traced("ssd_state_tail", side->s, [&] { return launch_state_tail(p, side->s); }));
-      SSD_TRY(cudaEventRecord(side->join, side->s));
+      SSD_TRY(side_stream(&side.side));
+      side.s = s;
+      SSD_TRY(cudaEventRecord(side.side->fork, s));
+      SSD_TRY(cudaStreamWaitEvent(side.side->s, side.side->fork, 0));
+      side.forked = true;
+      SSD_TRY(traced("ssd_state_tail", side.side->s, [&] { return launch_state_tail(p, side.side->s); }));
     }
     if (p.n_seg > 1) {
       SSD_TRY(traced("ssd_scan_tc_states", s, [&] { return launch_scan_tc(p, 1, s); }));
       SSD_TRY(traced("ssd_state_pass", s, [&] { return launch_state_pass(p, s); }));
     }
     SSD_TRY(traced("ssd_scan_tc", s, [&] { return launch_scan_tc(p, 0, s); }));
-    if (side) {
-      SSD_TRY(cudaStreamWaitEvent(s, side->join, 0));
+    if (side.forked) {
+      SSD_TRY(side.join());
       SSD_TRY(traced("ssd_tail_fold", s, [&] { return launch_tail_fold(p, s); }));
     }
     if (p.norm_groups > 0) SSD_TRY(traced("ssd_gated_norm", s, [&] { return launch_gated_norm(p, s); }));
