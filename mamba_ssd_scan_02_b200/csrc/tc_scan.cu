@@ -24,7 +24,7 @@
 // Warp roles (640 threads): warp 0 issues TMA loads (B and C tiles of the group, the head's
 // raw x rows with a 3-token halo, per-chunk dt and prefix sums), warp 1 allocates TMEM and
 // issues each MMA group as soon as its inputs are ready, warps 2-4, 6-8, 10-11 compute the x
-// channels (causal conv1d + SiLU) in place into X and into w o X, warps 12-15 turn S into S~,
+// channels (causal conv1d + SiLU) in place into w o X and into X, warps 12-15 turn S into S~,
 // warps 16-19 update the state (kept in fp32 in TMEM), refresh its fp16 copy and write y.
 // X, w o X, S (with Yi in its upper half), Ys and the B/C stages are double-buffered, so each
 // role can run a chunk ahead of the next.  Hand-offs use mbarriers (TMA transaction counts,
@@ -78,15 +78,15 @@ constexpr uint32_t OFF_B = 2 * kTile;         // B tile
 constexpr uint32_t OFF_DT = 4 * kTile;        // dt[128] fp32
 constexpr uint32_t OFF_CS = OFF_DT + 512;     // cs[128] fp32
 constexpr uint32_t kStage = 4 * kTile + 1024;  // 66560 = 65 * 1024
-// CTA layout.  X[b] (two buffers, chunk k uses b = k % 2) first receives by TMA the chunk's
-// raw bf16 x rows for times t0-3 .. t0+127 (131 rows of this head's 64 channels); the conv
-// overwrites row s with X row s.  w o X is double-buffered the same way.
-constexpr int kXBufs = 2;
+// CTA layout.  w o X[b] (two buffers, chunk k uses b = k % 2) first receives by TMA the
+// chunk's raw bf16 x rows for times t0-3 .. t0+127 (131 rows of this head's 64 channels); the
+// conv overwrites row s with the w o X row s and writes X row s into X[b].  The raw tile thus
+// waits only for MMA4 of chunk k-2 (which frees w o X[b]), not for MMA2, which comes later.
 constexpr uint32_t kXBuf = 17 * 1024;           // 131 rows of 128 bytes, padded
 constexpr uint32_t kRawRows = QC + 3;
-constexpr uint32_t OFF_X = 2 * kStage;              // X[2]  [s][p] fp16 (raw x rows first)
-constexpr uint32_t OFF_XW = OFF_X + kXBufs * kXBuf;  // w o X [2][s][p] fp16, 16 KB each
-constexpr uint32_t OFF_H = OFF_XW + 2 * kTile;      // h copy [n][p] fp16, 16 KB
+constexpr uint32_t OFF_X = 2 * kStage;              // X[2]  [s][p] fp16, 16 KB each
+constexpr uint32_t OFF_XW = OFF_X + 2 * kTile;      // w o X [2][s][p] fp16 (raw x rows first)
+constexpr uint32_t OFF_H = OFF_XW + 2 * kXBuf;      // h copy [n][p] fp16, 16 KB
 constexpr uint32_t OFF_CF = OFF_H + kTile;          // column factors, 128 fp32
 constexpr uint32_t OFF_CSM = OFF_CF + 512;          // the mask's copies of cs and dt
 constexpr uint32_t OFF_DTM = OFF_CSM + 512;
@@ -96,7 +96,7 @@ constexpr uint32_t OFF_BAR = OFF_DTM + 512;
 enum {
   BAR_FULL0, BAR_FULL1,        // stage k % 2 loaded (TMA)
   BAR_EMPTY0, BAR_EMPTY1,      // stage k % 2 released (conv, mask, state warps + MMA commit)
-  BAR_FULLX0, BAR_FULLX1,      // raw x of chunk k in X[k % 2] (TMA)
+  BAR_FULLX0, BAR_FULLX1,      // raw x of chunk k in w o X[k % 2] (TMA)
   BAR_XFREE0, BAR_XFREE1,      // X[k % 2] read by MMA2 of chunk k
   BAR_SREADY0, BAR_SREADY1,    // S of chunk k in TMEM (MMA1)
   BAR_STREADY0, BAR_STREADY1,  // S~ of chunk k in TMEM (mask warps)
@@ -288,16 +288,16 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    // Raw x rows of chunk k go to X[k % 2] once MMA2 of chunk k-2 has released it; the B/C
-    // tiles, dt and prefix sums go to stage k % 2 once chunk k-2's consumers released it.
+    // Raw x rows of chunk k go to w o X[k % 2] once MMA4 of chunk k-2 has released it; the
+    // B/C tiles, dt and prefix sums go to stage k % 2 once chunk k-2's consumers released it.
     if (lane == 0) {
       int k = 0, nx = 0, nbc = 0;
       for (; k < nck; ++k) {
         const int xb = k & 1, st = k & 1;
         const int t0 = t_begin + k * QC;
-        if (k >= 2 && !mbar_wait(BAR(BAR_XFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err)) break;
+        if (k >= 2 && !mbar_wait(BAR(BAR_XWFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err)) break;
         mbar_arrive_expect_tx(BAR(BAR_FULLX0 + xb), kRawRows * 128);
-        tma_load_3d(sb + OFF_X + xb * kXBuf, &tm_x, h * 64, t0 - 3, b, BAR(BAR_FULLX0 + xb));
+        tma_load_3d(sb + OFF_XW + xb * kXBuf, &tm_x, h * 64, t0 - 3, b, BAR(BAR_FULLX0 + xb));
         ++nx;
         if (k >= 2 && !mbar_wait(BAR(BAR_EMPTY0 + st), ((k >> 1) - 1) & 1, abort_flag, a.err)) break;
         const uint32_t sst = sb + st * kStage;
@@ -349,7 +349,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           tc_fence_after();
           TC_MARK(j, 11);
           const uint32_t tS = tmem + ((j & 1) ? TM_S1 : TM_S0);
-          issue_Yi(tS, sb + OFF_X + (j & 1) * kXBuf, tS + TM_YI_OFF);
+          issue_Yi(tS, sb + OFF_X + (j & 1) * kTile, tS + TM_YI_OFF);
           mma_commit(BAR(BAR_YREADY0 + (j & 1)));
           mma_commit(BAR(BAR_XFREE0 + (j & 1)));
           ++nYi;
@@ -374,9 +374,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           tc_fence_after();
           TC_MARK(j, 8);
           const uint32_t sst = sb + (j & 1) * kStage;
-          issue_dH(sst, sb + OFF_XW + (j & 1) * kTile, tmem + TM_DH, false);
+          issue_dH(sst, sb + OFF_XW + (j & 1) * kXBuf, tmem + TM_DH, false);
           // last chunk: the low part of w o X (in the other w o X buffer) for the final state
-          if (j == last) issue_dH(sst, sb + OFF_XW + ((j + 1) & 1) * kTile, tmem + TM_DH, true);
+          if (j == last) issue_dH(sst, sb + OFF_XW + ((j + 1) & 1) * kXBuf, tmem + TM_DH, true);
           mma_commit(BAR(BAR_XWFREE0 + (j & 1)));
           mma_commit(BAR(BAR_DHREADY));
           if (kStateOnly) mma_commit(BAR(BAR_XFREE0 + (j & 1)));
@@ -418,10 +418,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
   } else if (conv_index(warp) >= 0) {
     // ---------------------------------------------------------------- conv + SiLU -> X, w o X
-    // Warp cw makes tokens 16cw..16cw+15; lane l channels 2l, 2l+1.  Raw row r of the X
-    // buffer holds time t0-3+r; token s reads rows s..s+3 (a register window) and then
-    // overwrites row s with its X row.  Rows 16cw+16..+18 belong to the next warp's tokens,
-    // so every warp reads them before the group barrier that precedes all writes.
+    // Warp cw makes tokens 16cw..16cw+15; lane l channels 2l, 2l+1.  Raw row r of the w o X
+    // buffer holds time t0-3+r; token s reads rows s..s+3 (a register window), then
+    // overwrites row s with its w o X row and writes its X row to row s of X.  Rows
+    // 16cw+16..+18 belong to the next warp's tokens, so every warp reads them before the
+    // group barrier that precedes all writes.
     // SiLU(u) = u * sigmoid(u) = h + h * tanh(h) with h = u / 2.  The conv accumulates h
     // directly (halved weights) in fp16 pairs -- the precision of the MMA operand it feeds,
     // 11 significant bits -- and one half2 tanh serves both channels.  The last chunk of a
@@ -457,8 +458,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       if (leader) TC_MARK(k, 13);
       if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, 1, abort_flag, a.err, 256)) break;
       if (leader) TC_MARK(k, 14);
-      // w o X[k % 2] was last read by MMA4 of chunk k-2
-      if (k >= 2 && !wg_wait(BAR(BAR_XWFREE0 + xb), ((k >> 1) - 1) & 1, leader, 1, abort_flag, a.err, 256))
+      // X[k % 2] was last read by MMA2 of chunk k-2 (MMA4 of chunk k-2 released w o X[k % 2]
+      // before the raw rows were loaded into it)
+      if (k >= 2 && !wg_wait(BAR(BAR_XFREE0 + xb), ((k >> 1) - 1) & 1, leader, 1, abort_flag, a.err, 256))
         break;
       // the low part of w o X goes to the other w o X buffer, last read by MMA4 of chunk k-1
       if (is_last && k >= 1 &&
@@ -469,11 +471,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const float cs_end = cs[QC - 1];
       const float wl = lane < kTokPerConvWarp ? __expf(cs_end - cs[tok0 + lane]) * dtv[tok0 + lane] : 0.f;
       const uint32_t wl2 = pack_f16(wl, wl);
-      unsigned char *xt = smem + OFF_X + xb * kXBuf + tok0 * 128;   // row tok0
-      unsigned char *xwt = smem + OFF_XW + xb * kTile + tok0 * 128;
-      unsigned char *xlt = smem + OFF_XW + lb * kTile + tok0 * 128;
-      // rows tok0 + r for r = 0..18 (tok0 is a multiple of 8, so row mod 8 = r mod 8)
-#define RAW(r) (*reinterpret_cast<const uint32_t *>(xt + (r) * 128 + loff[(r) & 7]))
+      unsigned char *xt = smem + OFF_X + xb * kTile + tok0 * 128;   // row tok0
+      unsigned char *xwt = smem + OFF_XW + xb * kXBuf + tok0 * 128;
+      unsigned char *xlt = smem + OFF_XW + lb * kXBuf + tok0 * 128;
+      // raw rows tok0 + r for r = 0..18 (tok0 is a multiple of 8, so row mod 8 = r mod 8)
+#define RAW(r) (*reinterpret_cast<const uint32_t *>(xwt + (r) * 128 + loff[(r) & 7]))
       uint32_t r0 = RAW(0), r1 = RAW(1), r2 = RAW(2);
       const int t0 = t_begin + k * QC;
       if (cw == 0 && t0 == 0) {  // history before the first token comes from the conv cache
