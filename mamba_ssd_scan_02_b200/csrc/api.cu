@@ -5,6 +5,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "plan.h"
 
@@ -20,9 +22,11 @@ constexpr long long kTargetCtas = 2 * 148;  // scan CTAs wanted in flight (2 per
 constexpr size_t kAlign = 256;
 
 int *device_error_ptr() {
+  static std::mutex mu;
   static int *ptrs[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
   if (!ptrs[dev]) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;

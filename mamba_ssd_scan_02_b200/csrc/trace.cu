@@ -1,4 +1,5 @@
 // trace.cu -- optional CUDA-event tracing of the library's kernel launches (host code).
+#include <atomic>
 #include <mutex>
 #include <string.h>
 #include <vector>
@@ -15,16 +16,16 @@ struct Rec {
 };
 
 std::mutex g_mu;
-bool g_on = false;
+std::atomic<bool> g_on{false};  // read without the lock on every launch
 std::vector<Rec> g_recs;  // events are created once and reused after each read
 size_t g_next = 0;
 
 }  // namespace
 
-bool trace_enabled() { return g_on; }
+bool trace_enabled() { return g_on.load(); }
 
 int trace_begin(cudaStream_t s) {
-  if (!g_on) return -1;
+  if (!g_on.load()) return -1;
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_next == g_recs.size()) {
     Rec r{};
@@ -51,8 +52,7 @@ extern "C" {
 
 int ssd_trace_enable(int on) {
   std::lock_guard<std::mutex> lk(ssd::g_mu);
-  const int prev = ssd::g_on ? 1 : 0;
-  ssd::g_on = on != 0;
+  const int prev = ssd::g_on.exchange(on != 0) ? 1 : 0;
   return prev;
 }
 
