@@ -454,18 +454,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     for (int k = 0; k < nck; ++k) {
       const int st = k & 1, xb = k & 1, lb = (k + 1) & 1;
       const bool is_last = (k == last);
-      if (!wg_wait(BAR(BAR_FULLX0 + xb), (k >> 1) & 1, leader, 1, abort_flag, a.err, 256)) break;
-      if (leader) TC_MARK(k, 13);
-      if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, 1, abort_flag, a.err, 256)) break;
-      if (leader) TC_MARK(k, 14);
-      // X[k % 2] was last read by MMA2 of chunk k-2 (MMA4 of chunk k-2 released w o X[k % 2]
-      // before the raw rows were loaded into it)
-      if (k >= 2 && !wg_wait(BAR(BAR_XFREE0 + xb), ((k >> 1) - 1) & 1, leader, 1, abort_flag, a.err, 256))
-        break;
-      // the low part of w o X goes to the other w o X buffer, last read by MMA4 of chunk k-1
-      if (is_last && k >= 1 &&
-          !wg_wait(BAR(BAR_XWFREE0 + lb), ((k - 1) >> 1) & 1, leader, 1, abort_flag, a.err, 256))
-        break;
+      // the leader waits for every input of the chunk, then one group barrier releases all
+      if (leader) {
+        bool ok = mbar_wait(BAR(BAR_FULLX0 + xb), (k >> 1) & 1, abort_flag, a.err);
+        if (ok) ok = mbar_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, abort_flag, a.err);
+        if (ok && k >= 2) ok = mbar_wait(BAR(BAR_XFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err);
+        if (ok && is_last && k >= 1) mbar_wait(BAR(BAR_XWFREE0 + lb), ((k - 1) >> 1) & 1, abort_flag, a.err);
+      }
+      named_bar(1, 256);
+      if (*abort_flag) break;
       const float *cs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
       const float *dtv = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
       const float cs_end = cs[QC - 1];
