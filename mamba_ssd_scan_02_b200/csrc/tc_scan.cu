@@ -460,6 +460,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (ok) ok = mbar_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, abort_flag, a.err);
         if (ok && k >= 2) ok = mbar_wait(BAR(BAR_XFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err);
         if (ok && is_last && k >= 1) mbar_wait(BAR(BAR_XWFREE0 + lb), ((k - 1) >> 1) & 1, abort_flag, a.err);
+        TC_MARK(k, 14);
       }
       named_bar(1, 256);
       if (*abort_flag) break;
@@ -579,6 +580,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       };
       if (is_last) tokens(std::true_type{});
       else tokens(std::false_type{});
+      if (leader) TC_MARK(k, 13);
 #undef RAW
       fence_proxy_async();
       named_bar(1, 256);
