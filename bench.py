@@ -611,11 +611,33 @@ def cpu_baseline(target_s: float = 10.0):
         else:
             reps = int(reps * grow) + 1
     frac = groups / cfg["ngroups"]
+    # the same oracle on one thread, on a sample sized for a few seconds
+    tok1 = max(64, min(tok, int(tok * 3.0 / max(dt / reps * cores, 1e-3))))
+    t0 = time.time()
+    o.ssd_prefill(dict(cfg, seqlen=tok1), inp["xBC"][:, :tok1], inp["dt"][:, :tok1], inp["A"], inp["D"],
+                  inp["dt_bias"], conv_w=inp["conv_w"], heads=(0, hpg), threads=1)
+    dt1 = time.time() - t0
     return {"value": round(reps * tok * frac / dt, 2), "unit": "tokens/s", "cores": cores,
-            "kind": "oracle",
+            "kind": "oracle", "cpu_model": cpu_model(),
             "sample": f"prefill_8k inputs, first {tok} tokens x heads 0-{groups * hpg - 1} "
                       f"({groups}/{cfg['ngroups']} of the layer) x {reps} run(s), fp64, "
-                      f"{dt:.1f} s"}
+                      f"{dt:.1f} s",
+            "single_thread": {"value": round(tok1 / cfg["ngroups"] / dt1, 2), "unit": "tokens/s",
+                              "cores": 1,
+                              "sample": f"first {tok1} tokens x heads 0-{hpg - 1} (1/{cfg['ngroups']} "
+                                        f"of the layer), fp64, {dt1:.1f} s"}}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 def reference_arm(args):

@@ -214,6 +214,15 @@ ssd_status_t ssd_get_device_error(void *stream);
 /* Version of this library as MAJOR*10000 + MINOR*100 + PATCH. */
 int ssd_version(void);
 
+/* Test hook for the failure path of the bounded device waits (not for production use).
+ * While set (chunk >= 0), every tensor-core prefill scan withholds the loads of that chunk's
+ * B/C tile, so the CTAs that wait for it give up after wait_limit_ns nanoseconds of device
+ * time instead of the normal 2 s, leave cleanly (loads drained, MMAs complete, tensor memory
+ * released) and latch SSD_ERR_TIMEOUT for ssd_get_device_error().  The outputs of such a call
+ * are undefined.  chunk < 0 turns the hook off.  Process-wide; not thread-safe with respect
+ * to prefills running concurrently on other host threads. */
+void ssd_test_stall_scan(int chunk, unsigned long long wait_limit_ns);
+
 /* Kernel tracing for measurement tools.  While enabled, every kernel the library launches
  * is bracketed by two CUDA events recorded on the stream it is launched on (so the timing
  * covers exactly that kernel).  Off by default; do not enable it while a stream is being

@@ -5,6 +5,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -16,6 +17,11 @@ namespace ssd {
 __device__ int g_device_error_word;
 
 namespace {
+
+// Test hook (ssd_test_stall_scan): chunk index + 1 whose stage the tensor-core scan withholds,
+// and the wait limit its bounded waits then use; 0 = off.
+std::atomic<int> g_stall_chunk1{0};
+std::atomic<unsigned long long> g_stall_wait_ns{0};
 
 constexpr int kMaxDevices = 64;
 constexpr long long kTargetCtas = 2 * 148;  // scan CTAs wanted in flight (2 per B200 SM)
@@ -97,12 +103,30 @@ void tc_segments(const ssd_config_t *c, int *n, int *len) {
   choose_segments(c, kTcTile, kTcTarget, n, len);
 }
 
-// The two scan paths use the workspace differently; the layouts overlap (a call uses one).
+// The scan path a prefill with this config takes on the current device: the tensor-core scan
+// for bf16 unless the CUDA-core one is requested (an explicit tensor-core request on a device
+// without it is refused later, but is sized for that path).
+bool prefill_uses_tc(const ssd_config_t *c) {
+  if (c->kernel == SSD_KERNEL_SIMT) return false;
+  if (c->kernel == SSD_KERNEL_TENSOR) return true;
+  return c->io_dtype == SSD_BF16 && tc_scan_available();
+}
+
+// The tensor-core scan applies the z gate itself and leaves only a rescale for the group norm
+// when every norm group is made of whole heads (and the rescale's per-row factors fit in
+// shared memory); otherwise it writes the fp32 output and the separate gated norm follows.
+bool tc_fused_norm(const ssd_config_t *c) {
+  return c->io_dtype == SSD_BF16 && c->norm_groups > 0 && c->nheads % c->norm_groups == 0 &&
+         2LL * c->nheads + c->norm_groups <= 12 * 1024;
+}
+
+// The two scan paths use the workspace differently; the layouts overlap (a call uses one),
+// and the size asked for is that of the path the call takes.
 struct WsLayout {
   // CUDA-core path
   size_t u, dte, yf, seg_state, seg_decay, simt_end;
   // tensor-core path
-  size_t tc_bc, tc_dte, tc_cs, tc_yf, tc_seg_state, tc_seg_decay, tc_dh, tc_end;
+  size_t tc_bc, tc_dte, tc_cs, tc_yf, tc_q, tc_ssq, tc_seg_state, tc_seg_decay, tc_dh, tc_end;
   int Lpad;
   size_t total;
 };
@@ -132,7 +156,14 @@ WsLayout prefill_layout(const ssd_config_t *c) {
   w.tc_bc = off;   off = round_up(off + T * 2 * c->ngroups * c->dstate * 2, kAlign);
   w.tc_dte = off;  off = round_up(off + (size_t)c->batch * c->nheads * w.Lpad * 4, kAlign);
   w.tc_cs = off;   off = round_up(off + (size_t)c->batch * c->nheads * w.Lpad * 4, kAlign);
-  w.tc_yf = off;   if (c->norm_groups > 0) off = round_up(off + T * d_inner * 4, kAlign);
+  w.tc_yf = w.tc_q = w.tc_ssq = off;
+  if (tc_fused_norm(c)) {
+    off = round_up(off + T * d_inner * 2, kAlign);
+    w.tc_ssq = off;
+    off = round_up(off + T * c->nheads * 4, kAlign);
+  } else if (c->norm_groups > 0) {
+    off = round_up(off + T * d_inner * 4, kAlign);
+  }
   w.tc_seg_state = w.tc_seg_decay = off;
   if (n_seg > 1) {
     off = round_up(off + (size_t)n_seg * state, kAlign);
@@ -141,7 +172,7 @@ WsLayout prefill_layout(const ssd_config_t *c) {
   }
   w.tc_dh = off;   off = round_up(off + state + (size_t)c->batch * c->nheads * 4, kAlign);
   w.tc_end = off;
-  w.total = w.simt_end > w.tc_end ? w.simt_end : w.tc_end;
+  w.total = prefill_uses_tc(c) ? w.tc_end : w.simt_end;
   return w;
 }
 
@@ -239,22 +270,18 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
   p.csi = a->conv_state_in; p.y = a->y; p.ys = a->y_row_stride; p.h_final = a->h_final;
   p.cso = a->conv_state_out;
   p.err = device_error_ptr();
+  p.stall_chunk1 = g_stall_chunk1.load();
+  p.stall_wait_ns = g_stall_wait_ns.load();
 
   if (!has_tokens) return from_cuda(traced("ssd_carry", s, [&] { return launch_carry_only(p, s); }));
 
+  const bool use_tc = prefill_uses_tc(c);
+  if (use_tc && (!p.bf16 || !tc_scan_available())) return SSD_ERR_UNSUPPORTED;
   const WsLayout lay = prefill_layout(c);
   if (a->workspace_bytes < lay.total || (lay.total && !a->workspace) ||
       (reinterpret_cast<uintptr_t>(a->workspace) % kAlign) != 0)
     return SSD_ERR_WORKSPACE;
   char *ws = static_cast<char *>(a->workspace);
-
-  bool use_tc = false;
-  if (c->kernel == SSD_KERNEL_TENSOR) {
-    if (!p.bf16 || !tc_scan_available()) return SSD_ERR_UNSUPPORTED;
-    use_tc = true;
-  } else if (c->kernel == SSD_KERNEL_AUTO) {
-    use_tc = p.bf16 && tc_scan_available();
-  }
 
   if (use_tc) {
     tc_segments(c, &p.n_seg, &p.seg_len);
@@ -262,7 +289,11 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
     p.bc = ws + lay.tc_bc;
     p.dte_hm = reinterpret_cast<float *>(ws + lay.tc_dte);
     p.cs_hm = reinterpret_cast<float *>(ws + lay.tc_cs);
-    p.yf = c->norm_groups > 0 ? reinterpret_cast<float *>(ws + lay.tc_yf) : nullptr;
+    const bool fused_norm = tc_fused_norm(c);
+    if (fused_norm && a->norm_w && !aligned16(a->norm_w)) return SSD_ERR_ALIGNMENT;
+    p.yf = c->norm_groups > 0 && !fused_norm ? reinterpret_cast<float *>(ws + lay.tc_yf) : nullptr;
+    p.qn = fused_norm ? reinterpret_cast<__half *>(ws + lay.tc_q) : nullptr;
+    p.ssq = fused_norm ? reinterpret_cast<float *>(ws + lay.tc_ssq) : nullptr;
     p.seg_state = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.tc_seg_state) : nullptr;
     p.seg_decay = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.tc_seg_decay) : nullptr;
     p.tail_dh = p.h_final ? reinterpret_cast<float *>(ws + lay.tc_dh) : nullptr;
@@ -300,7 +331,11 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
       SSD_TRY(side.join());
       SSD_TRY(traced("ssd_tail_fold", s, [&] { return launch_tail_fold(p, s); }));
     }
-    if (p.norm_groups > 0) SSD_TRY(traced("ssd_gated_norm", s, [&] { return launch_gated_norm(p, s); }));
+    if (p.qn) {
+      SSD_TRY(traced("ssd_norm_rescale", s, [&] { return launch_norm_rescale(p, s); }));
+    } else if (p.norm_groups > 0) {
+      SSD_TRY(traced("ssd_gated_norm", s, [&] { return launch_gated_norm(p, s); }));
+    }
     if (!cso_early) SSD_TRY(traced("ssd_conv_state_out", s, [&] { return launch_conv_state_out(p, s); }));
     return SSD_OK;
   }
@@ -552,5 +587,10 @@ ssd_status_t ssd_get_device_error(void *stream) {
 }
 
 int ssd_version(void) { return 100; }
+
+void ssd_test_stall_scan(int chunk, unsigned long long wait_limit_ns) {
+  g_stall_wait_ns.store(wait_limit_ns);
+  g_stall_chunk1.store(chunk >= 0 ? chunk + 1 : 0);
+}
 
 }  // extern "C"

@@ -146,8 +146,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int m0, n0;
       tile_coords(tile, mb_count, nb_count, m0, n0);
       if (leader) mbar_wait(GB(G_ACCF + buf), (local >> 1) & 1, abort_flag, g.err);
-      named_bar(1, 128);
-      if (*abort_flag) break;
+      if (named_bar_or(1, 128, *abort_flag != 0)) break;
       tc_fence_after();
       const int m = m0 + 32 * ew + lane;
       __nv_bfloat16 *crow = g.C + (long long)m * g.ldc;

@@ -117,6 +117,73 @@ __global__ void __launch_bounds__(1024) gated_norm_v8_kernel(
   store8(out + row * os + c, g);
 }
 
+// Second half of the gated norm fused into the tensor-core scan.  The scan's output stage
+// has gated each token's head (g = y * silu(z), or g = y when normalising first) and stored
+//   q_h   = g / s_h  in fp16, with s_h = sqrt(mean of g^2 over the head's 64 channels)
+//   ssq_h = sum of g^2 over those channels (fp32, per token row and head),
+// so |q| <= 8 and fp16 keeps 11 significant bits of it with no risk of overflow.  A norm group
+// covers whole heads, and its statistic is the sum of its heads' ssq:
+//   out = q * s_h * rsqrt(sum_{h in group} ssq_h / gs + eps) * w   (* silu(z) normalising first).
+// One CTA per token row: the row's per-head factors are formed in shared memory, then every
+// thread rescales 8 channels at a time (16-byte loads and stores).
+constexpr int kRescaleThreads = 256;
+
+__global__ void __launch_bounds__(kRescaleThreads) norm_rescale_kernel(
+    const __half *__restrict__ q, const float *__restrict__ ssq, const __nv_bfloat16 *__restrict__ z,
+    long long zs, const __nv_bfloat16 *__restrict__ w, __nv_bfloat16 *__restrict__ out, long long os,
+    int H, int hpn, int ng, int d_inner, float eps, int nbg) {
+  extern __shared__ float rsm[];
+  float *sq = rsm, *fac = rsm + H, *gsum = rsm + 2 * H;
+  const long long row = blockIdx.x;
+  for (int i = threadIdx.x; i < H; i += kRescaleThreads) sq[i] = ssq[row * H + i];
+  __syncthreads();
+  for (int gi = threadIdx.x; gi < ng; gi += kRescaleThreads) {  // fixed order: reproducible
+    float t = 0.f;
+    for (int j = 0; j < hpn; ++j) t += sq[gi * hpn + j];
+    gsum[gi] = rsqrtf(t / (float)(hpn * kHeadDim) + eps);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < H; i += kRescaleThreads)
+    fac[i] = sqrtf(sq[i] * (1.f / kHeadDim)) * gsum[i / hpn];
+  __syncthreads();
+  const __half *qr = q + row * d_inner;
+  for (int c = threadIdx.x * 8; c < d_inner; c += kRescaleThreads * 8) {
+    const uint4 qu = __ldcs(reinterpret_cast<const uint4 *>(qr + c));
+    const __half2 *q2 = reinterpret_cast<const __half2 *>(&qu);
+    const float f = fac[c / kHeadDim];
+    float v[8], wv[8];
+    if (w) {
+      load8(w + c, wv);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) wv[i] = 1.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 qf = __half22float2(q2[i]);
+      v[2 * i] = qf.x * f * wv[2 * i];
+      v[2 * i + 1] = qf.y * f * wv[2 * i + 1];
+    }
+    if (nbg) {
+      float zv[8];
+      load8(z + row * zs + c, zv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] *= silu(zv[i]);
+    }
+    store8(out + row * os + c, v);
+  }
+}
+
+cudaError_t launch_norm_rescale(const PrefillPlan &p, cudaStream_t s) {
+  const int hpn = p.H / p.norm_groups;
+  const size_t smem = (size_t)(2 * p.H + p.norm_groups) * sizeof(float);
+  if (smem > 48 * 1024) return cudaErrorInvalidValue;
+  norm_rescale_kernel<<<(unsigned)((long long)p.B * p.L), kRescaleThreads, smem, s>>>(
+      p.qn, p.ssq, (const __nv_bfloat16 *)p.z, p.zs, (const __nv_bfloat16 *)p.norm_w,
+      (__nv_bfloat16 *)p.y, p.ys, p.H, hpn, p.norm_groups, p.d_inner, p.eps, p.nbg);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s) {
   const int gs = p.d_inner / p.norm_groups;
   dim3 grid((unsigned)((long long)p.B * p.L), p.norm_groups);

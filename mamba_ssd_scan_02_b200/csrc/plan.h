@@ -1,6 +1,7 @@
 // plan.h -- resolved launch parameters shared by the C-ABI layer and the kernel launchers.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 
@@ -40,8 +41,15 @@ struct PrefillPlan {
   float *tail_dh;    // [B, H, P, N] fp32 contribution of the final state's last chunks, from a
                      // zero state (tensor path; null when no final state is written)
   float *tail_dec;   // [B, H] decay over those chunks
+  __half *qn;        // [B, L, d_inner] fp16 head-normalised gated output (tensor path, fused
+                     // gate: the scan gates and writes these, the rescale finishes the norm)
+  float *ssq;        // [B, L, H] sum of squares of each head's gated output
   int Lpad;
   int *err;          // device error word
+  // test hook (tensor-core scan): 0 = off; c + 1 = the producer withholds chunk c's stage so
+  // that the bounded waits run out after stall_wait_ns
+  int stall_chunk1;
+  unsigned long long stall_wait_ns;
 };
 
 struct DecodePlan {
@@ -87,6 +95,7 @@ cudaError_t launch_state_tail(const PrefillPlan &p, cudaStream_t s);
 cudaError_t launch_tail_fold(const PrefillPlan &p, cudaStream_t s);
 // norms (norm.cu)
 cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s);          // fp32 yf -> y
+cudaError_t launch_norm_rescale(const PrefillPlan &p, cudaStream_t s);        // qn, ssq -> y
 cudaError_t launch_rmsnorm_bf16(const void *x, const void *w, void *out, long long rows, int width,
                                 float eps, cudaStream_t s);
 // decode (decode.cu)

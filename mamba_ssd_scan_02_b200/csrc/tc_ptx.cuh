@@ -60,18 +60,20 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete.  Gives up after ~2 s of device time
-// (the waits here normally last microseconds): sets *abort and latches SSD_ERR_TIMEOUT.
-// Each try sleeps up to ~0.2 ms, so the clock and the abort flag are checked every few tries.
+// Waits for the phase with the given parity to complete.  Gives up after `limit_ns` of device
+// time (2 s by default; the waits here normally last microseconds): sets *abort and latches
+// SSD_ERR_TIMEOUT.  Each try sleeps up to ~0.2 ms, so the clock and the abort flag are checked
+// every few tries.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                          int *err) {
+                                          int *err, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 3u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > 2000000000ull) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort = 1;
         if (err) atomicCAS(err, 0, (int)SSD_ERR_TIMEOUT);
         return false;
@@ -117,6 +119,22 @@ __device__ __forceinline__ void fence_proxy_async() {
 // Named barrier over `count` threads.
 __device__ __forceinline__ void named_bar(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier over `count` threads that also ORs one predicate over them: every thread gets
+// the same result, so a branch taken on it (such as leaving a loop after an abort) is uniform
+// across the group even when the predicate's source changes while the threads arrive.
+__device__ __forceinline__ bool named_bar_or(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
 }
 
 // ---- tcgen05 --------------------------------------------------------------------------------

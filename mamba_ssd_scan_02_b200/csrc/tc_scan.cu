@@ -68,9 +68,9 @@ namespace {
 using namespace tc;
 
 constexpr int QC = 128;              // tokens per chunk
-constexpr int kThreadsTC = 640;       // 20 warps
-constexpr int kConvWarps = 8;          // see conv_index()
-constexpr int kTokPerConvWarp = QC / kConvWarps;  // 16
+constexpr int kThreadsTC = 640;       // 20 warps (roles below)
+constexpr int kConvWarps = 4;
+constexpr int kTokPerConvWarp = QC / kConvWarps;  // 32
 constexpr uint32_t kTile = 16384;    // one 128-row x 128-byte operand box
 // per-stage layout (bytes)
 constexpr uint32_t OFF_C = 0;                 // C tile: channels 0-63 | 64-127
@@ -90,7 +90,8 @@ constexpr uint32_t OFF_H = OFF_XW + 2 * kXBuf;      // h copy [n][p] fp16, 16 KB
 constexpr uint32_t OFF_CF = OFF_H + kTile;          // column factors, 128 fp32
 constexpr uint32_t OFF_CSM = OFF_CF + 512;          // the mask's copies of cs and dt
 constexpr uint32_t OFF_DTM = OFF_CSM + 512;
-constexpr uint32_t OFF_BAR = OFF_DTM + 512;
+constexpr uint32_t OFF_ET = OFF_DTM + 512;          // e^{cs_t} of chunk k in ET[k % 2] (mask -> output)
+constexpr uint32_t OFF_BAR = OFF_ET + 1024;
 // Barriers.  Every event that can recur before its consumer has observed the previous
 // occurrence has one barrier per buffer, so that a parity test never sees two phases at once.
 enum {
@@ -106,10 +107,10 @@ enum {
   BAR_DHFREE,                  // dH of chunk k read by the state warps
   BAR_HTFREE,                  // h tile (h_{k-1}) read by MMA3 of chunk k
   BAR_HREADY,                  // h tile holds h_k (state warps)
-  BAR_YREADY0, BAR_YREADY1,    // Yi and Ys of chunk k in TMEM (MMA2 commit)
+  BAR_YREADY0, BAR_YREADY1,    // Yi and Ys of chunk k in TMEM (MMA2 and MMA3 commits)
   BAR_YFREE0, BAR_YFREE1,      // Yi and Ys of chunk k read by the output warps
   BAR_XLOREADY,                // low part of w o X of the last chunk written
-  BAR_DONE,
+  BAR_DONE_A, BAR_DONE_B,      // every MMA of issuer A / B complete (before TMEM is freed)
   kNumBars
 };
 constexpr uint32_t OFF_MISC = OFF_BAR + 8 * 32;   // [0] TMEM base, [1] abort flag
@@ -149,8 +150,17 @@ struct TcArgs {
   __nv_bfloat16 *y;        // output (no gate) ...
   long long ys;
   float *yf;               // ... or fp32 pre-norm output [B, L, d_inner] when a gated norm follows
+  __half *qn;              // ... or (fused gate) the gated output of each head divided by its RMS
+  float *ssq;              //     over the head's 64 channels, fp16 [B, L, d_inner], and its sum
+                           //     of squares, fp32 [B, L, H]; a rescale pass finishes the norm
+  const __nv_bfloat16 *z;  // gate [B, L, d_inner] (fused gate, gate first)
+  long long zs;
+  int nbg;                 // 1: normalise before gating (the gate is applied by the rescale)
   int d_inner;
   int *err;
+  unsigned long long wait_ns;  // limit of every bounded wait
+  int debug_skip_chunk;        // test hook (-1 = off): the producer stops before loading this
+                               // chunk's stage, so its consumers' bounded waits run out
 };
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -166,13 +176,14 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   return __bfloat1622float2(v);
 }
 
-// A warpgroup-uniform bounded wait: one leader thread waits on the mbarrier, then the
-// group syncs on its named barrier and reads the (shared) abort flag.
+// A group-uniform bounded wait: one leader thread waits on the mbarrier, then the group
+// syncs on its named barrier, which ORs every thread's view of the abort flag so that all of
+// them take the same branch.
 __device__ __forceinline__ bool wg_wait(uint32_t bar, uint32_t parity, bool leader, int nb,
-                                        volatile int *abort_flag, int *err, int nthreads = 128) {
-  if (leader) mbar_wait(bar, parity, abort_flag, err);
-  named_bar(nb, nthreads);
-  return *abort_flag == 0;
+                                        volatile int *abort_flag, int *err, uint64_t limit_ns,
+                                        int nthreads = 128) {
+  if (leader) mbar_wait(bar, parity, abort_flag, err, limit_ns);
+  return !named_bar_or(nb, nthreads, *abort_flag != 0);
 }
 
 // ---- MMA issue (single thread) ---------------------------------------------------------
@@ -213,21 +224,14 @@ __device__ __forceinline__ void issue_dH(uint32_t stage, uint32_t xwbase, uint32
     mma_f16_ss(tDH, desc_adv(a0, j * 2048), desc_adv(b0, j * 2048), IDESC_DH, (j > 0 || acc) ? 1u : 0u);
 }
 
-// Conv warps: 2, 3, 4, 6, 7, 8, 10, 11 -- none on the sub-partition of warp 1 (warps 1, 5, 9,
-// ...), whose single MMA-issuing thread would otherwise be starved of issue slots.
-__device__ __forceinline__ int conv_index(int warp) {
-  switch (warp) {
-    case 2: return 0;
-    case 3: return 1;
-    case 4: return 2;
-    case 6: return 3;
-    case 7: return 4;
-    case 8: return 5;
-    case 10: return 6;
-    case 11: return 7;
-    default: return -1;
-  }
-}
+// Warp roles.  Each warp index w runs on SM sub-partition w % 4, and a warp reaches only the
+// TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, so every role that touches TMEM rows (mask, state,
+// output) has one warp per sub-partition.  The two MMA-issuing threads sit on sub-partitions
+// 1 and 2; the conv warps, one per sub-partition, spread their issue slots evenly.
+constexpr int kWarpTma = 0, kWarpIssueA = 1, kWarpIssueB = 2;
+constexpr int kWarpMask0 = 4, kWarpState0 = 8, kWarpOut0 = 12, kWarpConv0 = 16;
+// named barriers (0 is __syncthreads)
+constexpr int kNbConv = 1, kNbMask = 2, kNbState = 3, kNbOut = 4;
 
 // Row r (128 bytes) of a 128-byte-swizzled tile: 16-byte chunk c sits at chunk c ^ (r & 7).
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
@@ -258,6 +262,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const int t_end = min(a.L, t_begin + a.seg_len);
   const int nck = t_end > t_begin ? (t_end - t_begin + QC - 1) / QC : 0;
   const int last = nck - 1;
+  const uint64_t lim = a.wait_ns;
   const uint32_t bar0 = sb + OFF_BAR;
 #define BAR(i) (bar0 + 8u * (uint32_t)(i))
   uint32_t *misc = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
@@ -266,18 +271,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   if (tid == 0) {
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t cnt = 1;
-      if (i == BAR_EMPTY0 || i == BAR_EMPTY1) cnt = kStateOnly ? 3 : 4;  // + mask warps
+      if (i == BAR_EMPTY0 || i == BAR_EMPTY1) cnt = kStateOnly ? 3 : 5;
+      if (i == BAR_YREADY0 || i == BAR_YREADY1) cnt = 2;
       mbar_init(BAR(i), cnt);
     }
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == kWarpTma && lane == 0) {
     prefetch_tmap(&tm_bc);
     prefetch_tmap(&tm_x);
   }
-  if (warp == 1) {
+  if (warp == kWarpIssueA) {
     tmem_alloc(sb + OFF_MISC, TM_COLS);
     tmem_relinquish();
   }
@@ -286,23 +292,25 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   tc_fence_after();
   const uint32_t tmem = misc[0];
 
-  if (warp == 0) {
+  if (warp == kWarpTma) {
     // ---------------------------------------------------------------- TMA producer
     // Raw x rows of chunk k go to w o X[k % 2] once MMA4 of chunk k-2 has released it; the
-    // B/C tiles, dt and prefix sums go to stage k % 2 once chunk k-2's consumers released it.
+    // B/C tiles, dt and prefix sums go to stage k % 2 once chunk k-2's readers released it.
     if (lane == 0) {
-      int k = 0, nx = 0, nbc = 0;
-      for (; k < nck; ++k) {
+      int nx = 0, nbc = 0;
+      for (int k = 0; k < nck; ++k) {
         const int xb = k & 1, st = k & 1;
         const int t0 = t_begin + k * QC;
-        if (k >= 2 && !mbar_wait(BAR(BAR_XWFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err)) break;
+        if (k >= 2 && !mbar_wait(BAR(BAR_XWFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err, lim)) break;
+        TC_MARK(k, 13);
         mbar_arrive_expect_tx(BAR(BAR_FULLX0 + xb), kRawRows * 128);
         tma_load_3d(sb + OFF_XW + xb * kXBuf, &tm_x, h * 64, t0 - 3, b, BAR(BAR_FULLX0 + xb));
         ++nx;
-        if (k >= 2 && !mbar_wait(BAR(BAR_EMPTY0 + st), ((k >> 1) - 1) & 1, abort_flag, a.err)) break;
+        if (a.debug_skip_chunk == k) break;  // test hook: stage k never arrives (see TcArgs)
+        if (k >= 2 && !mbar_wait(BAR(BAR_EMPTY0 + st), ((k >> 1) - 1) & 1, abort_flag, a.err, lim)) break;
         const uint32_t sst = sb + st * kStage;
         const uint32_t full = BAR(BAR_FULL0 + st);
-        TC_MARK(k, 12);
+        TC_MARK(k, 14);
         mbar_arrive_expect_tx(full, (kStateOnly ? 2 * kTile : 4 * kTile) + 1024);
         const int cB = g * 128, cC = a.G * 128 + g * 128;
         if (!kStateOnly) {
@@ -323,112 +331,93 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       for (int j = (nbc >= 2 ? nbc - 2 : 0); j < nbc; ++j)
         mbar_wait(BAR(BAR_FULL0 + (j & 1)), (j >> 1) & 1, &never_abort, a.err);
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    // Issues each chunk's four MMA groups as soon as their inputs are ready, whatever the
-    // order, so that no group waits behind another one that is still blocked:
-    //   MMA1 S(j)   stage j loaded; S[j % 2] free (MMA2 of chunk j-2 issued, its output read)
-    //   MMA4 dH(j)  X(j) and w o X(j) written; dH of chunk j-1 read by the state warps
-    //   MMA3 Ys(j)  after MMA1(j); h_{j-1} in the h tile
-    //   MMA2 Yi(j)  after MMA3(j) and MMA4(j); S~(j) written by the mask warps
-    // A commit after each group signals its consumers; stage j is released by a commit after
-    // the last of MMA1/MMA3/MMA4 of chunk j.  Polling sleeps briefly when nothing is ready and
-    // gives up (abort + SSD_ERR_TIMEOUT) after ~2 s without progress.
+  } else if (warp == kWarpIssueA) {
+    // ---------------------------------------------------------------- MMA issuer A: the state
+    // chain.  Per chunk k: MMA4 dH(k) (once w o X(k) is written and the state warps have read
+    // dH(k-1)), then MMA3 Ys(k) = C h_{k-1}^T (once the h tile holds h_{k-1} and the output
+    // warps have read Ys(k-2)).  Every wait blocks in hardware, so the thread issues nothing
+    // while it waits.
     if (lane == 0) {
-      int nS = kStateOnly ? nck : 0, nD = 0, nYs = kStateOnly ? nck : 0, nYi = kStateOnly ? nck : 0;
-      auto stage_done = [&](int j) {  // all readers of stage j issued?
-        return nD > j && (kStateOnly || (nS > j && nYs > j));
-      };
-      uint64_t t_prog = globaltimer();
-      uint32_t nap = 32;  // sleep between polls: doubles up to 256 ns while nothing is ready
-      bool ok = true;
-      while (ok && (nD < nck || nYi < nck)) {
-        bool prog = false;
-        if (nYi < nck && nYi < nYs && nYi < nD && mbar_test(BAR(BAR_STREADY0 + (nYi & 1)), (nYi >> 1) & 1)) {
-          const int j = nYi;
-          tc_fence_after();
-          TC_MARK(j, 11);
-          const uint32_t tS = tmem + ((j & 1) ? TM_S1 : TM_S0);
-          issue_Yi(tS, sb + OFF_X + (j & 1) * kTile, tS + TM_YI_OFF);
-          mma_commit(BAR(BAR_YREADY0 + (j & 1)));
-          mma_commit(BAR(BAR_XFREE0 + (j & 1)));
-          ++nYi;
-          prog = true;
+      for (int k = 0; k < nck; ++k) {
+        const int st = k & 1;
+        const uint32_t sst = sb + st * kStage;
+        if (!mbar_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, abort_flag, a.err, lim)) break;
+        if (!mbar_wait(BAR(BAR_XREADY0 + st), (k >> 1) & 1, abort_flag, a.err, lim)) break;
+        if (k == last && !mbar_wait(BAR(BAR_XLOREADY), 0, abort_flag, a.err, lim)) break;
+        if (k >= 1 && !mbar_wait(BAR(BAR_DHFREE), (k - 1) & 1, abort_flag, a.err, lim)) break;
+        tc_fence_after();
+        TC_MARK(k, 9);
+        issue_dH(sst, sb + OFF_XW + st * kXBuf, tmem + TM_DH, false);
+        // last chunk: the low part of w o X (in the other w o X buffer) for the final state
+        if (k == last) issue_dH(sst, sb + OFF_XW + ((k + 1) & 1) * kXBuf, tmem + TM_DH, true);
+        mma_commit(BAR(BAR_XWFREE0 + st));
+        mma_commit(BAR(BAR_DHREADY));
+        if (kStateOnly) {
+          mma_commit(BAR(BAR_EMPTY0 + st));
+          continue;
         }
-        if (nYs < nck && nYs < nS && mbar_test(BAR(BAR_HREADY), nYs & 1)) {
-          const int j = nYs;
-          tc_fence_after();
-          TC_MARK(j, 9);
-          issue_Ys(sb + (j & 1) * kStage, sb + OFF_H, tmem + ((j & 1) ? TM_YS1 : TM_YS0));
-          mma_commit(BAR(BAR_HTFREE));
-          ++nYs;
-          if (stage_done(j)) mma_commit(BAR(BAR_EMPTY0 + (j & 1)));
-          prog = true;
-        }
-        if (nD < nck && (kStateOnly || nD < nS) &&
-            mbar_test(BAR(BAR_XREADY0 + (nD & 1)), (nD >> 1) & 1) &&
-            (nD == 0 || mbar_test(BAR(BAR_DHFREE), (nD - 1) & 1)) &&
-            (nD != last || mbar_test(BAR(BAR_XLOREADY), 0)) &&
-            (!kStateOnly || mbar_test(BAR(BAR_FULL0 + (nD & 1)), (nD >> 1) & 1))) {
-          const int j = nD;
-          tc_fence_after();
-          TC_MARK(j, 8);
-          const uint32_t sst = sb + (j & 1) * kStage;
-          issue_dH(sst, sb + OFF_XW + (j & 1) * kXBuf, tmem + TM_DH, false);
-          // last chunk: the low part of w o X (in the other w o X buffer) for the final state
-          if (j == last) issue_dH(sst, sb + OFF_XW + ((j + 1) & 1) * kXBuf, tmem + TM_DH, true);
-          mma_commit(BAR(BAR_XWFREE0 + (j & 1)));
-          mma_commit(BAR(BAR_DHREADY));
-          if (kStateOnly) mma_commit(BAR(BAR_XFREE0 + (j & 1)));
-          ++nD;
-          if (stage_done(j)) mma_commit(BAR(BAR_EMPTY0 + (j & 1)));
-          prog = true;
-        }
-        if (nS < nck && nS <= nYi + 1 && mbar_test(BAR(BAR_FULL0 + (nS & 1)), (nS >> 1) & 1) &&
-            (nS < 2 || mbar_test(BAR(BAR_YFREE0 + (nS & 1)), ((nS >> 1) - 1) & 1))) {
-          const int j = nS;
-          tc_fence_after();
-          TC_MARK(j, 10);
-          issue_S(sb + (j & 1) * kStage, tmem + ((j & 1) ? TM_S1 : TM_S0));
-          mma_commit(BAR(BAR_SREADY0 + (j & 1)));
-          ++nS;
-          if (stage_done(j)) mma_commit(BAR(BAR_EMPTY0 + (j & 1)));
-          prog = true;
-        }
-        if (prog) {
-          t_prog = globaltimer();
-          nap = 32;
-        } else {
-          if (*abort_flag) {
-            ok = false;
-          } else if (globaltimer() - t_prog > 2000000000ull) {
-            *abort_flag = 1;
-            if (a.err) atomicCAS(a.err, 0, (int)SSD_ERR_TIMEOUT);
-            ok = false;
-          } else {
-            __nanosleep(nap);
-            nap = nap < 256 ? 2 * nap : 256;
-          }
-        }
+        if (!mbar_wait(BAR(BAR_HREADY), k & 1, abort_flag, a.err, lim)) break;
+        if (k >= 2 && !mbar_wait(BAR(BAR_YFREE0 + st), ((k >> 1) - 1) & 1, abort_flag, a.err, lim)) break;
+        tc_fence_after();
+        TC_MARK(k, 10);
+        issue_Ys(sst, sb + OFF_H, tmem + (st ? TM_YS1 : TM_YS0));
+        mma_commit(BAR(BAR_HTFREE));
+        mma_commit(BAR(BAR_YREADY0 + st));
+        mma_commit(BAR(BAR_EMPTY0 + st));
       }
       // no MMA may still be running when TMEM is released
-      mma_commit(BAR(BAR_DONE));
+      mma_commit(BAR(BAR_DONE_A));
       int never_abort = 0;
-      mbar_wait(BAR(BAR_DONE), 0, &never_abort, a.err);
+      mbar_wait(BAR(BAR_DONE_A), 0, &never_abort, a.err);
     }
-  } else if (conv_index(warp) >= 0) {
+  } else if (warp == kWarpIssueB) {
+    // ---------------------------------------------------------------- MMA issuer B: the S
+    // chain.  MMA1 S(j) = C B^T once stage j is loaded and S[j % 2] is free (the output warps
+    // have read Yi(j-2) from it); MMA2 Yi(k) = S~ X once the mask warps have written S~(k).
+    // MMA1 of chunk k+1 is issued before MMA2 of chunk k, so that the mask of chunk k+1 can
+    // run while MMA2 and the output of chunk k do.
+    if (!kStateOnly && lane == 0) {
+      auto mma1 = [&](int j) -> bool {
+        const int st = j & 1;
+        if (!mbar_wait(BAR(BAR_FULL0 + st), (j >> 1) & 1, abort_flag, a.err, lim)) return false;
+        if (j >= 2 && !mbar_wait(BAR(BAR_YFREE0 + st), ((j >> 1) - 1) & 1, abort_flag, a.err, lim)) return false;
+        tc_fence_after();
+        TC_MARK(j, 11);
+        issue_S(sb + st * kStage, tmem + (st ? TM_S1 : TM_S0));
+        mma_commit(BAR(BAR_SREADY0 + st));
+        mma_commit(BAR(BAR_EMPTY0 + st));
+        return true;
+      };
+      bool ok = nck > 0 ? mma1(0) : true;
+      for (int k = 0; ok && k < nck; ++k) {
+        const int st = k & 1;
+        if (k + 1 < nck && !(ok = mma1(k + 1))) break;
+        if (!(ok = mbar_wait(BAR(BAR_STREADY0 + st), (k >> 1) & 1, abort_flag, a.err, lim))) break;
+        if (!(ok = mbar_wait(BAR(BAR_XREADY0 + st), (k >> 1) & 1, abort_flag, a.err, lim))) break;
+        tc_fence_after();
+        TC_MARK(k, 12);
+        const uint32_t tS = tmem + (st ? TM_S1 : TM_S0);
+        issue_Yi(tS, sb + OFF_X + st * kTile, tS + TM_YI_OFF);
+        mma_commit(BAR(BAR_XFREE0 + st));
+        mma_commit(BAR(BAR_YREADY0 + st));
+      }
+      mma_commit(BAR(BAR_DONE_B));
+      int never_abort = 0;
+      mbar_wait(BAR(BAR_DONE_B), 0, &never_abort, a.err);
+    }
+  } else if (warp >= kWarpConv0 && warp < kWarpConv0 + kConvWarps) {
     // ---------------------------------------------------------------- conv + SiLU -> X, w o X
-    // Warp cw makes tokens 16cw..16cw+15; lane l channels 2l, 2l+1.  Raw row r of the w o X
+    // Warp cw makes tokens 32cw..32cw+31; lane l channels 2l, 2l+1.  Raw row r of the w o X
     // buffer holds time t0-3+r; token s reads rows s..s+3 (a register window), then
     // overwrites row s with its w o X row and writes its X row to row s of X.  Rows
-    // 16cw+16..+18 belong to the next warp's tokens, so every warp reads them before the
+    // 32cw+32..+34 belong to the next warp's tokens, so every warp reads them before the
     // group barrier that precedes all writes.
     // SiLU(u) = u * sigmoid(u) = h + h * tanh(h) with h = u / 2.  The conv accumulates h
     // directly (halved weights) in fp16 pairs -- the precision of the MMA operand it feeds,
     // 11 significant bits -- and one half2 tanh serves both channels.  The last chunk of a
     // segment, whose newest tokens dominate the final state, uses fp32 and the exact SiLU.
-    const int cw = conv_index(warp);
-    const bool leader = (tid == 2 * 32);  // leaders sit on different SM sub-partitions
+    const int cw = warp - kWarpConv0;
+    const bool leader = (warp == kWarpConv0 && lane == 0);
     const int ch = h * 64 + 2 * lane;
     const int W = a.W;
     float2 ew[4], bias2 = make_float2(0.f, 0.f);
@@ -456,23 +445,23 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const bool is_last = (k == last);
       // the leader waits for every input of the chunk, then one group barrier releases all
       if (leader) {
-        bool ok = mbar_wait(BAR(BAR_FULLX0 + xb), (k >> 1) & 1, abort_flag, a.err);
-        if (ok) ok = mbar_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, abort_flag, a.err);
-        if (ok && k >= 2) ok = mbar_wait(BAR(BAR_XFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err);
-        if (ok && is_last && k >= 1) mbar_wait(BAR(BAR_XWFREE0 + lb), ((k - 1) >> 1) & 1, abort_flag, a.err);
-        TC_MARK(k, 14);
+        bool ok = mbar_wait(BAR(BAR_FULLX0 + xb), (k >> 1) & 1, abort_flag, a.err, lim);
+        if (ok) ok = mbar_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, abort_flag, a.err, lim);
+        if (ok && !kStateOnly && k >= 2)
+          ok = mbar_wait(BAR(BAR_XFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err, lim);
+        if (ok && is_last && k >= 1) mbar_wait(BAR(BAR_XWFREE0 + lb), ((k - 1) >> 1) & 1, abort_flag, a.err, lim);
+        TC_MARK(k, 0);
       }
-      named_bar(1, 256);
-      if (*abort_flag) break;
+      if (named_bar_or(kNbConv, 32 * kConvWarps, *abort_flag != 0)) break;
       const float *cs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
       const float *dtv = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
       const float cs_end = cs[QC - 1];
-      const float wl = lane < kTokPerConvWarp ? __expf(cs_end - cs[tok0 + lane]) * dtv[tok0 + lane] : 0.f;
+      const float wl = __expf(cs_end - cs[tok0 + lane]) * dtv[tok0 + lane];  // w of token tok0+lane
       const uint32_t wl2 = pack_f16(wl, wl);
       unsigned char *xt = smem + OFF_X + xb * kTile + tok0 * 128;   // row tok0
       unsigned char *xwt = smem + OFF_XW + xb * kXBuf + tok0 * 128;
       unsigned char *xlt = smem + OFF_XW + lb * kXBuf + tok0 * 128;
-      // raw rows tok0 + r for r = 0..18 (tok0 is a multiple of 8, so row mod 8 = r mod 8)
+      // raw rows tok0 + r for r = 0..34 (tok0 is a multiple of 8, so row mod 8 = r mod 8)
 #define RAW(r) (*reinterpret_cast<const uint32_t *>(xwt + (r) * 128 + loff[(r) & 7]))
       uint32_t r0 = RAW(0), r1 = RAW(1), r2 = RAW(2);
       const int t0 = t_begin + k * QC;
@@ -488,12 +477,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         r1 = hist[1];
         r2 = hist[2];
       }
-      const uint32_t nb0 = RAW(16), nb1 = RAW(17), nb2 = RAW(18);
-      named_bar(1, 256);  // all boundary rows read before any row is overwritten
-      if (leader) {
-        TC_MARK(k, 0);
-        mbar_arrive(BAR(BAR_EMPTY0 + st));  // dt and prefix sums already read
-      }
+      constexpr int T = kTokPerConvWarp;
+      const uint32_t nb0 = RAW(T), nb1 = RAW(T + 1), nb2 = RAW(T + 2);
+      named_bar(kNbConv, 32 * kConvWarps);  // all boundary rows and prefix sums read
+      if (leader) mbar_arrive(BAR(BAR_EMPTY0 + st));
       // The token loop is compiled twice: the common chunks, and the last chunk of a segment.
       auto tokens = [&](auto last_tag) {
         constexpr bool kLast = decltype(last_tag)::value;
@@ -501,19 +488,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           __half2 xm3 = __float22half2_rn(unpack_bf16(r0)), xm2 = __float22half2_rn(unpack_bf16(r1)),
                   xm1 = __float22half2_rn(unpack_bf16(r2));
 #pragma unroll 1
-          for (int g = 0; g < 2; ++g) {
+          for (int gi = 0; gi < T / 8; ++gi) {
             __half2 xn[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-              const int nxt = 8 * g + u + 3;  // row of time t for token 8g+u
+              const int nxt = 8 * gi + u + 3;  // row of time t for token 8gi+u
               uint32_t w3;
-              if (nxt < 16) w3 = RAW(nxt);
-              else w3 = nxt == 16 ? nb0 : (nxt == 17 ? nb1 : nb2);
+              if (nxt < T) w3 = RAW(nxt);
+              else w3 = nxt == T ? nb0 : (nxt == T + 1 ? nb1 : nb2);
               xn[u] = __float22half2_rn(unpack_bf16(w3));
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-              const int i = 8 * g + u;
+              const int i = 8 * gi + u;
               const __half2 x0 = xn[u];
               __half2 xo = x0;
               if (W != 0) {
@@ -524,7 +511,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
                 xo = __hfma2(acc, h2tanh_approx(acc), acc);
               }
               const uint32_t off = i * 128 + loff[u];
-              *reinterpret_cast<__half2 *>(xt + off) = xo;
+              if (!kStateOnly) *reinterpret_cast<__half2 *>(xt + off) = xo;
               const uint32_t w2 = __shfl_sync(0xffffffffu, wl2, i);
               *reinterpret_cast<__half2 *>(xwt + off) = __hmul2(xo, *reinterpret_cast<const __half2 *>(&w2));
               xm3 = xm2;
@@ -536,19 +523,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         float2 xm3 = unpack_bf16(r0), xm2 = unpack_bf16(r1), xm1 = unpack_bf16(r2);
 #pragma unroll 1
-        for (int g = 0; g < 2; ++g) {
+        for (int gi = 0; gi < T / 8; ++gi) {
           float2 xn[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const int nxt = 8 * g + u + 3;  // row of time t for token 8g+u
+            const int nxt = 8 * gi + u + 3;  // row of time t for token 8gi+u
             uint32_t w3;
-            if (nxt < 16) w3 = RAW(nxt);
-            else w3 = nxt == 16 ? nb0 : (nxt == 17 ? nb1 : nb2);
+            if (nxt < T) w3 = RAW(nxt);
+            else w3 = nxt == T ? nb0 : (nxt == T + 1 ? nb1 : nb2);
             xn[u] = unpack_bf16(w3);
           }
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const int i = 8 * g + u;
+            const int i = 8 * gi + u;
             const float2 x0 = xn[u];
             float2 acc = x0;
             if (W != 0) {
@@ -568,7 +555,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
               const float2 v = make_float2(u0 * ws, u1 * ws);
               const __half2 hi = __float22half2_rn(v);
               const float2 hf = __half22float2(hi);
-              *reinterpret_cast<uint32_t *>(xt + off) = pack_f16(u0, u1);
+              if (!kStateOnly) *reinterpret_cast<uint32_t *>(xt + off) = pack_f16(u0, u1);
               *reinterpret_cast<__half2 *>(xwt + off) = hi;
               *reinterpret_cast<uint32_t *>(xlt + off) = pack_f16(v.x - hf.x, v.y - hf.y);
             }
@@ -580,43 +567,45 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       };
       if (is_last) tokens(std::true_type{});
       else tokens(std::false_type{});
-      if (leader) TC_MARK(k, 13);
 #undef RAW
       fence_proxy_async();
-      named_bar(1, 256);
+      named_bar(kNbConv, 32 * kConvWarps);
       if (leader) {
         TC_MARK(k, 1);
         mbar_arrive(BAR(BAR_XREADY0 + xb));
         if (is_last) mbar_arrive(BAR(BAR_XLOREADY));
       }
     }
-  } else if (warp >= 12 && warp < 16) {
+  } else if (warp >= kWarpMask0 && warp < kWarpMask0 + 4) {
     // ---------------------------------------------------------------- S -> S~ (decay mask)
     if (!kStateOnly) {
-      const int mw = warp - 12;
+      const int mw = warp - kWarpMask0;  // == warp % 4: TMEM lanes 32 mw .. 32 mw + 31
       const int t = 32 * mw + lane;
-      const bool leader = (tid == 14 * 32);
+      const bool leader = (warp == kWarpMask0 + 2 && lane == 0);
       float *cf = reinterpret_cast<float *>(smem + OFF_CF);
       const float Dh = a.D[h];
       for (int k = 0; k < nck; ++k) {
         const int st = k & 1;
-        if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, 2, abort_flag, a.err)) break;
-        if (!wg_wait(BAR(BAR_SREADY0 + st), (k >> 1) & 1, leader, 2, abort_flag, a.err)) break;
+        if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, kNbMask, abort_flag, a.err, lim)) break;
+        if (!wg_wait(BAR(BAR_SREADY0 + st), (k >> 1) & 1, leader, kNbMask, abort_flag, a.err, lim)) break;
         tc_fence_after();
+        if (leader) TC_MARK(k, 2);
         float *cs = reinterpret_cast<float *>(smem + OFF_CSM);
         float *dtv = reinterpret_cast<float *>(smem + OFF_DTM);
+        float *et = reinterpret_cast<float *>(smem + OFF_ET + st * 512);
         {  // private copies (the stage is released at once); column factor of column t:
-           // e^{r_J - cs_t} dt_t with r_J = cs at the end of t's block
+           // e^{r_J - cs_t} dt_t with r_J = cs at the end of t's block; and the output row
+           // factor e^{cs_t} of this chunk for the output warps
           const float *scs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
           const float *sdt = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
           const float rJ = scs[32 * (t >> 5) + 31];
           cs[t] = scs[t];
           dtv[t] = sdt[t];
           cf[t] = __expf(rJ - scs[t]) * sdt[t];
+          et[t] = __expf(scs[t]);
         }
-        named_bar(2, 128);
+        named_bar(kNbMask, 128);
         if (leader) mbar_arrive(BAR(BAR_EMPTY0 + st));
-        if (leader) TC_MARK(k, 2);
         const float cst = cs[t];
         const uint32_t trow = tmem + (st ? TM_S1 : TM_S0) + ((uint32_t)(32 * mw) << 16);
         // Blocks of 32 columns in increasing J: S~ columns 32J..32J+31 go to the packed TMEM
@@ -697,18 +686,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        named_bar(2, 128);
+        named_bar(kNbMask, 128);
         if (leader) {
           TC_MARK(k, 3);
           mbar_arrive(BAR(BAR_STREADY0 + st));
         }
       }
     }
-  } else if (warp >= 16) {
-    // ---------------------------------------------------------------- state update + output
-    const int ew = warp - 16;
-    const int n = 32 * ew + lane;  // TMEM lane: state row n, output row t = n
-    const bool leader = (tid == 19 * 32);
+  } else if (warp >= kWarpState0 && warp < kWarpState0 + 4) {
+    // ---------------------------------------------------------------- state update
+    const int ew = warp - kWarpState0;
+    const int n = 32 * ew + lane;  // TMEM lane: state row n
+    const bool leader = (warp == kWarpState0 + 3 && lane == 0);
     const uint32_t lane_off = (uint32_t)(32 * ew) << 16;
     const long long bh = (long long)b * a.H + h;
     float *hout = a.h_out ? a.h_out + seg * a.h_out_seg + bh * 8192 : nullptr;
@@ -727,7 +716,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           hu[i] = __float_as_uint(hr[i]);
         }
         tmem_st32(tmem + TM_H + 32 * half + lane_off, hu);
-        write_h_tile(smem, hr, n, half);
+        if (!kStateOnly) write_h_tile(smem, hr, n, half);
         if (tail && tail_k < 0) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) hout[(32 * half + i) * 128 + n] = hr[i];
@@ -737,20 +726,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
     fence_proxy_async();
     tc_fence_before();
-    named_bar(3, 128);
+    named_bar(kNbState, 128);
     if (leader) mbar_arrive(BAR(BAR_HREADY));
     float decay_sum = 0.f;
     for (int k = 0; k < nck; ++k) {
       const int st = k & 1;
-      if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, 3, abort_flag, a.err)) break;
-      const float *cs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
-      const float cs_end = cs[QC - 1];
-      const float et = __expf(cs[n]);
+      if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, kNbState, abort_flag, a.err, lim)) break;
+      const float cs_end = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS)[QC - 1];
       decay_sum += cs_end;
       const float ak = __expf(cs_end);
-      named_bar(3, 128);  // every thread has read the prefix sums
+      named_bar(kNbState, 128);  // every thread has read the prefix sums
       if (leader) mbar_arrive(BAR(BAR_EMPTY0 + st));
-      if (!wg_wait(BAR(BAR_DHREADY), k & 1, leader, 3, abort_flag, a.err)) break;
+      if (!wg_wait(BAR(BAR_DHREADY), k & 1, leader, kNbState, abort_flag, a.err, lim)) break;
       tc_fence_after();
       if (leader) TC_MARK(k, 4);
 #pragma unroll 1
@@ -764,8 +751,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         for (int i = 0; i < 32; i += 2) {
           const float2 r = __ffma2_rn(make_float2(ak, ak), make_float2(hr[i], hr[i + 1]),
                                       make_float2(dh[i], dh[i + 1]));
-          hr[i] = r.x;
-          hr[i + 1] = r.y;
           hu[i] = __float_as_uint(r.x);
           hu[i + 1] = __float_as_uint(r.y);
         }
@@ -773,8 +758,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      named_bar(3, 128);
-      if (leader) mbar_arrive(BAR(BAR_DHFREE));  // dH read: MMA4 of chunk k+1 may overwrite it
+      named_bar(kNbState, 128);
+      if (leader) {
+        TC_MARK(k, 5);
+        mbar_arrive(BAR(BAR_DHFREE));  // dH read: MMA4 of chunk k+1 may overwrite it
+      }
       if (tail && k == tail_k) {  // the state entering the tail, in fp32
         tc_fence_after();
 #pragma unroll 1
@@ -788,7 +776,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       if (!kStateOnly && k != last) {
         // fp16 copy of h_k for MMA3 of chunk k+1, once MMA3 of chunk k has read h_{k-1}
-        if (!wg_wait(BAR(BAR_HTFREE), k & 1, leader, 3, abort_flag, a.err)) break;
+        if (!wg_wait(BAR(BAR_HTFREE), k & 1, leader, kNbState, abort_flag, a.err, lim)) break;
         tc_fence_after();
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
@@ -798,23 +786,109 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           write_h_tile(smem, hr, n, half);
         }
         fence_proxy_async();
-        named_bar(3, 128);
+        named_bar(kNbState, 128);
         if (leader) {
-          TC_MARK(k, 5);
+          TC_MARK(k, 6);
           mbar_arrive(BAR(BAR_HREADY));
         }
       }
-      if (!kStateOnly) {
-        if (!wg_wait(BAR(BAR_YREADY0 + st), (k >> 1) & 1, leader, 3, abort_flag, a.err)) break;
+    }
+    if (*abort_flag == 0) {
+      if (hout && a.tail_chunks == 0) {
         tc_fence_after();
-        if (leader) TC_MARK(k, 6);
-        const int tok = t_begin + k * QC + n;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          float hr[32];
+          tmem_ld32(tmem + TM_H + 32 * half + lane_off, hr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) hout[(32 * half + i) * 128 + n] = hr[i];
+        }
+      }
+      if (a.seg_decay && n == 0) a.seg_decay[(long long)seg * a.B * a.H + bh] = __expf(decay_sum);
+    }
+  } else if (warp >= kWarpOut0 && warp < kWarpOut0 + 4) {
+    // ---------------------------------------------------------------- output y = Yi + e^{cs} Ys
+    if (!kStateOnly) {
+      const int ow = warp - kWarpOut0;
+      const int t = 32 * ow + lane;  // TMEM lane: output row t
+      const bool leader = (warp == kWarpOut0 + 1 && lane == 0);
+      const uint32_t lane_off = (uint32_t)(32 * ow) << 16;
+      const bool gate = a.qn != nullptr && !a.nbg;
+      for (int k = 0; k < nck; ++k) {
+        const int st = k & 1;
+        const int tok = t_begin + k * QC + t;
         const long long row = (long long)b * a.L + tok;
+        // fused gate: this row's z (64 channels, 128 bytes) is prefetched into L1 before the
+        // wait for the chunk's products
+        const __nv_bfloat16 *zrow = gate ? a.z + row * a.zs + h * 64 : nullptr;
+        if (gate && tok < t_end) {
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(zrow));
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(zrow + 63));
+        }
+        if (!wg_wait(BAR(BAR_STREADY0 + st), (k >> 1) & 1, leader, kNbOut, abort_flag, a.err, lim)) break;
+        if (!wg_wait(BAR(BAR_YREADY0 + st), (k >> 1) & 1, leader, kNbOut, abort_flag, a.err, lim)) break;
+        tc_fence_after();
+        if (leader) TC_MARK(k, 7);
+        const float et = reinterpret_cast<const float *>(smem + OFF_ET + st * 512)[t];
+        const uint32_t tYi = tmem + (st ? TM_S1 : TM_S0) + TM_YI_OFF + lane_off;
+        const uint32_t tYs = tmem + (st ? TM_YS1 : TM_YS0) + lane_off;
+        if (a.qn) {
+          // fused gate: g = y SiLU(z) (or g = y when normalising first) is stored as g / s in
+          // fp16, s the RMS of g over the head's 64 channels, with sum(g^2) for the rescale
+          // pass.  Pass 1 (16 columns at a time) forms g, keeps it in the Yi columns of TMEM
+          // and sums its squares; pass 2 scales and stores it.  SiLU(v) = v/2 + v/2 tanh(v/2).
+          float ssq = 0.f;
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd) {
+            float yi[16], ysv[16];
+            tmem_ld16(tYi + 16 * qd, yi);
+            tmem_ld16(tYs + 16 * qd, ysv);
+            uint4 zu[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+            if (gate && tok < t_end) {
+              zu[0] = __ldg(reinterpret_cast<const uint4 *>(zrow + 16 * qd));
+              zu[1] = __ldg(reinterpret_cast<const uint4 *>(zrow + 16 * qd + 8));
+            }
+            const uint32_t zw[8] = {zu[0].x, zu[0].y, zu[0].z, zu[0].w, zu[1].x, zu[1].y, zu[1].z, zu[1].w};
+            tmem_ld_wait();
+            uint32_t gu[16];
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+              float2 g2 = __ffma2_rn(make_float2(et, et), make_float2(ysv[i], ysv[i + 1]),
+                                     make_float2(yi[i], yi[i + 1]));
+              if (gate) {
+                const __half2 hh = __hmul2(__float22half2_rn(unpack_bf16(zw[i / 2])), __float2half2_rn(0.5f));
+                g2 = __fmul2_rn(g2, __half22float2(__hfma2(hh, h2tanh_approx(hh), hh)));
+              }
+              ssq = fmaf(g2.x, g2.x, fmaf(g2.y, g2.y, ssq));
+              gu[i] = __float_as_uint(g2.x);
+              gu[i + 1] = __float_as_uint(g2.y);
+            }
+            tmem_st16(tYi + 16 * qd, gu);
+          }
+          tmem_st_wait();
+          const float inv = ssq > 0.f ? rsqrtf(ssq * (1.f / 64.f)) : 0.f;
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd) {
+            float gv[16];
+            tmem_ld16(tYi + 16 * qd, gv);
+            tmem_ld_wait();
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) pk[i / 2] = pack_f16(gv[i] * inv, gv[i + 1] * inv);
+            if (tok < t_end) {
+              uint4 *dst = reinterpret_cast<uint4 *>(a.qn + row * a.d_inner + h * 64 + 16 * qd);
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+          }
+          if (tok < t_end) a.ssq[row * a.H + h] = ssq;
+        } else {
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
           float yi[32], ysv[32];
-          tmem_ld32(tmem + (st ? TM_S1 : TM_S0) + TM_YI_OFF + 32 * half + lane_off, yi);
-          tmem_ld32(tmem + (st ? TM_YS1 : TM_YS0) + 32 * half + lane_off, ysv);
+          tmem_ld32(tYi + 32 * half, yi);
+          tmem_ld32(tYs + 32 * half, ysv);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
@@ -837,33 +911,20 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             }
           }
         }
+        }
         tc_fence_before();
-        named_bar(3, 128);
+        named_bar(kNbOut, 128);
         if (leader) {
-          TC_MARK(k, 7);
+          TC_MARK(k, 8);
           mbar_arrive(BAR(BAR_YFREE0 + st));
         }
       }
-    }
-    if (*abort_flag == 0) {
-      if (hout && a.tail_chunks == 0) {
-        tc_fence_after();
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          float hr[32];
-          tmem_ld32(tmem + TM_H + 32 * half + lane_off, hr);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) hout[(32 * half + i) * 128 + n] = hr[i];
-        }
-      }
-      if (a.seg_decay && n == 0) a.seg_decay[(long long)seg * a.B * a.H + bh] = __expf(decay_sum);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpIssueA) {
     tc_fence_after();
     tmem_dealloc(tmem, TM_COLS);
   }
@@ -925,8 +986,15 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
   a.conv_w = (const __nv_bfloat16 *)p.conv_w; a.conv_b = (const __nv_bfloat16 *)p.conv_b;
   a.dte = p.dte_hm; a.cs = p.cs_hm; a.D = p.D;
   a.y = (__nv_bfloat16 *)p.y; a.ys = p.ys; a.err = p.err;
-  a.yf = p.norm_groups > 0 ? p.yf : nullptr;
+  a.yf = p.norm_groups > 0 && !p.qn ? p.yf : nullptr;
+  a.qn = p.norm_groups > 0 ? p.qn : nullptr;
+  a.ssq = p.ssq;
+  a.z = (const __nv_bfloat16 *)p.z;
+  a.zs = p.zs;
+  a.nbg = p.nbg;
   a.d_inner = p.d_inner;
+  a.wait_ns = p.stall_chunk1 > 0 ? p.stall_wait_ns : tc::kWaitLimitNs;
+  a.debug_skip_chunk = p.stall_chunk1 - 1;
   const long long seg_stride = (long long)p.B * p.H * p.P * p.N;
   dim3 grid(p.n_seg, p.H, p.B);
   cudaError_t e;

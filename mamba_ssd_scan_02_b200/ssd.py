@@ -78,7 +78,7 @@ class TraceRecord(ctypes.Structure):
 EXPORTS = ("ssd_workspace_size", "ssd_prefill", "ssd_decode_step", "ssd_mixer_workspace_size",
            "mamba2_mixer_forward", "ssd_status_string", "ssd_get_device_error", "ssd_version",
            "ssd_trace_enable", "ssd_trace_read", "ssd_prefill_noalloc", "ssd_varlen_workspace_size",
-           "ssd_prefill_varlen")
+           "ssd_prefill_varlen", "ssd_test_stall_scan")
 NOALLOC_WORKSPACE_BYTES = 64 << 20
 
 _lib = None
@@ -119,6 +119,8 @@ def load(path: str = LIB_PATH):
                                        ctypes.POINTER(c_int), c_int, vp]
     lib.ssd_prefill_noalloc.restype = c_int
     lib.ssd_prefill_noalloc.argtypes = [ctypes.POINTER(SsdConfig), ctypes.POINTER(PrefillArgs), vp]
+    lib.ssd_test_stall_scan.restype = None
+    lib.ssd_test_stall_scan.argtypes = [c_int, ctypes.c_ulonglong]
     lib.ssd_trace_enable.restype = c_int
     lib.ssd_trace_enable.argtypes = [c_int]
     lib.ssd_trace_read.restype = c_int
@@ -351,6 +353,12 @@ def mixer_forward(cfg: dict, hidden, rms_w, W_in, W_out, A, D, dt_bias, conv_w, 
 def get_device_error(stream=None) -> int:
     """Waits for the stream, returns and clears the library's device error status."""
     return load().ssd_get_device_error(_stream(stream))
+
+
+def test_stall_scan(chunk: int, wait_limit_ms: float = 20.0) -> None:
+    """Test hook: tensor-core prefills withhold chunk `chunk`'s stage so that their bounded
+    waits give up after wait_limit_ms (SSD_ERR_TIMEOUT); chunk < 0 turns it off."""
+    load().ssd_test_stall_scan(int(chunk), int(wait_limit_ms * 1e6))
 
 
 def trace_enable(on: bool) -> bool:

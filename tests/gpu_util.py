@@ -41,6 +41,10 @@ def assert_close(got, want, tol, what, out_dtype="f32", both_rounded=False):
     excess = np.abs(got - want) - (2 if both_rounded else 1) * UNIT_ROUNDOFF[out_dtype] * np.abs(want)
     r_ex = float(np.max(excess)) / rms
     r = rel_err(got, want)
+    # both figures: the plain one, and the one the bound applies to (the excess over the
+    # storage rounding); pytest shows them with -s or -rA
+    print(f"[parity] {what}: max|err|/RMS = {r:.3e}; max(|err| - {'2u' if both_rounded else 'u'}|ref|)/RMS"
+          f" = {r_ex:.3e} (bound {tol:.1e}, u = {UNIT_ROUNDOFF[out_dtype]:.3g})")
     assert r_ex <= tol, (f"{what}: max(|err| - u|ref|)/RMS = {r_ex:.3e} > {tol:.1e} "
                          f"(plain max|err|/RMS = {r:.3e})")
     return r

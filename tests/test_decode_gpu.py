@@ -91,8 +91,9 @@ def test_decode_equals_prefill(cuda_lib):
 
 def test_decode_16k_steps_full_size(cuda_lib, oracle):
     """Workload 2: B64 H128 G8, 16384 steps.
-    (a) rows 0 and 63 for all 16384 steps, starting from an 8192-token prefill computed
-        independently on the GPU (all 64 rows) and by the oracle (those two rows);
+    (a) rows 0 and 63 for all 16384 steps (y compared every 16th step, the state and cache
+        at the end), starting from an 8192-token prefill computed independently on the GPU
+        (all 64 rows) and by the oracle (those two rows);
     (b) all 64 rows for the first 64 steps from a seeded random state and conv cache."""
     import torch
     from mamba_ssd_scan_02_b200 import ssd
@@ -153,7 +154,7 @@ def test_decode_16k_steps_full_size(cuda_lib, oracle):
                                z_t=np.ascontiguousarray(pool["z"][i][rows]), norm_w=norm_w)
         ocache = np.ascontiguousarray(
             np.concatenate([ocache[:, 1:], pool["xBC"][i][rows][:, None]], axis=1))
-        if s % 1024 == 1023:
+        if s % 16 == 15:
             assert_close(y.float().cpu().numpy()[rows], r["out"], TOL_BF16, f"rows 0/63, step {s}",
                          out_dtype="bf16")
     assert_close(host(state)[rows], ost, TOL_BF16, "state after 16384 steps")

@@ -150,6 +150,15 @@ def test_prefill_8k_full_size(cuda_lib, oracle):
     _check(oracle, cfg, inp, kernel=None, tag="cfg1")
 
 
+@pytest.mark.parametrize("nseg", [3])
+def test_prefill_8k_full_size_internal_segments(cuda_lib, oracle, nseg):
+    """Workload 1 at full size with the sequence forced into internal segments (state-only
+    pass, inter-segment pass, output pass), all heads."""
+    cfg = dict(datagen.config(1), n_segments=nseg)
+    inp = datagen.make_inputs(1)
+    _check(oracle, cfg, inp, kernel=None, tag=f"cfg1 seg{nseg}")
+
+
 def test_long_context_split_equals_unsplit(cuda_lib, oracle):
     """Workload 3: 131072 tokens as 4 x 32768 with state + conv-cache carry equals one pass;
     the oracle checks the heads of groups 0 and 7 (heads and groups are independent)."""
