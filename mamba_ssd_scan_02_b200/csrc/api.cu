@@ -126,7 +126,7 @@ struct WsLayout {
   // CUDA-core path
   size_t u, dte, yf, seg_state, seg_decay, simt_end;
   // tensor-core path
-  size_t tc_bc, tc_dte, tc_cs, tc_yf, tc_q, tc_ssq, tc_seg_state, tc_seg_decay, tc_dh, tc_end;
+  size_t tc_bc, tc_dte, tc_cs, tc_yf, tc_q, tc_ssq, tc_seg_state, tc_seg_decay, tc_dh, tc_blo, tc_end;
   int Lpad;
   size_t total;
 };
@@ -171,6 +171,7 @@ WsLayout prefill_layout(const ssd_config_t *c) {
     off = round_up(off + (size_t)n_seg * c->batch * c->nheads * 4, kAlign);
   }
   w.tc_dh = off;   off = round_up(off + state + (size_t)c->batch * c->nheads * 4, kAlign);
+  w.tc_blo = off;  off = round_up(off + (size_t)c->batch * kTailChunks * kTcTile * c->ngroups * c->dstate * 2, kAlign);
   w.tc_end = off;
   w.total = prefill_uses_tc(c) ? w.tc_end : w.simt_end;
   return w;
@@ -184,8 +185,8 @@ ssd_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_E
     if (e_ != cudaSuccess) return SSD_ERR_CUDA;  \
   } while (0)
 
-// Per host thread and device: a side stream and two events that run the fp32 tail pass beside
-// the output scan (made on first use and kept for the life of the process).  Per thread, so
+// Per host thread and device: a side stream and two events that run the tail pass beside the
+// output scan (made on first use and kept for the life of the process).  Per thread, so
 // that a fork is always joined before the same objects are recorded again.
 struct SideStream {
   cudaStream_t s;
@@ -298,6 +299,15 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
     p.seg_decay = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.tc_seg_decay) : nullptr;
     p.tail_dh = p.h_final ? reinterpret_cast<float *>(ws + lay.tc_dh) : nullptr;
     p.tail_dec = p.h_final ? p.tail_dh + (size_t)c->batch * c->nheads * c->headdim * c->dstate : nullptr;
+    if (p.tail_dh) {  // the tail: the last kTailChunks chunks of the last segment
+      const int t_b = (p.n_seg - 1) * p.seg_len;
+      const int nck = (p.L - t_b + kTcTile - 1) / kTcTile;
+      p.t_tail = t_b + kTcTile * (nck > kTailChunks ? nck - kTailChunks : 0);
+      p.ntail = p.L - p.t_tail;
+      p.blo = reinterpret_cast<__half *>(ws + lay.tc_blo);
+    } else {
+      p.t_tail = p.L;
+    }
     // The outgoing conv cache may be written before the scan unless it overlaps an input
     // that later kernels read.
     const size_t x_span = ((size_t)c->batch * c->seqlen - 1) * (size_t)a->xBC_row_stride * es + (size_t)conv_dim * es;
@@ -311,8 +321,9 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
       SSD_TRY(traced("ssd_dt_cumsum", s, [&] { return launch_dt_cumsum(p, p.dte_hm, p.cs_hm, p.Lpad, s); }));
       SSD_TRY(traced("ssd_bc_conv", s, [&] { return launch_bc_conv_f16(p, s); }));
     }
-    // the fp32 tail needs only the front end's outputs: it runs on a side stream, on the SMs
-    // the scan leaves free, and is joined before the fold
+    // The tail pass needs only the front end's outputs: it is forked onto a side stream right
+    // after the front end and launched after the scan, so that it takes the SMs the scan
+    // leaves free; it is joined before the fold.
     SideJoin side;
     if (p.tail_dh) {
       SSD_TRY(side_stream(&side.side));
@@ -320,13 +331,14 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
       SSD_TRY(cudaEventRecord(side.side->fork, s));
       SSD_TRY(cudaStreamWaitEvent(side.side->s, side.side->fork, 0));
       side.forked = true;
-      SSD_TRY(traced("ssd_state_tail", side.side->s, [&] { return launch_state_tail(p, side.side->s); }));
     }
     if (p.n_seg > 1) {
       SSD_TRY(traced("ssd_scan_tc_states", s, [&] { return launch_scan_tc(p, 1, s); }));
       SSD_TRY(traced("ssd_state_pass", s, [&] { return launch_state_pass(p, s); }));
     }
     SSD_TRY(traced("ssd_scan_tc", s, [&] { return launch_scan_tc(p, 0, s); }));
+    if (side.forked)
+      SSD_TRY(traced("ssd_scan_tc_tail", side.side->s, [&] { return launch_scan_tc(p, 2, side.side->s); }));
     if (side.forked) {
       SSD_TRY(side.join());
       SSD_TRY(traced("ssd_tail_fold", s, [&] { return launch_tail_fold(p, s); }));

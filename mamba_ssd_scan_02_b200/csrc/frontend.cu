@@ -283,19 +283,24 @@ __device__ __forceinline__ void unpack8(const uint4 &r, float2 (&v)[4]) {
   for (int i = 0; i < 4; ++i) v[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
 }
 
+// The B channels of the final state's tail (tokens t >= t_tail, written when blo is set) use
+// the exact SiLU, and their fp16 rounding error goes to blo: the tail pass multiplies both
+// parts, so that the final state's newest tokens enter it with fp32 accuracy.
 template <int W>
 __device__ __forceinline__ void bc_conv_tile(const __nv_bfloat16 *__restrict__ xBC, long long xs,
                                              const __nv_bfloat16 *__restrict__ csi,
                                              const __nv_bfloat16 *__restrict__ w,
                                              const __nv_bfloat16 *__restrict__ bias,
                                              __half *__restrict__ out, int L, int conv_dim, int c_begin,
-                                             int C_out, int bx, int by, int bz) {
+                                             int C_out, int bx, int by, int bz, __half *__restrict__ blo,
+                                             int t_tail, int ntail, int n_b) {
   const int o8 = (bx * kBcThreads + threadIdx.x) * kBcCh;
   if (o8 >= C_out) return;
   const int c8 = c_begin + o8;
   const int b = bz;
   const int t0 = by * kBcTok;
   const int t1 = min(L, t0 + kBcTok);
+  const bool tail_tile = blo != nullptr && o8 < n_b && t1 > t_tail;
   const __nv_bfloat16 *xrow = xBC + (long long)b * L * xs + c8;
   float2 wt[4][4], bs[4];  // [tap][channel pair]: tap k multiplies time t-(W-1)+k
 #pragma unroll
@@ -338,8 +343,9 @@ __device__ __forceinline__ void bc_conv_tile(const __nv_bfloat16 *__restrict__ x
     for (int j = 0; j < 8; ++j) {
       const int t = tg + j;
       if (!kFull && t >= t1) break;
+      const bool exact = tail_tile && t >= t_tail;
       float2 x0[4];
-      uint32_t r[4];
+      uint32_t r[4], rl[4];
       unpack8(cur[j], x0);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -349,15 +355,21 @@ __device__ __forceinline__ void bc_conv_tile(const __nv_bfloat16 *__restrict__ x
           float2 acc = bs[i];
 #pragma unroll
           for (int k = 0; k < W; ++k) acc = __ffma2_rn(wt[k][i], xw[4 - W + k], acc);
-          v = make_float2(silu_tanh(acc.x), silu_tanh(acc.y));
+          v = exact ? make_float2(silu(acc.x), silu(acc.y)) : make_float2(silu_tanh(acc.x), silu_tanh(acc.y));
         }
         const __half2 hv = __floats2half2_rn(v.x, v.y);
         r[i] = *reinterpret_cast<const uint32_t *>(&hv);
+        const float2 hf = __half22float2(hv);
+        const __half2 lv = __floats2half2_rn(v.x - hf.x, v.y - hf.y);
+        rl[i] = *reinterpret_cast<const uint32_t *>(&lv);
         x3[i] = x2[i];
         x2[i] = x1[i];
         x1[i] = x0[i];
       }
       *reinterpret_cast<uint4 *>(out + ((long long)b * L + t) * C_out + o8) = make_uint4(r[0], r[1], r[2], r[3]);
+      if (exact)
+        *reinterpret_cast<uint4 *>(blo + ((long long)b * ntail + (t - t_tail)) * n_b + o8) =
+            make_uint4(rl[0], rl[1], rl[2], rl[3]);
     }
   };
   if (t1 - t0 == kBcTok) {
@@ -375,8 +387,10 @@ __global__ void __launch_bounds__(kBcThreads, 2) bc_conv_kernel(const __nv_bfloa
                                                              const __nv_bfloat16 *__restrict__ w,
                                                              const __nv_bfloat16 *__restrict__ bias,
                                                              __half *__restrict__ out, int L, int conv_dim,
-                                                             int c_begin, int C_out) {
-  bc_conv_tile<W>(xBC, xs, csi, w, bias, out, L, conv_dim, c_begin, C_out, blockIdx.x, blockIdx.y, blockIdx.z);
+                                                             int c_begin, int C_out, __half *__restrict__ blo,
+                                                             int t_tail, int ntail) {
+  bc_conv_tile<W>(xBC, xs, csi, w, bias, out, L, conv_dim, c_begin, C_out, blockIdx.x, blockIdx.y, blockIdx.z,
+                  blo, t_tail, ntail, C_out / 2);
 }
 
 // The tensor-core path's front end in one launch: dt + chunk prefix sums, the outgoing conv
@@ -387,8 +401,9 @@ struct FrontArgs {
   long long xs, ds;
   const float *dt_bias, *A;
   float *dte, *cs;
-  __half *bc;
+  __half *bc, *blo;
   __nv_bfloat16 *cso;
+  int t_tail, ntail;
   int B, L, H, Lpad, conv_dim, d_inner, C_out, W, sp;
   float lo, hi;
   int n_dt, dt_tiles, dt_nch, dt_nhg, n_cso, gx, gy;
@@ -416,12 +431,13 @@ __global__ void __launch_bounds__(kBcThreads, 2) front_tc_kernel(const FrontArgs
   }
   j -= f.n_cso;
   bc_conv_tile<W>(f.xBC, f.xs, f.csi, f.conv_w, f.conv_b, f.bc, f.L, f.conv_dim, f.d_inner, f.C_out,
-                  j % f.gx, (j / f.gx) % f.gy, j / (f.gx * f.gy));
+                  j % f.gx, (j / f.gx) % f.gy, j / (f.gx * f.gy), f.blo, f.t_tail, f.ntail, f.C_out / 2);
 }
 
 cudaError_t launch_bc_conv_f16(const PrefillPlan &p, cudaStream_t s) {
   const int C_out = 2 * p.G * p.N;
   if (C_out % 8 || p.xs % 8 || p.conv_dim % 8 || p.d_inner % 8) {  // 16-byte accesses; else the generic kernel
+    if (p.blo) return cudaErrorInvalidValue;  // the tail's low parts need the 16-byte kernel
     conv_dispatch<__nv_bfloat16, __half>(p, (__half *)p.bc, p.d_inner, C_out, s);
     return cudaGetLastError();
   }
@@ -432,11 +448,11 @@ cudaError_t launch_bc_conv_f16(const PrefillPlan &p, cudaStream_t s) {
   const auto *bb = (const __nv_bfloat16 *)p.conv_b;
   __half *o = (__half *)p.bc;
   switch (p.W) {
-    case 0: bc_conv_kernel<0><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
-    case 1: bc_conv_kernel<1><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
-    case 2: bc_conv_kernel<2><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
-    case 3: bc_conv_kernel<3><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
-    default: bc_conv_kernel<4><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
+    case 0: bc_conv_kernel<0><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out, p.blo, p.t_tail, p.ntail); break;
+    case 1: bc_conv_kernel<1><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out, p.blo, p.t_tail, p.ntail); break;
+    case 2: bc_conv_kernel<2><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out, p.blo, p.t_tail, p.ntail); break;
+    case 3: bc_conv_kernel<3><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out, p.blo, p.t_tail, p.ntail); break;
+    default: bc_conv_kernel<4><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out, p.blo, p.t_tail, p.ntail); break;
   }
   return cudaGetLastError();
 }
@@ -453,6 +469,7 @@ cudaError_t launch_front_tc(const PrefillPlan &p, bool with_cso, cudaStream_t s)
   f.csi = (const __nv_bfloat16 *)p.csi; f.conv_w = (const __nv_bfloat16 *)p.conv_w;
   f.conv_b = (const __nv_bfloat16 *)p.conv_b; f.xs = p.xs; f.ds = p.ds; f.dt_bias = p.dt_bias; f.A = p.A;
   f.dte = p.dte_hm; f.cs = p.cs_hm; f.bc = (__half *)p.bc; f.cso = (__nv_bfloat16 *)p.cso;
+  f.blo = p.blo; f.t_tail = p.t_tail; f.ntail = p.ntail;
   f.B = p.B; f.L = p.L; f.H = p.H; f.Lpad = p.Lpad; f.conv_dim = p.conv_dim; f.d_inner = p.d_inner;
   f.C_out = 2 * p.G * p.N; f.W = p.W; f.sp = p.softplus; f.lo = p.dt_min; f.hi = p.dt_max;
   f.dt_nch = p.Lpad / 128; f.dt_nhg = (p.H + 7) / 8; f.dt_tiles = f.dt_nch * f.dt_nhg * p.B;

@@ -7,7 +7,9 @@
 // and the state after the last segment is lambda_{n-1} h_in[n-1] + s_{n-1} = h_final.
 // This is the same linear recurrence as the token scan, applied at segment granularity.
 // One thread per 4 state elements (float4), sequential over the segments; h_in[k]
-// overwrites s_k in place (s_k is read first).
+// overwrites s_k in place (s_k is read first).  Within a segment the state never leaves the
+// scan CTA (it stays in tensor memory from chunk to chunk), so this pass only joins segments:
+// a few float4 streams of 4 MiB each, bound by memory, with no data shared between threads.
 #include "common.cuh"
 #include "plan.h"
 
@@ -33,7 +35,32 @@ __global__ void state_pass_kernel(float4 *__restrict__ seg_state, const float *_
   }
 }
 
+// The final state's fold after the tail pass: h = dec h + dh per (batch row, head), where
+// dh and dec are what the last chunks contribute from a zero state and their total decay.
+__global__ void tail_fold_kernel(float4 *__restrict__ h, const float4 *__restrict__ dh,
+                                 const float *__restrict__ dec, long long n4) {
+  constexpr int kPer = kHeadDim * kDState / 4;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float d = dec[i / kPer];
+    float4 v = h[i];
+    const float4 a = dh[i];
+    v.x = fmaf(d, v.x, a.x); v.y = fmaf(d, v.y, a.y); v.z = fmaf(d, v.z, a.z); v.w = fmaf(d, v.w, a.w);
+    h[i] = v;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_tail_fold(const PrefillPlan &p, cudaStream_t s) {
+  if (!p.tail_dh || p.L == 0) return cudaSuccess;
+  const long long n4 = (long long)p.B * p.H * kHeadDim * kDState / 4;
+  long long blocks = (n4 + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  tail_fold_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<float4 *>(p.h_final),
+                                                     reinterpret_cast<const float4 *>(p.tail_dh), p.tail_dec, n4);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_state_pass(const PrefillPlan &p, cudaStream_t s) {
   const long long BH = (long long)p.B * p.H;

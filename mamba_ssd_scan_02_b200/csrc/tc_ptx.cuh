@@ -63,11 +63,12 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 // Waits for the phase with the given parity to complete.  Gives up after `limit_ns` of device
 // time (2 s by default; the waits here normally last microseconds): sets *abort and latches
 // SSD_ERR_TIMEOUT.  Each try sleeps up to ~0.2 ms, so the clock and the abort flag are checked
-// every few tries.
+// every few tries.  The first try is inline; the retry loop is one shared out-of-line copy, so
+// that the many wait sites of a warp-specialised kernel do not each add the loop's code to the
+// instruction working set.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                          int *err, uint64_t limit_ns = kWaitLimitNs) {
-  if (mbar_try_wait(bar, parity)) return true;
+static __device__ __noinline__ bool mbar_wait_retry(uint32_t bar, uint32_t parity, volatile int *abort,
+                                                    int *err, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -80,6 +81,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
+                                          int *err, uint64_t limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_retry(bar, parity, abort, err, limit_ns);
 }
 
 // ---- TMA ----------------------------------------------------------------------------------

@@ -91,7 +91,8 @@ constexpr uint32_t OFF_CF = OFF_H + kTile;          // column factors, 128 fp32
 constexpr uint32_t OFF_CSM = OFF_CF + 512;          // the mask's copies of cs and dt
 constexpr uint32_t OFF_DTM = OFF_CSM + 512;
 constexpr uint32_t OFF_ET = OFF_DTM + 512;          // e^{cs_t} of chunk k in ET[k % 2] (mask -> output)
-constexpr uint32_t OFF_BAR = OFF_ET + 1024;
+constexpr uint32_t OFF_WTOK = OFF_ET + 1024;        // the conv's token weights w_s of the current chunk
+constexpr uint32_t OFF_BAR = OFF_WTOK + 512;
 // Barriers.  Every event that can recur before its consumer has observed the previous
 // occurrence has one barrier per buffer, so that a parity test never sees two phases at once.
 enum {
@@ -144,6 +145,7 @@ struct TcArgs {
   long long h_init_seg;
   float *h_out;            // final state destination or null
   long long h_out_seg;
+  int t_base;              // first token of segment 0 (the tail pass starts inside the sequence)
   int tail_chunks;         // > 0: instead of the final state, the last segment writes the state
                            // before its last tail_chunks chunks (an fp32 pass finishes it)
   float *seg_decay;        // [n_seg, B, H] total decay per segment, or null
@@ -217,8 +219,9 @@ __device__ __forceinline__ void issue_Yi(uint32_t tSt, uint32_t xbase, uint32_t 
 #pragma unroll
   for (int j = 0; j < 8; ++j) mma_f16_ts(tYi, tSt + 8 * j, desc_adv(b0, j * 2048), IDESC_YI, j > 0);
 }
-__device__ __forceinline__ void issue_dH(uint32_t stage, uint32_t xwbase, uint32_t tDH, bool acc) {
-  const uint64_t a0 = smem_desc_sw128(stage + OFF_B, kTile, 1024), b0 = smem_desc_sw128(xwbase, 8192, 1024);
+// bbase: the B^T operand (OFF_B of a stage, or OFF_C holding B's low parts in the tail pass)
+__device__ __forceinline__ void issue_dH(uint32_t bbase, uint32_t xwbase, uint32_t tDH, bool acc) {
+  const uint64_t a0 = smem_desc_sw128(bbase, kTile, 1024), b0 = smem_desc_sw128(xwbase, 8192, 1024);
 #pragma unroll
   for (int j = 0; j < 8; ++j)
     mma_f16_ss(tDH, desc_adv(a0, j * 2048), desc_adv(b0, j * 2048), IDESC_DH, (j > 0 || acc) ? 1u : 0u);
@@ -248,17 +251,22 @@ __device__ __forceinline__ void write_h_tile(unsigned char *smem, const float (&
   }
 }
 
-template <bool kStateOnly>
+// kMode 0: output scan; 1: state-only pass (the local state of each segment); 2: the final
+// state's tail in full precision (state-only over the last chunks, every product split)
+template <int kMode>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     ssd_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_bc,
-                       const __grid_constant__ CUtensorMap tm_x, const TcArgs a) {
+                       const __grid_constant__ CUtensorMap tm_x,
+                       const __grid_constant__ CUtensorMap tm_blo, const TcArgs a) {
+  constexpr bool kStateOnly = kMode != 0;
+  constexpr bool kPrecise = kMode == 2;
   extern __shared__ unsigned char smem_raw[];
   unsigned char *smem =
       reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z, g = h / a.hpg;
-  const int t_begin = seg * a.seg_len;
+  const int t_begin = a.t_base + seg * a.seg_len;
   const int t_end = min(a.L, t_begin + a.seg_len);
   const int nck = t_end > t_begin ? (t_end - t_begin + QC - 1) / QC : 0;
   const int last = nck - 1;
@@ -282,6 +290,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   if (warp == kWarpTma && lane == 0) {
     prefetch_tmap(&tm_bc);
     prefetch_tmap(&tm_x);
+    if (kPrecise) prefetch_tmap(&tm_blo);
   }
   if (warp == kWarpIssueA) {
     tmem_alloc(sb + OFF_MISC, TM_COLS);
@@ -311,11 +320,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const uint32_t sst = sb + st * kStage;
         const uint32_t full = BAR(BAR_FULL0 + st);
         TC_MARK(k, 14);
-        mbar_arrive_expect_tx(full, (kStateOnly ? 2 * kTile : 4 * kTile) + 1024);
+        mbar_arrive_expect_tx(full, (kStateOnly && !kPrecise ? 2 * kTile : 4 * kTile) + 1024);
         const int cB = g * 128, cC = a.G * 128 + g * 128;
         if (!kStateOnly) {
           tma_load_3d(sst + OFF_C, &tm_bc, cC, t0, b, full);
           tma_load_3d(sst + OFF_C + kTile, &tm_bc, cC + 64, t0, b, full);
+        }
+        if (kPrecise) {  // the low fp16 parts of B go where C would be
+          tma_load_3d(sst + OFF_C, &tm_blo, cB, t0 - a.t_base, b, full);
+          tma_load_3d(sst + OFF_C + kTile, &tm_blo, cB + 64, t0 - a.t_base, b, full);
         }
         tma_load_3d(sst + OFF_B, &tm_bc, cB, t0, b, full);
         tma_load_3d(sst + OFF_B + kTile, &tm_bc, cB + 64, t0, b, full);
@@ -343,13 +356,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const uint32_t sst = sb + st * kStage;
         if (!mbar_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, abort_flag, a.err, lim)) break;
         if (!mbar_wait(BAR(BAR_XREADY0 + st), (k >> 1) & 1, abort_flag, a.err, lim)) break;
-        if (k == last && !mbar_wait(BAR(BAR_XLOREADY), 0, abort_flag, a.err, lim)) break;
+        if (!kPrecise && k == last && !mbar_wait(BAR(BAR_XLOREADY), 0, abort_flag, a.err, lim)) break;
         if (k >= 1 && !mbar_wait(BAR(BAR_DHFREE), (k - 1) & 1, abort_flag, a.err, lim)) break;
         tc_fence_after();
         TC_MARK(k, 9);
-        issue_dH(sst, sb + OFF_XW + st * kXBuf, tmem + TM_DH, false);
-        // last chunk: the low part of w o X (in the other w o X buffer) for the final state
-        if (k == last) issue_dH(sst, sb + OFF_XW + ((k + 1) & 1) * kXBuf, tmem + TM_DH, true);
+        issue_dH(sst + OFF_B, sb + OFF_XW + st * kXBuf, tmem + TM_DH, false);
+        if (kPrecise) {
+          // B w o X = (B_hi + B_lo)(wX_hi + wX_lo) without the lo * lo term: fp32 accuracy
+          issue_dH(sst + OFF_B, sb + OFF_X + st * kTile, tmem + TM_DH, true);
+          issue_dH(sst + OFF_C, sb + OFF_XW + st * kXBuf, tmem + TM_DH, true);
+        } else if (k == last) {
+          // last chunk: the low part of w o X (in the other w o X buffer) for the final state
+          issue_dH(sst + OFF_B, sb + OFF_XW + ((k + 1) & 1) * kXBuf, tmem + TM_DH, true);
+        }
         mma_commit(BAR(BAR_XWFREE0 + st));
         mma_commit(BAR(BAR_DHREADY));
         if (kStateOnly) {
@@ -407,173 +426,182 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
   } else if (warp >= kWarpConv0 && warp < kWarpConv0 + kConvWarps) {
     // ---------------------------------------------------------------- conv + SiLU -> X, w o X
-    // Warp cw makes tokens 32cw..32cw+31; lane l channels 2l, 2l+1.  Raw row r of the w o X
-    // buffer holds time t0-3+r; token s reads rows s..s+3 (a register window), then
-    // overwrites row s with its w o X row and writes its X row to row s of X.  Rows
-    // 32cw+32..+34 belong to the next warp's tokens, so every warp reads them before the
-    // group barrier that precedes all writes.
-    // SiLU(u) = u * sigmoid(u) = h + h * tanh(h) with h = u / 2.  The conv accumulates h
-    // directly (halved weights) in fp16 pairs -- the precision of the MMA operand it feeds,
-    // 11 significant bits -- and one half2 tanh serves both channels.  The last chunk of a
-    // segment, whose newest tokens dominate the final state, uses fp32 and the exact SiLU.
-    const int cw = warp - kWarpConv0;
-    const bool leader = (warp == kWarpConv0 && lane == 0);
-    const int ch = h * 64 + 2 * lane;
+    // Lane layout: channel group cg = lane % 8 (the head's channels 8cg .. 8cg+7, one 16-byte
+    // piece of a 128-byte row) and token group tg = lane / 8; warp cw covers tokens
+    // 32cw .. 32cw+31, so a lane makes tokens s0 .. s0+7 with s0 = 32cw + 8tg.  Raw row r of
+    // the w o X buffer holds time t0-3+r, and token s reads rows s .. s+3: its own rows s0 ..
+    // s0+7 (which it overwrites with w o X in order, after reading them) and the 3 rows after
+    // them (the next token group's own rows, read before the group barrier that precedes all
+    // writes).  Every access moves 16 bytes; a warp's 4 token groups touch 4 whole rows, so the
+    // 128-byte swizzle keeps each access conflict-free.
+    // SiLU(u) = u * sigmoid(u) = h + h * tanh(h) with h = u / 2: the conv accumulates h
+    // directly (halved weights) in fp16 pairs -- the precision of the MMA operand it feeds --
+    // and one half2 tanh serves two channels.  The last chunk of a segment (and every chunk of
+    // the tail pass) runs in fp32 with the exact SiLU and stores w o X as fp16 hi + lo parts.
+    const int cw = warp - kWarpConv0, cg = lane & 7, tg = lane >> 3;
+    const int ctid = 32 * cw + lane;
+    const int s0 = 32 * cw + 8 * tg;
+    const bool leader = ctid == 0;
+    const int ch0 = h * 64 + 8 * cg;
     const int W = a.W;
-    float2 ew[4], bias2 = make_float2(0.f, 0.f);
+    float *wtok = reinterpret_cast<float *>(smem + OFF_WTOK);
+    __half2 hw[4][4], hb[4];  // [tap j: input at time t-3+j][channel pair], halved
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {  // half the weight for the input at time t-3+j
-      const int k = j - (4 - W);
-      ew[j].x = (W > 0 && k >= 0) ? 0.5f * __bfloat162float(a.conv_w[(long long)ch * W + k]) : 0.f;
-      ew[j].y = (W > 0 && k >= 0) ? 0.5f * __bfloat162float(a.conv_w[(long long)(ch + 1) * W + k]) : 0.f;
+    for (int i = 0; i < 4; ++i) {
+      float2 bb = make_float2(0.f, 0.f);
+      if (W > 0 && a.conv_b) bb = make_float2(__bfloat162float(a.conv_b[ch0 + 2 * i]), __bfloat162float(a.conv_b[ch0 + 2 * i + 1]));
+      hb[i] = __float22half2_rn(make_float2(0.5f * bb.x, 0.5f * bb.y));
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int kk = j - (4 - W);
+        float2 ww = make_float2(0.f, 0.f);
+        if (W > 0 && kk >= 0)
+          ww = make_float2(__bfloat162float(a.conv_w[(long long)(ch0 + 2 * i) * W + kk]),
+                           __bfloat162float(a.conv_w[(long long)(ch0 + 2 * i + 1) * W + kk]));
+        hw[j][i] = __float22half2_rn(make_float2(0.5f * ww.x, 0.5f * ww.y));
+      }
     }
-    if (W > 0 && a.conv_b) {
-      bias2.x = 0.5f * __bfloat162float(a.conv_b[ch]);
-      bias2.y = 0.5f * __bfloat162float(a.conv_b[ch + 1]);
-    }
-    __half2 hw[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) hw[j] = __float22half2_rn(ew[j]);
-    const __half2 hbias = __float22half2_rn(bias2);
-    // byte offset of this lane's 4 bytes within a swizzled row r, by r mod 8
-    uint32_t loff[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) loff[u] = ((uint32_t)((lane >> 2) ^ u) << 4) + ((uint32_t)(lane & 3) << 2);
-    const int tok0 = kTokPerConvWarp * cw;  // multiple of 8
     for (int k = 0; k < nck; ++k) {
       const int st = k & 1, xb = k & 1, lb = (k + 1) & 1;
       const bool is_last = (k == last);
+      const bool exact = kPrecise || is_last;  // fp32 conv, exact SiLU, w o X as hi + lo
       // the leader waits for every input of the chunk, then one group barrier releases all
       if (leader) {
         bool ok = mbar_wait(BAR(BAR_FULLX0 + xb), (k >> 1) & 1, abort_flag, a.err, lim);
         if (ok) ok = mbar_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, abort_flag, a.err, lim);
         if (ok && !kStateOnly && k >= 2)
           ok = mbar_wait(BAR(BAR_XFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err, lim);
-        if (ok && is_last && k >= 1) mbar_wait(BAR(BAR_XWFREE0 + lb), ((k - 1) >> 1) & 1, abort_flag, a.err, lim);
+        if (ok && !kPrecise && is_last && k >= 1)
+          mbar_wait(BAR(BAR_XWFREE0 + lb), ((k - 1) >> 1) & 1, abort_flag, a.err, lim);
         TC_MARK(k, 0);
       }
       if (named_bar_or(kNbConv, 32 * kConvWarps, *abort_flag != 0)) break;
-      const float *cs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
-      const float *dtv = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
-      const float cs_end = cs[QC - 1];
-      const float wl = __expf(cs_end - cs[tok0 + lane]) * dtv[tok0 + lane];  // w of token tok0+lane
-      const uint32_t wl2 = pack_f16(wl, wl);
-      unsigned char *xt = smem + OFF_X + xb * kTile + tok0 * 128;   // row tok0
-      unsigned char *xwt = smem + OFF_XW + xb * kXBuf + tok0 * 128;
-      unsigned char *xlt = smem + OFF_XW + lb * kXBuf + tok0 * 128;
-      // raw rows tok0 + r for r = 0..34 (tok0 is a multiple of 8, so row mod 8 = r mod 8)
-#define RAW(r) (*reinterpret_cast<const uint32_t *>(xwt + (r) * 128 + loff[(r) & 7]))
-      uint32_t r0 = RAW(0), r1 = RAW(1), r2 = RAW(2);
+      {  // this thread's token weight w = e^{cs_Q - cs_s} dt_s, for the whole group
+        const float *cs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
+        const float *dtv = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
+        wtok[ctid] = __expf(cs[QC - 1] - cs[ctid]) * dtv[ctid];
+      }
+      unsigned char *xt = smem + OFF_X + xb * kTile;   // X rows
+      unsigned char *xwt = smem + OFF_XW + xb * kXBuf;  // raw rows in, w o X rows out
+      // low parts: the other w o X buffer, or X (unused) in the tail pass
+      unsigned char *xlt = kPrecise ? xt : smem + OFF_XW + lb * kXBuf;
+#define ROW16(buf, r) (*reinterpret_cast<uint4 *>((buf) + (uint32_t)(r) * 128u + ((uint32_t)(cg ^ ((r) & 7)) << 4)))
+      const uint4 halo0 = ROW16(xwt, s0 + 8), halo1 = ROW16(xwt, s0 + 9), halo2 = ROW16(xwt, s0 + 10);
+      uint4 rw0 = ROW16(xwt, s0), rw1 = ROW16(xwt, s0 + 1), rw2 = ROW16(xwt, s0 + 2);
       const int t0 = t_begin + k * QC;
-      if (cw == 0 && t0 == 0) {  // history before the first token comes from the conv cache
-        uint32_t hist[3] = {0u, 0u, 0u};
+      if (s0 == 0 && t0 == 0) {  // history before the first token comes from the conv cache
+        uint4 hist[3];
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
           const int tau = j - 3;
-          if (a.csi && W + tau >= 0)
-            hist[j] = *reinterpret_cast<const uint32_t *>(a.csi + ((long long)b * W + (W + tau)) * a.conv_dim + ch);
+          hist[j] = (a.csi && W + tau >= 0)
+                        ? *reinterpret_cast<const uint4 *>(a.csi + ((long long)b * W + (W + tau)) * a.conv_dim + ch0)
+                        : make_uint4(0u, 0u, 0u, 0u);
         }
-        r0 = hist[0];
-        r1 = hist[1];
-        r2 = hist[2];
+        rw0 = hist[0];
+        rw1 = hist[1];
+        rw2 = hist[2];
       }
-      constexpr int T = kTokPerConvWarp;
-      const uint32_t nb0 = RAW(T), nb1 = RAW(T + 1), nb2 = RAW(T + 2);
-      named_bar(kNbConv, 32 * kConvWarps);  // all boundary rows and prefix sums read
+      named_bar(kNbConv, 32 * kConvWarps);  // halo rows read and token weights written
       if (leader) mbar_arrive(BAR(BAR_EMPTY0 + st));
-      // The token loop is compiled twice: the common chunks, and the last chunk of a segment.
-      auto tokens = [&](auto last_tag) {
-        constexpr bool kLast = decltype(last_tag)::value;
-        if constexpr (!kLast) {
-          __half2 xm3 = __float22half2_rn(unpack_bf16(r0)), xm2 = __float22half2_rn(unpack_bf16(r1)),
-                  xm1 = __float22half2_rn(unpack_bf16(r2));
-#pragma unroll 1
-          for (int gi = 0; gi < T / 8; ++gi) {
-            __half2 xn[8];
+      if (!exact) {
+        // 8 bf16 -> 4 fp16 pairs
+        auto cvt = [](const uint4 &r, __half2 (&o)[4]) {
+          const uint32_t u[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int nxt = 8 * gi + u + 3;  // row of time t for token 8gi+u
-              uint32_t w3;
-              if (nxt < T) w3 = RAW(nxt);
-              else w3 = nxt == T ? nb0 : (nxt == T + 1 ? nb1 : nb2);
-              xn[u] = __float22half2_rn(unpack_bf16(w3));
-            }
+          for (int i = 0; i < 4; ++i) o[i] = __float22half2_rn(unpack_bf16(u[i]));
+        };
+        __half2 xm3[4], xm2[4], xm1[4];
+        cvt(rw0, xm3);
+        cvt(rw1, xm2);
+        cvt(rw2, xm1);
+#pragma unroll 4
+        for (int j = 0; j < 8; ++j) {
+          const int s = s0 + j;
+          const uint4 rn = j + 3 < 8 ? ROW16(xwt, s + 3) : (j == 5 ? halo0 : (j == 6 ? halo1 : halo2));
+          __half2 x0[4], xo[4], xw[4];
+          cvt(rn, x0);
+          const __half2 w2 = __float2half2_rn(wtok[s]);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int i = 8 * gi + u;
-              const __half2 x0 = xn[u];
-              __half2 xo = x0;
-              if (W != 0) {
-                __half2 acc = __hfma2(hw[0], xm3, hbias);
-                acc = __hfma2(hw[1], xm2, acc);
-                acc = __hfma2(hw[2], xm1, acc);
-                acc = __hfma2(hw[3], x0, acc);
-                xo = __hfma2(acc, h2tanh_approx(acc), acc);
-              }
-              const uint32_t off = i * 128 + loff[u];
-              if (!kStateOnly) *reinterpret_cast<__half2 *>(xt + off) = xo;
-              const uint32_t w2 = __shfl_sync(0xffffffffu, wl2, i);
-              *reinterpret_cast<__half2 *>(xwt + off) = __hmul2(xo, *reinterpret_cast<const __half2 *>(&w2));
-              xm3 = xm2;
-              xm2 = xm1;
-              xm1 = x0;
-            }
+          for (int i = 0; i < 4; ++i) {
+            __half2 acc = __hfma2(hw[0][i], xm3[i], hb[i]);
+            acc = __hfma2(hw[1][i], xm2[i], acc);
+            acc = __hfma2(hw[2][i], xm1[i], acc);
+            acc = __hfma2(hw[3][i], x0[i], acc);
+            xo[i] = W != 0 ? __hfma2(acc, h2tanh_approx(acc), acc) : x0[i];
+            xw[i] = __hmul2(xo[i], w2);
+            xm3[i] = xm2[i];
+            xm2[i] = xm1[i];
+            xm1[i] = x0[i];
           }
-          return;
+          if (!kStateOnly)
+            ROW16(xt, s) = make_uint4(*reinterpret_cast<uint32_t *>(&xo[0]), *reinterpret_cast<uint32_t *>(&xo[1]),
+                                      *reinterpret_cast<uint32_t *>(&xo[2]), *reinterpret_cast<uint32_t *>(&xo[3]));
+          ROW16(xwt, s) = make_uint4(*reinterpret_cast<uint32_t *>(&xw[0]), *reinterpret_cast<uint32_t *>(&xw[1]),
+                                     *reinterpret_cast<uint32_t *>(&xw[2]), *reinterpret_cast<uint32_t *>(&xw[3]));
         }
-        float2 xm3 = unpack_bf16(r0), xm2 = unpack_bf16(r1), xm1 = unpack_bf16(r2);
+      } else {
+        // The final state's chunks: their newest tokens dominate the final state, so X comes
+        // from the fp32 conv and SiLU and w o X is stored as the fp16 hi + lo parts of the fp32
+        // product.  The halved bf16 weights are exact in fp16, so the fp16 copies serve here.
+        // One channel pair at a time (4-byte accesses) keeps this path's registers few.
+        auto word = [](const uint4 &r, int i) { return i == 0 ? r.x : (i == 1 ? r.y : (i == 2 ? r.z : r.w)); };
 #pragma unroll 1
-        for (int gi = 0; gi < T / 8; ++gi) {
-          float2 xn[8];
+        for (int i = 0; i < 4; ++i) {
+          // this pair's fp32 weights (tap j multiplies the input at time t-3+j) and bias
+          float2 wj[4];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int nxt = 8 * gi + u + 3;  // row of time t for token 8gi+u
-            uint32_t w3;
-            if (nxt < T) w3 = RAW(nxt);
-            else w3 = nxt == T ? nb0 : (nxt == T + 1 ? nb1 : nb2);
-            xn[u] = unpack_bf16(w3);
+          for (int j = 0; j < 4; ++j) {
+            const int kk = j - (4 - W);
+            wj[j] = (W > 0 && kk >= 0)
+                        ? make_float2(__bfloat162float(a.conv_w[(long long)(ch0 + 2 * i) * W + kk]),
+                                      __bfloat162float(a.conv_w[(long long)(ch0 + 2 * i + 1) * W + kk]))
+                        : make_float2(0.f, 0.f);
           }
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int i = 8 * gi + u;
-            const float2 x0 = xn[u];
-            float2 acc = x0;
+          const float2 hb2 = (W > 0 && a.conv_b)
+                                 ? make_float2(__bfloat162float(a.conv_b[ch0 + 2 * i]), __bfloat162float(a.conv_b[ch0 + 2 * i + 1]))
+                                 : make_float2(0.f, 0.f);
+          const float2 w0 = wj[0], w1 = wj[1], w2 = wj[2], w3 = wj[3];
+          float2 xm3 = unpack_bf16(word(rw0, i)), xm2 = unpack_bf16(word(rw1, i)), xm1 = unpack_bf16(word(rw2, i));
+          const uint32_t hw0 = word(halo0, i), hw1 = word(halo1, i), hw2 = word(halo2, i);
+          const uint32_t cofs = ((uint32_t)cg << 4) + 4u * (uint32_t)i;  // before the swizzle
+#pragma unroll 1
+          for (int j = 0; j < 8; ++j) {
+            const int s = s0 + j;
+            const int rr = s + 3;
+            const uint32_t un = j + 3 < 8
+                                    ? *reinterpret_cast<const uint32_t *>(xwt + (uint32_t)rr * 128u + (cofs ^ ((uint32_t)(rr & 7) << 4)))
+                                    : (j == 5 ? hw0 : (j == 6 ? hw1 : hw2));
+            const float2 x0 = unpack_bf16(un);
+            float2 v = x0;
             if (W != 0) {
-              acc = __ffma2_rn(ew[0], xm3, bias2);
-              acc = __ffma2_rn(ew[1], xm2, acc);
-              acc = __ffma2_rn(ew[2], xm1, acc);
-              acc = __ffma2_rn(ew[3], x0, acc);
+              float2 acc = __ffma2_rn(w0, xm3, hb2);
+              acc = __ffma2_rn(w1, xm2, acc);
+              acc = __ffma2_rn(w2, xm1, acc);
+              acc = __ffma2_rn(w3, x0, acc);
+              v = make_float2(silu(acc.x), silu(acc.y));
             }
-            const uint32_t off = i * 128 + loff[u];
-            {
-              // The final state's chunk: its newest tokens dominate the final state, so X
-              // comes from the fp32 SiLU and w o X is stored as the fp16 hi + lo parts of the
-              // fp32 product.
-              const float u0 = W != 0 ? silu(2.f * acc.x) : acc.x;
-              const float u1 = W != 0 ? silu(2.f * acc.y) : acc.y;
-              const float ws = __shfl_sync(0xffffffffu, wl, i);
-              const float2 v = make_float2(u0 * ws, u1 * ws);
-              const __half2 hi = __float22half2_rn(v);
-              const float2 hf = __half22float2(hi);
-              if (!kStateOnly) *reinterpret_cast<uint32_t *>(xt + off) = pack_f16(u0, u1);
-              *reinterpret_cast<__half2 *>(xwt + off) = hi;
-              *reinterpret_cast<uint32_t *>(xlt + off) = pack_f16(v.x - hf.x, v.y - hf.y);
-            }
+            const float ws = wtok[s];
+            const float2 p = make_float2(v.x * ws, v.y * ws);
+            const __half2 hi = __float22half2_rn(p);
+            const float2 hf = __half22float2(hi);
+            const uint32_t off = (uint32_t)s * 128u + (cofs ^ ((uint32_t)(s & 7) << 4));
+            if (!kStateOnly) *reinterpret_cast<uint32_t *>(xt + off) = pack_f16(v.x, v.y);
+            *reinterpret_cast<uint32_t *>(xwt + off) = *reinterpret_cast<const uint32_t *>(&hi);
+            *reinterpret_cast<uint32_t *>(xlt + off) = pack_f16(p.x - hf.x, p.y - hf.y);
             xm3 = xm2;
             xm2 = xm1;
             xm1 = x0;
           }
         }
-      };
-      if (is_last) tokens(std::true_type{});
-      else tokens(std::false_type{});
-#undef RAW
+      }
+#undef ROW16
       fence_proxy_async();
       named_bar(kNbConv, 32 * kConvWarps);
       if (leader) {
         TC_MARK(k, 1);
         mbar_arrive(BAR(BAR_XREADY0 + xb));
-        if (is_last) mbar_arrive(BAR(BAR_XLOREADY));
+        if (!kPrecise && is_last) mbar_arrive(BAR(BAR_XLOREADY));
       }
     }
   } else if (warp >= kWarpMask0 && warp < kWarpMask0 + 4) {
@@ -997,26 +1025,46 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
   a.debug_skip_chunk = p.stall_chunk1 - 1;
   const long long seg_stride = (long long)p.B * p.H * p.P * p.N;
   dim3 grid(p.n_seg, p.H, p.B);
+  // the low parts of B over the tail (tail pass only; else the B|C map stands in, unread)
+  CUtensorMap tml = tm;
+  if (mode == 2) {
+    const cuuint64_t GN = (cuuint64_t)p.G * p.N;
+    cuuint64_t ldims[3] = {GN, (cuuint64_t)p.ntail, (cuuint64_t)p.B};
+    cuuint64_t lstrides[2] = {GN * 2, GN * 2 * (cuuint64_t)p.ntail};
+    r = enc(&tml, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, p.blo, ldims, lstrides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
   cudaError_t e;
   if (mode == 1) {
     a.h_init = nullptr; a.h_init_seg = 0;
     a.h_out = p.seg_state; a.h_out_seg = seg_stride; a.seg_decay = p.seg_decay;
-    e = set_smem_attr(ssd_scan_tc_kernel<true>, kSmemAlloc, s);
+    e = set_smem_attr(ssd_scan_tc_kernel<1>, kSmemAlloc, s);
     if (e != cudaSuccess) return e;
-    ssd_scan_tc_kernel<true><<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, a);
+    ssd_scan_tc_kernel<1><<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, tml, a);
+  } else if (mode == 2) {
+    // the tail pass: tokens [t_tail, L) of every (batch row, head), from a zero state, into
+    // tail_dh and their total decay into tail_dec
+    a.t_base = p.t_tail; a.seg_len = p.L - p.t_tail;
+    a.h_init = nullptr; a.h_init_seg = 0;
+    a.h_out = p.tail_dh; a.h_out_seg = 0; a.seg_decay = p.tail_dec;
+    e = set_smem_attr(ssd_scan_tc_kernel<2>, kSmemAlloc, s);
+    if (e != cudaSuccess) return e;
+    ssd_scan_tc_kernel<2><<<dim3(1, p.H, p.B), kThreadsTC, kSmemAlloc, s>>>(tm, tmx, tml, a);
   } else {
     if (p.n_seg > 1) {
       a.h_init = p.seg_state; a.h_init_seg = seg_stride;
     } else {
       a.h_init = p.h0; a.h_init_seg = 0;
     }
-    // the last segment leaves the state before its last kTailChunks chunks; the fp32 tail pass
-    // adds what those chunks contribute
+    // the last segment leaves the state entering the tail; the tail pass adds what the tail's
+    // chunks contribute
     a.h_out = p.h_final; a.h_out_seg = 0; a.seg_decay = nullptr;
     a.tail_chunks = p.tail_dh ? kTailChunks : 0;
-    e = set_smem_attr(ssd_scan_tc_kernel<false>, kSmemAlloc, s);
+    e = set_smem_attr(ssd_scan_tc_kernel<0>, kSmemAlloc, s);
     if (e != cudaSuccess) return e;
-    ssd_scan_tc_kernel<false><<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, a);
+    ssd_scan_tc_kernel<0><<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, tml, a);
   }
   return cudaGetLastError();
 }
