@@ -126,7 +126,7 @@ struct WsLayout {
   // CUDA-core path
   size_t u, dte, yf, seg_state, seg_decay, simt_end;
   // tensor-core path
-  size_t tc_bc, tc_dte, tc_cs, tc_yf, tc_q, tc_ssq, tc_seg_state, tc_seg_decay, tc_dh, tc_blo, tc_end;
+  size_t tc_bc, tc_dte, tc_cs, tc_yf, tc_q, tc_ssq, tc_seg_state, tc_seg_decay, tc_dh, tc_end;
   int Lpad;
   size_t total;
 };
@@ -171,7 +171,6 @@ WsLayout prefill_layout(const ssd_config_t *c) {
     off = round_up(off + (size_t)n_seg * c->batch * c->nheads * 4, kAlign);
   }
   w.tc_dh = off;   off = round_up(off + state + (size_t)c->batch * c->nheads * 4, kAlign);
-  w.tc_blo = off;  off = round_up(off + (size_t)c->batch * kTailChunks * kTcTile * c->ngroups * c->dstate * 2, kAlign);
   w.tc_end = off;
   w.total = prefill_uses_tc(c) ? w.tc_end : w.simt_end;
   return w;
@@ -299,15 +298,6 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
     p.seg_decay = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.tc_seg_decay) : nullptr;
     p.tail_dh = p.h_final ? reinterpret_cast<float *>(ws + lay.tc_dh) : nullptr;
     p.tail_dec = p.h_final ? p.tail_dh + (size_t)c->batch * c->nheads * c->headdim * c->dstate : nullptr;
-    if (p.tail_dh) {  // the tail: the last kTailChunks chunks of the last segment
-      const int t_b = (p.n_seg - 1) * p.seg_len;
-      const int nck = (p.L - t_b + kTcTile - 1) / kTcTile;
-      p.t_tail = t_b + kTcTile * (nck > kTailChunks ? nck - kTailChunks : 0);
-      p.ntail = p.L - p.t_tail;
-      p.blo = reinterpret_cast<__half *>(ws + lay.tc_blo);
-    } else {
-      p.t_tail = p.L;
-    }
     // The outgoing conv cache may be written before the scan unless it overlaps an input
     // that later kernels read.
     const size_t x_span = ((size_t)c->batch * c->seqlen - 1) * (size_t)a->xBC_row_stride * es + (size_t)conv_dim * es;
@@ -338,7 +328,7 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
     }
     SSD_TRY(traced("ssd_scan_tc", s, [&] { return launch_scan_tc(p, 0, s); }));
     if (side.forked)
-      SSD_TRY(traced("ssd_scan_tc_tail", side.side->s, [&] { return launch_scan_tc(p, 2, side.side->s); }));
+      SSD_TRY(traced("ssd_state_tail", side.side->s, [&] { return launch_state_tail(p, side.side->s); }));
     if (side.forked) {
       SSD_TRY(side.join());
       SSD_TRY(traced("ssd_tail_fold", s, [&] { return launch_tail_fold(p, s); }));

@@ -258,13 +258,12 @@ cudaError_t launch_conv_silu_f32(const PrefillPlan &p, cudaStream_t s) {
 }
 
 // Conv + SiLU of the B and C channels into fp16 (the tensor-core scan's operand buffer).
-// A streaming kernel: one thread owns 8 channels (one 16-byte load per row, one 16-byte store
-// per output row) over kBcTok tokens, with the 4-row window kept in fp32 register pairs, and
-// loads 8 rows ahead; a warp moves 512 contiguous bytes per row.  The 3 rows before the
-// first token come from the rows above (or the conv cache / zeros at t < 0).
+// A streaming kernel: one thread owns 4 channels (one 8-byte load per row) over kBcTok
+// tokens with the 4-row window kept in fp32 registers, and loads 8 rows ahead; few registers
+// per thread keep several blocks per SM and tens of kilobytes of loads in flight.  The 3 rows
+// before the first token come from the rows above (or the conv cache / zeros at t < 0).
 constexpr int kBcTok = 16;
 constexpr int kBcThreads = 256;
-constexpr int kBcCh = 8;  // channels per thread
 
 // SiLU(u) = u sigmoid(u) = h + h tanh(h) with h = u / 2, using the hardware tanh
 // approximation (one special-function op instead of an exponential and a reciprocal).  Its
@@ -276,100 +275,85 @@ __device__ __forceinline__ float silu_tanh(float u) {
   return fmaf(h, t, h);
 }
 
-// 8 bf16 (one 16-byte row piece) -> 4 fp32 pairs
-__device__ __forceinline__ void unpack8(const uint4 &r, float2 (&v)[4]) {
-  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) v[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+__device__ __forceinline__ void unpack4(const uint2 &r, float (&v)[4]) {
+  v[0] = __uint_as_float(r.x << 16);
+  v[1] = __uint_as_float(r.x & 0xFFFF0000u);
+  v[2] = __uint_as_float(r.y << 16);
+  v[3] = __uint_as_float(r.y & 0xFFFF0000u);
 }
 
-// The B channels of the final state's tail (tokens t >= t_tail, written when blo is set) use
-// the exact SiLU, and their fp16 rounding error goes to blo: the tail pass multiplies both
-// parts, so that the final state's newest tokens enter it with fp32 accuracy.
 template <int W>
 __device__ __forceinline__ void bc_conv_tile(const __nv_bfloat16 *__restrict__ xBC, long long xs,
                                              const __nv_bfloat16 *__restrict__ csi,
                                              const __nv_bfloat16 *__restrict__ w,
                                              const __nv_bfloat16 *__restrict__ bias,
                                              __half *__restrict__ out, int L, int conv_dim, int c_begin,
-                                             int C_out, int bx, int by, int bz, __half *__restrict__ blo,
-                                             int t_tail, int ntail, int n_b) {
-  const int o8 = (bx * kBcThreads + threadIdx.x) * kBcCh;
-  if (o8 >= C_out) return;
-  const int c8 = c_begin + o8;
+                                             int C_out, int bx, int by, int bz) {
+  const int o4 = (bx * kBcThreads + threadIdx.x) * 4;
+  if (o4 >= C_out) return;
+  const int c4 = c_begin + o4;
   const int b = bz;
   const int t0 = by * kBcTok;
   const int t1 = min(L, t0 + kBcTok);
-  const bool tail_tile = blo != nullptr && o8 < n_b && t1 > t_tail;
-  const __nv_bfloat16 *xrow = xBC + (long long)b * L * xs + c8;
-  float2 wt[4][4], bs[4];  // [tap][channel pair]: tap k multiplies time t-(W-1)+k
+  const __nv_bfloat16 *xrow = xBC + (long long)b * L * xs + c4;
+  float wt[4][4], bs[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    bs[i] = bias ? make_float2(__bfloat162float(bias[c8 + 2 * i]), __bfloat162float(bias[c8 + 2 * i + 1]))
-                 : make_float2(0.f, 0.f);
+    bs[i] = bias ? __bfloat162float(bias[c4 + i]) : 0.f;
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      wt[k][i] = (k < W) ? make_float2(__bfloat162float(w[(long long)(c8 + 2 * i) * W + k]),
-                                       __bfloat162float(w[(long long)(c8 + 2 * i + 1) * W + k]))
-                         : make_float2(0.f, 0.f);
+    for (int k = 0; k < 4; ++k) wt[k][i] = (k < W) ? __bfloat162float(w[(long long)(c4 + i) * W + k]) : 0.f;
   }
-  float2 x3[4], x2[4], x1[4];  // times t-3, t-2, t-1
+  float x3[4], x2[4], x1[4];  // times t-3, t-2, t-1
   {
-    uint4 hist[3];
+    uint2 hist[3];
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
       const int tau = t0 - 3 + j;
       if (W > 0 && tau >= 0) {
-        hist[j] = *reinterpret_cast<const uint4 *>(xrow + (long long)tau * xs);
+        hist[j] = *reinterpret_cast<const uint2 *>(xrow + (long long)tau * xs);
       } else if (csi && W > 0 && W + tau >= 0) {
-        hist[j] = *reinterpret_cast<const uint4 *>(csi + ((long long)b * W + (W + tau)) * conv_dim + c8);
+        hist[j] = *reinterpret_cast<const uint2 *>(csi + ((long long)b * W + (W + tau)) * conv_dim + c4);
       } else {
-        hist[j] = make_uint4(0u, 0u, 0u, 0u);
+        hist[j] = make_uint2(0u, 0u);
       }
     }
-    unpack8(hist[0], x3);
-    unpack8(hist[1], x2);
-    unpack8(hist[2], x1);
+    unpack4(hist[0], x3);
+    unpack4(hist[1], x2);
+    unpack4(hist[2], x1);
   }
   // Rows in groups of 8; the common full tile runs without per-row bounds checks.
   auto group = [&](int tg, auto full_tag) {
     constexpr bool kFull = decltype(full_tag)::value;
-    uint4 cur[8];
+    uint2 cur[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      cur[j] = (kFull || tg + j < t1) ? __ldcs(reinterpret_cast<const uint4 *>(xrow + (long long)(tg + j) * xs))
-                                      : make_uint4(0u, 0u, 0u, 0u);
+      cur[j] = (kFull || tg + j < t1) ? __ldcs(reinterpret_cast<const uint2 *>(xrow + (long long)(tg + j) * xs))
+                                      : make_uint2(0u, 0u);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int t = tg + j;
       if (!kFull && t >= t1) break;
-      const bool exact = tail_tile && t >= t_tail;
-      float2 x0[4];
-      uint32_t r[4], rl[4];
-      unpack8(cur[j], x0);
+      float x0[4], r[4];
+      unpack4(cur[j], x0);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        float2 v = x0[i];
-        if (W > 0) {
-          const float2 xw[4] = {x3[i], x2[i], x1[i], x0[i]};
-          float2 acc = bs[i];
+        if (W == 0) {
+          r[i] = x0[i];
+        } else {
+          // tap k multiplies time t-(W-1)+k
+          const float xs4[4] = {x3[i], x2[i], x1[i], x0[i]};
+          float acc = bs[i];
 #pragma unroll
-          for (int k = 0; k < W; ++k) acc = __ffma2_rn(wt[k][i], xw[4 - W + k], acc);
-          v = exact ? make_float2(silu(acc.x), silu(acc.y)) : make_float2(silu_tanh(acc.x), silu_tanh(acc.y));
+          for (int k = 0; k < W; ++k) acc = fmaf(wt[k][i], xs4[4 - W + k], acc);
+          r[i] = silu_tanh(acc);
         }
-        const __half2 hv = __floats2half2_rn(v.x, v.y);
-        r[i] = *reinterpret_cast<const uint32_t *>(&hv);
-        const float2 hf = __half22float2(hv);
-        const __half2 lv = __floats2half2_rn(v.x - hf.x, v.y - hf.y);
-        rl[i] = *reinterpret_cast<const uint32_t *>(&lv);
         x3[i] = x2[i];
         x2[i] = x1[i];
         x1[i] = x0[i];
       }
-      *reinterpret_cast<uint4 *>(out + ((long long)b * L + t) * C_out + o8) = make_uint4(r[0], r[1], r[2], r[3]);
-      if (exact)
-        *reinterpret_cast<uint4 *>(blo + ((long long)b * ntail + (t - t_tail)) * n_b + o8) =
-            make_uint4(rl[0], rl[1], rl[2], rl[3]);
+      const __half2 h01 = __floats2half2_rn(r[0], r[1]), h23 = __floats2half2_rn(r[2], r[3]);
+      *reinterpret_cast<uint2 *>(out + ((long long)b * L + t) * C_out + o4) =
+          make_uint2(*reinterpret_cast<const uint32_t *>(&h01), *reinterpret_cast<const uint32_t *>(&h23));
     }
   };
   if (t1 - t0 == kBcTok) {
@@ -382,15 +366,13 @@ __device__ __forceinline__ void bc_conv_tile(const __nv_bfloat16 *__restrict__ x
 }
 
 template <int W>
-__global__ void __launch_bounds__(kBcThreads, 2) bc_conv_kernel(const __nv_bfloat16 *__restrict__ xBC, long long xs,
+__global__ void __launch_bounds__(kBcThreads) bc_conv_kernel(const __nv_bfloat16 *__restrict__ xBC, long long xs,
                                                              const __nv_bfloat16 *__restrict__ csi,
                                                              const __nv_bfloat16 *__restrict__ w,
                                                              const __nv_bfloat16 *__restrict__ bias,
                                                              __half *__restrict__ out, int L, int conv_dim,
-                                                             int c_begin, int C_out, __half *__restrict__ blo,
-                                                             int t_tail, int ntail) {
-  bc_conv_tile<W>(xBC, xs, csi, w, bias, out, L, conv_dim, c_begin, C_out, blockIdx.x, blockIdx.y, blockIdx.z,
-                  blo, t_tail, ntail, C_out / 2);
+                                                             int c_begin, int C_out) {
+  bc_conv_tile<W>(xBC, xs, csi, w, bias, out, L, conv_dim, c_begin, C_out, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
 // The tensor-core path's front end in one launch: dt + chunk prefix sums, the outgoing conv
@@ -401,16 +383,15 @@ struct FrontArgs {
   long long xs, ds;
   const float *dt_bias, *A;
   float *dte, *cs;
-  __half *bc, *blo;
+  __half *bc;
   __nv_bfloat16 *cso;
-  int t_tail, ntail;
   int B, L, H, Lpad, conv_dim, d_inner, C_out, W, sp;
   float lo, hi;
   int n_dt, dt_tiles, dt_nch, dt_nhg, n_cso, gx, gy;
 };
 
 template <int W>
-__global__ void __launch_bounds__(kBcThreads, 2) front_tc_kernel(const FrontArgs f) {
+__global__ void __launch_bounds__(kBcThreads) front_tc_kernel(const FrontArgs f) {
   __shared__ float v[2][128][9];
   int j = blockIdx.x;
   if (j < f.n_dt) {  // two 128-thread dt tiles per CTA
@@ -431,35 +412,34 @@ __global__ void __launch_bounds__(kBcThreads, 2) front_tc_kernel(const FrontArgs
   }
   j -= f.n_cso;
   bc_conv_tile<W>(f.xBC, f.xs, f.csi, f.conv_w, f.conv_b, f.bc, f.L, f.conv_dim, f.d_inner, f.C_out,
-                  j % f.gx, (j / f.gx) % f.gy, j / (f.gx * f.gy), f.blo, f.t_tail, f.ntail, f.C_out / 2);
+                  j % f.gx, (j / f.gx) % f.gy, j / (f.gx * f.gy));
 }
 
 cudaError_t launch_bc_conv_f16(const PrefillPlan &p, cudaStream_t s) {
   const int C_out = 2 * p.G * p.N;
-  if (C_out % 8 || p.xs % 8 || p.conv_dim % 8 || p.d_inner % 8) {  // 16-byte accesses; else the generic kernel
-    if (p.blo) return cudaErrorInvalidValue;  // the tail's low parts need the 16-byte kernel
+  if (C_out % 4 || p.xs % 4 || p.conv_dim % 4 || p.d_inner % 4) {  // 8-byte accesses; else the generic kernel
     conv_dispatch<__nv_bfloat16, __half>(p, (__half *)p.bc, p.d_inner, C_out, s);
     return cudaGetLastError();
   }
-  dim3 grid((C_out / kBcCh + kBcThreads - 1) / kBcThreads, (p.L + kBcTok - 1) / kBcTok, p.B);
+  dim3 grid((C_out / 4 + kBcThreads - 1) / kBcThreads, (p.L + kBcTok - 1) / kBcTok, p.B);
   const auto *x = (const __nv_bfloat16 *)p.xBC;
   const auto *csi = (const __nv_bfloat16 *)p.csi;
   const auto *w = (const __nv_bfloat16 *)p.conv_w;
   const auto *bb = (const __nv_bfloat16 *)p.conv_b;
   __half *o = (__half *)p.bc;
   switch (p.W) {
-    case 0: bc_conv_kernel<0><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out, p.blo, p.t_tail, p.ntail); break;
-    case 1: bc_conv_kernel<1><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out, p.blo, p.t_tail, p.ntail); break;
-    case 2: bc_conv_kernel<2><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out, p.blo, p.t_tail, p.ntail); break;
-    case 3: bc_conv_kernel<3><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out, p.blo, p.t_tail, p.ntail); break;
-    default: bc_conv_kernel<4><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out, p.blo, p.t_tail, p.ntail); break;
+    case 0: bc_conv_kernel<0><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
+    case 1: bc_conv_kernel<1><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
+    case 2: bc_conv_kernel<2><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
+    case 3: bc_conv_kernel<3><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
+    default: bc_conv_kernel<4><<<grid, kBcThreads, 0, s>>>(x, p.xs, csi, w, bb, o, p.L, p.conv_dim, p.d_inner, C_out); break;
   }
   return cudaGetLastError();
 }
 
-// False when the shapes need the separate front-end kernels (unaligned 16-byte B/C accesses).
+// False when the shapes need the separate front-end kernels (unaligned 8-byte B/C accesses).
 bool front_tc_fusable(const PrefillPlan &p) {
-  return p.bf16 && (2 * p.G * p.N) % 8 == 0 && p.xs % 8 == 0 && p.conv_dim % 8 == 0 && p.d_inner % 8 == 0 &&
+  return p.bf16 && (2 * p.G * p.N) % 4 == 0 && p.xs % 4 == 0 && p.conv_dim % 4 == 0 && p.d_inner % 4 == 0 &&
          p.H % 8 == 0 && p.ds % 8 == 0;
 }
 
@@ -469,14 +449,13 @@ cudaError_t launch_front_tc(const PrefillPlan &p, bool with_cso, cudaStream_t s)
   f.csi = (const __nv_bfloat16 *)p.csi; f.conv_w = (const __nv_bfloat16 *)p.conv_w;
   f.conv_b = (const __nv_bfloat16 *)p.conv_b; f.xs = p.xs; f.ds = p.ds; f.dt_bias = p.dt_bias; f.A = p.A;
   f.dte = p.dte_hm; f.cs = p.cs_hm; f.bc = (__half *)p.bc; f.cso = (__nv_bfloat16 *)p.cso;
-  f.blo = p.blo; f.t_tail = p.t_tail; f.ntail = p.ntail;
   f.B = p.B; f.L = p.L; f.H = p.H; f.Lpad = p.Lpad; f.conv_dim = p.conv_dim; f.d_inner = p.d_inner;
   f.C_out = 2 * p.G * p.N; f.W = p.W; f.sp = p.softplus; f.lo = p.dt_min; f.hi = p.dt_max;
   f.dt_nch = p.Lpad / 128; f.dt_nhg = (p.H + 7) / 8; f.dt_tiles = f.dt_nch * f.dt_nhg * p.B;
   f.n_dt = (f.dt_tiles + 1) / 2;
   const long long ncso = (with_cso && p.cso && p.W > 0) ? (long long)p.B * p.W * ((long long)p.conv_dim * 2 / 16) : 0;
   f.n_cso = ncso ? (int)std::min<long long>((ncso + kBcThreads - 1) / kBcThreads, 64) : 0;
-  f.gx = (f.C_out / kBcCh + kBcThreads - 1) / kBcThreads; f.gy = (p.L + kBcTok - 1) / kBcTok;
+  f.gx = (f.C_out / 4 + kBcThreads - 1) / kBcThreads; f.gy = (p.L + kBcTok - 1) / kBcTok;
   const long long blocks = (long long)f.n_dt + f.n_cso + (long long)f.gx * f.gy * p.B;
   switch (p.W) {
     case 0: front_tc_kernel<0><<<(unsigned)blocks, kBcThreads, 0, s>>>(f); break;

@@ -41,8 +41,6 @@ struct PrefillPlan {
   float *tail_dh;    // [B, H, P, N] fp32 contribution of the final state's last chunks, from a
                      // zero state (tensor path; null when no final state is written)
   float *tail_dec;   // [B, H] decay over those chunks
-  __half *blo;       // [B, ntail, G*N] low fp16 parts of B over the tail (B - fp16(B))
-  int t_tail, ntail; // the tail: tokens [t_tail, L) of the last segment (ntail = L - t_tail)
   __half *qn;        // [B, L, d_inner] fp16 head-normalised gated output (tensor path, fused
                      // gate: the scan gates and writes these, the rescale finishes the norm)
   float *ssq;        // [B, L, H] sum of squares of each head's gated output
@@ -83,17 +81,17 @@ cudaError_t launch_front_tc(const PrefillPlan &p, bool with_cso, cudaStream_t s)
 cudaError_t launch_dt_cumsum(const PrefillPlan &p, float *dte, float *cs, int Lpad, cudaStream_t s);
 // chunked scan on CUDA cores (scan_simt.cu); mode 0 full, 1 state-only, 2 output-only
 cudaError_t launch_scan_simt(const PrefillPlan &p, int mode, cudaStream_t s);
-// chunked scan on tcgen05 tensor cores (tc_scan.cu); mode 0 full/output, 1 state-only,
-// 2 the final state's tail in full precision
+// chunked scan on tcgen05 tensor cores (tc_scan.cu); mode 0 full/output, 1 state-only
 bool tc_scan_available();
 cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s);
 // inter-segment state pass (state_pass.cu)
 cudaError_t launch_state_pass(const PrefillPlan &p, cudaStream_t s);
-// The final state's last kTailChunks chunks in full precision (tensor-core path): the output
-// scan leaves the state entering them in h_final; the tail pass (launch_scan_tc mode 2) adds
-// up, from a zero state, what those chunks contribute, into p.tail_dh / p.tail_dec, on a side
-// stream beside the output scan; the fold then sets h_final = tail_dec * h_final + tail_dh.
+// fp32 recomputation of the final state's last kTailChunks chunks (tensor-core path): what
+// those chunks add to a zero state, into p.tail_dh / p.tail_dec.  It runs on a side stream
+// beside the output scan, which leaves the state entering those chunks in h_final; the fold
+// then sets h_final = tail_dec * h_final + tail_dh.
 constexpr int kTailChunks = 2;
+cudaError_t launch_state_tail(const PrefillPlan &p, cudaStream_t s);
 cudaError_t launch_tail_fold(const PrefillPlan &p, cudaStream_t s);
 // norms (norm.cu)
 cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s);          // fp32 yf -> y

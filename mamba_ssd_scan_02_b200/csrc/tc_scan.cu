@@ -68,9 +68,9 @@ namespace {
 using namespace tc;
 
 constexpr int QC = 128;              // tokens per chunk
-constexpr int kThreadsTC = 640;       // 20 warps (roles below)
-constexpr int kConvWarps = 4;
-constexpr int kTokPerConvWarp = QC / kConvWarps;  // 32
+constexpr int kThreadsTC = 640;       // 20 warps
+constexpr int kConvWarps = 8;          // see conv_index()
+constexpr int kTokPerConvWarp = QC / kConvWarps;  // 16
 constexpr uint32_t kTile = 16384;    // one 128-row x 128-byte operand box
 // per-stage layout (bytes)
 constexpr uint32_t OFF_C = 0;                 // C tile: channels 0-63 | 64-127
@@ -90,9 +90,7 @@ constexpr uint32_t OFF_H = OFF_XW + 2 * kXBuf;      // h copy [n][p] fp16, 16 KB
 constexpr uint32_t OFF_CF = OFF_H + kTile;          // column factors, 128 fp32
 constexpr uint32_t OFF_CSM = OFF_CF + 512;          // the mask's copies of cs and dt
 constexpr uint32_t OFF_DTM = OFF_CSM + 512;
-constexpr uint32_t OFF_ET = OFF_DTM + 512;          // e^{cs_t} of chunk k in ET[k % 2] (mask -> output)
-constexpr uint32_t OFF_WTOK = OFF_ET + 1024;        // the conv's token weights w_s of the current chunk
-constexpr uint32_t OFF_BAR = OFF_WTOK + 512;
+constexpr uint32_t OFF_BAR = OFF_DTM + 512;
 // Barriers.  Every event that can recur before its consumer has observed the previous
 // occurrence has one barrier per buffer, so that a parity test never sees two phases at once.
 enum {
@@ -108,10 +106,10 @@ enum {
   BAR_DHFREE,                  // dH of chunk k read by the state warps
   BAR_HTFREE,                  // h tile (h_{k-1}) read by MMA3 of chunk k
   BAR_HREADY,                  // h tile holds h_k (state warps)
-  BAR_YREADY0, BAR_YREADY1,    // Yi and Ys of chunk k in TMEM (MMA2 and MMA3 commits)
+  BAR_YREADY0, BAR_YREADY1,    // Yi and Ys of chunk k in TMEM (MMA2 commit)
   BAR_YFREE0, BAR_YFREE1,      // Yi and Ys of chunk k read by the output warps
   BAR_XLOREADY,                // low part of w o X of the last chunk written
-  BAR_DONE_A, BAR_DONE_B,      // every MMA of issuer A / B complete (before TMEM is freed)
+  BAR_DONE,
   kNumBars
 };
 constexpr uint32_t OFF_MISC = OFF_BAR + 8 * 32;   // [0] TMEM base, [1] abort flag
@@ -145,7 +143,6 @@ struct TcArgs {
   long long h_init_seg;
   float *h_out;            // final state destination or null
   long long h_out_seg;
-  int t_base;              // first token of segment 0 (the tail pass starts inside the sequence)
   int tail_chunks;         // > 0: instead of the final state, the last segment writes the state
                            // before its last tail_chunks chunks (an fp32 pass finishes it)
   float *seg_decay;        // [n_seg, B, H] total decay per segment, or null
@@ -219,22 +216,28 @@ __device__ __forceinline__ void issue_Yi(uint32_t tSt, uint32_t xbase, uint32_t 
 #pragma unroll
   for (int j = 0; j < 8; ++j) mma_f16_ts(tYi, tSt + 8 * j, desc_adv(b0, j * 2048), IDESC_YI, j > 0);
 }
-// bbase: the B^T operand (OFF_B of a stage, or OFF_C holding B's low parts in the tail pass)
-__device__ __forceinline__ void issue_dH(uint32_t bbase, uint32_t xwbase, uint32_t tDH, bool acc) {
-  const uint64_t a0 = smem_desc_sw128(bbase, kTile, 1024), b0 = smem_desc_sw128(xwbase, 8192, 1024);
+__device__ __forceinline__ void issue_dH(uint32_t stage, uint32_t xwbase, uint32_t tDH, bool acc) {
+  const uint64_t a0 = smem_desc_sw128(stage + OFF_B, kTile, 1024), b0 = smem_desc_sw128(xwbase, 8192, 1024);
 #pragma unroll
   for (int j = 0; j < 8; ++j)
     mma_f16_ss(tDH, desc_adv(a0, j * 2048), desc_adv(b0, j * 2048), IDESC_DH, (j > 0 || acc) ? 1u : 0u);
 }
 
-// Warp roles.  Each warp index w runs on SM sub-partition w % 4, and a warp reaches only the
-// TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, so every role that touches TMEM rows (mask, state,
-// output) has one warp per sub-partition.  The two MMA-issuing threads sit on sub-partitions
-// 1 and 2; the conv warps, one per sub-partition, spread their issue slots evenly.
-constexpr int kWarpTma = 0, kWarpIssueA = 1, kWarpIssueB = 2;
-constexpr int kWarpMask0 = 4, kWarpState0 = 8, kWarpOut0 = 12, kWarpConv0 = 16;
-// named barriers (0 is __syncthreads)
-constexpr int kNbConv = 1, kNbMask = 2, kNbState = 3, kNbOut = 4;
+// Conv warps: 2, 3, 4, 6, 7, 8, 10, 11 -- none on the sub-partition of warp 1 (warps 1, 5, 9,
+// ...), whose single MMA-issuing thread would otherwise be starved of issue slots.
+__device__ __forceinline__ int conv_index(int warp) {
+  switch (warp) {
+    case 2: return 0;
+    case 3: return 1;
+    case 4: return 2;
+    case 6: return 3;
+    case 7: return 4;
+    case 8: return 5;
+    case 10: return 6;
+    case 11: return 7;
+    default: return -1;
+  }
+}
 
 // Row r (128 bytes) of a 128-byte-swizzled tile: 16-byte chunk c sits at chunk c ^ (r & 7).
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
@@ -251,22 +254,17 @@ __device__ __forceinline__ void write_h_tile(unsigned char *smem, const float (&
   }
 }
 
-// kMode 0: output scan; 1: state-only pass (the local state of each segment); 2: the final
-// state's tail in full precision (state-only over the last chunks, every product split)
-template <int kMode>
+template <bool kStateOnly>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     ssd_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_bc,
-                       const __grid_constant__ CUtensorMap tm_x,
-                       const __grid_constant__ CUtensorMap tm_blo, const TcArgs a) {
-  constexpr bool kStateOnly = kMode != 0;
-  constexpr bool kPrecise = kMode == 2;
+                       const __grid_constant__ CUtensorMap tm_x, const TcArgs a) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char *smem =
       reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z, g = h / a.hpg;
-  const int t_begin = a.t_base + seg * a.seg_len;
+  const int t_begin = seg * a.seg_len;
   const int t_end = min(a.L, t_begin + a.seg_len);
   const int nck = t_end > t_begin ? (t_end - t_begin + QC - 1) / QC : 0;
   const int last = nck - 1;
@@ -279,20 +277,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   if (tid == 0) {
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t cnt = 1;
-      if (i == BAR_EMPTY0 || i == BAR_EMPTY1) cnt = kStateOnly ? 3 : 5;
-      if (i == BAR_YREADY0 || i == BAR_YREADY1) cnt = 2;
+      if (i == BAR_EMPTY0 || i == BAR_EMPTY1) cnt = kStateOnly ? 3 : 4;  // + mask warps
       mbar_init(BAR(i), cnt);
     }
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async();
   }
-  if (warp == kWarpTma && lane == 0) {
+  if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_bc);
     prefetch_tmap(&tm_x);
-    if (kPrecise) prefetch_tmap(&tm_blo);
   }
-  if (warp == kWarpIssueA) {
+  if (warp == 1) {
     tmem_alloc(sb + OFF_MISC, TM_COLS);
     tmem_relinquish();
   }
@@ -301,17 +297,16 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   tc_fence_after();
   const uint32_t tmem = misc[0];
 
-  if (warp == kWarpTma) {
+  if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     // Raw x rows of chunk k go to w o X[k % 2] once MMA4 of chunk k-2 has released it; the
-    // B/C tiles, dt and prefix sums go to stage k % 2 once chunk k-2's readers released it.
+    // B/C tiles, dt and prefix sums go to stage k % 2 once chunk k-2's consumers released it.
     if (lane == 0) {
-      int nx = 0, nbc = 0;
-      for (int k = 0; k < nck; ++k) {
+      int k = 0, nx = 0, nbc = 0;
+      for (; k < nck; ++k) {
         const int xb = k & 1, st = k & 1;
         const int t0 = t_begin + k * QC;
         if (k >= 2 && !mbar_wait(BAR(BAR_XWFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err, lim)) break;
-        TC_MARK(k, 13);
         mbar_arrive_expect_tx(BAR(BAR_FULLX0 + xb), kRawRows * 128);
         tma_load_3d(sb + OFF_XW + xb * kXBuf, &tm_x, h * 64, t0 - 3, b, BAR(BAR_FULLX0 + xb));
         ++nx;
@@ -319,16 +314,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (k >= 2 && !mbar_wait(BAR(BAR_EMPTY0 + st), ((k >> 1) - 1) & 1, abort_flag, a.err, lim)) break;
         const uint32_t sst = sb + st * kStage;
         const uint32_t full = BAR(BAR_FULL0 + st);
-        TC_MARK(k, 14);
-        mbar_arrive_expect_tx(full, (kStateOnly && !kPrecise ? 2 * kTile : 4 * kTile) + 1024);
+        TC_MARK(k, 12);
+        mbar_arrive_expect_tx(full, (kStateOnly ? 2 * kTile : 4 * kTile) + 1024);
         const int cB = g * 128, cC = a.G * 128 + g * 128;
         if (!kStateOnly) {
           tma_load_3d(sst + OFF_C, &tm_bc, cC, t0, b, full);
           tma_load_3d(sst + OFF_C + kTile, &tm_bc, cC + 64, t0, b, full);
-        }
-        if (kPrecise) {  // the low fp16 parts of B go where C would be
-          tma_load_3d(sst + OFF_C, &tm_blo, cB, t0 - a.t_base, b, full);
-          tma_load_3d(sst + OFF_C + kTile, &tm_blo, cB + 64, t0 - a.t_base, b, full);
         }
         tma_load_3d(sst + OFF_B, &tm_bc, cB, t0, b, full);
         tma_load_3d(sst + OFF_B + kTile, &tm_bc, cB + 64, t0, b, full);
@@ -344,296 +335,299 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       for (int j = (nbc >= 2 ? nbc - 2 : 0); j < nbc; ++j)
         mbar_wait(BAR(BAR_FULL0 + (j & 1)), (j >> 1) & 1, &never_abort, a.err);
     }
-  } else if (warp == kWarpIssueA) {
-    // ---------------------------------------------------------------- MMA issuer A: the state
-    // chain.  Per chunk k: MMA4 dH(k) (once w o X(k) is written and the state warps have read
-    // dH(k-1)), then MMA3 Ys(k) = C h_{k-1}^T (once the h tile holds h_{k-1} and the output
-    // warps have read Ys(k-2)).  Every wait blocks in hardware, so the thread issues nothing
-    // while it waits.
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    // Issues each chunk's four MMA groups as soon as their inputs are ready, whatever the
+    // order, so that no group waits behind another one that is still blocked:
+    //   MMA1 S(j)   stage j loaded; S[j % 2] free (MMA2 of chunk j-2 issued, its output read)
+    //   MMA4 dH(j)  X(j) and w o X(j) written; dH of chunk j-1 read by the state warps
+    //   MMA3 Ys(j)  after MMA1(j); h_{j-1} in the h tile
+    //   MMA2 Yi(j)  after MMA3(j) and MMA4(j); S~(j) written by the mask warps
+    // A commit after each group signals its consumers; stage j is released by a commit after
+    // the last of MMA1/MMA3/MMA4 of chunk j.  Polling sleeps briefly when nothing is ready and
+    // gives up (abort + SSD_ERR_TIMEOUT) after ~2 s without progress.
     if (lane == 0) {
-      for (int k = 0; k < nck; ++k) {
-        const int st = k & 1;
-        const uint32_t sst = sb + st * kStage;
-        if (!mbar_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, abort_flag, a.err, lim)) break;
-        if (!mbar_wait(BAR(BAR_XREADY0 + st), (k >> 1) & 1, abort_flag, a.err, lim)) break;
-        if (!kPrecise && k == last && !mbar_wait(BAR(BAR_XLOREADY), 0, abort_flag, a.err, lim)) break;
-        if (k >= 1 && !mbar_wait(BAR(BAR_DHFREE), (k - 1) & 1, abort_flag, a.err, lim)) break;
-        tc_fence_after();
-        TC_MARK(k, 9);
-        issue_dH(sst + OFF_B, sb + OFF_XW + st * kXBuf, tmem + TM_DH, false);
-        if (kPrecise) {
-          // B w o X = (B_hi + B_lo)(wX_hi + wX_lo) without the lo * lo term: fp32 accuracy
-          issue_dH(sst + OFF_B, sb + OFF_X + st * kTile, tmem + TM_DH, true);
-          issue_dH(sst + OFF_C, sb + OFF_XW + st * kXBuf, tmem + TM_DH, true);
-        } else if (k == last) {
+      int nS = kStateOnly ? nck : 0, nD = 0, nYs = kStateOnly ? nck : 0, nYi = kStateOnly ? nck : 0;
+      auto stage_done = [&](int j) {  // all readers of stage j issued?
+        return nD > j && (kStateOnly || (nS > j && nYs > j));
+      };
+      uint64_t t_prog = globaltimer();
+      uint32_t nap = 32;  // sleep between polls: doubles up to 256 ns while nothing is ready
+      bool ok = true;
+      while (ok && (nD < nck || nYi < nck)) {
+        bool prog = false;
+        if (nYi < nck && nYi < nYs && nYi < nD && mbar_test(BAR(BAR_STREADY0 + (nYi & 1)), (nYi >> 1) & 1)) {
+          const int j = nYi;
+          tc_fence_after();
+          TC_MARK(j, 11);
+          const uint32_t tS = tmem + ((j & 1) ? TM_S1 : TM_S0);
+          issue_Yi(tS, sb + OFF_X + (j & 1) * kTile, tS + TM_YI_OFF);
+          mma_commit(BAR(BAR_YREADY0 + (j & 1)));
+          mma_commit(BAR(BAR_XFREE0 + (j & 1)));
+          ++nYi;
+          prog = true;
+        }
+        if (nYs < nck && nYs < nS && mbar_test(BAR(BAR_HREADY), nYs & 1)) {
+          const int j = nYs;
+          tc_fence_after();
+          TC_MARK(j, 9);
+          issue_Ys(sb + (j & 1) * kStage, sb + OFF_H, tmem + ((j & 1) ? TM_YS1 : TM_YS0));
+          mma_commit(BAR(BAR_HTFREE));
+          ++nYs;
+          if (stage_done(j)) mma_commit(BAR(BAR_EMPTY0 + (j & 1)));
+          prog = true;
+        }
+        if (nD < nck && (kStateOnly || nD < nS) &&
+            mbar_test(BAR(BAR_XREADY0 + (nD & 1)), (nD >> 1) & 1) &&
+            (nD == 0 || mbar_test(BAR(BAR_DHFREE), (nD - 1) & 1)) &&
+            (nD != last || mbar_test(BAR(BAR_XLOREADY), 0)) &&
+            (!kStateOnly || mbar_test(BAR(BAR_FULL0 + (nD & 1)), (nD >> 1) & 1))) {
+          const int j = nD;
+          tc_fence_after();
+          TC_MARK(j, 8);
+          const uint32_t sst = sb + (j & 1) * kStage;
+          issue_dH(sst, sb + OFF_XW + (j & 1) * kXBuf, tmem + TM_DH, false);
           // last chunk: the low part of w o X (in the other w o X buffer) for the final state
-          issue_dH(sst + OFF_B, sb + OFF_XW + ((k + 1) & 1) * kXBuf, tmem + TM_DH, true);
+          if (j == last) issue_dH(sst, sb + OFF_XW + ((j + 1) & 1) * kXBuf, tmem + TM_DH, true);
+          mma_commit(BAR(BAR_XWFREE0 + (j & 1)));
+          mma_commit(BAR(BAR_DHREADY));
+          if (kStateOnly) mma_commit(BAR(BAR_XFREE0 + (j & 1)));
+          ++nD;
+          if (stage_done(j)) mma_commit(BAR(BAR_EMPTY0 + (j & 1)));
+          prog = true;
         }
-        mma_commit(BAR(BAR_XWFREE0 + st));
-        mma_commit(BAR(BAR_DHREADY));
-        if (kStateOnly) {
-          mma_commit(BAR(BAR_EMPTY0 + st));
-          continue;
+        if (nS < nck && nS <= nYi + 1 && mbar_test(BAR(BAR_FULL0 + (nS & 1)), (nS >> 1) & 1) &&
+            (nS < 2 || mbar_test(BAR(BAR_YFREE0 + (nS & 1)), ((nS >> 1) - 1) & 1))) {
+          const int j = nS;
+          tc_fence_after();
+          TC_MARK(j, 10);
+          issue_S(sb + (j & 1) * kStage, tmem + ((j & 1) ? TM_S1 : TM_S0));
+          mma_commit(BAR(BAR_SREADY0 + (j & 1)));
+          ++nS;
+          if (stage_done(j)) mma_commit(BAR(BAR_EMPTY0 + (j & 1)));
+          prog = true;
         }
-        if (!mbar_wait(BAR(BAR_HREADY), k & 1, abort_flag, a.err, lim)) break;
-        if (k >= 2 && !mbar_wait(BAR(BAR_YFREE0 + st), ((k >> 1) - 1) & 1, abort_flag, a.err, lim)) break;
-        tc_fence_after();
-        TC_MARK(k, 10);
-        issue_Ys(sst, sb + OFF_H, tmem + (st ? TM_YS1 : TM_YS0));
-        mma_commit(BAR(BAR_HTFREE));
-        mma_commit(BAR(BAR_YREADY0 + st));
-        mma_commit(BAR(BAR_EMPTY0 + st));
+        if (prog) {
+          t_prog = globaltimer();
+          nap = 32;
+        } else {
+          if (*abort_flag) {
+            ok = false;
+          } else if (globaltimer() - t_prog > lim) {
+            *abort_flag = 1;
+            if (a.err) atomicCAS(a.err, 0, (int)SSD_ERR_TIMEOUT);
+            ok = false;
+          } else {
+            __nanosleep(nap);
+            nap = nap < 256 ? 2 * nap : 256;
+          }
+        }
       }
       // no MMA may still be running when TMEM is released
-      mma_commit(BAR(BAR_DONE_A));
+      mma_commit(BAR(BAR_DONE));
       int never_abort = 0;
-      mbar_wait(BAR(BAR_DONE_A), 0, &never_abort, a.err);
+      mbar_wait(BAR(BAR_DONE), 0, &never_abort, a.err);
     }
-  } else if (warp == kWarpIssueB) {
-    // ---------------------------------------------------------------- MMA issuer B: the S
-    // chain.  MMA1 S(j) = C B^T once stage j is loaded and S[j % 2] is free (the output warps
-    // have read Yi(j-2) from it); MMA2 Yi(k) = S~ X once the mask warps have written S~(k).
-    // MMA1 of chunk k+1 is issued before MMA2 of chunk k, so that the mask of chunk k+1 can
-    // run while MMA2 and the output of chunk k do.
-    if (!kStateOnly && lane == 0) {
-      auto mma1 = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(BAR(BAR_FULL0 + st), (j >> 1) & 1, abort_flag, a.err, lim)) return false;
-        if (j >= 2 && !mbar_wait(BAR(BAR_YFREE0 + st), ((j >> 1) - 1) & 1, abort_flag, a.err, lim)) return false;
-        tc_fence_after();
-        TC_MARK(j, 11);
-        issue_S(sb + st * kStage, tmem + (st ? TM_S1 : TM_S0));
-        mma_commit(BAR(BAR_SREADY0 + st));
-        mma_commit(BAR(BAR_EMPTY0 + st));
-        return true;
-      };
-      bool ok = nck > 0 ? mma1(0) : true;
-      for (int k = 0; ok && k < nck; ++k) {
-        const int st = k & 1;
-        if (k + 1 < nck && !(ok = mma1(k + 1))) break;
-        if (!(ok = mbar_wait(BAR(BAR_STREADY0 + st), (k >> 1) & 1, abort_flag, a.err, lim))) break;
-        if (!(ok = mbar_wait(BAR(BAR_XREADY0 + st), (k >> 1) & 1, abort_flag, a.err, lim))) break;
-        tc_fence_after();
-        TC_MARK(k, 12);
-        const uint32_t tS = tmem + (st ? TM_S1 : TM_S0);
-        issue_Yi(tS, sb + OFF_X + st * kTile, tS + TM_YI_OFF);
-        mma_commit(BAR(BAR_XFREE0 + st));
-        mma_commit(BAR(BAR_YREADY0 + st));
-      }
-      mma_commit(BAR(BAR_DONE_B));
-      int never_abort = 0;
-      mbar_wait(BAR(BAR_DONE_B), 0, &never_abort, a.err);
-    }
-  } else if (warp >= kWarpConv0 && warp < kWarpConv0 + kConvWarps) {
+  } else if (conv_index(warp) >= 0) {
     // ---------------------------------------------------------------- conv + SiLU -> X, w o X
-    // Lane layout: channel group cg = lane % 8 (the head's channels 8cg .. 8cg+7, one 16-byte
-    // piece of a 128-byte row) and token group tg = lane / 8; warp cw covers tokens
-    // 32cw .. 32cw+31, so a lane makes tokens s0 .. s0+7 with s0 = 32cw + 8tg.  Raw row r of
-    // the w o X buffer holds time t0-3+r, and token s reads rows s .. s+3: its own rows s0 ..
-    // s0+7 (which it overwrites with w o X in order, after reading them) and the 3 rows after
-    // them (the next token group's own rows, read before the group barrier that precedes all
-    // writes).  Every access moves 16 bytes; a warp's 4 token groups touch 4 whole rows, so the
-    // 128-byte swizzle keeps each access conflict-free.
-    // SiLU(u) = u * sigmoid(u) = h + h * tanh(h) with h = u / 2: the conv accumulates h
-    // directly (halved weights) in fp16 pairs -- the precision of the MMA operand it feeds --
-    // and one half2 tanh serves two channels.  The last chunk of a segment (and every chunk of
-    // the tail pass) runs in fp32 with the exact SiLU and stores w o X as fp16 hi + lo parts.
-    const int cw = warp - kWarpConv0, cg = lane & 7, tg = lane >> 3;
-    const int ctid = 32 * cw + lane;
-    const int s0 = 32 * cw + 8 * tg;
-    const bool leader = ctid == 0;
-    const int ch0 = h * 64 + 8 * cg;
+    // Warp cw makes tokens 16cw..16cw+15; lane l channels 2l, 2l+1.  Raw row r of the w o X
+    // buffer holds time t0-3+r; token s reads rows s..s+3 (a register window), then
+    // overwrites row s with its w o X row and writes its X row to row s of X.  Rows
+    // 16cw+16..+18 belong to the next warp's tokens, so every warp reads them before the
+    // group barrier that precedes all writes.
+    // SiLU(u) = u * sigmoid(u) = h + h * tanh(h) with h = u / 2.  The conv accumulates h
+    // directly (halved weights) in fp16 pairs -- the precision of the MMA operand it feeds,
+    // 11 significant bits -- and one half2 tanh serves both channels.  The last chunk of a
+    // segment, whose newest tokens dominate the final state, uses fp32 and the exact SiLU.
+    const int cw = conv_index(warp);
+    const bool leader = (tid == 2 * 32);  // leaders sit on different SM sub-partitions
+    const int ch = h * 64 + 2 * lane;
     const int W = a.W;
-    float *wtok = reinterpret_cast<float *>(smem + OFF_WTOK);
-    __half2 hw[4][4], hb[4];  // [tap j: input at time t-3+j][channel pair], halved
+    float2 ew[4], bias2 = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float2 bb = make_float2(0.f, 0.f);
-      if (W > 0 && a.conv_b) bb = make_float2(__bfloat162float(a.conv_b[ch0 + 2 * i]), __bfloat162float(a.conv_b[ch0 + 2 * i + 1]));
-      hb[i] = __float22half2_rn(make_float2(0.5f * bb.x, 0.5f * bb.y));
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int kk = j - (4 - W);
-        float2 ww = make_float2(0.f, 0.f);
-        if (W > 0 && kk >= 0)
-          ww = make_float2(__bfloat162float(a.conv_w[(long long)(ch0 + 2 * i) * W + kk]),
-                           __bfloat162float(a.conv_w[(long long)(ch0 + 2 * i + 1) * W + kk]));
-        hw[j][i] = __float22half2_rn(make_float2(0.5f * ww.x, 0.5f * ww.y));
-      }
+    for (int j = 0; j < 4; ++j) {  // half the weight for the input at time t-3+j
+      const int k = j - (4 - W);
+      ew[j].x = (W > 0 && k >= 0) ? 0.5f * __bfloat162float(a.conv_w[(long long)ch * W + k]) : 0.f;
+      ew[j].y = (W > 0 && k >= 0) ? 0.5f * __bfloat162float(a.conv_w[(long long)(ch + 1) * W + k]) : 0.f;
     }
+    if (W > 0 && a.conv_b) {
+      bias2.x = 0.5f * __bfloat162float(a.conv_b[ch]);
+      bias2.y = 0.5f * __bfloat162float(a.conv_b[ch + 1]);
+    }
+    __half2 hw[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) hw[j] = __float22half2_rn(ew[j]);
+    const __half2 hbias = __float22half2_rn(bias2);
+    // byte offset of this lane's 4 bytes within a swizzled row r, by r mod 8
+    uint32_t loff[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) loff[u] = ((uint32_t)((lane >> 2) ^ u) << 4) + ((uint32_t)(lane & 3) << 2);
+    const int tok0 = kTokPerConvWarp * cw;  // multiple of 8
     for (int k = 0; k < nck; ++k) {
       const int st = k & 1, xb = k & 1, lb = (k + 1) & 1;
       const bool is_last = (k == last);
-      const bool exact = kPrecise || is_last;  // fp32 conv, exact SiLU, w o X as hi + lo
       // the leader waits for every input of the chunk, then one group barrier releases all
       if (leader) {
         bool ok = mbar_wait(BAR(BAR_FULLX0 + xb), (k >> 1) & 1, abort_flag, a.err, lim);
         if (ok) ok = mbar_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, abort_flag, a.err, lim);
-        if (ok && !kStateOnly && k >= 2)
-          ok = mbar_wait(BAR(BAR_XFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err, lim);
-        if (ok && !kPrecise && is_last && k >= 1)
-          mbar_wait(BAR(BAR_XWFREE0 + lb), ((k - 1) >> 1) & 1, abort_flag, a.err, lim);
-        TC_MARK(k, 0);
+        if (ok && k >= 2) ok = mbar_wait(BAR(BAR_XFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err, lim);
+        if (ok && is_last && k >= 1) mbar_wait(BAR(BAR_XWFREE0 + lb), ((k - 1) >> 1) & 1, abort_flag, a.err, lim);
+        TC_MARK(k, 14);
       }
-      if (named_bar_or(kNbConv, 32 * kConvWarps, *abort_flag != 0)) break;
-      {  // this thread's token weight w = e^{cs_Q - cs_s} dt_s, for the whole group
-        const float *cs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
-        const float *dtv = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
-        wtok[ctid] = __expf(cs[QC - 1] - cs[ctid]) * dtv[ctid];
-      }
-      unsigned char *xt = smem + OFF_X + xb * kTile;   // X rows
-      unsigned char *xwt = smem + OFF_XW + xb * kXBuf;  // raw rows in, w o X rows out
-      // low parts: the other w o X buffer, or X (unused) in the tail pass
-      unsigned char *xlt = kPrecise ? xt : smem + OFF_XW + lb * kXBuf;
-#define ROW16(buf, r) (*reinterpret_cast<uint4 *>((buf) + (uint32_t)(r) * 128u + ((uint32_t)(cg ^ ((r) & 7)) << 4)))
-      const uint4 halo0 = ROW16(xwt, s0 + 8), halo1 = ROW16(xwt, s0 + 9), halo2 = ROW16(xwt, s0 + 10);
-      uint4 rw0 = ROW16(xwt, s0), rw1 = ROW16(xwt, s0 + 1), rw2 = ROW16(xwt, s0 + 2);
+      if (named_bar_or(1, 256, *abort_flag != 0)) break;
+      const float *cs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
+      const float *dtv = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
+      const float cs_end = cs[QC - 1];
+      const float wl = lane < kTokPerConvWarp ? __expf(cs_end - cs[tok0 + lane]) * dtv[tok0 + lane] : 0.f;
+      const uint32_t wl2 = pack_f16(wl, wl);
+      unsigned char *xt = smem + OFF_X + xb * kTile + tok0 * 128;   // row tok0
+      unsigned char *xwt = smem + OFF_XW + xb * kXBuf + tok0 * 128;
+      unsigned char *xlt = smem + OFF_XW + lb * kXBuf + tok0 * 128;
+      // raw rows tok0 + r for r = 0..18 (tok0 is a multiple of 8, so row mod 8 = r mod 8)
+#define RAW(r) (*reinterpret_cast<const uint32_t *>(xwt + (r) * 128 + loff[(r) & 7]))
+      uint32_t r0 = RAW(0), r1 = RAW(1), r2 = RAW(2);
       const int t0 = t_begin + k * QC;
-      if (s0 == 0 && t0 == 0) {  // history before the first token comes from the conv cache
-        uint4 hist[3];
+      if (cw == 0 && t0 == 0) {  // history before the first token comes from the conv cache
+        uint32_t hist[3] = {0u, 0u, 0u};
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
           const int tau = j - 3;
-          hist[j] = (a.csi && W + tau >= 0)
-                        ? *reinterpret_cast<const uint4 *>(a.csi + ((long long)b * W + (W + tau)) * a.conv_dim + ch0)
-                        : make_uint4(0u, 0u, 0u, 0u);
+          if (a.csi && W + tau >= 0)
+            hist[j] = *reinterpret_cast<const uint32_t *>(a.csi + ((long long)b * W + (W + tau)) * a.conv_dim + ch);
         }
-        rw0 = hist[0];
-        rw1 = hist[1];
-        rw2 = hist[2];
+        r0 = hist[0];
+        r1 = hist[1];
+        r2 = hist[2];
       }
-      named_bar(kNbConv, 32 * kConvWarps);  // halo rows read and token weights written
-      if (leader) mbar_arrive(BAR(BAR_EMPTY0 + st));
-      if (!exact) {
-        // 8 bf16 -> 4 fp16 pairs
-        auto cvt = [](const uint4 &r, __half2 (&o)[4]) {
-          const uint32_t u[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) o[i] = __float22half2_rn(unpack_bf16(u[i]));
-        };
-        __half2 xm3[4], xm2[4], xm1[4];
-        cvt(rw0, xm3);
-        cvt(rw1, xm2);
-        cvt(rw2, xm1);
-#pragma unroll 4
-        for (int j = 0; j < 8; ++j) {
-          const int s = s0 + j;
-          const uint4 rn = j + 3 < 8 ? ROW16(xwt, s + 3) : (j == 5 ? halo0 : (j == 6 ? halo1 : halo2));
-          __half2 x0[4], xo[4], xw[4];
-          cvt(rn, x0);
-          const __half2 w2 = __float2half2_rn(wtok[s]);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            __half2 acc = __hfma2(hw[0][i], xm3[i], hb[i]);
-            acc = __hfma2(hw[1][i], xm2[i], acc);
-            acc = __hfma2(hw[2][i], xm1[i], acc);
-            acc = __hfma2(hw[3][i], x0[i], acc);
-            xo[i] = W != 0 ? __hfma2(acc, h2tanh_approx(acc), acc) : x0[i];
-            xw[i] = __hmul2(xo[i], w2);
-            xm3[i] = xm2[i];
-            xm2[i] = xm1[i];
-            xm1[i] = x0[i];
-          }
-          if (!kStateOnly)
-            ROW16(xt, s) = make_uint4(*reinterpret_cast<uint32_t *>(&xo[0]), *reinterpret_cast<uint32_t *>(&xo[1]),
-                                      *reinterpret_cast<uint32_t *>(&xo[2]), *reinterpret_cast<uint32_t *>(&xo[3]));
-          ROW16(xwt, s) = make_uint4(*reinterpret_cast<uint32_t *>(&xw[0]), *reinterpret_cast<uint32_t *>(&xw[1]),
-                                     *reinterpret_cast<uint32_t *>(&xw[2]), *reinterpret_cast<uint32_t *>(&xw[3]));
-        }
-      } else {
-        // The final state's chunks: their newest tokens dominate the final state, so X comes
-        // from the fp32 conv and SiLU and w o X is stored as the fp16 hi + lo parts of the fp32
-        // product.  The halved bf16 weights are exact in fp16, so the fp16 copies serve here.
-        // One channel pair at a time (4-byte accesses) keeps this path's registers few.
-        auto word = [](const uint4 &r, int i) { return i == 0 ? r.x : (i == 1 ? r.y : (i == 2 ? r.z : r.w)); };
+      const uint32_t nb0 = RAW(16), nb1 = RAW(17), nb2 = RAW(18);
+      named_bar(1, 256);  // all boundary rows read before any row is overwritten
+      if (leader) {
+        TC_MARK(k, 0);
+        mbar_arrive(BAR(BAR_EMPTY0 + st));  // dt and prefix sums already read
+      }
+      // The token loop is compiled twice: the common chunks, and the last chunk of a segment.
+      auto tokens = [&](auto last_tag) {
+        constexpr bool kLast = decltype(last_tag)::value;
+        if constexpr (!kLast) {
+          __half2 xm3 = __float22half2_rn(unpack_bf16(r0)), xm2 = __float22half2_rn(unpack_bf16(r1)),
+                  xm1 = __float22half2_rn(unpack_bf16(r2));
 #pragma unroll 1
-        for (int i = 0; i < 4; ++i) {
-          // this pair's fp32 weights (tap j multiplies the input at time t-3+j) and bias
-          float2 wj[4];
+          for (int g = 0; g < 2; ++g) {
+            __half2 xn[8];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int kk = j - (4 - W);
-            wj[j] = (W > 0 && kk >= 0)
-                        ? make_float2(__bfloat162float(a.conv_w[(long long)(ch0 + 2 * i) * W + kk]),
-                                      __bfloat162float(a.conv_w[(long long)(ch0 + 2 * i + 1) * W + kk]))
-                        : make_float2(0.f, 0.f);
-          }
-          const float2 hb2 = (W > 0 && a.conv_b)
-                                 ? make_float2(__bfloat162float(a.conv_b[ch0 + 2 * i]), __bfloat162float(a.conv_b[ch0 + 2 * i + 1]))
-                                 : make_float2(0.f, 0.f);
-          const float2 w0 = wj[0], w1 = wj[1], w2 = wj[2], w3 = wj[3];
-          float2 xm3 = unpack_bf16(word(rw0, i)), xm2 = unpack_bf16(word(rw1, i)), xm1 = unpack_bf16(word(rw2, i));
-          const uint32_t hw0 = word(halo0, i), hw1 = word(halo1, i), hw2 = word(halo2, i);
-          const uint32_t cofs = ((uint32_t)cg << 4) + 4u * (uint32_t)i;  // before the swizzle
-#pragma unroll 1
-          for (int j = 0; j < 8; ++j) {
-            const int s = s0 + j;
-            const int rr = s + 3;
-            const uint32_t un = j + 3 < 8
-                                    ? *reinterpret_cast<const uint32_t *>(xwt + (uint32_t)rr * 128u + (cofs ^ ((uint32_t)(rr & 7) << 4)))
-                                    : (j == 5 ? hw0 : (j == 6 ? hw1 : hw2));
-            const float2 x0 = unpack_bf16(un);
-            float2 v = x0;
-            if (W != 0) {
-              float2 acc = __ffma2_rn(w0, xm3, hb2);
-              acc = __ffma2_rn(w1, xm2, acc);
-              acc = __ffma2_rn(w2, xm1, acc);
-              acc = __ffma2_rn(w3, x0, acc);
-              v = make_float2(silu(acc.x), silu(acc.y));
+            for (int u = 0; u < 8; ++u) {
+              const int nxt = 8 * g + u + 3;  // row of time t for token 8g+u
+              uint32_t w3;
+              if (nxt < 16) w3 = RAW(nxt);
+              else w3 = nxt == 16 ? nb0 : (nxt == 17 ? nb1 : nb2);
+              xn[u] = __float22half2_rn(unpack_bf16(w3));
             }
-            const float ws = wtok[s];
-            const float2 p = make_float2(v.x * ws, v.y * ws);
-            const __half2 hi = __float22half2_rn(p);
-            const float2 hf = __half22float2(hi);
-            const uint32_t off = (uint32_t)s * 128u + (cofs ^ ((uint32_t)(s & 7) << 4));
-            if (!kStateOnly) *reinterpret_cast<uint32_t *>(xt + off) = pack_f16(v.x, v.y);
-            *reinterpret_cast<uint32_t *>(xwt + off) = *reinterpret_cast<const uint32_t *>(&hi);
-            *reinterpret_cast<uint32_t *>(xlt + off) = pack_f16(p.x - hf.x, p.y - hf.y);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int i = 8 * g + u;
+              const __half2 x0 = xn[u];
+              __half2 xo = x0;
+              if (W != 0) {
+                __half2 acc = __hfma2(hw[0], xm3, hbias);
+                acc = __hfma2(hw[1], xm2, acc);
+                acc = __hfma2(hw[2], xm1, acc);
+                acc = __hfma2(hw[3], x0, acc);
+                xo = __hfma2(acc, h2tanh_approx(acc), acc);
+              }
+              const uint32_t off = i * 128 + loff[u];
+              *reinterpret_cast<__half2 *>(xt + off) = xo;
+              const uint32_t w2 = __shfl_sync(0xffffffffu, wl2, i);
+              *reinterpret_cast<__half2 *>(xwt + off) = __hmul2(xo, *reinterpret_cast<const __half2 *>(&w2));
+              xm3 = xm2;
+              xm2 = xm1;
+              xm1 = x0;
+            }
+          }
+          return;
+        }
+        float2 xm3 = unpack_bf16(r0), xm2 = unpack_bf16(r1), xm1 = unpack_bf16(r2);
+#pragma unroll 1
+        for (int g = 0; g < 2; ++g) {
+          float2 xn[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int nxt = 8 * g + u + 3;  // row of time t for token 8g+u
+            uint32_t w3;
+            if (nxt < 16) w3 = RAW(nxt);
+            else w3 = nxt == 16 ? nb0 : (nxt == 17 ? nb1 : nb2);
+            xn[u] = unpack_bf16(w3);
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int i = 8 * g + u;
+            const float2 x0 = xn[u];
+            float2 acc = x0;
+            if (W != 0) {
+              acc = __ffma2_rn(ew[0], xm3, bias2);
+              acc = __ffma2_rn(ew[1], xm2, acc);
+              acc = __ffma2_rn(ew[2], xm1, acc);
+              acc = __ffma2_rn(ew[3], x0, acc);
+            }
+            const uint32_t off = i * 128 + loff[u];
+            {
+              // The final state's chunk: its newest tokens dominate the final state, so X
+              // comes from the fp32 SiLU and w o X is stored as the fp16 hi + lo parts of the
+              // fp32 product.
+              const float u0 = W != 0 ? silu(2.f * acc.x) : acc.x;
+              const float u1 = W != 0 ? silu(2.f * acc.y) : acc.y;
+              const float ws = __shfl_sync(0xffffffffu, wl, i);
+              const float2 v = make_float2(u0 * ws, u1 * ws);
+              const __half2 hi = __float22half2_rn(v);
+              const float2 hf = __half22float2(hi);
+              *reinterpret_cast<uint32_t *>(xt + off) = pack_f16(u0, u1);
+              *reinterpret_cast<__half2 *>(xwt + off) = hi;
+              *reinterpret_cast<uint32_t *>(xlt + off) = pack_f16(v.x - hf.x, v.y - hf.y);
+            }
             xm3 = xm2;
             xm2 = xm1;
             xm1 = x0;
           }
         }
-      }
-#undef ROW16
+      };
+      if (is_last) tokens(std::true_type{});
+      else tokens(std::false_type{});
+      if (leader) TC_MARK(k, 13);
+#undef RAW
       fence_proxy_async();
-      named_bar(kNbConv, 32 * kConvWarps);
+      named_bar(1, 256);
       if (leader) {
         TC_MARK(k, 1);
         mbar_arrive(BAR(BAR_XREADY0 + xb));
-        if (!kPrecise && is_last) mbar_arrive(BAR(BAR_XLOREADY));
+        if (is_last) mbar_arrive(BAR(BAR_XLOREADY));
       }
     }
-  } else if (warp >= kWarpMask0 && warp < kWarpMask0 + 4) {
+  } else if (warp >= 12 && warp < 16) {
     // ---------------------------------------------------------------- S -> S~ (decay mask)
     if (!kStateOnly) {
-      const int mw = warp - kWarpMask0;  // == warp % 4: TMEM lanes 32 mw .. 32 mw + 31
+      const int mw = warp - 12;
       const int t = 32 * mw + lane;
-      const bool leader = (warp == kWarpMask0 + 2 && lane == 0);
+      const bool leader = (tid == 14 * 32);
       float *cf = reinterpret_cast<float *>(smem + OFF_CF);
       const float Dh = a.D[h];
       for (int k = 0; k < nck; ++k) {
         const int st = k & 1;
-        if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, kNbMask, abort_flag, a.err, lim)) break;
-        if (!wg_wait(BAR(BAR_SREADY0 + st), (k >> 1) & 1, leader, kNbMask, abort_flag, a.err, lim)) break;
+        if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, 2, abort_flag, a.err, lim)) break;
+        if (!wg_wait(BAR(BAR_SREADY0 + st), (k >> 1) & 1, leader, 2, abort_flag, a.err, lim)) break;
         tc_fence_after();
-        if (leader) TC_MARK(k, 2);
         float *cs = reinterpret_cast<float *>(smem + OFF_CSM);
         float *dtv = reinterpret_cast<float *>(smem + OFF_DTM);
-        float *et = reinterpret_cast<float *>(smem + OFF_ET + st * 512);
         {  // private copies (the stage is released at once); column factor of column t:
-           // e^{r_J - cs_t} dt_t with r_J = cs at the end of t's block; and the output row
-           // factor e^{cs_t} of this chunk for the output warps
+           // e^{r_J - cs_t} dt_t with r_J = cs at the end of t's block
           const float *scs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
           const float *sdt = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
           const float rJ = scs[32 * (t >> 5) + 31];
           cs[t] = scs[t];
           dtv[t] = sdt[t];
           cf[t] = __expf(rJ - scs[t]) * sdt[t];
-          et[t] = __expf(scs[t]);
         }
-        named_bar(kNbMask, 128);
+        named_bar(2, 128);
         if (leader) mbar_arrive(BAR(BAR_EMPTY0 + st));
+        if (leader) TC_MARK(k, 2);
         const float cst = cs[t];
         const uint32_t trow = tmem + (st ? TM_S1 : TM_S0) + ((uint32_t)(32 * mw) << 16);
         // Blocks of 32 columns in increasing J: S~ columns 32J..32J+31 go to the packed TMEM
@@ -714,18 +708,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        named_bar(kNbMask, 128);
+        named_bar(2, 128);
         if (leader) {
           TC_MARK(k, 3);
           mbar_arrive(BAR(BAR_STREADY0 + st));
         }
       }
     }
-  } else if (warp >= kWarpState0 && warp < kWarpState0 + 4) {
-    // ---------------------------------------------------------------- state update
-    const int ew = warp - kWarpState0;
-    const int n = 32 * ew + lane;  // TMEM lane: state row n
-    const bool leader = (warp == kWarpState0 + 3 && lane == 0);
+  } else if (warp >= 16) {
+    // ---------------------------------------------------------------- state update + output
+    const int ew = warp - 16;
+    const int n = 32 * ew + lane;  // TMEM lane: state row n, output row t = n
+    const bool leader = (tid == 19 * 32);
     const uint32_t lane_off = (uint32_t)(32 * ew) << 16;
     const long long bh = (long long)b * a.H + h;
     float *hout = a.h_out ? a.h_out + seg * a.h_out_seg + bh * 8192 : nullptr;
@@ -744,7 +738,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           hu[i] = __float_as_uint(hr[i]);
         }
         tmem_st32(tmem + TM_H + 32 * half + lane_off, hu);
-        if (!kStateOnly) write_h_tile(smem, hr, n, half);
+        write_h_tile(smem, hr, n, half);
         if (tail && tail_k < 0) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) hout[(32 * half + i) * 128 + n] = hr[i];
@@ -754,18 +748,20 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
     fence_proxy_async();
     tc_fence_before();
-    named_bar(kNbState, 128);
+    named_bar(3, 128);
     if (leader) mbar_arrive(BAR(BAR_HREADY));
     float decay_sum = 0.f;
     for (int k = 0; k < nck; ++k) {
       const int st = k & 1;
-      if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, kNbState, abort_flag, a.err, lim)) break;
-      const float cs_end = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS)[QC - 1];
+      if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, 3, abort_flag, a.err, lim)) break;
+      const float *cs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
+      const float cs_end = cs[QC - 1];
+      const float et = __expf(cs[n]);
       decay_sum += cs_end;
       const float ak = __expf(cs_end);
-      named_bar(kNbState, 128);  // every thread has read the prefix sums
+      named_bar(3, 128);  // every thread has read the prefix sums
       if (leader) mbar_arrive(BAR(BAR_EMPTY0 + st));
-      if (!wg_wait(BAR(BAR_DHREADY), k & 1, leader, kNbState, abort_flag, a.err, lim)) break;
+      if (!wg_wait(BAR(BAR_DHREADY), k & 1, leader, 3, abort_flag, a.err, lim)) break;
       tc_fence_after();
       if (leader) TC_MARK(k, 4);
 #pragma unroll 1
@@ -779,6 +775,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         for (int i = 0; i < 32; i += 2) {
           const float2 r = __ffma2_rn(make_float2(ak, ak), make_float2(hr[i], hr[i + 1]),
                                       make_float2(dh[i], dh[i + 1]));
+          hr[i] = r.x;
+          hr[i + 1] = r.y;
           hu[i] = __float_as_uint(r.x);
           hu[i + 1] = __float_as_uint(r.y);
         }
@@ -786,11 +784,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      named_bar(kNbState, 128);
-      if (leader) {
-        TC_MARK(k, 5);
-        mbar_arrive(BAR(BAR_DHFREE));  // dH read: MMA4 of chunk k+1 may overwrite it
-      }
+      named_bar(3, 128);
+      if (leader) mbar_arrive(BAR(BAR_DHFREE));  // dH read: MMA4 of chunk k+1 may overwrite it
       if (tail && k == tail_k) {  // the state entering the tail, in fp32
         tc_fence_after();
 #pragma unroll 1
@@ -804,7 +799,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       if (!kStateOnly && k != last) {
         // fp16 copy of h_k for MMA3 of chunk k+1, once MMA3 of chunk k has read h_{k-1}
-        if (!wg_wait(BAR(BAR_HTFREE), k & 1, leader, kNbState, abort_flag, a.err, lim)) break;
+        if (!wg_wait(BAR(BAR_HTFREE), k & 1, leader, 3, abort_flag, a.err, lim)) break;
         tc_fence_after();
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
@@ -814,51 +809,26 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           write_h_tile(smem, hr, n, half);
         }
         fence_proxy_async();
-        named_bar(kNbState, 128);
+        named_bar(3, 128);
         if (leader) {
-          TC_MARK(k, 6);
+          TC_MARK(k, 5);
           mbar_arrive(BAR(BAR_HREADY));
         }
       }
-    }
-    if (*abort_flag == 0) {
-      if (hout && a.tail_chunks == 0) {
-        tc_fence_after();
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          float hr[32];
-          tmem_ld32(tmem + TM_H + 32 * half + lane_off, hr);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) hout[(32 * half + i) * 128 + n] = hr[i];
-        }
-      }
-      if (a.seg_decay && n == 0) a.seg_decay[(long long)seg * a.B * a.H + bh] = __expf(decay_sum);
-    }
-  } else if (warp >= kWarpOut0 && warp < kWarpOut0 + 4) {
-    // ---------------------------------------------------------------- output y = Yi + e^{cs} Ys
-    if (!kStateOnly) {
-      const int ow = warp - kWarpOut0;
-      const int t = 32 * ow + lane;  // TMEM lane: output row t
-      const bool leader = (warp == kWarpOut0 + 1 && lane == 0);
-      const uint32_t lane_off = (uint32_t)(32 * ow) << 16;
-      const bool gate = a.qn != nullptr && !a.nbg;
-      for (int k = 0; k < nck; ++k) {
-        const int st = k & 1;
-        const int tok = t_begin + k * QC + t;
+      if (!kStateOnly) {
+        const int tok = t_begin + k * QC + n;
         const long long row = (long long)b * a.L + tok;
-        // fused gate: this row's z (64 channels, 128 bytes) is prefetched into L1 before the
-        // wait for the chunk's products
+        // fused gate (gate first): this row's z (64 channels, 128 bytes) is prefetched into L1
+        // before the wait for the chunk's products
+        const bool gate = a.qn != nullptr && !a.nbg;
         const __nv_bfloat16 *zrow = gate ? a.z + row * a.zs + h * 64 : nullptr;
         if (gate && tok < t_end) {
           asm volatile("prefetch.global.L1 [%0];" ::"l"(zrow));
           asm volatile("prefetch.global.L1 [%0];" ::"l"(zrow + 63));
         }
-        if (!wg_wait(BAR(BAR_STREADY0 + st), (k >> 1) & 1, leader, kNbOut, abort_flag, a.err, lim)) break;
-        if (!wg_wait(BAR(BAR_YREADY0 + st), (k >> 1) & 1, leader, kNbOut, abort_flag, a.err, lim)) break;
+        if (!wg_wait(BAR(BAR_YREADY0 + st), (k >> 1) & 1, leader, 3, abort_flag, a.err, lim)) break;
         tc_fence_after();
-        if (leader) TC_MARK(k, 7);
-        const float et = reinterpret_cast<const float *>(smem + OFF_ET + st * 512)[t];
+        if (leader) TC_MARK(k, 6);
         const uint32_t tYi = tmem + (st ? TM_S1 : TM_S0) + TM_YI_OFF + lane_off;
         const uint32_t tYs = tmem + (st ? TM_YS1 : TM_YS0) + lane_off;
         if (a.qn) {
@@ -941,18 +911,32 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         }
         tc_fence_before();
-        named_bar(kNbOut, 128);
+        named_bar(3, 128);
         if (leader) {
-          TC_MARK(k, 8);
+          TC_MARK(k, 7);
           mbar_arrive(BAR(BAR_YFREE0 + st));
         }
       }
+    }
+    if (*abort_flag == 0) {
+      if (hout && a.tail_chunks == 0) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          float hr[32];
+          tmem_ld32(tmem + TM_H + 32 * half + lane_off, hr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) hout[(32 * half + i) * 128 + n] = hr[i];
+        }
+      }
+      if (a.seg_decay && n == 0) a.seg_decay[(long long)seg * a.B * a.H + bh] = __expf(decay_sum);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kWarpIssueA) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, TM_COLS);
   }
@@ -1020,51 +1004,31 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
   a.z = (const __nv_bfloat16 *)p.z;
   a.zs = p.zs;
   a.nbg = p.nbg;
-  a.d_inner = p.d_inner;
   a.wait_ns = p.stall_chunk1 > 0 ? p.stall_wait_ns : tc::kWaitLimitNs;
   a.debug_skip_chunk = p.stall_chunk1 - 1;
+  a.d_inner = p.d_inner;
   const long long seg_stride = (long long)p.B * p.H * p.P * p.N;
   dim3 grid(p.n_seg, p.H, p.B);
-  // the low parts of B over the tail (tail pass only; else the B|C map stands in, unread)
-  CUtensorMap tml = tm;
-  if (mode == 2) {
-    const cuuint64_t GN = (cuuint64_t)p.G * p.N;
-    cuuint64_t ldims[3] = {GN, (cuuint64_t)p.ntail, (cuuint64_t)p.B};
-    cuuint64_t lstrides[2] = {GN * 2, GN * 2 * (cuuint64_t)p.ntail};
-    r = enc(&tml, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, p.blo, ldims, lstrides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  }
   cudaError_t e;
   if (mode == 1) {
     a.h_init = nullptr; a.h_init_seg = 0;
     a.h_out = p.seg_state; a.h_out_seg = seg_stride; a.seg_decay = p.seg_decay;
-    e = set_smem_attr(ssd_scan_tc_kernel<1>, kSmemAlloc, s);
+    e = set_smem_attr(ssd_scan_tc_kernel<true>, kSmemAlloc, s);
     if (e != cudaSuccess) return e;
-    ssd_scan_tc_kernel<1><<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, tml, a);
-  } else if (mode == 2) {
-    // the tail pass: tokens [t_tail, L) of every (batch row, head), from a zero state, into
-    // tail_dh and their total decay into tail_dec
-    a.t_base = p.t_tail; a.seg_len = p.L - p.t_tail;
-    a.h_init = nullptr; a.h_init_seg = 0;
-    a.h_out = p.tail_dh; a.h_out_seg = 0; a.seg_decay = p.tail_dec;
-    e = set_smem_attr(ssd_scan_tc_kernel<2>, kSmemAlloc, s);
-    if (e != cudaSuccess) return e;
-    ssd_scan_tc_kernel<2><<<dim3(1, p.H, p.B), kThreadsTC, kSmemAlloc, s>>>(tm, tmx, tml, a);
+    ssd_scan_tc_kernel<true><<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, a);
   } else {
     if (p.n_seg > 1) {
       a.h_init = p.seg_state; a.h_init_seg = seg_stride;
     } else {
       a.h_init = p.h0; a.h_init_seg = 0;
     }
-    // the last segment leaves the state entering the tail; the tail pass adds what the tail's
-    // chunks contribute
+    // the last segment leaves the state before its last kTailChunks chunks; the fp32 tail pass
+    // adds what those chunks contribute
     a.h_out = p.h_final; a.h_out_seg = 0; a.seg_decay = nullptr;
     a.tail_chunks = p.tail_dh ? kTailChunks : 0;
-    e = set_smem_attr(ssd_scan_tc_kernel<0>, kSmemAlloc, s);
+    e = set_smem_attr(ssd_scan_tc_kernel<false>, kSmemAlloc, s);
     if (e != cudaSuccess) return e;
-    ssd_scan_tc_kernel<0><<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, tml, a);
+    ssd_scan_tc_kernel<false><<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, a);
   }
   return cudaGetLastError();
 }
