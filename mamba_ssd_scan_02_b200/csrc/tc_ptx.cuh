@@ -126,6 +126,10 @@ __device__ __forceinline__ void fence_proxy_async() {
 __device__ __forceinline__ void named_bar(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Arrive on a named barrier without waiting for it (the waiting side uses named_bar).
+__device__ __forceinline__ void named_bar_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 // Named barrier over `count` threads that also ORs one predicate over them: every thread gets
 // the same result, so a branch taken on it (such as leaving a loop after an abort) is uniform

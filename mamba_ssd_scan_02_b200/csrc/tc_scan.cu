@@ -23,9 +23,9 @@
 //
 // Warp roles (640 threads): warp 0 issues TMA loads (B and C tiles of the group, the head's
 // raw x rows with a 3-token halo, per-chunk dt and prefix sums), warp 1 allocates TMEM and
-// issues each MMA group as soon as its inputs are ready, warps 2-4, 6-8, 10-11 compute the x
-// channels (causal conv1d + SiLU) in place into w o X and into X, warps 12-15 turn S into S~,
-// warps 16-19 update the state (kept in fp32 in TMEM), refresh its fp16 copy and write y.
+// issues each MMA group as soon as its inputs are ready, warps 2-9 compute the x channels
+// (causal conv1d + SiLU) in place into w o X and into X, warps 10-15 turn S into S~, warps
+// 16-19 update the state (kept in fp32 in TMEM), refresh its fp16 copy and write y.
 // X, w o X, S (with Yi in its upper half), Ys and the B/C stages are double-buffered, so each
 // role can run a chunk ahead of the next.  Hand-offs use mbarriers (TMA transaction counts,
 // tcgen05.commit, thread arrivals); every wait is bounded and a timeout aborts the CTA
@@ -223,21 +223,9 @@ __device__ __forceinline__ void issue_dH(uint32_t stage, uint32_t xwbase, uint32
     mma_f16_ss(tDH, desc_adv(a0, j * 2048), desc_adv(b0, j * 2048), IDESC_DH, (j > 0 || acc) ? 1u : 0u);
 }
 
-// Conv warps: 2, 3, 4, 6, 7, 8, 10, 11 -- none on the sub-partition of warp 1 (warps 1, 5, 9,
-// ...), whose single MMA-issuing thread would otherwise be starved of issue slots.
-__device__ __forceinline__ int conv_index(int warp) {
-  switch (warp) {
-    case 2: return 0;
-    case 3: return 1;
-    case 4: return 2;
-    case 6: return 3;
-    case 7: return 4;
-    case 8: return 5;
-    case 10: return 6;
-    case 11: return 7;
-    default: return -1;
-  }
-}
+// Conv warps: 2-9, two on each SM sub-partition (warp % 4), the issuer's included: spreading
+// them evenly measured faster than keeping the issuer's sub-partition free of them.
+__device__ __forceinline__ int conv_index(int warp) { return warp >= 2 && warp < 10 ? warp - 2 : -1; }
 
 // Row r (128 bytes) of a 128-byte-swizzled tile: 16-byte chunk c sits at chunk c ^ (r & 7).
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
@@ -268,6 +256,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const int t_end = min(a.L, t_begin + a.seg_len);
   const int nck = t_end > t_begin ? (t_end - t_begin + QC - 1) / QC : 0;
   const int last = nck - 1;
+  // The last chunk's exact path (fp32 SiLU, split-precision w o X) serves only the final
+  // state; in tail mode an fp32 pass recomputes the last chunks, and without h_out nothing
+  // reads it.
+  const bool exact_last = kStateOnly || (a.tail_chunks == 0 && a.h_out != nullptr);
   const uint64_t lim = a.wait_ns;
   const uint32_t bar0 = sb + OFF_BAR;
 #define BAR(i) (bar0 + 8u * (uint32_t)(i))
@@ -380,7 +372,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (nD < nck && (kStateOnly || nD < nS) &&
             mbar_test(BAR(BAR_XREADY0 + (nD & 1)), (nD >> 1) & 1) &&
             (nD == 0 || mbar_test(BAR(BAR_DHFREE), (nD - 1) & 1)) &&
-            (nD != last || mbar_test(BAR(BAR_XLOREADY), 0)) &&
+            (nD != last || !exact_last || mbar_test(BAR(BAR_XLOREADY), 0)) &&
             (!kStateOnly || mbar_test(BAR(BAR_FULL0 + (nD & 1)), (nD >> 1) & 1))) {
           const int j = nD;
           tc_fence_after();
@@ -388,7 +380,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           const uint32_t sst = sb + (j & 1) * kStage;
           issue_dH(sst, sb + OFF_XW + (j & 1) * kXBuf, tmem + TM_DH, false);
           // last chunk: the low part of w o X (in the other w o X buffer) for the final state
-          if (j == last) issue_dH(sst, sb + OFF_XW + ((j + 1) & 1) * kXBuf, tmem + TM_DH, true);
+          if (j == last && exact_last) issue_dH(sst, sb + OFF_XW + ((j + 1) & 1) * kXBuf, tmem + TM_DH, true);
           mma_commit(BAR(BAR_XWFREE0 + (j & 1)));
           mma_commit(BAR(BAR_DHREADY));
           if (kStateOnly) mma_commit(BAR(BAR_XFREE0 + (j & 1)));
@@ -465,7 +457,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     const int tok0 = kTokPerConvWarp * cw;  // multiple of 8
     for (int k = 0; k < nck; ++k) {
       const int st = k & 1, xb = k & 1, lb = (k + 1) & 1;
-      const bool is_last = (k == last);
+      const bool is_last = (k == last) && exact_last;
       // the leader waits for every input of the chunk, then one group barrier releases all
       if (leader) {
         bool ok = mbar_wait(BAR(BAR_FULLX0 + xb), (k >> 1) & 1, abort_flag, a.err, lim);
@@ -601,23 +593,35 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (is_last) mbar_arrive(BAR(BAR_XLOREADY));
       }
     }
-  } else if (warp >= 12 && warp < 16) {
+  } else if (warp >= 10 && warp < 16) {
     // ---------------------------------------------------------------- S -> S~ (decay mask)
+    // Row t of S sits in TMEM lane t, and a warp reaches only the 32 lanes of its SM
+    // sub-partition (warp % 4): lane quarter q (rows 32q..32q+31) needs the blocks J <= q of
+    // 32 columns, one to four of them.  Warps 12-15 own the quarters; warps 10 and 11 take
+    // blocks 2..q of quarters 2 and 3, so that no warp handles more than two blocks.
+    // S~ columns 32J..32J+31 go to the packed TMEM columns 16J..16J+15, which lie in S block
+    // J/2: blocks 0 and 1 land in block 0, read by the same warp before; blocks 2 and 3 land
+    // in block 1, so a helper stores only after its owner has read block 1 (named barrier
+    // 4 or 5, owner arrives, helper waits).
     if (!kStateOnly) {
-      const int mw = warp - 12;
-      const int t = 32 * mw + lane;
+      const int q = warp & 3;
+      const bool helper = warp < 12;
+      const bool split = q >= 2;
+      const int jlo = helper ? 2 : 0, jhi = (split && !helper) ? 1 : q;
+      const int pair_bar = 4 + (q & 1);  // quarters 2 and 3
+      const int t = 32 * q + lane;
       const bool leader = (tid == 14 * 32);
       float *cf = reinterpret_cast<float *>(smem + OFF_CF);
       const float Dh = a.D[h];
       for (int k = 0; k < nck; ++k) {
         const int st = k & 1;
-        if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, 2, abort_flag, a.err, lim)) break;
-        if (!wg_wait(BAR(BAR_SREADY0 + st), (k >> 1) & 1, leader, 2, abort_flag, a.err, lim)) break;
+        if (!wg_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, leader, 2, abort_flag, a.err, lim, 192)) break;
+        if (!wg_wait(BAR(BAR_SREADY0 + st), (k >> 1) & 1, leader, 2, abort_flag, a.err, lim, 192)) break;
         tc_fence_after();
         float *cs = reinterpret_cast<float *>(smem + OFF_CSM);
         float *dtv = reinterpret_cast<float *>(smem + OFF_DTM);
-        {  // private copies (the stage is released at once); column factor of column t:
-           // e^{r_J - cs_t} dt_t with r_J = cs at the end of t's block
+        if (!helper) {  // private copies (the stage is released at once); column factor of
+                        // column t: e^{r_J - cs_t} dt_t with r_J = cs at the end of t's block
           const float *scs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
           const float *sdt = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
           const float rJ = scs[32 * (t >> 5) + 31];
@@ -625,50 +629,24 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           dtv[t] = sdt[t];
           cf[t] = __expf(rJ - scs[t]) * sdt[t];
         }
-        named_bar(2, 128);
+        named_bar(2, 192);
         if (leader) mbar_arrive(BAR(BAR_EMPTY0 + st));
         if (leader) TC_MARK(k, 2);
         const float cst = cs[t];
-        const uint32_t trow = tmem + (st ? TM_S1 : TM_S0) + ((uint32_t)(32 * mw) << 16);
-        // Blocks of 32 columns in increasing J: S~ columns 32J..32J+31 go to the packed TMEM
-        // columns 16J..16J+15, which only hold S columns of blocks already read.
-        // Blocks J < mw lie wholly below the diagonal: S~ = S * rf * cf (a block whose cs
-        // span is too steep to factor takes the direct exponential instead).
+        const uint32_t trow = tmem + (st ? TM_S1 : TM_S0) + ((uint32_t)(32 * q) << 16);
+        // S~ = S * e^{cs_t - cs_s} dt_s, factored per block as rf_t * cf_s with rf_t = e^{cs_t -
+        // r_J}; a block whose cs span is too steep to factor takes the direct exponential.  The
+        // diagonal block J = q also applies the causal mask (column c <= row lane) and adds the
+        // D x skip on its diagonal.
 #pragma unroll 1
-        for (int J = 0; J < mw; ++J) {
-          uint32_t pk[16];
+        for (int J = jlo; J <= jhi; ++J) {
           float v[32];
           tmem_ld32(trow + 32 * J, v);
           tmem_ld_wait();
-          const float rJ = cs[32 * J + 31];
-          if (cs[32 * J] - rJ > 60.f) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) v[c] *= __expf(cst - cs[32 * J + c]) * dtv[32 * J + c];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) pk[c] = pack_f16(v[2 * c], v[2 * c + 1]);
-          } else {
-            const float rf = __expf(cst - rJ);
-            const float2 rf2 = make_float2(rf, rf);
-            const float4 *cf4 = reinterpret_cast<const float4 *>(cf + 32 * J);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 c4 = cf4[q];
-              const float2 lo = __fmul2_rn(__fmul2_rn(make_float2(v[4 * q], v[4 * q + 1]), rf2),
-                                           make_float2(c4.x, c4.y));
-              const float2 hi = __fmul2_rn(__fmul2_rn(make_float2(v[4 * q + 2], v[4 * q + 3]), rf2),
-                                           make_float2(c4.z, c4.w));
-              pk[2 * q] = pack_f16(lo.x, lo.y);
-              pk[2 * q + 1] = pack_f16(hi.x, hi.y);
-            }
+          if (split && !helper && J == 1) {  // block 1 read: the helper may write over it
+            tc_fence_before();
+            named_bar_arrive(pair_bar, 64);
           }
-          tmem_st16(trow + 16 * J, pk);
-        }
-        {  // diagonal block J = mw: causal mask (column c <= row lane) and the D x skip
-          const int J = mw;
-          uint32_t pk[16];
-          float v[32];
-          tmem_ld32(trow + 32 * J, v);
-          tmem_ld_wait();
           const float rJ = cs[32 * J + 31];
           if (cs[32 * J] - rJ > 60.f) {
 #pragma unroll
@@ -678,37 +656,44 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             const float2 rf2 = make_float2(rf, rf);
             const float4 *cf4 = reinterpret_cast<const float4 *>(cf + 32 * J);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 c4 = cf4[q];
-              const float2 lo = __fmul2_rn(__fmul2_rn(make_float2(v[4 * q], v[4 * q + 1]), rf2),
+            for (int qq = 0; qq < 8; ++qq) {
+              const float4 c4 = cf4[qq];
+              const float2 lo = __fmul2_rn(__fmul2_rn(make_float2(v[4 * qq], v[4 * qq + 1]), rf2),
                                            make_float2(c4.x, c4.y));
-              const float2 hi = __fmul2_rn(__fmul2_rn(make_float2(v[4 * q + 2], v[4 * q + 3]), rf2),
+              const float2 hi = __fmul2_rn(__fmul2_rn(make_float2(v[4 * qq + 2], v[4 * qq + 3]), rf2),
                                            make_float2(c4.z, c4.w));
-              v[4 * q] = lo.x;
-              v[4 * q + 1] = lo.y;
-              v[4 * q + 2] = hi.x;
-              v[4 * q + 3] = hi.y;
+              v[4 * qq] = lo.x;
+              v[4 * qq + 1] = lo.y;
+              v[4 * qq + 2] = hi.x;
+              v[4 * qq + 3] = hi.y;
             }
           }
+          if (J == q) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float val = c <= lane ? v[c] : 0.f;
-            v[c] = c == lane ? val + Dh : val;
+            for (int c = 0; c < 32; ++c) {
+              const float val = c <= lane ? v[c] : 0.f;
+              v[c] = c == lane ? val + Dh : val;
+            }
           }
+          uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) pk[c] = pack_f16(v[2 * c], v[2 * c + 1]);
+          if (helper && J == jlo) {  // the owner has read block 1
+            named_bar(pair_bar, 64);
+            tc_fence_after();
+          }
           tmem_st16(trow + 16 * J, pk);
         }
-        {  // blocks J > mw lie above the diagonal: zeros
+        if (helper || !split) {  // blocks J > q lie above the diagonal: zeros
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) pk[c] = 0u;
 #pragma unroll 1
-          for (int J = mw + 1; J < 4; ++J) tmem_st16(trow + 16 * J, pk);
+          for (int J = q + 1; J < 4; ++J) tmem_st16(trow + 16 * J, pk);
         }
         tmem_st_wait();
         tc_fence_before();
-        named_bar(2, 128);
+        named_bar(2, 192);
         if (leader) {
           TC_MARK(k, 3);
           mbar_arrive(BAR(BAR_STREADY0 + st));
@@ -761,7 +746,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const float ak = __expf(cs_end);
       named_bar(3, 128);  // every thread has read the prefix sums
       if (leader) mbar_arrive(BAR(BAR_EMPTY0 + st));
-      if (!wg_wait(BAR(BAR_DHREADY), k & 1, leader, 3, abort_flag, a.err, lim)) break;
+      // h_k = e^{cs_end} h_{k-1} + dH_k in TMEM, and its fp16 copy for MMA3 of chunk k+1, which
+      // may overwrite the h tile once MMA3 of chunk k has read h_{k-1} from it
+      const bool htile = !kStateOnly && k != last;
+      if (leader) {
+        bool ok = mbar_wait(BAR(BAR_DHREADY), k & 1, abort_flag, a.err, lim);
+        if (ok && htile) mbar_wait(BAR(BAR_HTFREE), k & 1, abort_flag, a.err, lim);
+      }
+      if (named_bar_or(3, 128, *abort_flag != 0)) break;
       tc_fence_after();
       if (leader) TC_MARK(k, 4);
 #pragma unroll 1
@@ -781,36 +773,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           hu[i + 1] = __float_as_uint(r.y);
         }
         tmem_st32(tmem + TM_H + 32 * half + lane_off, hu);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      named_bar(3, 128);
-      if (leader) mbar_arrive(BAR(BAR_DHFREE));  // dH read: MMA4 of chunk k+1 may overwrite it
-      if (tail && k == tail_k) {  // the state entering the tail, in fp32
-        tc_fence_after();
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          float hr[32];
-          tmem_ld32(tmem + TM_H + 32 * half + lane_off, hr);
-          tmem_ld_wait();
+        if (htile) write_h_tile(smem, hr, n, half);
+        if (tail && k == tail_k) {  // the state entering the tail, in fp32
 #pragma unroll
           for (int i = 0; i < 32; ++i) hout[(32 * half + i) * 128 + n] = hr[i];
         }
       }
-      if (!kStateOnly && k != last) {
-        // fp16 copy of h_k for MMA3 of chunk k+1, once MMA3 of chunk k has read h_{k-1}
-        if (!wg_wait(BAR(BAR_HTFREE), k & 1, leader, 3, abort_flag, a.err, lim)) break;
-        tc_fence_after();
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          float hr[32];
-          tmem_ld32(tmem + TM_H + 32 * half + lane_off, hr);
-          tmem_ld_wait();
-          write_h_tile(smem, hr, n, half);
-        }
-        fence_proxy_async();
-        named_bar(3, 128);
-        if (leader) {
+      tmem_st_wait();
+      if (htile) fence_proxy_async();
+      tc_fence_before();
+      named_bar(3, 128);
+      if (leader) {
+        mbar_arrive(BAR(BAR_DHFREE));  // dH read: MMA4 of chunk k+1 may overwrite it
+        if (htile) {
           TC_MARK(k, 5);
           mbar_arrive(BAR(BAR_HREADY));
         }
@@ -888,6 +863,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           tmem_ld32(tYi + 32 * half, yi);
           tmem_ld32(tYs + 32 * half, ysv);
           tmem_ld_wait();
+          if (half == 1) {  // every product read: the buffers are free before the stores
+            tc_fence_before();
+            named_bar(3, 128);
+            if (leader) {
+              TC_MARK(k, 7);
+              mbar_arrive(BAR(BAR_YFREE0 + st));
+            }
+          }
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             const float2 r = __ffma2_rn(make_float2(et, et), make_float2(ysv[i], ysv[i + 1]),
@@ -910,11 +893,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           }
         }
         }
-        tc_fence_before();
-        named_bar(3, 128);
-        if (leader) {
-          TC_MARK(k, 7);
-          mbar_arrive(BAR(BAR_YFREE0 + st));
+        if (a.qn) {
+          tc_fence_before();
+          named_bar(3, 128);
+          if (leader) {
+            TC_MARK(k, 7);
+            mbar_arrive(BAR(BAR_YFREE0 + st));
+          }
         }
       }
     }
