@@ -270,6 +270,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t cnt = 1;
       if (i == BAR_EMPTY0 || i == BAR_EMPTY1) cnt = kStateOnly ? 3 : 4;  // + mask warps
+      if (i == BAR_XREADY0 || i == BAR_XREADY1 || i == BAR_XLOREADY) cnt = kConvWarps;
       mbar_init(BAR(i), cnt);
     }
     *abort_flag = 0;
@@ -432,7 +433,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     // 11 significant bits -- and one half2 tanh serves both channels.  The last chunk of a
     // segment, whose newest tokens dominate the final state, uses fp32 and the exact SiLU.
     const int cw = conv_index(warp);
-    const bool leader = (tid == 2 * 32);  // leaders sit on different SM sub-partitions
+    const bool leader = (tid == 2 * 32);  // releases the stage
     const int ch = h * 64 + 2 * lane;
     const int W = a.W;
     float2 ew[4], bias2 = make_float2(0.f, 0.f);
@@ -458,15 +459,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     for (int k = 0; k < nck; ++k) {
       const int st = k & 1, xb = k & 1, lb = (k + 1) & 1;
       const bool is_last = (k == last) && exact_last;
-      // the leader waits for every input of the chunk, then one group barrier releases all
-      if (leader) {
-        bool ok = mbar_wait(BAR(BAR_FULLX0 + xb), (k >> 1) & 1, abort_flag, a.err, lim);
-        if (ok) ok = mbar_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, abort_flag, a.err, lim);
-        if (ok && k >= 2) ok = mbar_wait(BAR(BAR_XFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err, lim);
-        if (ok && is_last && k >= 1) mbar_wait(BAR(BAR_XWFREE0 + lb), ((k - 1) >> 1) & 1, abort_flag, a.err, lim);
-        TC_MARK(k, 14);
-      }
-      if (named_bar_or(1, 256, *abort_flag != 0)) break;
+      // every thread waits for the chunk's inputs itself; one barrier per chunk (after the
+      // boundary rows are read) keeps the warps together and makes an abort uniform, and each
+      // warp signals its own rows of X and w o X (XREADY counts eight arrivals)
+      bool ok = mbar_wait(BAR(BAR_FULLX0 + xb), (k >> 1) & 1, abort_flag, a.err, lim);
+      if (ok) ok = mbar_wait(BAR(BAR_FULL0 + st), (k >> 1) & 1, abort_flag, a.err, lim);
+      if (ok && k >= 2) ok = mbar_wait(BAR(BAR_XFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err, lim);
+      if (ok && is_last && k >= 1) ok = mbar_wait(BAR(BAR_XWFREE0 + lb), ((k - 1) >> 1) & 1, abort_flag, a.err, lim);
+      if (leader) TC_MARK(k, 14);
       const float *cs = reinterpret_cast<const float *>(smem + st * kStage + OFF_CS);
       const float *dtv = reinterpret_cast<const float *>(smem + st * kStage + OFF_DT);
       const float cs_end = cs[QC - 1];
@@ -492,7 +492,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         r2 = hist[2];
       }
       const uint32_t nb0 = RAW(16), nb1 = RAW(17), nb2 = RAW(18);
-      named_bar(1, 256);  // all boundary rows read before any row is overwritten
+      // all boundary rows read before any row is overwritten; a failed wait anywhere ends all
+      if (named_bar_or(1, 256, !ok || *abort_flag != 0)) break;
       if (leader) {
         TC_MARK(k, 0);
         mbar_arrive(BAR(BAR_EMPTY0 + st));  // dt and prefix sums already read
@@ -586,9 +587,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       if (leader) TC_MARK(k, 13);
 #undef RAW
       fence_proxy_async();
-      named_bar(1, 256);
-      if (leader) {
-        TC_MARK(k, 1);
+      __syncwarp();
+      if (leader) TC_MARK(k, 1);
+      if (lane == 0) {
         mbar_arrive(BAR(BAR_XREADY0 + xb));
         if (is_last) mbar_arrive(BAR(BAR_XLOREADY));
       }
