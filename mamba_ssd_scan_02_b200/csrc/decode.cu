@@ -36,16 +36,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodePlan p) {
   float *dts = ys + nx;                     // [hpg]
   __shared__ float red[32];
 
-  // The first rows of each warp's first head do not depend on the conv: their loads are
-  // issued now, so that the state stream is already in flight during the conv below.
-  float4 hv[kRowsInFlight];
-  if (warp < p.hpg) {
-    const float4 *st0 = reinterpret_cast<const float4 *>(
-        p.state + ((long long)b * p.H + g * p.hpg + warp) * kHeadDim * kDState);
-#pragma unroll
-    for (int i = 0; i < kRowsInFlight; ++i) hv[i] = __ldcs(st0 + i * (kDState / 4) + lane);
-  }
-
   // ---- conv of the group's channels (x: nx, B: N, C: N), cache shift -------------------
   const int nvec = (nx + 2 * kDState) / 8;
   const T *xrow = reinterpret_cast<const T *>(p.xBC) + (long long)b * p.xs;
@@ -120,10 +110,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(DecodePlan p) {
     const float Dh = p.D[h];
     float4 *st = reinterpret_cast<float4 *>(p.state + ((long long)b * p.H + h) * kHeadDim * kDState);
     for (int p0 = 0; p0 < kHeadDim; p0 += kRowsInFlight) {
-      if (hi != warp || p0 != 0) {  // (the first rows of the first head are already loaded)
+      float4 hv[kRowsInFlight];
 #pragma unroll
-        for (int i = 0; i < kRowsInFlight; ++i) hv[i] = __ldcs(st + (p0 + i) * (kDState / 4) + lane);
-      }
+      for (int i = 0; i < kRowsInFlight; ++i) hv[i] = __ldcs(st + (p0 + i) * (kDState / 4) + lane);
 #pragma unroll
       for (int i = 0; i < kRowsInFlight; ++i) {
         const float xp = ux[hi * kHeadDim + p0 + i];
