@@ -172,6 +172,38 @@ size_t ssd_varlen_workspace_size(const ssd_config_t *cfg, const int *cu_seqlens,
 ssd_status_t ssd_prefill_varlen(const ssd_config_t *cfg, const ssd_prefill_args_t *args,
                                 const int *cu_seqlens, int nseq, void *stream);
 
+/* Sequence parallelism (one exchange).  A sequence too long for one GPU is split into spans
+ * of consecutive tokens, one per rank.  The recurrence is linear in the state, so the state
+ * entering span k is h_in[k] = lambda_{k-1} h_in[k-1] + s_{k-1} (h_in[0] = h0), where s_k is
+ * the state span k produces from a zero state and lambda_k = exp(sum over its tokens of
+ * dt A), per (batch row, head).  This is the chunked form's inter-chunk recurrence of the
+ * Mamba-2 scan applied at span granularity; the pages fix only the fp32 state it carries
+ * (neurohive.io article, section "Deployment and usage") and 128k-token contexts (abstract).
+ * Per rank: (1) ssd_prefill_span_state on its span; (2) the caller all-gathers (s_k,
+ * lambda_k) over the ranks (its own collective, e.g. NCCL all-gather: n_spans * B*H*P*N +
+ * n_spans * B*H floats); (3) ssd_span_prefix gives h_in[k]; (4) ssd_prefill on the span with
+ * h0 = h_in[own k] gives its y, and the last rank's h_final is the sequence's final state.
+ * The conv of a span's first W-1 tokens reads the previous span's last W raw rows: each rank
+ * is given them as conv_state_in (a W-row halo of its input), so no exchange is needed for it.
+ *
+ * ssd_prefill_span_state: args as for ssd_prefill (xBC, dt, A, dt_bias, conv_w, conv_b,
+ *   conv_state_in and the workspace are used; y, D, z, norm_w, h0, h_final and
+ *   conv_state_out are ignored and may be NULL).  Writes span_state [B, H, P, N] fp32
+ *   (16-byte aligned) and span_decay [B, H] fp32.  seqlen = 0 gives zeros and ones.  Errors
+ *   as for ssd_prefill. */
+ssd_status_t ssd_prefill_span_state(const ssd_config_t *cfg, const ssd_prefill_args_t *args,
+                                    float *span_state, float *span_decay, void *stream);
+
+/* ssd_span_prefix: span_states [n_spans, B, H, P, N] and span_decays [n_spans, B, H] (fp32,
+ * span-major, as an all-gather leaves them); h0 [B, H, P, N] or NULL (zero).  Writes
+ * h_in [n_spans, B, H, P, N] (the state entering each span; may be span_states itself, in
+ * place; otherwise the two must not overlap) and/or h_final [B, H, P, N] (the state after the
+ * last span); either may be NULL but not both.  Device pointers, 16-byte aligned
+ * (SSD_ERR_ALIGNMENT); headdim * dstate a multiple of 4 (SSD_ERR_INVALID_ARG). */
+ssd_status_t ssd_span_prefix(const float *span_states, const float *span_decays, int n_spans,
+                             int batch, int nheads, int headdim, int dstate, const float *h0,
+                             float *h_in, float *h_final, void *stream);
+
 /* One token per batch row: conv-cache shift + conv + SiLU, softplus dt, the state update
  * h = exp(dt A) h + dt x B^T (fp32 state in place), y = h C + D x, optional gated RMSNorm.
  * cfg->seqlen and cfg->chunk are ignored.  norm_groups must be 0 or a multiple of ngroups. */

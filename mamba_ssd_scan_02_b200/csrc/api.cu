@@ -230,23 +230,41 @@ struct SideJoin {
   ~SideJoin() { join(); }
 };
 
-ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cudaStream_t s) {
+// Span mode (sequence parallelism): instead of y and the final state, the call leaves the
+// state its tokens produce from a zero state, and their total decay exp(sum dt A), per
+// (batch row, head).  y, h0, z and the norm, and the outgoing conv cache are not used.
+struct SpanOut {
+  float *state;  // [B, H, P, N]
+  float *decay;  // [B, H]
+};
+
+ssd_status_t run_prefill(const ssd_config_t *c_in, const ssd_prefill_args_t *a, cudaStream_t s,
+                         const SpanOut *span = nullptr) {
+  ssd_config_t c_span;
+  const ssd_config_t *c = c_in;
+  if (span && c_in) {  // the norm does not touch the state
+    c_span = *c_in;
+    c_span.norm_groups = 0;
+    c = &c_span;
+  }
   ssd_status_t st = check_config(c, true);
   if (st != SSD_OK) return st;
   if (!a) return SSD_ERR_INVALID_ARG;
+  if (span && (!span->state || !span->decay || !aligned16(span->state))) return SSD_ERR_INVALID_ARG;
   const int H = c->nheads, P = c->headdim, N = c->dstate, G = c->ngroups, W = c->conv_width;
   const long long d_inner = (long long)H * P, conv_dim = d_inner + 2LL * G * N;
   const size_t es = elt_size(c->io_dtype);
   const bool has_tokens = c->seqlen > 0;
   if (has_tokens) {
-    if (!a->xBC || !a->dt || !a->A || !a->D || !a->dt_bias || !a->y) return SSD_ERR_INVALID_ARG;
+    if (!a->xBC || !a->dt || !a->A || !a->dt_bias || (!span && (!a->D || !a->y))) return SSD_ERR_INVALID_ARG;
     if (W > 0 && !a->conv_w) return SSD_ERR_INVALID_ARG;
     if (c->norm_groups > 0 && !a->z) return SSD_ERR_INVALID_ARG;
-    if (a->xBC_row_stride < conv_dim || a->dt_row_stride < H || a->y_row_stride < d_inner)
+    if (a->xBC_row_stride < conv_dim || a->dt_row_stride < H || (!span && a->y_row_stride < d_inner))
       return SSD_ERR_INVALID_ARG;
     if (c->norm_groups > 0 && a->z_row_stride < d_inner) return SSD_ERR_INVALID_ARG;
-    if (!aligned16(a->xBC) || !aligned16(a->y) || (a->z && !aligned16(a->z)) ||
-        a->xBC_row_stride % 8 || a->y_row_stride % 8 || (a->z && a->z_row_stride % 8))
+    if (!aligned16(a->xBC) || a->xBC_row_stride % 8) return SSD_ERR_ALIGNMENT;
+    if (!span && (!aligned16(a->y) || (a->z && !aligned16(a->z)) || a->y_row_stride % 8 ||
+                  (a->z && a->z_row_stride % 8)))
       return SSD_ERR_ALIGNMENT;
   }
   if ((a->h0 && !aligned16(a->h0)) || (a->h_final && !aligned16(a->h_final)) ||
@@ -269,10 +287,27 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
   p.conv_w = a->conv_w; p.conv_b = a->conv_b; p.norm_w = a->norm_w; p.h0 = a->h0;
   p.csi = a->conv_state_in; p.y = a->y; p.ys = a->y_row_stride; p.h_final = a->h_final;
   p.cso = a->conv_state_out;
+  if (span) {
+    p.z = nullptr; p.norm_w = nullptr; p.h0 = nullptr; p.y = nullptr; p.h_final = nullptr;
+    p.cso = nullptr;
+  }
   p.err = device_error_ptr();
   p.stall_chunk1 = g_stall_chunk1.load();
   p.stall_wait_ns = g_stall_wait_ns.load();
 
+  if (span) {
+    // the combine of internal segments (or of none) into the span's own state and decay
+    auto combine = [&](const char *name) {
+      return traced(name, s, [&] {
+        return launch_span_prefix(p.seg_state, nullptr, p.seg_decay, p.n_seg, (long long)p.B * p.H,
+                                  p.P * p.N, nullptr, span->state, span->decay, s);
+      });
+    };
+    if (!has_tokens) {
+      p.n_seg = 0;
+      return from_cuda(combine("ssd_span_combine"));
+    }
+  }
   if (!has_tokens) return from_cuda(traced("ssd_carry", s, [&] { return launch_carry_only(p, s); }));
 
   const bool use_tc = prefill_uses_tc(c);
@@ -310,6 +345,18 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
     } else {
       SSD_TRY(traced("ssd_dt_cumsum", s, [&] { return launch_dt_cumsum(p, p.dte_hm, p.cs_hm, p.Lpad, s); }));
       SSD_TRY(traced("ssd_bc_conv", s, [&] { return launch_bc_conv_f16(p, s); }));
+    }
+    if (span) {
+      if (p.n_seg == 1) {
+        p.seg_state = span->state;
+        p.seg_decay = span->decay;
+        return from_cuda(traced("ssd_scan_tc_states", s, [&] { return launch_scan_tc(p, 1, s); }));
+      }
+      SSD_TRY(traced("ssd_scan_tc_states", s, [&] { return launch_scan_tc(p, 1, s); }));
+      return from_cuda(traced("ssd_span_combine", s, [&] {
+        return launch_span_prefix(p.seg_state, nullptr, p.seg_decay, p.n_seg, (long long)p.B * p.H,
+                                  p.P * p.N, nullptr, span->state, span->decay, s);
+      }));
     }
     // The tail pass needs only the front end's outputs: it is forked onto a side stream right
     // after the front end and launched after the scan, so that it takes the SMs the scan
@@ -350,6 +397,18 @@ ssd_status_t run_prefill(const ssd_config_t *c, const ssd_prefill_args_t *a, cud
   p.seg_decay = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.seg_decay) : nullptr;
   SSD_TRY(traced("ssd_dt", s, [&] { return launch_dt(p, s); }));
   SSD_TRY(traced("ssd_conv_silu", s, [&] { return launch_conv_silu_f32(p, s); }));
+  if (span) {
+    if (p.n_seg == 1) {
+      p.seg_state = span->state;
+      p.seg_decay = span->decay;
+      return from_cuda(traced("ssd_scan_simt_states", s, [&] { return launch_scan_simt(p, 1, s); }));
+    }
+    SSD_TRY(traced("ssd_scan_simt_states", s, [&] { return launch_scan_simt(p, 1, s); }));
+    return from_cuda(traced("ssd_span_combine", s, [&] {
+      return launch_span_prefix(p.seg_state, nullptr, p.seg_decay, p.n_seg, (long long)p.B * p.H,
+                                p.P * p.N, nullptr, span->state, span->decay, s);
+    }));
+  }
   if (p.n_seg == 1) {
     SSD_TRY(traced("ssd_scan_simt", s, [&] { return launch_scan_simt(p, 0, s); }));
   } else {
@@ -586,6 +645,34 @@ ssd_status_t ssd_get_device_error(void *stream) {
     if (cudaMemcpy(p, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return SSD_ERR_CUDA;
   }
   return static_cast<ssd_status_t>(v);
+}
+
+ssd_status_t ssd_prefill_span_state(const ssd_config_t *cfg, const ssd_prefill_args_t *args,
+                                    float *span_state, float *span_decay, void *stream) {
+  const SpanOut out{span_state, span_decay};
+  return run_prefill(cfg, args, static_cast<cudaStream_t>(stream), &out);
+}
+
+ssd_status_t ssd_span_prefix(const float *span_states, const float *span_decays, int n_spans,
+                             int batch, int nheads, int headdim, int dstate, const float *h0,
+                             float *h_in, float *h_final, void *stream) {
+  if (n_spans < 0 || batch < 0 || nheads < 0 || headdim < 1 || dstate < 1 ||
+      (headdim * dstate) % 4 != 0)
+    return SSD_ERR_INVALID_ARG;
+  if (n_spans > 0 && (!span_states || !span_decays)) return SSD_ERR_INVALID_ARG;
+  if (!h_in && !h_final) return SSD_ERR_INVALID_ARG;
+  if ((span_states && !aligned16(span_states)) || (h0 && !aligned16(h0)) ||
+      (h_in && !aligned16(h_in)) || (h_final && !aligned16(h_final)))
+    return SSD_ERR_ALIGNMENT;
+  const long long BH = (long long)batch * nheads;
+  if (h_in && h_in != span_states && n_spans > 0) {
+    const size_t bytes = (size_t)n_spans * BH * headdim * dstate * sizeof(float);
+    if (ranges_overlap(h_in, bytes, span_states, bytes)) return SSD_ERR_INVALID_ARG;
+  }
+  return from_cuda(traced("ssd_span_prefix", static_cast<cudaStream_t>(stream), [&] {
+    return launch_span_prefix(span_states, h_in, span_decays, n_spans, BH, headdim * dstate, h0,
+                              h_final, nullptr, static_cast<cudaStream_t>(stream));
+  }));
 }
 
 int ssd_version(void) { return 100; }

@@ -86,6 +86,11 @@ bool tc_scan_available();
 cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s);
 // inter-segment state pass (state_pass.cu)
 cudaError_t launch_state_pass(const PrefillPlan &p, cudaStream_t s);
+// The same linear recurrence over spans held elsewhere (sequence parallelism): h_in[k] (may be
+// `states` itself, in place) = the state entering span k; h_final and decay_total optional.
+cudaError_t launch_span_prefix(const float *states, float *h_in, const float *decays, int n_spans,
+                               long long BH, int PN, const float *h0, float *h_final,
+                               float *decay_total, cudaStream_t s);
 // fp32 recomputation of the final state's last kTailChunks chunks (tensor-core path): what
 // those chunks add to a zero state, into p.tail_dh / p.tail_dec.  It runs on a side stream
 // beside the output scan, which leaves the state entering those chunks in h_final; the fold

@@ -78,7 +78,7 @@ class TraceRecord(ctypes.Structure):
 EXPORTS = ("ssd_workspace_size", "ssd_prefill", "ssd_decode_step", "ssd_mixer_workspace_size",
            "mamba2_mixer_forward", "ssd_status_string", "ssd_get_device_error", "ssd_version",
            "ssd_trace_enable", "ssd_trace_read", "ssd_prefill_noalloc", "ssd_varlen_workspace_size",
-           "ssd_prefill_varlen", "ssd_test_stall_scan")
+           "ssd_prefill_varlen", "ssd_test_stall_scan", "ssd_prefill_span_state", "ssd_span_prefix")
 NOALLOC_WORKSPACE_BYTES = 64 << 20
 
 _lib = None
@@ -119,6 +119,10 @@ def load(path: str = LIB_PATH):
                                        ctypes.POINTER(c_int), c_int, vp]
     lib.ssd_prefill_noalloc.restype = c_int
     lib.ssd_prefill_noalloc.argtypes = [ctypes.POINTER(SsdConfig), ctypes.POINTER(PrefillArgs), vp]
+    lib.ssd_prefill_span_state.restype = c_int
+    lib.ssd_prefill_span_state.argtypes = [ctypes.POINTER(SsdConfig), ctypes.POINTER(PrefillArgs), vp, vp, vp]
+    lib.ssd_span_prefix.restype = c_int
+    lib.ssd_span_prefix.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int, vp, vp, vp, vp]
     lib.ssd_test_stall_scan.restype = None
     lib.ssd_test_stall_scan.argtypes = [c_int, ctypes.c_ulonglong]
     lib.ssd_trace_enable.restype = c_int
@@ -297,6 +301,48 @@ def prefill_varlen(cfg: dict, cu_seqlens, xBC, dt, A, D, dt_bias, conv_w=None, c
     _check(lib.ssd_prefill_varlen(ctypes.byref(c), ctypes.byref(a), cu_arr, nseq, _stream(stream)),
            "ssd_prefill_varlen")
     return y, h_final, cso
+
+
+def prefill_span_state(cfg: dict, xBC, dt, A, dt_bias, conv_w=None, conv_b=None, conv_state_in=None,
+                       *, span_state=None, span_decay=None, workspace=None, stream=None,
+                       kernel: int | None = None):
+    """ssd_prefill_span_state: the state this span's tokens produce from a zero state and their
+    total decay; returns (span_state [B, H, P, N], span_decay [B, H])."""
+    import torch
+    lib = load()
+    Bn, L = xBC.shape[0], xBC.shape[1]
+    c = make_config(cfg, seqlen=L, kernel=kernel)
+    dev = xBC.device
+    if span_state is None:
+        span_state = torch.empty((Bn, c.nheads, c.headdim, c.dstate), dtype=torch.float32, device=dev)
+    if span_decay is None:
+        span_decay = torch.empty((Bn, c.nheads), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(lib.ssd_workspace_size(ctypes.byref(c)), dev)
+    a = PrefillArgs(
+        xBC=_ptr(xBC), xBC_row_stride=_row_stride(xBC), dt=_ptr(dt), dt_row_stride=_row_stride(dt),
+        A=_ptr(A), dt_bias=_ptr(dt_bias), conv_w=_ptr(conv_w), conv_b=_ptr(conv_b),
+        conv_state_in=_ptr(conv_state_in), workspace=_ptr(workspace), workspace_bytes=workspace.numel())
+    _check(lib.ssd_prefill_span_state(ctypes.byref(c), ctypes.byref(a), _ptr(span_state), _ptr(span_decay),
+                                      _stream(stream)), "ssd_prefill_span_state")
+    return span_state, span_decay
+
+
+def span_prefix(span_states, span_decays, h0=None, *, h_in=None, h_final=None, want_h_in=True,
+                want_h_final=True, stream=None):
+    """ssd_span_prefix over gathered span states [S, B, H, P, N] and decays [S, B, H]; returns
+    (h_in [S, B, H, P, N] or None, h_final [B, H, P, N] or None)."""
+    import torch
+    lib = load()
+    S, Bn, H, P, N = span_states.shape
+    if want_h_in and h_in is None:
+        h_in = torch.empty_like(span_states)
+    if want_h_final and h_final is None:
+        h_final = torch.empty((Bn, H, P, N), dtype=torch.float32, device=span_states.device)
+    _check(lib.ssd_span_prefix(_ptr(span_states), _ptr(span_decays), S, Bn, H, P, N, _ptr(h0),
+                               _ptr(h_in) if want_h_in else None, _ptr(h_final) if want_h_final else None,
+                               _stream(stream)), "ssd_span_prefix")
+    return (h_in if want_h_in else None), (h_final if want_h_final else None)
 
 
 def decode_step(cfg: dict, xBC_t, dt_t, A, D, dt_bias, conv_w, conv_b, state, conv_state_in,
