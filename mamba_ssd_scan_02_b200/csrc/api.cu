@@ -5,6 +5,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -238,13 +239,33 @@ struct SpanOut {
   float *decay;  // [B, H]
 };
 
+// Variable-length batch in one pass (tensor path): nseq sequences packed back to back, with
+// host offsets cu_host[0..nseq]; the plan is that of a batch of nseq rows of the longest
+// length, whose row b reads and writes the packed rows of sequence b (PrefillPlan::cu).
+struct VarlenIn {
+  const int *cu_host;
+  int nseq, Lmax;
+  long long total;
+};
+
+// Workspace of the one-pass variable-length prefill: the plan's layout, then the device copy
+// of the offsets.
+size_t varlen_cu_offset(const ssd_config_t *cv) { return round_up(prefill_layout(cv).total, kAlign); }
+
 ssd_status_t run_prefill(const ssd_config_t *c_in, const ssd_prefill_args_t *a, cudaStream_t s,
-                         const SpanOut *span = nullptr) {
+                         const SpanOut *span = nullptr, const VarlenIn *vl = nullptr) {
   ssd_config_t c_span;
   const ssd_config_t *c = c_in;
   if (span && c_in) {  // the norm does not touch the state
     c_span = *c_in;
     c_span.norm_groups = 0;
+    c = &c_span;
+  }
+  if (vl && c_in) {  // nseq rows of the longest length, one internal segment per sequence
+    c_span = *c_in;
+    c_span.batch = vl->nseq;
+    c_span.seqlen = vl->Lmax;
+    c_span.n_segments = 1;
     c = &c_span;
   }
   ssd_status_t st = check_config(c, true);
@@ -254,7 +275,8 @@ ssd_status_t run_prefill(const ssd_config_t *c_in, const ssd_prefill_args_t *a, 
   const int H = c->nheads, P = c->headdim, N = c->dstate, G = c->ngroups, W = c->conv_width;
   const long long d_inner = (long long)H * P, conv_dim = d_inner + 2LL * G * N;
   const size_t es = elt_size(c->io_dtype);
-  const bool has_tokens = c->seqlen > 0;
+  const long long rows = vl ? vl->total : (long long)c->batch * c->seqlen;  // token rows
+  const bool has_tokens = rows > 0;
   if (has_tokens) {
     if (!a->xBC || !a->dt || !a->A || !a->dt_bias || (!span && (!a->D || !a->y))) return SSD_ERR_INVALID_ARG;
     if (W > 0 && !a->conv_w) return SSD_ERR_INVALID_ARG;
@@ -292,6 +314,7 @@ ssd_status_t run_prefill(const ssd_config_t *c_in, const ssd_prefill_args_t *a, 
     p.cso = nullptr;
   }
   p.err = device_error_ptr();
+  p.rows = rows;
   p.stall_chunk1 = g_stall_chunk1.load();
   p.stall_wait_ns = g_stall_wait_ns.load();
 
@@ -312,11 +335,19 @@ ssd_status_t run_prefill(const ssd_config_t *c_in, const ssd_prefill_args_t *a, 
 
   const bool use_tc = prefill_uses_tc(c);
   if (use_tc && (!p.bf16 || !tc_scan_available())) return SSD_ERR_UNSUPPORTED;
+  if (vl && (!use_tc || !front_tc_fusable(p))) return SSD_ERR_UNSUPPORTED;
   const WsLayout lay = prefill_layout(c);
-  if (a->workspace_bytes < lay.total || (lay.total && !a->workspace) ||
+  const size_t ws_need = vl ? varlen_cu_offset(c) + (size_t)(vl->nseq + 1) * sizeof(int) : lay.total;
+  if (a->workspace_bytes < ws_need || (ws_need && !a->workspace) ||
       (reinterpret_cast<uintptr_t>(a->workspace) % kAlign) != 0)
     return SSD_ERR_WORKSPACE;
   char *ws = static_cast<char *>(a->workspace);
+  if (vl) {  // the offsets on the device (a pageable host source is staged before the return)
+    int *cu_dev = reinterpret_cast<int *>(ws + varlen_cu_offset(c));
+    SSD_TRY(cudaMemcpyAsync(cu_dev, vl->cu_host, (size_t)(vl->nseq + 1) * sizeof(int),
+                            cudaMemcpyHostToDevice, s));
+    p.cu = cu_dev;
+  }
 
   if (use_tc) {
     tc_segments(c, &p.n_seg, &p.seg_len);
@@ -335,8 +366,8 @@ ssd_status_t run_prefill(const ssd_config_t *c_in, const ssd_prefill_args_t *a, 
     p.tail_dec = p.h_final ? p.tail_dh + (size_t)c->batch * c->nheads * c->headdim * c->dstate : nullptr;
     // The outgoing conv cache may be written before the scan unless it overlaps an input
     // that later kernels read.
-    const size_t x_span = ((size_t)c->batch * c->seqlen - 1) * (size_t)a->xBC_row_stride * es + (size_t)conv_dim * es;
-    const size_t z_span = a->z ? ((size_t)c->batch * c->seqlen - 1) * (size_t)a->z_row_stride * es + (size_t)d_inner * es : 0;
+    const size_t x_span = ((size_t)rows - 1) * (size_t)a->xBC_row_stride * es + (size_t)conv_dim * es;
+    const size_t z_span = a->z ? ((size_t)rows - 1) * (size_t)a->z_row_stride * es + (size_t)d_inner * es : 0;
     const bool fused = front_tc_fusable(p);
     const bool cso_early = fused && !(a->conv_state_out && (ranges_overlap(a->conv_state_out, cache_bytes, a->xBC, x_span) ||
                                                             (a->z && ranges_overlap(a->conv_state_out, cache_bytes, a->z, z_span))));
@@ -556,8 +587,17 @@ ssd_status_t ssd_decode_step(const ssd_config_t *cfg, const ssd_decode_args_t *a
   return run_decode(cfg, args, static_cast<cudaStream_t>(stream));
 }
 
-// Variable-length batch: each packed sequence is one batch-1 prefill on the same stream,
-// its token tensors addressed at the sequence's first row and its carries at its index.
+// Variable-length batch.  On the tensor path (bf16, shapes the fused front end takes) it is one
+// pass: the front end, the scan (a CTA per (sequence, head)), the tail pass and the norm each
+// launch once for all the packed sequences.  Otherwise each packed sequence is one batch-1
+// prefill on the same stream, its token tensors addressed at the sequence's first row and its
+// carries at its index.
+static VarlenIn varlen_in(const int *cu, int nseq) {
+  VarlenIn v{cu, nseq, 0, cu[nseq]};
+  for (int i = 0; i < nseq; ++i) v.Lmax = std::max(v.Lmax, cu[i + 1] - cu[i]);
+  return v;
+}
+
 static bool varlen_ok(const ssd_config_t *cfg, const int *cu, int nseq) {
   if (!cfg || !cu || nseq < 1 || cfg->batch != 1 || cu[0] != 0 || cu[nseq] != cfg->seqlen) return false;
   for (int i = 0; i < nseq; ++i)
@@ -568,6 +608,12 @@ static bool varlen_ok(const ssd_config_t *cfg, const int *cu, int nseq) {
 size_t ssd_varlen_workspace_size(const ssd_config_t *cfg, const int *cu_seqlens, int nseq) {
   if (!varlen_ok(cfg, cu_seqlens, nseq) || check_config(cfg, true) != SSD_OK) return 0;
   size_t ws = 0;
+  if (prefill_uses_tc(cfg)) {  // the one-pass layout (the call may still take the loop)
+    const VarlenIn v = varlen_in(cu_seqlens, nseq);
+    ssd_config_t cv = *cfg;
+    cv.batch = nseq; cv.seqlen = v.Lmax; cv.n_segments = 1;
+    ws = varlen_cu_offset(&cv) + (size_t)(nseq + 1) * sizeof(int);
+  }
   for (int i = 0; i < nseq; ++i) {
     ssd_config_t c = *cfg;
     c.seqlen = cu_seqlens[i + 1] - cu_seqlens[i];
@@ -587,6 +633,11 @@ ssd_status_t ssd_prefill_varlen(const ssd_config_t *cfg, const ssd_prefill_args_
   const long long conv_dim = d_inner + 2LL * cfg->ngroups * cfg->dstate;
   const long long state = (long long)cfg->nheads * cfg->headdim * cfg->dstate;
   const long long cache = (long long)cfg->conv_width * conv_dim;
+  if (prefill_uses_tc(cfg)) {
+    const VarlenIn v = varlen_in(cu_seqlens, nseq);
+    st = run_prefill(cfg, args, static_cast<cudaStream_t>(stream), nullptr, &v);
+    if (st != SSD_ERR_UNSUPPORTED) return st;
+  }
   for (int i = 0; i < nseq; ++i) {
     ssd_config_t c = *cfg;
     const long long t0 = cu_seqlens[i];

@@ -20,6 +20,15 @@ __device__ __forceinline__ void latch_error(int *err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
+// ---- row geometry of a batch -----------------------------------------------------------------
+// A uniform batch stores batch row b's token t at row b*L + t.  A variable-length batch packs
+// its sequences back to back: sequence b is rows cu[b] .. cu[b+1]-1 (cu: device offsets, B + 1
+// of them) and L is the longest length, which sizes the grids.
+__device__ __forceinline__ long long seq_base(const int *cu, int b, int L) {
+  return cu ? (long long)cu[b] : (long long)b * L;
+}
+__device__ __forceinline__ int seq_len(const int *cu, int b, int L) { return cu ? cu[b + 1] - cu[b] : L; }
+
 // ---- element loads / stores in the io dtype ------------------------------------------------
 template <typename T> struct io;
 template <> struct io<float> {

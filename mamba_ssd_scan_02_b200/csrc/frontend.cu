@@ -116,12 +116,13 @@ __device__ __forceinline__ void dt_cumsum_tile(const T *__restrict__ dt, long lo
                                                const float *__restrict__ A, float *__restrict__ dte,
                                                float *__restrict__ cs, int L, int H, int Lpad, int sp,
                                                float lo, float hi, int c0, int h0, int b, int tid,
-                                               float (*v)[9], bool active) {
+                                               float (*v)[9], bool active, const int *cu = nullptr) {
   const int warp = tid / 32, lane = tid % 32;
   if (active) {
     const int tt = c0 + tid;
     float raw[8];
-    const T *row = dt + ((long long)b * L + tt) * ds + h0;
+    const T *row = dt + (seq_base(cu, b, L) + tt) * ds + h0;
+    L = seq_len(cu, b, L);  // this row's tokens; the tile's others are padding (dt = 0)
     if (tt < L && sizeof(T) == 2 && (H % 8) == 0 && (ds % 8) == 0) {
       load8(reinterpret_cast<const __nv_bfloat16 *>(row), raw);
     } else {
@@ -179,7 +180,7 @@ template <int ELT>
 __device__ __forceinline__ void conv_state_out_range(const char *__restrict__ xBC, long long xs_bytes,
                                                      const char *__restrict__ csi, char *__restrict__ cso,
                                                      int B, int L, int W, int C, long long i0,
-                                                     long long stride) {
+                                                     long long stride, const int *cu = nullptr) {
   const long long row_bytes = (long long)C * ELT;
   const long long vec_per_row = row_bytes / 16;
   const long long n = (long long)B * W * vec_per_row;
@@ -187,10 +188,10 @@ __device__ __forceinline__ void conv_state_out_range(const char *__restrict__ xB
     const long long v = i % vec_per_row;
     const int k = (int)((i / vec_per_row) % W);
     const int b = (int)(i / (vec_per_row * W));
-    const int tau = L - W + k;
+    const int tau = seq_len(cu, b, L) - W + k;
     uint4 val = make_uint4(0, 0, 0, 0);
     if (tau >= 0)
-      val = *reinterpret_cast<const uint4 *>(xBC + ((long long)b * L + tau) * xs_bytes + v * 16);
+      val = *reinterpret_cast<const uint4 *>(xBC + (seq_base(cu, b, L) + tau) * xs_bytes + v * 16);
     else if (csi)
       val = *reinterpret_cast<const uint4 *>(csi + ((long long)b * W + (W + tau)) * row_bytes + v * 16);
     *reinterpret_cast<uint4 *>(cso + ((long long)b * W + k) * row_bytes + v * 16) = val;
@@ -200,10 +201,10 @@ __device__ __forceinline__ void conv_state_out_range(const char *__restrict__ xB
 template <int ELT>
 __global__ void conv_state_out_kernel(const char *__restrict__ xBC, long long xs_bytes,
                                       const char *__restrict__ csi, char *__restrict__ cso, int B,
-                                      int L, int W, int C) {
+                                      int L, int W, int C, const int *cu) {
   conv_state_out_range<ELT>(xBC, xs_bytes, csi, cso, B, L, W, C,
                             blockIdx.x * (long long)blockDim.x + threadIdx.x,
-                            (long long)gridDim.x * blockDim.x);
+                            (long long)gridDim.x * blockDim.x, cu);
 }
 
 // seqlen == 0: the state passes through unchanged and so does the conv cache.
@@ -288,14 +289,16 @@ __device__ __forceinline__ void bc_conv_tile(const __nv_bfloat16 *__restrict__ x
                                              const __nv_bfloat16 *__restrict__ w,
                                              const __nv_bfloat16 *__restrict__ bias,
                                              __half *__restrict__ out, int L, int conv_dim, int c_begin,
-                                             int C_out, int bx, int by, int bz) {
+                                             int C_out, int bx, int by, int bz, const int *cu = nullptr) {
   const int o4 = (bx * kBcThreads + threadIdx.x) * 4;
   if (o4 >= C_out) return;
   const int c4 = c_begin + o4;
   const int b = bz;
   const int t0 = by * kBcTok;
-  const int t1 = min(L, t0 + kBcTok);
-  const __nv_bfloat16 *xrow = xBC + (long long)b * L * xs + c4;
+  const int t1 = min(seq_len(cu, b, L), t0 + kBcTok);
+  if (t0 >= t1) return;  // past this row's tokens (a shorter sequence of a packed batch)
+  const long long rb = seq_base(cu, b, L);
+  const __nv_bfloat16 *xrow = xBC + rb * xs + c4;
   float wt[4][4], bs[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -352,7 +355,7 @@ __device__ __forceinline__ void bc_conv_tile(const __nv_bfloat16 *__restrict__ x
         x1[i] = x0[i];
       }
       const __half2 h01 = __floats2half2_rn(r[0], r[1]), h23 = __floats2half2_rn(r[2], r[3]);
-      *reinterpret_cast<uint2 *>(out + ((long long)b * L + t) * C_out + o4) =
+      *reinterpret_cast<uint2 *>(out + (rb + t) * C_out + o4) =
           make_uint2(*reinterpret_cast<const uint32_t *>(&h01), *reinterpret_cast<const uint32_t *>(&h23));
     }
   };
@@ -388,6 +391,7 @@ struct FrontArgs {
   int B, L, H, Lpad, conv_dim, d_inner, C_out, W, sp;
   float lo, hi;
   int n_dt, dt_tiles, dt_nch, dt_nhg, n_cso, gx, gy;
+  const int *cu;  // packed variable-length batch offsets (device), or null
 };
 
 template <int W>
@@ -400,19 +404,19 @@ __global__ void __launch_bounds__(kBcThreads) front_tc_kernel(const FrontArgs f)
     const int qq = active ? q : 0;
     const int cx = qq % f.dt_nch, hy = (qq / f.dt_nch) % f.dt_nhg, b = qq / (f.dt_nch * f.dt_nhg);
     dt_cumsum_tile<__nv_bfloat16>(f.dt, f.ds, f.dt_bias, f.A, f.dte, f.cs, f.L, f.H, f.Lpad, f.sp, f.lo,
-                                  f.hi, cx * 128, hy * 8, b, threadIdx.x & 127, v[half], active);
+                                  f.hi, cx * 128, hy * 8, b, threadIdx.x & 127, v[half], active, f.cu);
     return;
   }
   j -= f.n_dt;
   if (j < f.n_cso) {
     conv_state_out_range<2>((const char *)f.xBC, f.xs * 2, (const char *)f.csi, (char *)f.cso, f.B, f.L,
                             f.W, f.conv_dim, j * (long long)kBcThreads + threadIdx.x,
-                            (long long)f.n_cso * kBcThreads);
+                            (long long)f.n_cso * kBcThreads, f.cu);
     return;
   }
   j -= f.n_cso;
   bc_conv_tile<W>(f.xBC, f.xs, f.csi, f.conv_w, f.conv_b, f.bc, f.L, f.conv_dim, f.d_inner, f.C_out,
-                  j % f.gx, (j / f.gx) % f.gy, j / (f.gx * f.gy));
+                  j % f.gx, (j / f.gx) % f.gy, j / (f.gx * f.gy), f.cu);
 }
 
 cudaError_t launch_bc_conv_f16(const PrefillPlan &p, cudaStream_t s) {
@@ -451,6 +455,7 @@ cudaError_t launch_front_tc(const PrefillPlan &p, bool with_cso, cudaStream_t s)
   f.dte = p.dte_hm; f.cs = p.cs_hm; f.bc = (__half *)p.bc; f.cso = (__nv_bfloat16 *)p.cso;
   f.B = p.B; f.L = p.L; f.H = p.H; f.Lpad = p.Lpad; f.conv_dim = p.conv_dim; f.d_inner = p.d_inner;
   f.C_out = 2 * p.G * p.N; f.W = p.W; f.sp = p.softplus; f.lo = p.dt_min; f.hi = p.dt_max;
+  f.cu = p.cu;
   f.dt_nch = p.Lpad / 128; f.dt_nhg = (p.H + 7) / 8; f.dt_tiles = f.dt_nch * f.dt_nhg * p.B;
   f.n_dt = (f.dt_tiles + 1) / 2;
   const long long ncso = (with_cso && p.cso && p.W > 0) ? (long long)p.B * p.W * ((long long)p.conv_dim * 2 / 16) : 0;
@@ -498,10 +503,10 @@ cudaError_t launch_conv_state_out(const PrefillPlan &p, cudaStream_t s) {
   const int g = grid_for(n, 256);
   if (p.bf16)
     conv_state_out_kernel<2><<<g, 256, 0, s>>>((const char *)p.xBC, p.xs * 2, (const char *)p.csi,
-                                                (char *)p.cso, p.B, p.L, p.W, p.conv_dim);
+                                                (char *)p.cso, p.B, p.L, p.W, p.conv_dim, p.cu);
   else
     conv_state_out_kernel<4><<<g, 256, 0, s>>>((const char *)p.xBC, p.xs * 4, (const char *)p.csi,
-                                                (char *)p.cso, p.B, p.L, p.W, p.conv_dim);
+                                                (char *)p.cso, p.B, p.L, p.W, p.conv_dim, p.cu);
   return cudaGetLastError();
 }
 

@@ -178,7 +178,7 @@ cudaError_t launch_norm_rescale(const PrefillPlan &p, cudaStream_t s) {
   const int hpn = p.H / p.norm_groups;
   const size_t smem = (size_t)(2 * p.H + p.norm_groups) * sizeof(float);
   if (smem > 48 * 1024) return cudaErrorInvalidValue;
-  norm_rescale_kernel<<<(unsigned)((long long)p.B * p.L), kRescaleThreads, smem, s>>>(
+  norm_rescale_kernel<<<(unsigned)p.rows, kRescaleThreads, smem, s>>>(
       p.qn, p.ssq, (const __nv_bfloat16 *)p.z, p.zs, (const __nv_bfloat16 *)p.norm_w,
       (__nv_bfloat16 *)p.y, p.ys, p.H, hpn, p.norm_groups, p.d_inner, p.eps, p.nbg);
   return cudaGetLastError();
@@ -186,7 +186,7 @@ cudaError_t launch_norm_rescale(const PrefillPlan &p, cudaStream_t s) {
 
 cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s) {
   const int gs = p.d_inner / p.norm_groups;
-  dim3 grid((unsigned)((long long)p.B * p.L), p.norm_groups);
+  dim3 grid((unsigned)p.rows, p.norm_groups);
   const bool v8 = p.bf16 && gs % 256 == 0 && gs / 8 <= 1024 &&  // whole warps of 8 channels
                   (reinterpret_cast<uintptr_t>(p.norm_w) & 15u) == 0;
   if (v8)

@@ -12,6 +12,12 @@ namespace ssd {
 // Everything a prefill launch needs, after validation: shapes, pointers, workspace carve-outs.
 struct PrefillPlan {
   int B, L, H, P, N, G, Q, W, norm_groups;
+  // Variable-length batch (tensor path): the B sequences are packed back to back, sequence b
+  // being rows cu[b] .. cu[b+1]-1 of every token tensor (cu: device, B + 1 offsets), and L is
+  // the longest length; null for a uniform batch (row b*L + t).  rows = the number of token
+  // rows (B*L, or cu[B]).
+  const int *cu;
+  long long rows;
   int nbg;           // 1: normalise before gating (out = rmsnorm(y) * w * silu(z))
   int hpg, d_inner, conv_dim;
   float eps, dt_min, dt_max;

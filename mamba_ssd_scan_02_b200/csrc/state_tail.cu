@@ -55,20 +55,28 @@ __global__ void __launch_bounds__(kTailThreads) state_tail_kernel(
     const __nv_bfloat16 *__restrict__ conv_b, const __nv_bfloat16 *__restrict__ csi,
     const float *__restrict__ dte, const float *__restrict__ cs, float *__restrict__ dh_out,
     float *__restrict__ dec_out, int L, int B, int H, int hpg, int conv_dim, int d_inner, int W,
-    int Lpad, int t_tail) {
+    int Lpad, int t_tail_uniform, const int *__restrict__ cu) {
   extern __shared__ __align__(16) unsigned char tsm[];
   __nv_bfloat16 *raw = reinterpret_cast<__nv_bfloat16 *>(tsm);       // [kRawRows][192]
   float *uo = reinterpret_cast<float *>(tsm + kRawBytes);             // [128][192]
   float *ws = reinterpret_cast<float *>(tsm + kRawBytes + kOutBytes);  // [256]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int p0 = 16 * (warp >> 2) + 4 * (lane >> 3), n0 = 32 * (warp & 3) + 4 * (lane & 7);
-  const int ntok = L - t_tail;  // 1 .. kTailMax
   // conv role: channel ch (column of raw / uo), token half hf of each chunk; tap j reads time t-3+j
   const bool conv_thread = tid < kConvThreads;
   const int ch = tid % kTailCh, hf = tid / kTailCh;
   for (int item = blockIdx.x; item < B * H; item += gridDim.x) {
     const int h = item % H, b = item / H, g = h / hpg;
-    const __nv_bfloat16 *xrow = xBC + (long long)b * L * xs;
+    // this row's tokens and tail (a packed variable-length batch has one segment per sequence,
+    // its tail the last two chunks of the sequence)
+    const int Lb = seq_len(cu, b, L);
+    int t_tail = t_tail_uniform;
+    if (cu) {
+      const int nckb = (Lb + 127) / 128;
+      t_tail = 128 * (nckb > kTailChunks ? nckb - kTailChunks : 0);
+    }
+    const int ntok = Lb - t_tail;  // 0 .. kTailMax
+    const __nv_bfloat16 *xrow = xBC + seq_base(cu, b, L) * xs;
     const float *csr = cs + ((long long)b * H + h) * Lpad;
     const float *dtr = dte + ((long long)b * H + h) * Lpad;
 
@@ -183,7 +191,7 @@ cudaError_t launch_state_tail(const PrefillPlan &p, cudaStream_t s) {
   state_tail_kernel<<<(unsigned)grid, kTailThreads, kTailSmem, s>>>(
       (const __nv_bfloat16 *)p.xBC, p.xs, (const __nv_bfloat16 *)p.conv_w, (const __nv_bfloat16 *)p.conv_b,
       (const __nv_bfloat16 *)p.csi, p.dte_hm, p.cs_hm, p.tail_dh, p.tail_dec, p.L, p.B, p.H, p.hpg,
-      p.conv_dim, p.d_inner, p.W, p.Lpad, t_tail);
+      p.conv_dim, p.d_inner, p.W, p.Lpad, t_tail, p.cu);
   return cudaGetLastError();
 }
 

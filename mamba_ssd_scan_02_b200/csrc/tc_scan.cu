@@ -160,6 +160,9 @@ struct TcArgs {
   unsigned long long wait_ns;  // limit of every bounded wait
   int debug_skip_chunk;        // test hook (-1 = off): the producer stops before loading this
                                // chunk's stage, so its consumers' bounded waits run out
+  const int *cu;               // packed variable-length batch: sequence b is token rows
+                               // cu[b] .. cu[b+1]-1 (the tensor maps then have one batch row
+                               // of all the tokens); null: row b*L + t
 };
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -253,7 +256,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z, g = h / a.hpg;
   const int t_begin = seg * a.seg_len;
-  const int t_end = min(a.L, t_begin + a.seg_len);
+  const int t_end = min(seq_len(a.cu, b, a.L), t_begin + a.seg_len);
+  // TMA coordinates of this row's token t: (t + tma_t0, batch tma_b)
+  const int tma_t0 = a.cu ? a.cu[b] : 0, tma_b = a.cu ? 0 : b;
   const int nck = t_end > t_begin ? (t_end - t_begin + QC - 1) / QC : 0;
   const int last = nck - 1;
   // The last chunk's exact path (fp32 SiLU, split-precision w o X) serves only the final
@@ -301,7 +306,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const int t0 = t_begin + k * QC;
         if (k >= 2 && !mbar_wait(BAR(BAR_XWFREE0 + xb), ((k >> 1) - 1) & 1, abort_flag, a.err, lim)) break;
         mbar_arrive_expect_tx(BAR(BAR_FULLX0 + xb), kRawRows * 128);
-        tma_load_3d(sb + OFF_XW + xb * kXBuf, &tm_x, h * 64, t0 - 3, b, BAR(BAR_FULLX0 + xb));
+        tma_load_3d(sb + OFF_XW + xb * kXBuf, &tm_x, h * 64, tma_t0 + t0 - 3, tma_b, BAR(BAR_FULLX0 + xb));
         ++nx;
         if (a.debug_skip_chunk == k) break;  // test hook: stage k never arrives (see TcArgs)
         if (k >= 2 && !mbar_wait(BAR(BAR_EMPTY0 + st), ((k >> 1) - 1) & 1, abort_flag, a.err, lim)) break;
@@ -311,11 +316,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         mbar_arrive_expect_tx(full, (kStateOnly ? 2 * kTile : 4 * kTile) + 1024);
         const int cB = g * 128, cC = a.G * 128 + g * 128;
         if (!kStateOnly) {
-          tma_load_3d(sst + OFF_C, &tm_bc, cC, t0, b, full);
-          tma_load_3d(sst + OFF_C + kTile, &tm_bc, cC + 64, t0, b, full);
+          tma_load_3d(sst + OFF_C, &tm_bc, cC, tma_t0 + t0, tma_b, full);
+          tma_load_3d(sst + OFF_C + kTile, &tm_bc, cC + 64, tma_t0 + t0, tma_b, full);
         }
-        tma_load_3d(sst + OFF_B, &tm_bc, cB, t0, b, full);
-        tma_load_3d(sst + OFF_B + kTile, &tm_bc, cB + 64, t0, b, full);
+        tma_load_3d(sst + OFF_B, &tm_bc, cB, tma_t0 + t0, tma_b, full);
+        tma_load_3d(sst + OFF_B + kTile, &tm_bc, cB + 64, tma_t0 + t0, tma_b, full);
         const long long hoff = ((long long)b * a.H + h) * a.Lpad + t0;
         bulk_load(sst + OFF_DT, a.dte + hoff, 512, full);
         bulk_load(sst + OFF_CS, a.cs + hoff, 512, full);
@@ -793,7 +798,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       if (!kStateOnly) {
         const int tok = t_begin + k * QC + n;
-        const long long row = (long long)b * a.L + tok;
+        const long long row = seq_base(a.cu, b, a.L) + tok;
         // fused gate (gate first): this row's z (64 channels, 128 bytes) is prefetched into L1
         // before the wait for the chunk's products
         const bool gate = a.qn != nullptr && !a.nbg;
@@ -960,8 +965,10 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap tm;
   const cuuint64_t C2 = 2ull * p.G * p.N;
-  cuuint64_t dims[3] = {C2, (cuuint64_t)p.L, (cuuint64_t)p.B};
-  cuuint64_t strides[2] = {C2 * 2, C2 * 2 * (cuuint64_t)p.L};
+  // a packed variable-length batch is one batch row of all its tokens
+  const cuuint64_t T = p.cu ? (cuuint64_t)p.rows : (cuuint64_t)p.L, NB = p.cu ? 1 : (cuuint64_t)p.B;
+  cuuint64_t dims[3] = {C2, T, NB};
+  cuuint64_t strides[2] = {C2 * 2, C2 * 2 * T};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, p.bc, dims, strides, box, estr,
@@ -970,8 +977,8 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   // raw x rows of one head: box of 64 channels x (128 + 3) tokens of the bf16 input
   CUtensorMap tmx;
-  cuuint64_t xdims[3] = {(cuuint64_t)p.conv_dim, (cuuint64_t)p.L, (cuuint64_t)p.B};
-  cuuint64_t xstrides[2] = {(cuuint64_t)p.xs * 2, (cuuint64_t)p.xs * 2 * (cuuint64_t)p.L};
+  cuuint64_t xdims[3] = {(cuuint64_t)p.conv_dim, T, NB};
+  cuuint64_t xstrides[2] = {(cuuint64_t)p.xs * 2, (cuuint64_t)p.xs * 2 * T};
   cuuint32_t xbox[3] = {64, kRawRows, 1};
   r = enc(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(p.xBC), xdims, xstrides, xbox,
           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -993,6 +1000,7 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
   a.wait_ns = p.stall_chunk1 > 0 ? p.stall_wait_ns : tc::kWaitLimitNs;
   a.debug_skip_chunk = p.stall_chunk1 - 1;
   a.d_inner = p.d_inner;
+  a.cu = p.cu;
   const long long seg_stride = (long long)p.B * p.H * p.P * p.N;
   dim3 grid(p.n_seg, p.H, p.B);
   cudaError_t e;

@@ -68,3 +68,58 @@ def test_varlen_equals_separate_calls(cuda_lib):
                                  dev(inp["z"][:, a:b]), dev(inp["norm_w"]), dev(inp["h0"][i:i + 1]),
                                  dev(inp["conv_state_in"][i:i + 1]))
         assert torch.equal(yi[0], y[a:b]) and torch.equal(hi[0], hf[i]) and torch.equal(ci[0], cso[i])
+
+
+def test_varlen_is_one_pass(cuda_lib):
+    """On the tensor path the packed batch is one front end, one scan, one tail pass and one
+    norm launch, whatever the number of sequences."""
+    from mamba_ssd_scan_02_b200 import ssd
+    cfg, cu, inp = _case()
+    ssd.trace_enable(True)
+    ssd.trace_read()
+    try:
+        _gpu(cfg, cu, inp)
+        names = [n for n, _ in ssd.trace_read()]
+    finally:
+        ssd.trace_enable(False)
+    for k in ("ssd_front", "ssd_scan_tc", "ssd_state_tail", "ssd_norm_rescale"):
+        assert names.count(k) == 1, names
+
+
+def test_many_short_sequences_at_full_width(cuda_lib, oracle):
+    """64 packed sequences of 1 to 700 tokens at the 8k layer's width (128 heads, 8 groups):
+    bit-exact against one ssd_prefill call per sequence, and the oracle on three of them."""
+    import torch
+    from mamba_ssd_scan_02_b200 import ssd
+    rng = np.random.default_rng(datagen.SEED_BASE + 64)
+    lens = rng.integers(1, 701, 64)
+    lens[5], lens[17] = 1, 128
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(int)
+    T, nseq = int(cu[-1]), len(lens)
+    cfg = dict(datagen.config(1), batch=1, seqlen=T)
+    inp = datagen.make_inputs(1, cfg)
+    H, P, N, W = cfg["nheads"], cfg["headdim"], cfg["dstate"], cfg["conv_width"]
+    seed = datagen.SEED_BASE + 301
+    h0 = datagen.random_state(seed, (nseq, H, P, N))
+    csi = datagen.random_conv_state(seed, (nseq, W, datagen.conv_dim(cfg)))
+    d = {k: dev(inp[k]) for k in ("A", "D", "dt_bias", "conv_w")}
+    x, dtt = dev(inp["xBC"][0]), dev(inp["dt"][0])
+    y, hf, cso = ssd.prefill_varlen(cfg, cu, x, dtt, d["A"], d["D"], d["dt_bias"], d["conv_w"], None,
+                                    None, None, dev(h0), dev(csi))
+    for i in range(nseq):
+        a, b = int(cu[i]), int(cu[i + 1])
+        yi, hi, ci = ssd.prefill(dict(cfg, seqlen=b - a), x[None, a:b], dtt[None, a:b], d["A"], d["D"],
+                                 d["dt_bias"], d["conv_w"], None, None, None, dev(h0[i:i + 1]),
+                                 dev(csi[i:i + 1]))
+        assert torch.equal(yi[0], y[a:b]), f"seq {i} y"
+        assert torch.equal(hi[0], hf[i]) and torch.equal(ci[0], cso[i]), f"seq {i} carries"
+    yh = y.float().cpu().numpy()
+    for i in (0, 5, 40):
+        a, b = int(cu[i]), int(cu[i + 1])
+        sub = {k: inp[k] for k in ("A", "D", "dt_bias", "conv_w")}
+        sub.update(xBC=inp["xBC"][:, a:b], dt=inp["dt"][:, a:b], h0=h0[i:i + 1],
+                   conv_state_in=csi[i:i + 1], conv_b=None)
+        scfg = dict(cfg, seqlen=b - a)
+        ref = run_oracle_prefill(oracle, scfg, sub, heads=(0, 16))
+        assert_close(yh[a:b, :16 * P], oracle_output(ref, scfg)[0], TOL_BF16, f"seq {i} y", out_dtype="bf16")
+        assert_close(host(hf)[i, :16], ref["h_final"][0], TOL_BF16, f"seq {i} h_final")
