@@ -593,6 +593,72 @@ def bench_mixer(c: Ctx):
             "dominant_kernel": dom}
 
 
+def bench_varlen(c: Ctx, nseq=128):
+    """A packed batch of many short sequences (the 8k layer's shape: 128 heads, 8 groups), each
+    with its own state and conv cache: ssd_prefill_varlen (one pass) against one ssd_prefill
+    call per sequence on the same stream."""
+    torch, ssd, args = c.torch, c.ssd, c.args
+    rng = np.random.default_rng(datagen.SEED_BASE + 128)
+    lens = rng.integers(64, 1025, nseq)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(int)
+    T = int(cu[-1])
+    cfg = dict(datagen.config(1), batch=1, seqlen=T)
+    inp = datagen.make_inputs(1, cfg)
+    H, P, N, W = cfg["nheads"], cfg["headdim"], cfg["dstate"], cfg["conv_width"]
+    d = {k: ssd.to_device(inp[k]) for k in ("A", "D", "dt_bias", "conv_w")}
+    x, dtt = ssd.to_device(inp["xBC"][0]), ssd.to_device(inp["dt"][0])
+    del inp
+    seed = datagen.SEED_BASE + 129
+    h0 = ssd.to_device(datagen.random_state(seed, (nseq, H, P, N)))
+    csi = ssd.to_device(datagen.random_conv_state(seed, (nseq, W, datagen.conv_dim(cfg))))
+
+    def one_pass():
+        ssd.prefill_varlen(cfg, cu, x, dtt, d["A"], d["D"], d["dt_bias"], d["conv_w"], None, None,
+                           None, h0, csi)
+
+    ws = ssd.alloc_workspace(max(ssd.workspace_size(dict(cfg, seqlen=int(L))) for L in lens), c.dev)
+
+    def per_sequence():
+        for i in range(nseq):
+            a, b = int(cu[i]), int(cu[i + 1])
+            ssd.prefill(dict(cfg, seqlen=b - a), x[None, a:b], dtt[None, a:b], d["A"], d["D"],
+                        d["dt_bias"], d["conv_w"], None, None, None, h0[i:i + 1], csi[i:i + 1],
+                        workspace=ws)
+
+    res = {}
+    for name, fn in (("one_pass", one_pass), ("per_sequence_calls", per_sequence)):
+        for _ in range(args.warmup):
+            fn()
+        ms, recs, _ = c.timed(fn, args.steps, flush=True, trace=(name == "one_pass"))
+        res[name] = {"ms_per_step": round(ms / args.steps, 4),
+                     "tokens_per_s": round(job_throughput(T, c.world, args.steps, ms), 1)}
+        if name == "one_pass":
+            res[name]["gpu_launches_per_step"] = len(recs) / args.steps
+    return {"metric": METRIC, "workload": "varlen_128_short", "sequences": nseq, "tokens": T,
+            "lengths": "uniform 64..1024 (seeded)", "value": res["one_pass"]["tokens_per_s"],
+            "unit": "tokens/s", **res}
+
+
+def summarize(rec):
+    """The figures of a workload record that a reader needs first (None stays None)."""
+    if not rec:
+        return rec
+    out = {k: rec[k] for k in ("workload", "metric", "value", "unit", "ms_per_step") if k in rec}
+    rf = rec.get("roofline")
+    if rf:
+        out["roofline"] = {k: rf[k] for k in ("bound", "kernel", "kernel_ms", "achieved", "peak",
+                                              "unit", "frac", "traffic") if k in rf}
+    for k in ("layer_tflops", "tokens", "sequences"):
+        if k in rec:
+            out[k] = rec[k]
+    for k in ("one_pass", "per_sequence_calls"):
+        if k in rec:
+            out[k] = rec[k]
+    if "clocks" in rec:
+        out["clocks"] = {k: rec["clocks"][k] for k in ("sm_mhz", "reasons") if k in rec["clocks"]}
+    return out
+
+
 def cpu_baseline(target_s: float = 10.0):
     """fp64 oracle on a bounded sample of the prefill workload (a token prefix of whole norm
     groups of heads), scaled to tokens/s of the whole layer."""
@@ -690,7 +756,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true",
                     help="headline prefill only (no decode, long-context, mixer or CPU legs)")
-    ap.add_argument("--workload", choices=["all", "prefill", "decode", "long_context", "mixer"],
+    ap.add_argument("--workload", choices=["all", "prefill", "decode", "long_context", "mixer", "varlen"],
                     default="all", help="run one workload alone (for profiling); prints its object")
     ap.add_argument("--mixer-batch", type=int, default=8,
                     help="batch of the mixer workload (smaller only for profiling captures)")
@@ -718,7 +784,7 @@ def main():
     c = Ctx(args, torch, ssd, dist, rank, world, clk)
     if args.workload != "all":
         fn = {"prefill": bench_prefill, "decode": bench_decode, "long_context": bench_long_context,
-              "mixer": bench_mixer}[args.workload]
+              "mixer": bench_mixer, "varlen": bench_varlen}[args.workload]
         try:
             r = fn(c)
             r["device_status"] = ssd.get_device_error()
@@ -732,13 +798,15 @@ def main():
         return
     try:
         res = bench_prefill(c)
-        dec = lng = mix = None
+        dec = lng = mix = vln = None
         if not args.quick:
             dec = bench_decode(c)
             torch.cuda.empty_cache()
             lng = bench_long_context(c)
             torch.cuda.empty_cache()
             mix = bench_mixer(c)
+            torch.cuda.empty_cache()
+            vln = bench_varlen(c)
         status = ssd.get_device_error()
     finally:
         clk.stop()
@@ -756,9 +824,14 @@ def main():
         "config": dict(HEADLINE_CONFIG, parallelism=f"replicas x{world}"),
         "roofline": res["roofline"], "e2e": res["e2e"], "gpu_launches": res["gpu_launches"],
         "clocks": res["clocks"], "kernels": res["kernels"],
-        "path_bytes_per_step": res["path_bytes_per_step"], "decode": dec, "long_context": lng,
-        "mixer": mix, "cpu_baseline": cpu, "device_status": status,
+        "path_bytes_per_step": res["path_bytes_per_step"], "cpu_baseline": cpu,
+        "device_status": status,
     }
+    # The other workloads: their full records on stderr, a short summary of each at the end
+    # of the line (where a truncated tail of the output still shows them).
+    detail = {"decode": dec, "long_context": lng, "mixer": mix, "varlen": vln}
+    print(json.dumps({"detail": detail}), file=sys.stderr, flush=True)
+    line.update({k: summarize(v) for k, v in detail.items()})
     print(json.dumps(line))
 
 
