@@ -113,13 +113,9 @@ bool prefill_uses_tc(const ssd_config_t *c) {
   return c->io_dtype == SSD_BF16 && tc_scan_available();
 }
 
-// The tensor-core scan applies the z gate itself and leaves only a rescale for the group norm
-// when every norm group is made of whole heads (and the rescale's per-row factors fit in
-// shared memory); otherwise it writes the fp32 output and the separate gated norm follows.
-bool tc_fused_norm(const ssd_config_t *c) {
-  return c->io_dtype == SSD_BF16 && c->norm_groups > 0 && c->nheads % c->norm_groups == 0 &&
-         2LL * c->nheads + c->norm_groups <= 12 * 1024;
-}
+// On the tensor path the scan hands y to the gated norm in fp16 (2 bytes per channel): the
+// norm's pass reads it with z once, so the scan's output stage needs no memory read.
+bool tc_norm_f16(const ssd_config_t *c) { return c->io_dtype == SSD_BF16 && c->norm_groups > 0; }
 
 // The two scan paths use the workspace differently; the layouts overlap (a call uses one),
 // and the size asked for is that of the path the call takes.
@@ -127,7 +123,7 @@ struct WsLayout {
   // CUDA-core path
   size_t u, dte, yf, seg_state, seg_decay, simt_end;
   // tensor-core path
-  size_t tc_bc, tc_dte, tc_cs, tc_yf, tc_q, tc_ssq, tc_seg_state, tc_seg_decay, tc_dh, tc_end;
+  size_t tc_bc, tc_dte, tc_cs, tc_yf, tc_yh, tc_seg_state, tc_seg_decay, tc_dh, tc_end;
   int Lpad;
   size_t total;
 };
@@ -157,11 +153,9 @@ WsLayout prefill_layout(const ssd_config_t *c) {
   w.tc_bc = off;   off = round_up(off + T * 2 * c->ngroups * c->dstate * 2, kAlign);
   w.tc_dte = off;  off = round_up(off + (size_t)c->batch * c->nheads * w.Lpad * 4, kAlign);
   w.tc_cs = off;   off = round_up(off + (size_t)c->batch * c->nheads * w.Lpad * 4, kAlign);
-  w.tc_yf = w.tc_q = w.tc_ssq = off;
-  if (tc_fused_norm(c)) {
+  w.tc_yf = w.tc_yh = off;
+  if (tc_norm_f16(c)) {
     off = round_up(off + T * d_inner * 2, kAlign);
-    w.tc_ssq = off;
-    off = round_up(off + T * c->nheads * 4, kAlign);
   } else if (c->norm_groups > 0) {
     off = round_up(off + T * d_inner * 4, kAlign);
   }
@@ -355,11 +349,9 @@ ssd_status_t run_prefill(const ssd_config_t *c_in, const ssd_prefill_args_t *a, 
     p.bc = ws + lay.tc_bc;
     p.dte_hm = reinterpret_cast<float *>(ws + lay.tc_dte);
     p.cs_hm = reinterpret_cast<float *>(ws + lay.tc_cs);
-    const bool fused_norm = tc_fused_norm(c);
-    if (fused_norm && a->norm_w && !aligned16(a->norm_w)) return SSD_ERR_ALIGNMENT;
-    p.yf = c->norm_groups > 0 && !fused_norm ? reinterpret_cast<float *>(ws + lay.tc_yf) : nullptr;
-    p.qn = fused_norm ? reinterpret_cast<__half *>(ws + lay.tc_q) : nullptr;
-    p.ssq = fused_norm ? reinterpret_cast<float *>(ws + lay.tc_ssq) : nullptr;
+    const bool norm_f16 = tc_norm_f16(c);
+    p.yf = c->norm_groups > 0 && !norm_f16 ? reinterpret_cast<float *>(ws + lay.tc_yf) : nullptr;
+    p.yh = norm_f16 ? reinterpret_cast<__half *>(ws + lay.tc_yh) : nullptr;
     p.seg_state = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.tc_seg_state) : nullptr;
     p.seg_decay = p.n_seg > 1 ? reinterpret_cast<float *>(ws + lay.tc_seg_decay) : nullptr;
     p.tail_dh = p.h_final ? reinterpret_cast<float *>(ws + lay.tc_dh) : nullptr;
@@ -411,9 +403,7 @@ ssd_status_t run_prefill(const ssd_config_t *c_in, const ssd_prefill_args_t *a, 
       SSD_TRY(side.join());
       SSD_TRY(traced("ssd_tail_fold", s, [&] { return launch_tail_fold(p, s); }));
     }
-    if (p.qn) {
-      SSD_TRY(traced("ssd_norm_rescale", s, [&] { return launch_norm_rescale(p, s); }));
-    } else if (p.norm_groups > 0) {
+    if (p.norm_groups > 0) {
       SSD_TRY(traced("ssd_gated_norm", s, [&] { return launch_gated_norm(p, s); }));
     }
     if (!cso_early) SSD_TRY(traced("ssd_conv_state_out", s, [&] { return launch_conv_state_out(p, s); }));

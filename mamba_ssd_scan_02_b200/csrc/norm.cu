@@ -30,19 +30,25 @@ __device__ float block_sum(float v, float *red) {
   return red[0];
 }
 
-// One CTA per (row, norm group).  y is fp32 [rows, d_inner] dense; z/out/w in the io dtype.
-template <typename T>
+// y as the scan left it: fp32 (the CUDA-core path) or fp16 (the tensor-core path).
+__device__ __forceinline__ float ld_y(const float *p) { return *p; }
+__device__ __forceinline__ float ld_y(const __half *p) { return __half2float(*p); }
+
+// One CTA per (row, norm group).  y is [rows, d_inner] dense (YT: float or __half); z/out/w in
+// the io dtype.
+template <typename T, typename YT>
 __global__ void __launch_bounds__(kNormThreads) gated_norm_kernel(
-    const float *__restrict__ y, const T *__restrict__ z, long long zs, const T *__restrict__ w,
-    T *__restrict__ out, long long os, int d_inner, int gs, float eps, int L, int nbg) {
+    const YT *__restrict__ y, const T *__restrict__ z, long long zs, const T *__restrict__ w,
+    T *__restrict__ out, long long os, int d_inner, int gs, float eps, int nbg) {
   __shared__ float red[32];
   const long long row = blockIdx.x;
   const int c0 = blockIdx.y * gs;
-  const float *yr = y + row * d_inner + c0;
+  const YT *yr = y + row * d_inner + c0;
   const T *zr = z + row * zs + c0;
   float ss = 0.f;
   for (int i = threadIdx.x; i < gs; i += kNormThreads) {
-    const float gv = nbg ? yr[i] : yr[i] * silu(io<T>::ld(zr + i));
+    const float yv = ld_y(yr + i);
+    const float gv = nbg ? yv : yv * silu(io<T>::ld(zr + i));
     ss += gv * gv;
   }
   ss = block_sum(ss, red);
@@ -50,7 +56,8 @@ __global__ void __launch_bounds__(kNormThreads) gated_norm_kernel(
   T *orow = out + row * os + c0;
   for (int i = threadIdx.x; i < gs; i += kNormThreads) {
     const float sz = silu(io<T>::ld(zr + i));
-    const float gv = nbg ? yr[i] : yr[i] * sz;
+    const float yv = ld_y(yr + i);
+    const float gv = nbg ? yv : yv * sz;
     io<T>::st(orow + i, gv * r * (w ? io<T>::ld(w + c0 + i) : 1.f) * (nbg ? sz : 1.f));
   }
 }
@@ -82,20 +89,35 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_bf16_kernel(
 
 }  // namespace
 
+// 8 consecutive channels of y (streaming loads: each is read once)
+__device__ __forceinline__ void ld_y8(const float *p, float (&v)[8]) {
+  const float4 a = __ldcs(reinterpret_cast<const float4 *>(p)), b = __ldcs(reinterpret_cast<const float4 *>(p + 4));
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void ld_y8(const __half *p, float (&v)[8]) {
+  const uint4 u = __ldcs(reinterpret_cast<const uint4 *>(p));
+  const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
 // The same for bf16 tensors in one pass: a CTA of gs / 8 threads per (row, norm group), each
 // thread holding 8 consecutive channels in registers (16-byte loads and stores).
+template <typename YT>
 __global__ void __launch_bounds__(1024) gated_norm_v8_kernel(
-    const float *__restrict__ y, const __nv_bfloat16 *__restrict__ z, long long zs,
+    const YT *__restrict__ y, const __nv_bfloat16 *__restrict__ z, long long zs,
     const __nv_bfloat16 *__restrict__ w, __nv_bfloat16 *__restrict__ out, long long os, int d_inner,
     int gs, float eps, int nbg) {
   __shared__ float red[32];
   const long long row = blockIdx.x;
   const int c = blockIdx.y * gs + 8 * threadIdx.x;
-  const float4 ya = __ldcs(reinterpret_cast<const float4 *>(y + row * d_inner + c));
-  const float4 yb = __ldcs(reinterpret_cast<const float4 *>(y + row * d_inner + c + 4));
-  float zv[8], g[8];
+  float yv[8], zv[8], g[8];
+  ld_y8(y + row * d_inner + c, yv);
   load8(z + row * zs + c, zv);
-  const float yv[8] = {ya.x, ya.y, ya.z, ya.w, yb.x, yb.y, yb.z, yb.w};
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -117,90 +139,31 @@ __global__ void __launch_bounds__(1024) gated_norm_v8_kernel(
   store8(out + row * os + c, g);
 }
 
-// Second half of the gated norm fused into the tensor-core scan.  The scan's output stage
-// has gated each token's head (g = y * silu(z), or g = y when normalising first) and stored
-//   q_h   = g / s_h  in fp16, with s_h = sqrt(mean of g^2 over the head's 64 channels)
-//   ssq_h = sum of g^2 over those channels (fp32, per token row and head),
-// so |q| <= 8 and fp16 keeps 11 significant bits of it with no risk of overflow.  A norm group
-// covers whole heads, and its statistic is the sum of its heads' ssq:
-//   out = q * s_h * rsqrt(sum_{h in group} ssq_h / gs + eps) * w   (* silu(z) normalising first).
-// One CTA per token row: the row's per-head factors are formed in shared memory, then every
-// thread rescales 8 channels at a time (16-byte loads and stores).
-constexpr int kRescaleThreads = 256;
-
-__global__ void __launch_bounds__(kRescaleThreads) norm_rescale_kernel(
-    const __half *__restrict__ q, const float *__restrict__ ssq, const __nv_bfloat16 *__restrict__ z,
-    long long zs, const __nv_bfloat16 *__restrict__ w, __nv_bfloat16 *__restrict__ out, long long os,
-    int H, int hpn, int ng, int d_inner, float eps, int nbg) {
-  extern __shared__ float rsm[];
-  float *sq = rsm, *fac = rsm + H, *gsum = rsm + 2 * H;
-  const long long row = blockIdx.x;
-  for (int i = threadIdx.x; i < H; i += kRescaleThreads) sq[i] = ssq[row * H + i];
-  __syncthreads();
-  for (int gi = threadIdx.x; gi < ng; gi += kRescaleThreads) {  // fixed order: reproducible
-    float t = 0.f;
-    for (int j = 0; j < hpn; ++j) t += sq[gi * hpn + j];
-    gsum[gi] = rsqrtf(t / (float)(hpn * kHeadDim) + eps);
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < H; i += kRescaleThreads)
-    fac[i] = sqrtf(sq[i] * (1.f / kHeadDim)) * gsum[i / hpn];
-  __syncthreads();
-  const __half *qr = q + row * d_inner;
-  for (int c = threadIdx.x * 8; c < d_inner; c += kRescaleThreads * 8) {
-    const uint4 qu = __ldcs(reinterpret_cast<const uint4 *>(qr + c));
-    const __half2 *q2 = reinterpret_cast<const __half2 *>(&qu);
-    const float f = fac[c / kHeadDim];
-    float v[8], wv[8];
-    if (w) {
-      load8(w + c, wv);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) wv[i] = 1.f;
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 qf = __half22float2(q2[i]);
-      v[2 * i] = qf.x * f * wv[2 * i];
-      v[2 * i + 1] = qf.y * f * wv[2 * i + 1];
-    }
-    if (nbg) {
-      float zv[8];
-      load8(z + row * zs + c, zv);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] *= silu(zv[i]);
-    }
-    store8(out + row * os + c, v);
-  }
-}
-
-cudaError_t launch_norm_rescale(const PrefillPlan &p, cudaStream_t s) {
-  const int hpn = p.H / p.norm_groups;
-  const size_t smem = (size_t)(2 * p.H + p.norm_groups) * sizeof(float);
-  if (smem > 48 * 1024) return cudaErrorInvalidValue;
-  norm_rescale_kernel<<<(unsigned)p.rows, kRescaleThreads, smem, s>>>(
-      p.qn, p.ssq, (const __nv_bfloat16 *)p.z, p.zs, (const __nv_bfloat16 *)p.norm_w,
-      (__nv_bfloat16 *)p.y, p.ys, p.H, hpn, p.norm_groups, p.d_inner, p.eps, p.nbg);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s) {
   const int gs = p.d_inner / p.norm_groups;
   dim3 grid((unsigned)p.rows, p.norm_groups);
   const bool v8 = p.bf16 && gs % 256 == 0 && gs / 8 <= 1024 &&  // whole warps of 8 channels
                   (reinterpret_cast<uintptr_t>(p.norm_w) & 15u) == 0;
-  if (v8)
-    gated_norm_v8_kernel<<<grid, gs / 8, 0, s>>>(p.yf, (const __nv_bfloat16 *)p.z, p.zs,
-                                                 (const __nv_bfloat16 *)p.norm_w, (__nv_bfloat16 *)p.y,
-                                                 p.ys, p.d_inner, gs, p.eps, p.nbg);
-  else if (p.bf16)
-    gated_norm_kernel<__nv_bfloat16><<<grid, kNormThreads, 0, s>>>(
-        p.yf, (const __nv_bfloat16 *)p.z, p.zs, (const __nv_bfloat16 *)p.norm_w,
-        (__nv_bfloat16 *)p.y, p.ys, p.d_inner, gs, p.eps, p.L, p.nbg);
-  else
-    gated_norm_kernel<float><<<grid, kNormThreads, 0, s>>>(p.yf, (const float *)p.z, p.zs,
-                                                           (const float *)p.norm_w, (float *)p.y,
-                                                           p.ys, p.d_inner, gs, p.eps, p.L, p.nbg);
+  const auto *z = (const __nv_bfloat16 *)p.z;
+  const auto *w = (const __nv_bfloat16 *)p.norm_w;
+  auto *o = (__nv_bfloat16 *)p.y;
+  if (p.yh) {  // tensor path: fp16 y, bf16 tensors
+    if (!p.bf16) return cudaErrorInvalidValue;
+    if (v8)
+      gated_norm_v8_kernel<__half><<<grid, gs / 8, 0, s>>>(p.yh, z, p.zs, w, o, p.ys, p.d_inner, gs, p.eps, p.nbg);
+    else
+      gated_norm_kernel<__nv_bfloat16, __half><<<grid, kNormThreads, 0, s>>>(p.yh, z, p.zs, w, o, p.ys,
+                                                                             p.d_inner, gs, p.eps, p.nbg);
+  } else if (v8) {
+    gated_norm_v8_kernel<float><<<grid, gs / 8, 0, s>>>(p.yf, z, p.zs, w, o, p.ys, p.d_inner, gs, p.eps, p.nbg);
+  } else if (p.bf16) {
+    gated_norm_kernel<__nv_bfloat16, float><<<grid, kNormThreads, 0, s>>>(p.yf, z, p.zs, w, o, p.ys, p.d_inner,
+                                                                          gs, p.eps, p.nbg);
+  } else {
+    gated_norm_kernel<float, float><<<grid, kNormThreads, 0, s>>>(p.yf, (const float *)p.z, p.zs,
+                                                                  (const float *)p.norm_w, (float *)p.y,
+                                                                  p.ys, p.d_inner, gs, p.eps, p.nbg);
+  }
   return cudaGetLastError();
 }
 

@@ -47,9 +47,8 @@ struct PrefillPlan {
   float *tail_dh;    // [B, H, P, N] fp32 contribution of the final state's last chunks, from a
                      // zero state (tensor path; null when no final state is written)
   float *tail_dec;   // [B, H] decay over those chunks
-  __half *qn;        // [B, L, d_inner] fp16 head-normalised gated output (tensor path, fused
-                     // gate: the scan gates and writes these, the rescale finishes the norm)
-  float *ssq;        // [B, L, H] sum of squares of each head's gated output
+  __half *yh;        // [rows, d_inner] fp16 pre-norm output (tensor path, when the gated
+                     // norm follows: its pass reads y with z)
   int Lpad;
   int *err;          // device error word
   // test hook (tensor-core scan): 0 = off; c + 1 = the producer withholds chunk c's stage so
@@ -105,8 +104,7 @@ constexpr int kTailChunks = 2;
 cudaError_t launch_state_tail(const PrefillPlan &p, cudaStream_t s);
 cudaError_t launch_tail_fold(const PrefillPlan &p, cudaStream_t s);
 // norms (norm.cu)
-cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s);          // fp32 yf -> y
-cudaError_t launch_norm_rescale(const PrefillPlan &p, cudaStream_t s);        // qn, ssq -> y
+cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s);  // yh (fp16) or yf (fp32) -> y
 cudaError_t launch_rmsnorm_bf16(const void *x, const void *w, void *out, long long rows, int width,
                                 float eps, cudaStream_t s);
 // decode (decode.cu)

@@ -148,13 +148,9 @@ struct TcArgs {
   float *seg_decay;        // [n_seg, B, H] total decay per segment, or null
   __nv_bfloat16 *y;        // output (no gate) ...
   long long ys;
-  float *yf;               // ... or fp32 pre-norm output [B, L, d_inner] when a gated norm follows
-  __half *qn;              // ... or (fused gate) the gated output of each head divided by its RMS
-  float *ssq;              //     over the head's 64 channels, fp16 [B, L, d_inner], and its sum
-                           //     of squares, fp32 [B, L, H]; a rescale pass finishes the norm
-  const __nv_bfloat16 *z;  // gate [B, L, d_inner] (fused gate, gate first)
-  long long zs;
-  int nbg;                 // 1: normalise before gating (the gate is applied by the rescale)
+  float *yf;               // ... or fp32 pre-norm output [rows, d_inner] when a gated norm follows
+  __half *yh;              // ... or fp16 pre-norm output [rows, d_inner] (the gated norm's pass
+                           //     reads it with z)
   int d_inner;
   int *err;
   unsigned long long wait_ns;  // limit of every bounded wait
@@ -799,70 +795,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       if (!kStateOnly) {
         const int tok = t_begin + k * QC + n;
         const long long row = seq_base(a.cu, b, a.L) + tok;
-        // fused gate (gate first): this row's z (64 channels, 128 bytes) is prefetched into L1
-        // before the wait for the chunk's products
-        const bool gate = a.qn != nullptr && !a.nbg;
-        const __nv_bfloat16 *zrow = gate ? a.z + row * a.zs + h * 64 : nullptr;
-        if (gate && tok < t_end) {
-          asm volatile("prefetch.global.L1 [%0];" ::"l"(zrow));
-          asm volatile("prefetch.global.L1 [%0];" ::"l"(zrow + 63));
-        }
         if (!wg_wait(BAR(BAR_YREADY0 + st), (k >> 1) & 1, leader, 3, abort_flag, a.err, lim)) break;
         tc_fence_after();
         if (leader) TC_MARK(k, 6);
         const uint32_t tYi = tmem + (st ? TM_S1 : TM_S0) + TM_YI_OFF + lane_off;
         const uint32_t tYs = tmem + (st ? TM_YS1 : TM_YS0) + lane_off;
-        if (a.qn) {
-          // fused gate: g = y SiLU(z) (or g = y when normalising first) is stored as g / s in
-          // fp16, s the RMS of g over the head's 64 channels, with sum(g^2) for the rescale
-          // pass.  Pass 1 (16 columns at a time) forms g, keeps it in the Yi columns of TMEM
-          // and sums its squares; pass 2 scales and stores it.  SiLU(v) = v/2 + v/2 tanh(v/2).
-          float ssq = 0.f;
-#pragma unroll
-          for (int qd = 0; qd < 4; ++qd) {
-            float yi[16], ysv[16];
-            tmem_ld16(tYi + 16 * qd, yi);
-            tmem_ld16(tYs + 16 * qd, ysv);
-            uint4 zu[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
-            if (gate && tok < t_end) {
-              zu[0] = __ldg(reinterpret_cast<const uint4 *>(zrow + 16 * qd));
-              zu[1] = __ldg(reinterpret_cast<const uint4 *>(zrow + 16 * qd + 8));
-            }
-            const uint32_t zw[8] = {zu[0].x, zu[0].y, zu[0].z, zu[0].w, zu[1].x, zu[1].y, zu[1].z, zu[1].w};
-            tmem_ld_wait();
-            uint32_t gu[16];
-#pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-              float2 g2 = __ffma2_rn(make_float2(et, et), make_float2(ysv[i], ysv[i + 1]),
-                                     make_float2(yi[i], yi[i + 1]));
-              if (gate) {
-                const __half2 hh = __hmul2(__float22half2_rn(unpack_bf16(zw[i / 2])), __float2half2_rn(0.5f));
-                g2 = __fmul2_rn(g2, __half22float2(__hfma2(hh, h2tanh_approx(hh), hh)));
-              }
-              ssq = fmaf(g2.x, g2.x, fmaf(g2.y, g2.y, ssq));
-              gu[i] = __float_as_uint(g2.x);
-              gu[i + 1] = __float_as_uint(g2.y);
-            }
-            tmem_st16(tYi + 16 * qd, gu);
-          }
-          tmem_st_wait();
-          const float inv = ssq > 0.f ? rsqrtf(ssq * (1.f / 64.f)) : 0.f;
-#pragma unroll
-          for (int qd = 0; qd < 4; ++qd) {
-            float gv[16];
-            tmem_ld16(tYi + 16 * qd, gv);
-            tmem_ld_wait();
-            uint32_t pk[8];
-#pragma unroll
-            for (int i = 0; i < 16; i += 2) pk[i / 2] = pack_f16(gv[i] * inv, gv[i + 1] * inv);
-            if (tok < t_end) {
-              uint4 *dst = reinterpret_cast<uint4 *>(a.qn + row * a.d_inner + h * 64 + 16 * qd);
-              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            }
-          }
-          if (tok < t_end) a.ssq[row * a.H + h] = ssq;
-        } else {
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
           float yi[32], ysv[32];
@@ -885,7 +822,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             yi[i + 1] = r.y;
           }
           if (tok < t_end) {
-            if (a.yf) {
+            if (a.yh) {
+              uint4 *dst = reinterpret_cast<uint4 *>(a.yh + row * a.d_inner + h * 64 + 32 * half);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(pack_f16(yi[8 * i], yi[8 * i + 1]), pack_f16(yi[8 * i + 2], yi[8 * i + 3]),
+                                    pack_f16(yi[8 * i + 4], yi[8 * i + 5]), pack_f16(yi[8 * i + 6], yi[8 * i + 7]));
+            } else if (a.yf) {
               float4 *dst = reinterpret_cast<float4 *>(a.yf + row * a.d_inner + h * 64 + 32 * half);
 #pragma unroll
               for (int i = 0; i < 8; ++i) dst[i] = make_float4(yi[4 * i], yi[4 * i + 1], yi[4 * i + 2], yi[4 * i + 3]);
@@ -896,15 +839,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
                 dst[i] = make_uint4(pack_bf16(yi[8 * i], yi[8 * i + 1]), pack_bf16(yi[8 * i + 2], yi[8 * i + 3]),
                                     pack_bf16(yi[8 * i + 4], yi[8 * i + 5]), pack_bf16(yi[8 * i + 6], yi[8 * i + 7]));
             }
-          }
-        }
-        }
-        if (a.qn) {
-          tc_fence_before();
-          named_bar(3, 128);
-          if (leader) {
-            TC_MARK(k, 7);
-            mbar_arrive(BAR(BAR_YFREE0 + st));
           }
         }
       }
@@ -991,12 +925,8 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
   a.conv_w = (const __nv_bfloat16 *)p.conv_w; a.conv_b = (const __nv_bfloat16 *)p.conv_b;
   a.dte = p.dte_hm; a.cs = p.cs_hm; a.D = p.D;
   a.y = (__nv_bfloat16 *)p.y; a.ys = p.ys; a.err = p.err;
-  a.yf = p.norm_groups > 0 && !p.qn ? p.yf : nullptr;
-  a.qn = p.norm_groups > 0 ? p.qn : nullptr;
-  a.ssq = p.ssq;
-  a.z = (const __nv_bfloat16 *)p.z;
-  a.zs = p.zs;
-  a.nbg = p.nbg;
+  a.yh = p.norm_groups > 0 ? p.yh : nullptr;
+  a.yf = p.norm_groups > 0 && !p.yh ? p.yf : nullptr;
   a.wait_ns = p.stall_chunk1 > 0 ? p.stall_wait_ns : tc::kWaitLimitNs;
   a.debug_skip_chunk = p.stall_chunk1 - 1;
   a.d_inner = p.d_inner;

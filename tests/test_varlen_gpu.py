@@ -82,7 +82,7 @@ def test_varlen_is_one_pass(cuda_lib):
         names = [n for n, _ in ssd.trace_read()]
     finally:
         ssd.trace_enable(False)
-    for k in ("ssd_front", "ssd_scan_tc", "ssd_state_tail", "ssd_norm_rescale"):
+    for k in ("ssd_front", "ssd_scan_tc", "ssd_state_tail", "ssd_gated_norm"):
         assert names.count(k) == 1, names
 
 
