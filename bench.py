@@ -437,9 +437,10 @@ def e2e_prefill(c: Ctx, cfg, d, ws, tokens):
 
 def bench_decode(c: Ctx, steps_total=16384, graph_steps=256):
     torch, ssd = c.torch, c.ssd
+    steps_total = c.args.decode_steps or steps_total
     cfg = datagen.config(2)
     Bn, H, P = cfg["batch"], cfg["nheads"], cfg["headdim"]
-    pcfg = dict(cfg, seqlen=cfg["prefill_len"], norm_groups=0)
+    pcfg = dict(cfg, seqlen=c.args.decode_prefill_len or cfg["prefill_len"], norm_groups=0)
     pin = datagen.make_inputs(2, pcfg)
     dp = {k: ssd.to_device(pin[k]) for k in ("A", "D", "dt_bias", "conv_w")}
     _, state, cache = ssd.prefill(pcfg, ssd.to_device(pin["xBC"]), ssd.to_device(pin["dt"]),
@@ -760,6 +761,13 @@ def main():
                     default="all", help="run one workload alone (for profiling); prints its object")
     ap.add_argument("--mixer-batch", type=int, default=8,
                     help="batch of the mixer workload (smaller only for profiling captures)")
+    ap.add_argument("--decode-steps", type=int, default=0,
+                    help="decode steps timed (0: the workload's 16384; fewer only for profiling "
+                         "captures)")
+    ap.add_argument("--decode-prefill-len", type=int, default=0,
+                    help="tokens of the prefill that gives the decode its starting state (0: the "
+                         "workload's 8192; shorter only for profiling captures, whose device "
+                         "memory it bounds)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))
