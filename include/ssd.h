@@ -230,7 +230,7 @@ const char *ssd_status_string(ssd_status_t status);
  * array of SSD_NOALLOC_WORKSPACE_BYTES that the library reserves on every device it is loaded
  * on and keeps until the process exits; the call itself allocates and frees nothing.
  *  - Returns SSD_ERR_WORKSPACE when ssd_workspace_size(cfg) exceeds that size.  On the
- *    tensor-core path that is about 2,800 tokens per call of a 128-head, 8-group layer with
+ *    tensor-core path that is about 2,900 tokens per call of a 128-head, 8-group layer with
  *    the gated norm, and about 12,000 without it; more for smaller layers.
  *  - The first call on a device looks up the array's device address; make that first call
  *    before starting any stream capture.
