@@ -479,8 +479,11 @@ ssd_status_t run_decode(const ssd_config_t *c, const ssd_decode_args_t *a, cudaS
   return from_cuda(traced("ssd_decode", s, [&] { return launch_decode(p, s); }));
 }
 
+// The input RMSNorm is folded into the in_proj GEMM: rmsnorm(x) W_in^T = diag(r) x (W_in diag(w))^T,
+// with r the per-row factor (computed by a light pass over x) applied in the GEMM's epilogue and
+// the norm weight w folded into a copy of W_in, so the normalised activations never reach HBM.
 struct MixerLayout {
-  size_t hn, zxbcdt, g, ssd, total;
+  size_t rs, wf, zxbcdt, g, ssd, total;
   ssd_config_t scfg;
 };
 
@@ -492,7 +495,8 @@ MixerLayout mixer_layout(const ssd_mixer_config_t *m) {
   const size_t proj = 2 * d_inner + 2 * (size_t)m->ssd.ngroups * m->ssd.dstate + m->ssd.nheads;
   const size_t proj_pad = round_up(proj, 8);
   size_t off = 0;
-  l.hn = off;      off = round_up(off + T * m->d_model * 2, kAlign);
+  l.rs = off;      off = round_up(off + T * 4, kAlign);
+  l.wf = off;      off = round_up(off + proj * m->d_model * 2, kAlign);
   l.zxbcdt = off;  off = round_up(off + T * proj_pad * 2, kAlign);
   l.g = off;       off = round_up(off + T * d_inner * 2, kAlign);
   l.ssd = off;     off = round_up(off + prefill_layout(&l.scfg).total, kAlign);
@@ -520,13 +524,21 @@ ssd_status_t run_mixer(const ssd_mixer_config_t *m, const ssd_mixer_args_t *a, c
   const long long T = (long long)m->ssd.batch * m->ssd.seqlen;
   if (T > INT32_MAX) return SSD_ERR_UNSUPPORTED;
   char *ws = static_cast<char *>(a->workspace);
-  void *hn = ws + l.hn, *zx = ws + l.zxbcdt, *g = ws + l.g;
-  SSD_TRY(traced("ssd_rmsnorm", s, [&] {
-    return launch_rmsnorm_bf16(a->hidden, a->rms_w, hn, T, m->d_model, m->rms_eps, s);
+  float *rs = reinterpret_cast<float *>(ws + l.rs);
+  void *zx = ws + l.zxbcdt, *g = ws + l.g;
+  const void *w_in = a->W_in;
+  SSD_TRY(traced("ssd_rms_rowscale", s, [&] {
+    return launch_rms_rowscale_bf16(a->hidden, rs, T, m->d_model, m->rms_eps, s);
   }));
+  if (a->rms_w) {
+    SSD_TRY(traced("ssd_fold_rms_w", s, [&] {
+      return launch_fold_cols_bf16(a->W_in, a->rms_w, ws + l.wf, proj, m->d_model, s);
+    }));
+    w_in = ws + l.wf;
+  }
   SSD_TRY(traced("gemm_in_proj", s, [&] {
-    return launch_gemm_bf16_tn(hn, m->d_model, a->W_in, m->d_model, zx, proj_pad, (int)T, (int)proj,
-                               m->d_model, s);
+    return launch_gemm_bf16_tn(a->hidden, m->d_model, w_in, m->d_model, zx, proj_pad, (int)T, (int)proj,
+                               m->d_model, s, rs);
   }));
   const __nv_bfloat16 *zxb = static_cast<const __nv_bfloat16 *>(zx);
   ssd_prefill_args_t pa{};
@@ -550,12 +562,12 @@ ssd_status_t run_mixer(const ssd_mixer_config_t *m, const ssd_mixer_args_t *a, c
 
 // Tensor-core GEMM on sm_100 when the operands satisfy TMA's alignment rules, else CUDA cores.
 cudaError_t launch_gemm_bf16_tn(const void *A, long long lda, const void *Bm, long long ldb, void *C,
-                                long long ldc, int M, int N, int K, cudaStream_t s) {
+                                long long ldc, int M, int N, int K, cudaStream_t s, const float *row_scale) {
   const bool aligned = aligned16(A) && aligned16(Bm) && aligned16(C) && lda % 8 == 0 && ldb % 8 == 0 &&
                        ldc % 8 == 0;
   if (aligned && tc_scan_available())
-    return launch_gemm_tc_bf16_tn(A, lda, Bm, ldb, C, ldc, M, N, K, device_error_ptr(), s);
-  return launch_gemm_simt_bf16_tn(A, lda, Bm, ldb, C, ldc, M, N, K, s);
+    return launch_gemm_tc_bf16_tn(A, lda, Bm, ldb, C, ldc, M, N, K, device_error_ptr(), s, row_scale);
+  return launch_gemm_simt_bf16_tn(A, lda, Bm, ldb, C, ldc, M, N, K, s, row_scale);
 }
 
 }  // namespace ssd

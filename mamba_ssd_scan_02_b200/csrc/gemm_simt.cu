@@ -11,7 +11,8 @@ constexpr int BM = 64, BN = 64, BK = 32;
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const __nv_bfloat16 *__restrict__ A, long long lda,
                                                         const __nv_bfloat16 *__restrict__ Bm, long long ldb,
                                                         __nv_bfloat16 *__restrict__ C, long long ldc,
-                                                        int M, int N, int K) {
+                                                        int M, int N, int K,
+                                                        const float *__restrict__ row_scale) {
   __shared__ float As[BK][BM + 1];
   __shared__ float Bs[BK][BN + 1];
   const int tid = threadIdx.x;
@@ -44,17 +45,18 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const __nv_bfloat16 *__r
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const long long m = m0 + tr * 4 + i, n = n0 + tc + 16 * j;
-      if (m < M && n < N) C[m * ldc + n] = __float2bfloat16_rn(acc[i][j]);
+      if (m < M && n < N) C[m * ldc + n] = __float2bfloat16_rn(row_scale ? acc[i][j] * row_scale[m] : acc[i][j]);
     }
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_simt_bf16_tn(const void *A, long long lda, const void *Bm, long long ldb, void *C,
-                                     long long ldc, int M, int N, int K, cudaStream_t s) {
+                                     long long ldc, int M, int N, int K, cudaStream_t s,
+                                     const float *row_scale) {
   dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
   gemm_simt_kernel<<<grid, 256, 0, s>>>((const __nv_bfloat16 *)A, lda, (const __nv_bfloat16 *)Bm, ldb,
-                                        (__nv_bfloat16 *)C, ldc, M, N, K);
+                                        (__nv_bfloat16 *)C, ldc, M, N, K, row_scale);
   return cudaGetLastError();
 }
 

@@ -38,6 +38,7 @@ struct GemmArgs {
   __nv_bfloat16 *C;
   long long ldc;
   int *err;
+  const float *row_scale;  // fp32 [M], applied in the epilogue, or null
 };
 
 __device__ __forceinline__ void tile_coords(int tile, int mb_count, int nb_count, int &m0, int &n0) {
@@ -150,11 +151,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const int m = m0 + 32 * ew + lane;
       __nv_bfloat16 *crow = g.C + (long long)m * g.ldc;
+      const float rs = (g.row_scale && m < g.M) ? g.row_scale[m] : 1.f;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         float v[32];
         tmem_ld32(tmem + buf * BN + 32 * c + lane_off, v);
         tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= rs;
         const int n = n0 + 32 * c;
         if (m < g.M && n < g.N) {
           if (n + 32 <= g.N) {
@@ -213,7 +217,8 @@ bool make_kmajor_map(CUtensorMap *map, const void *ptr, long long rows, long lon
 
 // Requirements: 16-byte aligned A, B, C; lda, ldb, ldc multiples of 8 elements.
 cudaError_t launch_gemm_tc_bf16_tn(const void *A, long long lda, const void *Bm, long long ldb, void *C,
-                                   long long ldc, int M, int N, int K, int *err, cudaStream_t s) {
+                                   long long ldc, int M, int N, int K, int *err, cudaStream_t s,
+                                   const float *row_scale) {
   CUtensorMap ta, tb;
   if (!make_kmajor_map(&ta, A, M, K, lda, BM) || !make_kmajor_map(&tb, Bm, N, K, ldb, BN))
     return cudaErrorInvalidValue;
@@ -221,7 +226,7 @@ cudaError_t launch_gemm_tc_bf16_tn(const void *A, long long lda, const void *Bm,
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long tiles = (long long)((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = (int)(tiles < sms ? tiles : sms);
-  GemmArgs g{M, N, K, (__nv_bfloat16 *)C, ldc, err};
+  GemmArgs g{M, N, K, (__nv_bfloat16 *)C, ldc, err, row_scale};
   cudaError_t e = set_smem_attr(gemm_tc_kernel, kGemmSmem, s);
   if (e != cudaSuccess) return e;
   gemm_tc_kernel<<<grid, kGemmThreads, kGemmSmem, s>>>(ta, tb, g);

@@ -1,5 +1,5 @@
 // norm.cu -- the z-gated RMSNorm applied to the scan output, and the plain RMSNorm at the
-// mixer input.  The Nemotron Nano 2 layers normalise with RMSNorm ("NVIDIA Nemotron Nano 2"
+// mixer input (as a per-row factor and a folded weight, applied by the in_proj GEMM).  The Nemotron Nano 2 layers normalise with RMSNorm ("NVIDIA Nemotron Nano 2"
 // summary, section "Method"); in the Mamba-2 mixer the scan output is gated by SiLU(z) and
 // then normalised over groups of d_inner / norm_groups consecutive channels:
 //   g = y * silu(z);   out = g / sqrt(mean_group(g^2) + eps) * w
@@ -62,9 +62,9 @@ __global__ void __launch_bounds__(kNormThreads) gated_norm_kernel(
   }
 }
 
-__global__ void __launch_bounds__(kNormThreads) rmsnorm_bf16_kernel(
-    const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w,
-    __nv_bfloat16 *__restrict__ out, int width, float eps) {
+// The RMSNorm's per-row factor alone (the projection that follows applies it): one CTA per row.
+__global__ void __launch_bounds__(kNormThreads) rms_rowscale_bf16_kernel(
+    const __nv_bfloat16 *__restrict__ x, float *__restrict__ r, int width, float eps) {
   __shared__ float red[32];
   const long long row = blockIdx.x;
   const __nv_bfloat16 *xr = x + row * width;
@@ -76,14 +76,20 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_bf16_kernel(
     for (int k = 0; k < 8; ++k) ss += v[k] * v[k];
   }
   ss = block_sum(ss, red);
-  const float r = rsqrtf(ss / width + eps);
-  for (int i = threadIdx.x * 8; i < width; i += kNormThreads * 8) {
+  if (threadIdx.x == 0) r[row] = rsqrtf(ss / width + eps);
+}
+
+// W'[n][k] = W[n][k] * w[k], 8 elements per thread (16-byte accesses).
+__global__ void fold_cols_bf16_kernel(const __nv_bfloat16 *__restrict__ W, const __nv_bfloat16 *__restrict__ w,
+                                      __nv_bfloat16 *__restrict__ out, long long n8, int K) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
+    const int k = (int)((i * 8) % K);
     float v[8], wv[8];
-    load8(xr + i, v);
-    if (w) load8(w + i, wv);
+    load8(W + i * 8, v);
+    load8(w + k, wv);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = v[k] * r * (w ? wv[k] : 1.f);
-    store8(out + row * width + i, v);
+    for (int j = 0; j < 8; ++j) v[j] *= wv[j];
+    store8(out + i * 8, v);
   }
 }
 
@@ -168,10 +174,21 @@ cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s) {
 }
 
 
-cudaError_t launch_rmsnorm_bf16(const void *x, const void *w, void *out, long long rows, int width,
-                                float eps, cudaStream_t s) {
-  rmsnorm_bf16_kernel<<<(unsigned)rows, kNormThreads, 0, s>>>(
-      (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)w, (__nv_bfloat16 *)out, width, eps);
+cudaError_t launch_rms_rowscale_bf16(const void *x, float *r, long long rows, int width, float eps,
+                                     cudaStream_t s) {
+  if (width % 8) return cudaErrorInvalidValue;
+  rms_rowscale_bf16_kernel<<<(unsigned)rows, kNormThreads, 0, s>>>((const __nv_bfloat16 *)x, r, width, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fold_cols_bf16(const void *W, const void *w, void *out, long long rows, int K,
+                                  cudaStream_t s) {
+  if (K % 8) return cudaErrorInvalidValue;
+  const long long n8 = rows * K / 8;
+  long long blocks = (n8 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  fold_cols_bf16_kernel<<<(unsigned)blocks, 256, 0, s>>>((const __nv_bfloat16 *)W, (const __nv_bfloat16 *)w,
+                                                         (__nv_bfloat16 *)out, n8, K);
   return cudaGetLastError();
 }
 

@@ -105,17 +105,25 @@ cudaError_t launch_state_tail(const PrefillPlan &p, cudaStream_t s);
 cudaError_t launch_tail_fold(const PrefillPlan &p, cudaStream_t s);
 // norms (norm.cu)
 cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s);  // yh (fp16) or yf (fp32) -> y
-cudaError_t launch_rmsnorm_bf16(const void *x, const void *w, void *out, long long rows, int width,
-                                float eps, cudaStream_t s);
+// RMSNorm folded into the projection that follows it: r[row] = 1 / sqrt(mean(x[row]^2) + eps)
+// (fp32), and W'[n][k] = W[n][k] * w[k] (bf16), so that rmsnorm(x) W^T = diag(r) x W'^T.
+cudaError_t launch_rms_rowscale_bf16(const void *x, float *r, long long rows, int width, float eps,
+                                     cudaStream_t s);
+cudaError_t launch_fold_cols_bf16(const void *W, const void *w, void *out, long long rows, int K,
+                                  cudaStream_t s);
 // decode (decode.cu)
 cudaError_t launch_decode(const DecodePlan &p, cudaStream_t s);
-// GEMM C[M,N] = A[M,K] . B[N,K]^T, bf16 in/out, fp32 accumulate
+// GEMM C[M,N] = diag(row_scale) A[M,K] . B[N,K]^T, bf16 in/out, fp32 accumulate (row_scale:
+// fp32 [M] or null for none)
 cudaError_t launch_gemm_bf16_tn(const void *A, long long lda, const void *Bm, long long ldb, void *C,
-                                long long ldc, int M, int N, int K, cudaStream_t s);
+                                long long ldc, int M, int N, int K, cudaStream_t s,
+                                const float *row_scale = nullptr);
 cudaError_t launch_gemm_tc_bf16_tn(const void *A, long long lda, const void *Bm, long long ldb, void *C,
-                                   long long ldc, int M, int N, int K, int *err, cudaStream_t s);
+                                   long long ldc, int M, int N, int K, int *err, cudaStream_t s,
+                                   const float *row_scale = nullptr);
 cudaError_t launch_gemm_simt_bf16_tn(const void *A, long long lda, const void *Bm, long long ldb,
-                                     void *C, long long ldc, int M, int N, int K, cudaStream_t s);
+                                     void *C, long long ldc, int M, int N, int K, cudaStream_t s,
+                                     const float *row_scale = nullptr);
 
 // ---- tracing (trace.cu): event pairs around each launch while enabled ------------------
 bool trace_enabled();

@@ -148,9 +148,8 @@ struct TcArgs {
   float *seg_decay;        // [n_seg, B, H] total decay per segment, or null
   __nv_bfloat16 *y;        // output (no gate) ...
   long long ys;
-  float *yf;               // ... or fp32 pre-norm output [rows, d_inner] when a gated norm follows
-  __half *yh;              // ... or fp16 pre-norm output [rows, d_inner] (the gated norm's pass
-                           //     reads it with z)
+  __half *yh;              // ... or fp16 pre-norm output [rows, d_inner] when the gated norm
+                           //     follows (its pass reads it with z)
   int d_inner;
   int *err;
   unsigned long long wait_ns;  // limit of every bounded wait
@@ -258,9 +257,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const int nck = t_end > t_begin ? (t_end - t_begin + QC - 1) / QC : 0;
   const int last = nck - 1;
   // The last chunk's exact path (fp32 SiLU, split-precision w o X) serves only the final
-  // state; in tail mode an fp32 pass recomputes the last chunks, and without h_out nothing
-  // reads it.
-  const bool exact_last = kStateOnly || (a.tail_chunks == 0 && a.h_out != nullptr);
+  // state, which the full pass never takes from here: with a final state requested it runs
+  // in tail mode (an fp32 pass recomputes the last chunks), and otherwise nothing reads it.
+  // So only the states-only pass compiles it.
+  constexpr bool exact_last = kStateOnly;
   const uint64_t lim = a.wait_ns;
   const uint32_t bar0 = sb + OFF_BAR;
 #define BAR(i) (bar0 + 8u * (uint32_t)(i))
@@ -828,10 +828,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
               for (int i = 0; i < 4; ++i)
                 dst[i] = make_uint4(pack_f16(yi[8 * i], yi[8 * i + 1]), pack_f16(yi[8 * i + 2], yi[8 * i + 3]),
                                     pack_f16(yi[8 * i + 4], yi[8 * i + 5]), pack_f16(yi[8 * i + 6], yi[8 * i + 7]));
-            } else if (a.yf) {
-              float4 *dst = reinterpret_cast<float4 *>(a.yf + row * a.d_inner + h * 64 + 32 * half);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) dst[i] = make_float4(yi[4 * i], yi[4 * i + 1], yi[4 * i + 2], yi[4 * i + 3]);
             } else {
               uint4 *dst = reinterpret_cast<uint4 *>(a.y + row * a.ys + h * 64 + 32 * half);
 #pragma unroll
@@ -925,8 +921,8 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
   a.conv_w = (const __nv_bfloat16 *)p.conv_w; a.conv_b = (const __nv_bfloat16 *)p.conv_b;
   a.dte = p.dte_hm; a.cs = p.cs_hm; a.D = p.D;
   a.y = (__nv_bfloat16 *)p.y; a.ys = p.ys; a.err = p.err;
+  if (p.norm_groups > 0 && !p.yh) return cudaErrorInvalidValue;  // the norm reads fp16 y
   a.yh = p.norm_groups > 0 ? p.yh : nullptr;
-  a.yf = p.norm_groups > 0 && !p.yh ? p.yf : nullptr;
   a.wait_ns = p.stall_chunk1 > 0 ? p.stall_wait_ns : tc::kWaitLimitNs;
   a.debug_skip_chunk = p.stall_chunk1 - 1;
   a.d_inner = p.d_inner;

@@ -1,4 +1,9 @@
-"""GPU parity of mamba2_mixer_forward (through the C ABI) against the fp64 oracle."""
+"""GPU parity of mamba2_mixer_forward (through the C ABI) against the fp64 oracle.
+
+The layer is held to the oracle with no rounding anywhere (fp64 end to end), at the bf16
+bound.  The oracle that rounds the activations a plain bf16 layer stores between its steps
+(RMSNorm output, in_proj output, gated-norm output) is reported beside it: this layer keeps
+the RMSNorm output in fp32 (folded into the in_proj GEMM), so it sits between the two."""
 import numpy as np
 import pytest
 
@@ -27,7 +32,8 @@ def test_mixer_small(cuda_lib, oracle):
                norm_groups=2)
     inp = datagen.make_inputs(4, cfg)
     out = _mixer(cfg, inp)
-    assert_close(out.float().cpu().numpy(), _oracle(oracle, cfg, inp), TOL_BF16, "mixer small", out_dtype="bf16")
+    assert_close(out.float().cpu().numpy(), _oracle(oracle, cfg, inp, bf16_activations=False), TOL_BF16,
+                 "mixer small", out_dtype="bf16")
 
 
 def test_mixer_odd_tokens_and_width(cuda_lib, oracle):
@@ -35,7 +41,8 @@ def test_mixer_odd_tokens_and_width(cuda_lib, oracle):
                norm_groups=2)
     inp = datagen.make_inputs(4, cfg)
     out = _mixer(cfg, inp)
-    assert_close(out.float().cpu().numpy(), _oracle(oracle, cfg, inp), TOL_BF16, "mixer odd", out_dtype="bf16")
+    assert_close(out.float().cpu().numpy(), _oracle(oracle, cfg, inp, bf16_activations=False), TOL_BF16,
+                 "mixer odd", out_dtype="bf16")
 
 
 def test_mixer_12b_width_full_size(cuda_lib, oracle):
@@ -45,25 +52,23 @@ def test_mixer_12b_width_full_size(cuda_lib, oracle):
     inp = datagen.make_inputs(4)
     out = _mixer(cfg, inp)
     got = out[[0, 7], :1024].float().cpu().numpy()
-    want = _oracle(oracle, cfg, inp, rows=[0, 7], tokens=1024)
+    want = _oracle(oracle, cfg, inp, rows=[0, 7], tokens=1024, bf16_activations=False)
     assert_close(got, want, TOL_BF16, "mixer 12B width", out_dtype="bf16")
 
 
-def test_mixer_against_the_unrounded_oracle(cuda_lib, oracle):
-    """The layer against the oracle with no rounding anywhere (fp64 end to end), beside the
-    oracle that rounds the three activations the layer stores in bf16 (its definition: the
-    layer runs in bf16).  All three figures are printed: GPU vs rounded oracle (the asserted
-    parity bound), GPU vs unrounded oracle, and rounded vs unrounded oracle -- the part of the
-    gap that the bf16 storage of the activations alone accounts for.  Measured on B200: the
-    unrounded comparison exceeds 2e-2 by a little (about 2.2e-2 over the storage rounding),
-    so it is held to the bound plus the rounding-only gap."""
+def test_mixer_between_the_two_oracles(cuda_lib, oracle):
+    """All three figures are printed: GPU vs the unrounded oracle (held to the bf16 bound), GPU
+    vs the oracle of a plain bf16 layer (which rounds the RMSNorm output, the in_proj output and
+    the gated-norm output), and the two oracles against each other -- how far the bf16 storage of
+    those activations alone moves the output.  The layer rounds only the last two, so against
+    the rounded oracle it is held to the bound plus that gap."""
     cfg = dict(datagen.config(4), batch=2, seqlen=300, d_model=256, nheads=8, ngroups=2,
                norm_groups=2)
     inp = datagen.make_inputs(4, cfg)
     got = _mixer(cfg, inp).float().cpu().numpy()
     rounded = _oracle(oracle, cfg, inp)
     exact = _oracle(oracle, cfg, inp, bf16_activations=False)
-    assert_close(got, rounded, TOL_BF16, "mixer vs bf16-activation oracle", out_dtype="bf16")
+    assert_close(got, exact, TOL_BF16, "mixer vs unrounded fp64 oracle", out_dtype="bf16")
     gap = rel_err(rounded, exact)
     print(f"[parity] bf16-activation oracle vs unrounded oracle: max|diff|/RMS = {gap:.3e}")
-    assert_close(got, exact, TOL_BF16 + gap, "mixer vs unrounded fp64 oracle", out_dtype="bf16")
+    assert_close(got, rounded, TOL_BF16 + gap, "mixer vs bf16-activation oracle", out_dtype="bf16")
