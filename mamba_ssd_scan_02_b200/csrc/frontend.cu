@@ -399,6 +399,7 @@ struct FrontArgs {
 template <int W>
 __global__ void __launch_bounds__(kBcThreads, 4) front_tc_kernel(const FrontArgs f) {
   __shared__ float v[2][128][9];
+  asm volatile("griddepcontrol.launch_dependents;");  // the scan may launch and set up now
   int j = blockIdx.x;
   if (j < f.n_dt) {  // two 128-thread dt tiles per CTA
     const int half = threadIdx.x >> 7, q = 2 * j + half;

@@ -306,6 +306,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         ++nx;
         if (a.debug_skip_chunk == k) break;  // test hook: stage k never arrives (see TcArgs)
         if (k >= 2 && !mbar_wait(BAR(BAR_EMPTY0 + st), ((k >> 1) - 1) & 1, abort_flag, a.err, lim)) break;
+        // the stage holds the front end's outputs: the kernel may have been launched before
+        // the front end finished (programmatic dependent launch), and waits for it here; the
+        // raw x rows above are the caller's input, complete before the front end started
+        if (k == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
         const uint32_t sst = sb + st * kStage;
         const uint32_t full = BAR(BAR_FULL0 + st);
         TC_MARK(k, 12);
@@ -948,7 +952,18 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
     a.tail_chunks = p.tail_dh ? kTailChunks : 0;
     e = set_smem_attr(ssd_scan_tc_kernel<false>, kSmemAlloc, s);
     if (e != cudaSuccess) return e;
-    ssd_scan_tc_kernel<false><<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, a);
+    // Programmatic dependent launch when the front end directly precedes the scan: the scan's
+    // set-up (TMEM, barriers, tensor maps, its first raw x loads) overlaps the front end's tail,
+    // and its producer waits for the front end before loading a stage.  Not after the
+    // states-only pass (the state warps read its output at once).
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid; lc.blockDim = dim3(kThreadsTC); lc.dynamicSmemBytes = kSmemAlloc; lc.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = p.n_seg == 1 ? 1 : 0;
+    lc.attrs = at; lc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&lc, ssd_scan_tc_kernel<false>, tm, tmx, a);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

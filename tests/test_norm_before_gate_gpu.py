@@ -37,9 +37,9 @@ def test_decode_norm_before_gate(cuda_lib, oracle):
 
 
 def test_mixer_norm_before_gate(cuda_lib, oracle):
-    from tests.test_mixer_gpu import _mixer, _oracle
+    from tests.test_mixer_gpu import _mixer, check_mixer
     cfg = dict(datagen.config(4), batch=1, seqlen=200, d_model=256, nheads=8, ngroups=2,
                norm_groups=2, norm_before_gate=True)
     inp = datagen.make_inputs(4, cfg)
     out = _mixer(cfg, inp)
-    assert_close(out.float().cpu().numpy(), _oracle(oracle, cfg, inp), TOL_BF16, "mixer nbg", out_dtype="bf16")
+    check_mixer(out.float().cpu().numpy(), oracle, cfg, inp, "mixer nbg")

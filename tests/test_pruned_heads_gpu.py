@@ -33,10 +33,9 @@ def test_decode_pruned_heads(cuda_lib, oracle):
 
 def test_mixer_pruned_width(cuda_lib, oracle):
     """The compressed model's width: d_model 4480 with 112 heads (in_proj width 16496)."""
-    from tests.test_mixer_gpu import _mixer, _oracle
+    from tests.test_mixer_gpu import _mixer, check_mixer
     cfg = dict(datagen.config(4), batch=1, seqlen=160, d_model=4480, nheads=112, ngroups=8,
                norm_groups=8)
     inp = datagen.make_inputs(4, cfg)
     out = _mixer(cfg, inp)
-    assert_close(out.float().cpu().numpy(), _oracle(oracle, cfg, inp), TOL_BF16, "mixer d4480 H112",
-                 out_dtype="bf16")
+    check_mixer(out.float().cpu().numpy(), oracle, cfg, inp, "mixer d4480 H112")
