@@ -1,49 +1,72 @@
-// state_tail.cu -- the final state's last chunks in fp32.
+// state_tail.cu -- the final state's last chunks at fp32 accuracy.
 //
 // The tensor-core scan carries the state in fp32 but multiplies fp16 operands, and the final
 // state's largest entries often come from a few recent tokens, whose products are not
-// averaged over many terms.  So this pass computes, in fp32 from the raw inputs, what the last
+// averaged over many terms.  So this pass computes, from the raw inputs, what the last
 // kTailChunks chunks (at most 256 tokens) of the sequence's last segment add to the final
 // state, starting from a zero state:
 //   per chunk:  dH <- e^{cs_Q} dH + sum_s e^{cs_Q - cs_s} dt_s x_s B_s^T
 // with x_s, B_s the causal conv1d + SiLU of the raw channels (history from the incoming conv
 // cache before token 0) and dt_s, cs_s the chunk-local prefix sums of dt*A already computed
-// for the scan.  The output scan leaves the state entering those chunks, and a fold sets
-// h = e^{sum of their cs_Q} h + dH.
+// for the scan.  Unrolled over the (at most two) chunks, dH = sum_s w_s x_s B_s^T with
+// w_s = e^{cs_Q(s) - cs_s + cs_Q of the later chunk, if any} dt_s.  The output scan leaves the
+// state entering those chunks, and a fold sets h = e^{sum of their cs_Q} h + dH.
 //
-// It needs only the front end's outputs, so it runs on a side stream beside the output scan:
-// on the SMs the scan leaves free, a few persistent CTAs work through the (head, batch row)
-// items.
-//
-// Per item, a CTA of 512 threads computes every tail token's weight w_s = e^{cs_Q - cs_s}
-// dt_s; per chunk it copies the chunk's raw rows of its 64 x channels and its group's 128 B
-// channels (plus 3 history rows) into shared memory with asynchronous 16-byte copies (all in
-// flight together).  Per 64 tokens, threads 0..383 then run the conv + SiLU, one channel and
-// 32 tokens each (a sliding window over the staged rows), writing fp32 outputs with the x
-// channels already multiplied by w_s; after one barrier all 16 warps apply those tokens'
-// rank-1 updates.  The staging of one chunk (about 100 KB of shared memory in all) lets two
-// CTAs share an SM, so that one's copies overlap the other's arithmetic.  For those, warp w owns state rows 16 (w >> 2) .. +15 and
-// columns 32 (w & 3) .. +31, and a lane a 4 x 4 block, so one token costs a warp two
-// conflict-free 16-byte shared loads (4 x values, 4 B values) and eight paired FMAs.
+// It needs only the front end's outputs, so it runs on a side stream beside the output scan,
+// on the SMs the scan leaves free: persistent CTAs (one per SM) work through items of up to
+// four heads of one group and batch row, which share the group's B channels.  Per item the CTA
+// computes every tail token's weight w_s per head; then, per 64 tokens (a round), it copies the
+// raw rows of the heads' x channels and the group's B channels (plus 3 history rows) into
+// shared memory with asynchronous 16-byte copies (the next round's copies, or the next item's
+// first, run during this round), and each thread runs the conv + SiLU in fp32 for two adjacent
+// channels over 16 tokens, multiplies the x channels by w_s, and splits each value v into fp16
+// parts, v = hi + lo + e with hi = fp16(v), lo = fp16(v - hi) and |e| <= 2^-22 |v| (plus an
+// absolute 2^-25 where lo falls below fp16's normal range), written into 128-byte-swizzled
+// operand tiles.  One thread then issues the round's update on the tensor cores, one MMA per
+// 16 tokens and product for all the item's heads (N = 64 per head), into a tensor-memory
+// accumulator (128 lanes = state column n, 64 columns per head), as three fp16 products with
+// fp32 accumulation:
+//   dH^T += B_hi^T X_hi + B_hi^T X_lo + B_lo^T X_hi
+// (the dropped lo*lo term is below 2^-22 of the product), which keeps the update at fp32
+// accuracy.  Sixteen warps finally read the accumulator and store dH.
 #include <algorithm>
 
 #include "common.cuh"
 #include "plan.h"
+#include "tc_ptx.cuh"
 
 namespace ssd {
 namespace {
 
-constexpr int kTailThreads = 512;
-constexpr int kTailMax = 256;                      // tokens in the tail at most (2 chunks)
-constexpr int kTailCh = kHeadDim + kDState;        // 192 channels: the head's x, the group's B
-constexpr int kConvThreads = 2 * kTailCh;          // two 32-token strips per channel
-constexpr int kStep = 64;                          // tokens per conv + update round
-constexpr int kRawRows = 128 + 3;                  // one chunk and its 3 history rows
-constexpr size_t kRawBytes = (size_t)kRawRows * kTailCh * 2;           // bf16 raw rows
-constexpr size_t kOutBytes = (size_t)kStep * kTailCh * 4;              // one round's fp32 outputs
-constexpr size_t kTailSmem = kRawBytes + kOutBytes + kTailMax * 4;     // + token weights
-static_assert(2 * kTailSmem + 2048 <= 228 * 1024, "two tail CTAs per SM");
-static_assert(kTailThreads == 16 * 32 && kHeadDim == 64 && kDState == 128, "warp tiling assumes 64 x 128");
+using namespace tc;
+
+constexpr int kTailThreads = 768;
+constexpr int kTailHeads = 4;                        // heads per item
+constexpr int kTailMax = 256;                        // tokens in the tail at most (2 chunks)
+constexpr int kRound = 64;                           // tokens per round (the MMAs' K)
+constexpr int kRawCh = kTailHeads * kHeadDim + kDState;  // 384 staged channels: x of 4 heads, B
+constexpr int kPairs = kRawCh / 2;                   // a thread converts two adjacent channels
+constexpr int kStrips = kTailThreads / kPairs;       // 4 strips of 16 tokens per round
+constexpr int kStripTok = kRound / kStrips;
+constexpr int kRawRows = kRound + 3;                 // a round's rows and their 3 history rows
+// shared memory, bytes from a 1024-aligned base (the operand tiles need the alignment for the
+// 128-byte swizzle)
+constexpr uint32_t kRawBuf = (uint32_t)kRawRows * kRawCh * 2;  // bf16 raw rows, double-buffered
+constexpr uint32_t OFF_AH = 103424;                  // B^T high parts: 2 boxes of 64 tokens x 64 n
+constexpr uint32_t OFF_AL = OFF_AH + 16384;          // B^T low parts
+constexpr uint32_t OFF_XH = OFF_AL + 16384;          // w x high parts: 4 boxes of 64 tokens x 64 p
+constexpr uint32_t OFF_XL = OFF_XH + 32768;          // w x low parts
+constexpr uint32_t OFF_WS = OFF_XL + 32768;          // token weights [4 heads][256] fp32
+constexpr uint32_t OFF_BAR = OFF_WS + kTailHeads * kTailMax * 4;
+constexpr uint32_t OFF_MISC = OFF_BAR + 8;           // [0] TMEM base, [1] abort flag, [2] drain flag
+constexpr uint32_t kTailSmem = OFF_MISC + 16 + 1024;  // + room to align the base
+constexpr uint32_t kTailCols = kTailHeads * kHeadDim;  // the accumulator: 64 columns per head
+static_assert(2 * kRawBuf <= OFF_AH && OFF_AH % 1024 == 0 && OFF_XH % 1024 == 0 && OFF_XL % 1024 == 0,
+              "tile layout");
+static_assert(kTailSmem <= 232448, "shared memory budget");
+static_assert(kPairs * kStrips == kTailThreads && kPairs % 32 == 0 && kStripTok % 8 == 0,
+              "warps are uniform in role and strip");
+static_assert(kHeadDim == 64 && kDState == 128, "tiles assume 64 x 128");
 
 // 16-byte global -> shared copy that zero-fills when src_bytes is 0 (the source is not read).
 __device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_bytes) {
@@ -52,157 +75,308 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_b
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(g), "r"(src_bytes) : "memory");
 }
 
-__global__ void __launch_bounds__(kTailThreads, 2) state_tail_kernel(
+__device__ __forceinline__ float2 ld_bf16x2(const __nv_bfloat16 *p) {
+  const uint32_t u = *reinterpret_cast<const uint32_t *>(p);
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+
+// One item: heads h0 .. h0+nh-1 of group g of batch row b, and its tail tokens.
+struct TailItem {
+  int b, g, nh, h0, t_tail, ntok;
+  long long base;  // token row of the sequence's first token
+};
+
+__device__ __forceinline__ TailItem tail_item(int item, int nq, int G, int hpg, int L, int t_tail_uniform,
+                                              const int *cu) {
+  TailItem it;
+  const int q = item % nq, bg = item / nq;
+  it.g = bg % G;
+  it.b = bg / G;
+  it.nh = min(kTailHeads, hpg - kTailHeads * q);
+  it.h0 = it.g * hpg + kTailHeads * q;
+  // a packed variable-length batch has one segment per sequence, its tail the last two chunks
+  // of the sequence
+  const int Lb = seq_len(cu, it.b, L);
+  int t_tail = t_tail_uniform;
+  if (cu) {
+    const int nckb = (Lb + 127) / 128;
+    t_tail = 128 * (nckb > kTailChunks ? nckb - kTailChunks : 0);
+  }
+  it.t_tail = t_tail;
+  it.ntok = Lb - t_tail;  // 0 .. kTailMax
+  it.base = seq_base(cu, it.b, L);
+  return it;
+}
+
+// Asynchronous copies of round r's raw rows (times t_tail + 64r - 3 ..) of the item's x and B
+// channels into raw[row][384] (x of head i at columns 64i.., B at 256..), as one commit group.
+__device__ __forceinline__ void tail_stage(const TailItem &it, int r, __nv_bfloat16 *raw,
+                                           const __nv_bfloat16 *__restrict__ xBC, long long xs,
+                                           const __nv_bfloat16 *__restrict__ csi, int W, int conv_dim,
+                                           int d_inner, int tid) {
+  const int tok0 = r * kRound;
+  const int rows = min(kRawRows, it.ntok - tok0 + 3);
+  const int nx = 8 * it.nh, per = nx + 16;  // 16-byte pieces per row
+  const __nv_bfloat16 *xrow = xBC + it.base * xs;
+  for (int i = tid; i < rows * per; i += kTailThreads) {
+    const int k = i / per, v = i - k * per, tau = it.t_tail + tok0 - 3 + k;
+    int rc, c;
+    if (v < nx) {
+      rc = 64 * (v >> 3) + 8 * (v & 7);
+      c = (it.h0 + (v >> 3)) * kHeadDim + 8 * (v & 7);
+    } else {
+      rc = kTailHeads * kHeadDim + 8 * (v - nx);
+      c = d_inner + it.g * kDState + 8 * (v - nx);
+    }
+    const void *src = xBC;  // not read when zero-filling
+    int bytes = 0;
+    if (tau >= 0) {
+      src = xrow + (long long)tau * xs + c; bytes = 16;
+    } else if (csi && W + tau >= 0) {
+      src = csi + ((long long)it.b * W + (W + tau)) * conv_dim + c; bytes = 16;
+    }
+    cp_async16(raw + k * kRawCh + rc, src, bytes);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kTailThreads, 1) state_tail_kernel(
     const __nv_bfloat16 *__restrict__ xBC, long long xs, const __nv_bfloat16 *__restrict__ conv_w,
     const __nv_bfloat16 *__restrict__ conv_b, const __nv_bfloat16 *__restrict__ csi,
     const float *__restrict__ dte, const float *__restrict__ cs, float *__restrict__ dh_out,
-    float *__restrict__ dec_out, int L, int B, int H, int hpg, int conv_dim, int d_inner, int W,
-    int Lpad, int t_tail_uniform, const int *__restrict__ cu) {
-  extern __shared__ __align__(16) unsigned char tsm[];
-  __nv_bfloat16 *raw = reinterpret_cast<__nv_bfloat16 *>(tsm);       // [kRawRows][192]
-  float *uo = reinterpret_cast<float *>(tsm + kRawBytes);             // [64][192]
-  float *ws = reinterpret_cast<float *>(tsm + kRawBytes + kOutBytes);  // [256]
+    float *__restrict__ dec_out, int L, int B, int H, int G, int hpg, int conv_dim, int d_inner, int W,
+    int Lpad, int t_tail_uniform, const int *__restrict__ cu, int *err) {
+  extern __shared__ unsigned char tsm_raw[];
+  unsigned char *tsm =
+      reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(tsm);
+  float *ws = reinterpret_cast<float *>(tsm + OFF_WS);  // [4][256]
+  uint32_t *misc = reinterpret_cast<uint32_t *>(tsm + OFF_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
+  volatile int *drain_flag = reinterpret_cast<volatile int *>(misc + 2);
+  const uint32_t bar = sb + OFF_BAR;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int p0 = 16 * (warp >> 2) + 4 * (lane >> 3), n0 = 32 * (warp & 3) + 4 * (lane & 7);
-  // conv role: channel ch (column of raw / uo), 32-token strip hf of each round; tap j reads
-  // time t-3+j
-  const bool conv_thread = tid < kConvThreads;
-  const int ch = tid % kTailCh, hf = tid / kTailCh;
-  for (int item = blockIdx.x; item < B * H; item += gridDim.x) {
-    const int h = item % H, b = item / H, g = h / hpg;
-    // this row's tokens and tail (a packed variable-length batch has one segment per sequence,
-    // its tail the last two chunks of the sequence)
-    const int Lb = seq_len(cu, b, L);
-    int t_tail = t_tail_uniform;
-    if (cu) {
-      const int nckb = (Lb + 127) / 128;
-      t_tail = 128 * (nckb > kTailChunks ? nckb - kTailChunks : 0);
-    }
-    const int ntok = Lb - t_tail;  // 0 .. kTailMax
-    const __nv_bfloat16 *xrow = xBC + seq_base(cu, b, L) * xs;
-    const float *csr = cs + ((long long)b * H + h) * Lpad;
-    const float *dtr = dte + ((long long)b * H + h) * Lpad;
-
-    // token weights w_s = e^{cs_Q - cs_s} dt_s, cs_Q the prefix at the end of the token's chunk
-    // (chunk-local prefix sums; the padding past L has dt = 0, so the prefix stays flat there)
-    for (int i = tid; i < ntok; i += kTailThreads)
-      ws[i] = __expf(csr[t_tail + (i & ~127) + 127] - csr[t_tail + i]) * dtr[t_tail + i];
-    float acc[16];  // acc[4 i + j] = dH[p0 + i][n0 + j]
+  // conv role: channel pair `pair` (0-127: x of head pair / 32, 128-191: B), 16-token strip
+  const int pair = tid % kPairs, strip = tid / kPairs;
+  const bool is_x = pair < kTailHeads * 32;
+  const int xhead = pair >> 5;                        // x pairs: the head within the item
+  const int rcol = 2 * pair;                          // raw column (x of head i at 64i, B at 256)
+  const int tcol = is_x ? 2 * (pair & 31) : (2 * (pair - 128)) & 63;  // column within its box
+  unsigned char *hi_tile = tsm + (is_x ? OFF_XH + (uint32_t)xhead * 8192u
+                                       : OFF_AH + (uint32_t)((2 * (pair - 128)) >> 6) * 8192u);
+  unsigned char *lo_tile = hi_tile + (is_x ? OFF_XL - OFF_XH : OFF_AL - OFF_AH);
+  // byte offset of this thread's 4 bytes in a swizzled row r, by r mod 8 (16-byte chunk
+  // c / 8 of row r sits at chunk (c / 8) ^ (r % 8))
+  uint32_t loff[8];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-    const int cch = ch < kHeadDim ? h * kHeadDim + ch : d_inner + g * kDState + (ch - kHeadDim);
-    float wt[4] = {0.f, 0.f, 0.f, 0.f}, bias = 0.f;
-    if (conv_thread && W > 0) {
+  for (int u = 0; u < 8; ++u) loff[u] = ((uint32_t)(((tcol >> 3) ^ u) & 7) << 4) + (uint32_t)(tcol & 7) * 2u;
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    *abort_flag = 0;
+    *drain_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(sb + OFF_MISC, kTailCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  const int nq = (hpg + kTailHeads - 1) / kTailHeads;
+  const int items = B * G * nq;
+  uint32_t phase = 0;   // parity of the next commit's phase
+  uint32_t gr = 0;      // rounds staged so far (raw buffer gr % 2)
+  bool staged = false;  // the current item's first round is already staged
+  bool failed = false;  // a bounded wait ran out (uniform across the CTA)
+
+  for (int item = blockIdx.x; item < items && !failed; item += gridDim.x) {
+    const TailItem it = tail_item(item, nq, G, hpg, L, t_tail_uniform, cu);
+    const int nr = (it.ntok + kRound - 1) / kRound;
+    if (!staged && nr > 0)
+      tail_stage(it, 0, reinterpret_cast<__nv_bfloat16 *>(tsm + (gr & 1) * kRawBuf), xBC, xs, csi, W,
+                 conv_dim, d_inner, tid);
+    staged = false;
+    const int nch = (it.ntok + 127) / 128;
+    // token weights (the previous item's readers finished at its last barrier)
+    for (int i = tid; i < it.nh * kTailMax; i += kTailThreads) {
+      const int hh = i >> 8, t = i & (kTailMax - 1);
+      if (t < it.ntok) {
+        const long long row = ((long long)it.b * H + it.h0 + hh) * Lpad + it.t_tail;
+        const float later = (nch == 2 && t < 128) ? cs[row + 255] : 0.f;
+        ws[i] = __expf(cs[row + (t & ~127) + 127] - cs[row + t] + later) * dte[row + t];
+      }
+    }
+    const bool active = !is_x || xhead < it.nh;
+    const int cch = is_x ? (it.h0 + xhead) * kHeadDim + 2 * (pair & 31) : d_inner + it.g * kDState + 2 * (pair - 128);
+    float2 wt[4], bias = make_float2(0.f, 0.f);  // tap j multiplies time t-3+j
+#pragma unroll
+    for (int j = 0; j < 4; ++j) wt[j] = make_float2(0.f, 0.f);
+    if (W > 0 && active) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int k = j - (4 - W);
-        if (k >= 0) wt[j] = __bfloat162float(conv_w[(long long)cch * W + k]);
+        if (k >= 0)
+          wt[j] = make_float2(__bfloat162float(conv_w[(long long)cch * W + k]),
+                              __bfloat162float(conv_w[(long long)(cch + 1) * W + k]));
       }
-      if (conv_b) bias = __bfloat162float(conv_b[cch]);
+      if (conv_b) bias = make_float2(__bfloat162float(conv_b[cch]), __bfloat162float(conv_b[cch + 1]));
     }
+    const uint32_t idesc = idesc_f16(128, kHeadDim * it.nh, true, true, kFmtF16);
 
-    for (int c0 = 0; c0 < ntok; c0 += 128) {  // chunks of the tail (t_tail is chunk-aligned)
-      const int n = min(128, ntok - c0);
-      // raw rows of times t_tail+c0-3 .. t_tail+c0+n-1: 24 16-byte pieces per row (8 of x,
-      // 16 of B); the previous chunk's readers finished at the barrier that ended it
-      for (int i = tid; i < (n + 3) * 24; i += kTailThreads) {
-        const int r = i / 24, v = i % 24, tau = t_tail + c0 - 3 + r;
-        const int c = v < 8 ? h * kHeadDim + 8 * v : d_inner + g * kDState + 8 * (v - 8);
-        const void *src = xBC;  // not read when zero-filling
-        int bytes = 0;
-        if (tau >= 0) {
-          src = xrow + (long long)tau * xs + c; bytes = 16;
-        } else if (csi && W + tau >= 0) {
-          src = csi + ((long long)b * W + (W + tau)) * conv_dim + c; bytes = 16;
-        }
-        cp_async16(raw + r * kTailCh + 8 * v, src, bytes);
-      }
-      asm volatile("cp.async.commit_group;" ::: "memory");
+    for (int r = 0; r < nr && !failed; ++r, ++gr) {
+      const __nv_bfloat16 *raw = reinterpret_cast<const __nv_bfloat16 *>(tsm + (gr & 1) * kRawBuf);
       asm volatile("cp.async.wait_all;" ::: "memory");
-      __syncthreads();
-      const float decay = __expf(csr[t_tail + c0 + 127]);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) acc[j] *= decay;
-      for (int h0 = 0; h0 < n; h0 += kStep) {
-        const int m = min(kStep, n - h0);
-        if (conv_thread) {
-          const int s_lo = h0 + hf * (kStep / 2), s_hi = min(s_lo + kStep / 2, n);
-          if (s_lo < s_hi) {
-            const __nv_bfloat16 *col = raw + s_lo * kTailCh + ch;  // raw row of time t-3 for s_lo
-            float xm3 = __bfloat162float(col[0]), xm2 = __bfloat162float(col[kTailCh]),
-                  xm1 = __bfloat162float(col[2 * kTailCh]);
-            const bool is_x = ch < kHeadDim;
+      __syncthreads();  // this round's rows landed; the other buffer's last readers are done
+      {  // the next round's rows (or the next item's first) into the other buffer
+        __nv_bfloat16 *nxt = reinterpret_cast<__nv_bfloat16 *>(tsm + ((gr + 1) & 1) * kRawBuf);
+        if (r + 1 < nr) {
+          tail_stage(it, r + 1, nxt, xBC, xs, csi, W, conv_dim, d_inner, tid);
+        } else if (item + (int)gridDim.x < items) {
+          const TailItem nx = tail_item(item + gridDim.x, nq, G, hpg, L, t_tail_uniform, cu);
+          if (nx.ntok > 0) {
+            tail_stage(nx, 0, nxt, xBC, xs, csi, W, conv_dim, d_inner, tid);
+            staged = true;
+          }
+        }
+      }
+      // the previous round's products read the tiles that this round rewrites
+      if (r > 0) {
+        mbar_wait(bar, phase, abort_flag, err);
+        phase ^= 1u;
+      }
+      const int tok0 = r * kRound, s_lo = strip * kStripTok;
+      if (active) {  // conv + SiLU of 16 tokens of two channels; rows past the tail are zero
+        const __nv_bfloat16 *colp = raw + s_lo * kRawCh + rcol;  // raw row of time t-3 for s_lo
+        float2 xm3 = ld_bf16x2(colp), xm2 = ld_bf16x2(colp + kRawCh), xm1 = ld_bf16x2(colp + 2 * kRawCh);
+        const int nvalid = it.ntok - tok0 - s_lo;
+        const float *wsr = ws + xhead * kTailMax + tok0 + s_lo;
 #pragma unroll 8
-            for (int s = s_lo; s < s_hi; ++s) {
-              const float x0 = __bfloat162float(raw[(s + 3) * kTailCh + ch]);
-              float v = x0;
-              if (W > 0) v = silu(fmaf(wt[0], xm3, fmaf(wt[1], xm2, fmaf(wt[2], xm1, fmaf(wt[3], x0, bias)))));
-              uo[(s - h0) * kTailCh + ch] = is_x ? v * ws[c0 + s] : v;
-              xm3 = xm2; xm2 = xm1; xm1 = x0;
+        for (int i = 0; i < kStripTok; ++i) {
+          uint32_t hw = 0u, lw = 0u;
+          if (i < nvalid) {
+            const float2 x0 = ld_bf16x2(colp + (i + 3) * kRawCh);
+            float2 v = x0;
+            if (W > 0) {
+              const float2 a = __ffma2_rn(wt[3], x0, __ffma2_rn(wt[2], xm1, __ffma2_rn(wt[1], xm2, __ffma2_rn(wt[0], xm3, bias))));
+              v = make_float2(silu(a.x), silu(a.y));
             }
+            if (is_x) {
+              const float w = wsr[i];
+              v = make_float2(v.x * w, v.y * w);
+            }
+            const __half2 hi = __float22half2_rn(v);
+            const float2 hf = __half22float2(hi);
+            const __half2 lo = __float22half2_rn(make_float2(v.x - hf.x, v.y - hf.y));
+            hw = *reinterpret_cast<const uint32_t *>(&hi);
+            lw = *reinterpret_cast<const uint32_t *>(&lo);
+            xm3 = xm2; xm2 = xm1; xm1 = x0;
           }
+          const uint32_t off = (uint32_t)(s_lo + i) * 128u + loff[i & 7];
+          *reinterpret_cast<uint32_t *>(hi_tile + off) = hw;
+          *reinterpret_cast<uint32_t *>(lo_tile + off) = lw;
         }
-        __syncthreads();  // the round's conv outputs are ready
-#pragma unroll 4
-        for (int s = 0; s < m; ++s) {
-          const float4 xv = *reinterpret_cast<const float4 *>(uo + s * kTailCh + p0);  // weighted x
-          const float4 bv = *reinterpret_cast<const float4 *>(uo + s * kTailCh + kHeadDim + n0);
-          const float2 b01 = make_float2(bv.x, bv.y), b23 = make_float2(bv.z, bv.w);
-          const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
+      }
+      fence_proxy_async();  // the tiles' generic writes, visible to the tensor cores
+      if (__syncthreads_or(*abort_flag != 0)) {
+        failed = true;
+        break;
+      }
+      if (tid == 0) {  // dH^T (128 n x 64 nh p) += the round's three fp16 products
+        tc_fence_after();
+        const uint64_t ah = smem_desc_sw128(sb + OFF_AH, 8192, 1024), al = smem_desc_sw128(sb + OFF_AL, 8192, 1024);
+        const uint64_t xh = smem_desc_sw128(sb + OFF_XH, 8192, 1024), xl = smem_desc_sw128(sb + OFF_XL, 8192, 1024);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 a2 = make_float2(xa[i], xa[i]);
-            const float2 lo = __ffma2_rn(a2, b01, make_float2(acc[4 * i], acc[4 * i + 1]));
-            const float2 hi = __ffma2_rn(a2, b23, make_float2(acc[4 * i + 2], acc[4 * i + 3]));
-            acc[4 * i] = lo.x; acc[4 * i + 1] = lo.y; acc[4 * i + 2] = hi.x; acc[4 * i + 3] = hi.y;
-          }
+        for (int j = 0; j < kRound / 16; ++j) {
+          // K step j: 16 token rows of 128 bytes further (the descriptors' address field is in
+          // 16-byte units and every address here lies below 256 KB, so the add stays in it)
+          const uint64_t o = (uint64_t)((j * 2048) >> 4);
+          mma_f16_ss(tmem, ah + o, xh + o, idesc, (r > 0 || j > 0) ? 1u : 0u);
+          mma_f16_ss(tmem, ah + o, xl + o, idesc, 1u);
+          mma_f16_ss(tmem, al + o, xh + o, idesc, 1u);
         }
-        __syncthreads();  // the outputs (and raw rows, weights) are consumed before they are rewritten
+        mma_commit(bar);
       }
     }
-    if (tid == 0) {  // decay over the tail's chunks
-      float sum = 0.f;
-      for (int c0 = 0; c0 < ntok; c0 += 128) sum += csr[t_tail + c0 + 127];
-      dec_out[(long long)b * H + h] = __expf(sum);
+    if (failed) break;
+    if (nr > 0) {  // the last round's products
+      mbar_wait(bar, phase, abort_flag, err);
+      phase ^= 1u;
+      tc_fence_after();
+      if (__syncthreads_or(*abort_flag != 0)) {
+        failed = true;
+        break;
+      }
     }
-    float *dblk = dh_out + (((long long)b * H + h) * kHeadDim + p0) * kDState + n0;
+    if (tid < it.nh) {  // decay over the tail's chunks
+      const float *csr = cs + ((long long)it.b * H + it.h0 + tid) * Lpad + it.t_tail;
+      float sum = 0.f;
+      for (int c0 = 0; c0 < it.ntok; c0 += 128) sum += csr[c0 + 127];
+      dec_out[(long long)it.b * H + it.h0 + tid] = __expf(sum);
+    }
+    if (warp < 4 * kTailHeads && (warp >> 2) < it.nh) {  // dH of head warp / 4, lanes 32 (warp % 4) ..
+      const int hh = warp >> 2, qd = warp & 3, nn = 32 * qd + lane;
+      float *dst = dh_out + ((long long)it.b * H + it.h0 + hh) * kHeadDim * kDState + nn;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {  // 16 columns (p) at a time
+        float a[16];
+        if (nr > 0) {
+          tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + (uint32_t)(kHeadDim * hh + 16 * c), a);
+          tmem_ld_wait();
+        }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      *reinterpret_cast<float4 *>(dblk + i * kDState) = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+        for (int i = 0; i < 16; ++i) dst[(16 * c + i) * kDState] = nr > 0 ? a[i] : 0.f;  // 32 consecutive n
+      }
+    }
+    tc_fence_before();
+    __syncthreads();  // the accumulator is read before the next item's first product
+    tc_fence_after();
   }  // item
+  // after a wait ran out, the products it waited for may still be in flight: wait for them
+  // (within 0.1 s, on a flag of its own, since the abort flag ends a wait at once) before the
+  // accumulator is freed; copies still in flight land in this CTA's own shared memory
+  if (failed && tid == 0) mbar_wait(bar, phase ^ 1u, drain_flag, nullptr, 100000000ull);
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTailCols);
+  }
 }
 
 }  // namespace
 
-// One tail item (a head of a batch row) costs about as much as this many chunks of the scan.
-constexpr int kItemChunks = 8;
+// One tail item (four heads of a batch row) costs about as much as this many chunks of the scan.
+constexpr int kItemChunks = 4;
 
 // The tail starts at chunk nck-kTailChunks of the last segment (its first chunk when it has
-// fewer).  Grid: two CTAs on each SM the output scan (one CTA per SM, n_seg x H x B of them)
-// leaves free, when they finish all items within the scan's time; otherwise two per SM of the
+// fewer).  Grid: one CTA on each SM the output scan (one CTA per SM, n_seg x H x B of them)
+// leaves free, when they finish all items within the scan's time; otherwise one per SM of the
 // whole GPU, up to one CTA per item.
 cudaError_t launch_state_tail(const PrefillPlan &p, cudaStream_t s) {
-  static_assert(kTailChunks * 128 <= kTailMax, "tail longer than the staging buffers");
+  static_assert(kTailChunks * 128 <= kTailMax, "tail longer than the weight buffer");
   if (!p.tail_dh || p.L == 0) return cudaSuccess;
+  if (p.xs % 8 || p.conv_dim % 8 || p.d_inner % 8) return cudaErrorInvalidValue;  // 16-byte copies
   const int t_b = (p.n_seg - 1) * p.seg_len;
   const int nck = (p.L - t_b + 127) / 128;
   const int t_tail = t_b + 128 * (nck > kTailChunks ? nck - kTailChunks : 0);
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long items = (long long)p.B * p.H;
+  const long long items = (long long)p.B * p.G * ((p.hpg + kTailHeads - 1) / kTailHeads);
   const long long scan_ctas = (long long)p.n_seg * p.H * p.B;
   const long long seg_chunks = (p.seg_len + 127) / 128;
   const long long free_sms = sms - scan_ctas;
   const long long need = (items * kItemChunks + seg_chunks - 1) / seg_chunks;  // CTAs to keep pace
-  // two CTAs per SM
-  long long grid = 2 * (free_sms >= need && free_sms >= 1 ? free_sms : sms);
+  long long grid = free_sms >= need && free_sms >= 1 ? free_sms : sms;
   if (grid > items) grid = items;
   cudaError_t e = set_smem_attr(state_tail_kernel, kTailSmem, s);
   if (e != cudaSuccess) return e;
   state_tail_kernel<<<(unsigned)grid, kTailThreads, kTailSmem, s>>>(
       (const __nv_bfloat16 *)p.xBC, p.xs, (const __nv_bfloat16 *)p.conv_w, (const __nv_bfloat16 *)p.conv_b,
-      (const __nv_bfloat16 *)p.csi, p.dte_hm, p.cs_hm, p.tail_dh, p.tail_dec, p.L, p.B, p.H, p.hpg,
-      p.conv_dim, p.d_inner, p.W, p.Lpad, t_tail, p.cu);
+      (const __nv_bfloat16 *)p.csi, p.dte_hm, p.cs_hm, p.tail_dh, p.tail_dec, p.L, p.B, p.H, p.G, p.hpg,
+      p.conv_dim, p.d_inner, p.W, p.Lpad, t_tail, p.cu, p.err);
   return cudaGetLastError();
 }
 
