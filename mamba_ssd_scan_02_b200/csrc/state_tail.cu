@@ -30,6 +30,7 @@
 // (the dropped lo*lo term is below 2^-22 of the product), which keeps the update at fp32
 // accuracy.  Sixteen warps finally read the accumulator and store dH.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "plan.h"
@@ -110,28 +111,31 @@ __device__ __forceinline__ TailItem tail_item(int item, int nq, int G, int hpg, 
 
 // Asynchronous copies of round r's raw rows (times t_tail + 64r - 3 ..) of the item's x and B
 // channels into raw[row][384] (x of head i at columns 64i.., B at 256..), as one commit group.
+// A row is 48 pieces of 16 bytes; thread tid copies piece tid % 48 of rows tid / 48, +16, ...
+constexpr int kPieces = kRawCh / 8;
+constexpr int kRowsPerPass = kTailThreads / kPieces;
+static_assert(kTailThreads % kPieces == 0, "whole rows per pass");
 __device__ __forceinline__ void tail_stage(const TailItem &it, int r, __nv_bfloat16 *raw,
                                            const __nv_bfloat16 *__restrict__ xBC, long long xs,
                                            const __nv_bfloat16 *__restrict__ csi, int W, int conv_dim,
                                            int d_inner, int tid) {
   const int tok0 = r * kRound;
   const int rows = min(kRawRows, it.ntok - tok0 + 3);
-  const int nx = 8 * it.nh, per = nx + 16;  // 16-byte pieces per row
-  const __nv_bfloat16 *xrow = xBC + it.base * xs;
-  for (int i = tid; i < rows * per; i += kTailThreads) {
-    const int k = i / per, v = i - k * per, tau = it.t_tail + tok0 - 3 + k;
-    int rc, c;
-    if (v < nx) {
-      rc = 64 * (v >> 3) + 8 * (v & 7);
-      c = (it.h0 + (v >> 3)) * kHeadDim + 8 * (v & 7);
-    } else {
-      rc = kTailHeads * kHeadDim + 8 * (v - nx);
-      c = d_inner + it.g * kDState + 8 * (v - nx);
-    }
+  const int v = tid % kPieces;
+  const bool vx = v < 8 * kTailHeads;
+  if (vx && (v >> 3) >= it.nh) {  // a head the item does not have
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    return;
+  }
+  const int rc = 8 * v;  // raw column: x of head v / 8, then B
+  const int c = vx ? (it.h0 + (v >> 3)) * kHeadDim + 8 * (v & 7) : d_inner + it.g * kDState + 8 * (v - 8 * kTailHeads);
+  const __nv_bfloat16 *xcol = xBC + it.base * xs + c;
+  for (int k = tid / kPieces; k < rows; k += kRowsPerPass) {
+    const int tau = it.t_tail + tok0 - 3 + k;
     const void *src = xBC;  // not read when zero-filling
     int bytes = 0;
     if (tau >= 0) {
-      src = xrow + (long long)tau * xs + c; bytes = 16;
+      src = xcol + (long long)tau * xs; bytes = 16;
     } else if (csi && W + tau >= 0) {
       src = csi + ((long long)it.b * W + (W + tau)) * conv_dim + c; bytes = 16;
     }
@@ -147,8 +151,9 @@ __global__ void __launch_bounds__(kTailThreads, 1) state_tail_kernel(
     float *__restrict__ dec_out, int L, int B, int H, int G, int hpg, int conv_dim, int d_inner, int W,
     int Lpad, int t_tail_uniform, const int *__restrict__ cu, int *err) {
   extern __shared__ unsigned char tsm_raw[];
-  unsigned char *tsm =
-      reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~uintptr_t(1023));
+  // aligned by an offset from the shared array itself (not through an integer), so that the
+  // compiler keeps every access derived from it in the shared address space
+  unsigned char *tsm = tsm_raw + ((1024u - (smem_u32(tsm_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(tsm);
   float *ws = reinterpret_cast<float *>(tsm + OFF_WS);  // [4][256]
   uint32_t *misc = reinterpret_cast<uint32_t *>(tsm + OFF_MISC);
@@ -249,34 +254,40 @@ __global__ void __launch_bounds__(kTailThreads, 1) state_tail_kernel(
       const int tok0 = r * kRound, s_lo = strip * kStripTok;
       if (active) {  // conv + SiLU of 16 tokens of two channels; rows past the tail are zero
         const __nv_bfloat16 *colp = raw + s_lo * kRawCh + rcol;  // raw row of time t-3 for s_lo
-        float2 xm3 = ld_bf16x2(colp), xm2 = ld_bf16x2(colp + kRawCh), xm1 = ld_bf16x2(colp + 2 * kRawCh);
         const int nvalid = it.ntok - tok0 - s_lo;
         const float *wsr = ws + xhead * kTailMax + tok0 + s_lo;
+        // the strip's tokens, all present (kFull) or checked one by one
+        auto strip_tokens = [&](auto full_tag) {
+          constexpr bool kFull = decltype(full_tag)::value;
+          float2 xm3 = ld_bf16x2(colp), xm2 = ld_bf16x2(colp + kRawCh), xm1 = ld_bf16x2(colp + 2 * kRawCh);
 #pragma unroll 8
-        for (int i = 0; i < kStripTok; ++i) {
-          uint32_t hw = 0u, lw = 0u;
-          if (i < nvalid) {
-            const float2 x0 = ld_bf16x2(colp + (i + 3) * kRawCh);
-            float2 v = x0;
-            if (W > 0) {
-              const float2 a = __ffma2_rn(wt[3], x0, __ffma2_rn(wt[2], xm1, __ffma2_rn(wt[1], xm2, __ffma2_rn(wt[0], xm3, bias))));
-              v = make_float2(silu(a.x), silu(a.y));
+          for (int i = 0; i < kStripTok; ++i) {
+            uint32_t hw = 0u, lw = 0u;
+            if (kFull || i < nvalid) {
+              const float2 x0 = ld_bf16x2(colp + (i + 3) * kRawCh);
+              float2 v = x0;
+              if (W > 0) {
+                const float2 a = __ffma2_rn(wt[3], x0, __ffma2_rn(wt[2], xm1, __ffma2_rn(wt[1], xm2, __ffma2_rn(wt[0], xm3, bias))));
+                v = make_float2(silu(a.x), silu(a.y));
+              }
+              if (is_x) {
+                const float w = wsr[i];
+                v = __fmul2_rn(v, make_float2(w, w));
+              }
+              const __half2 hi = __float22half2_rn(v);
+              const float2 hf = __half22float2(hi);
+              const __half2 lo = __float22half2_rn(make_float2(v.x - hf.x, v.y - hf.y));
+              hw = *reinterpret_cast<const uint32_t *>(&hi);
+              lw = *reinterpret_cast<const uint32_t *>(&lo);
+              xm3 = xm2; xm2 = xm1; xm1 = x0;
             }
-            if (is_x) {
-              const float w = wsr[i];
-              v = make_float2(v.x * w, v.y * w);
-            }
-            const __half2 hi = __float22half2_rn(v);
-            const float2 hf = __half22float2(hi);
-            const __half2 lo = __float22half2_rn(make_float2(v.x - hf.x, v.y - hf.y));
-            hw = *reinterpret_cast<const uint32_t *>(&hi);
-            lw = *reinterpret_cast<const uint32_t *>(&lo);
-            xm3 = xm2; xm2 = xm1; xm1 = x0;
+            const uint32_t off = (uint32_t)(s_lo + i) * 128u + loff[i & 7];
+            *reinterpret_cast<uint32_t *>(hi_tile + off) = hw;
+            *reinterpret_cast<uint32_t *>(lo_tile + off) = lw;
           }
-          const uint32_t off = (uint32_t)(s_lo + i) * 128u + loff[i & 7];
-          *reinterpret_cast<uint32_t *>(hi_tile + off) = hw;
-          *reinterpret_cast<uint32_t *>(lo_tile + off) = lw;
-        }
+        };
+        if (nvalid >= kStripTok) strip_tokens(std::true_type{});
+        else strip_tokens(std::false_type{});
       }
       fence_proxy_async();  // the tiles' generic writes, visible to the tensor cores
       if (__syncthreads_or(*abort_flag != 0)) {

@@ -245,8 +245,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     ssd_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_bc,
                        const __grid_constant__ CUtensorMap tm_x, const TcArgs a) {
   extern __shared__ unsigned char smem_raw[];
-  unsigned char *smem =
-      reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // aligned by an offset from the shared array itself (not through an integer), so that the
+  // compiler keeps every access derived from it in the shared address space
+  unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z, g = h / a.hpg;
