@@ -240,7 +240,9 @@ __device__ __forceinline__ void write_h_tile(unsigned char *smem, const float (&
   }
 }
 
-template <bool kStateOnly>
+// kStateOnly: the states-only pass (no y); kConv: the x channels have a causal conv (W > 0),
+// a compile-time switch so that the token loops carry no branch on it.
+template <bool kStateOnly, bool kConv>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     ssd_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_bc,
                        const __grid_constant__ CUtensorMap tm_x, const TcArgs a) {
@@ -441,7 +443,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     const int cw = conv_index(warp);
     const bool leader = (tid == 2 * 32);  // releases the stage
     const int ch = h * 64 + 2 * lane;
-    const int W = a.W;
+    const int W = kConv ? a.W : 0;
     float2 ew[4], bias2 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {  // half the weight for the input at time t-3+j
@@ -526,7 +528,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
               const int i = 8 * g + u;
               const __half2 x0 = xn[u];
               __half2 xo = x0;
-              if (W != 0) {
+              if (kConv) {
                 __half2 acc = __hfma2(hw[0], xm3, hbias);
                 acc = __hfma2(hw[1], xm2, acc);
                 acc = __hfma2(hw[2], xm1, acc);
@@ -561,7 +563,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             const int i = 8 * g + u;
             const float2 x0 = xn[u];
             float2 acc = x0;
-            if (W != 0) {
+            if (kConv) {
               acc = __ffma2_rn(ew[0], xm3, bias2);
               acc = __ffma2_rn(ew[1], xm2, acc);
               acc = __ffma2_rn(ew[2], xm1, acc);
@@ -572,8 +574,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
               // The final state's chunk: its newest tokens dominate the final state, so X
               // comes from the fp32 SiLU and w o X is stored as the fp16 hi + lo parts of the
               // fp32 product.
-              const float u0 = W != 0 ? silu(2.f * acc.x) : acc.x;
-              const float u1 = W != 0 ? silu(2.f * acc.y) : acc.y;
+              const float u0 = kConv ? silu(2.f * acc.x) : acc.x;
+              const float u1 = kConv ? silu(2.f * acc.y) : acc.y;
               const float ws = __shfl_sync(0xffffffffu, wl, i);
               const float2 v = make_float2(u0 * ws, u1 * ws);
               const __half2 hi = __float22half2_rn(v);
@@ -938,9 +940,10 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
   if (mode == 1) {
     a.h_init = nullptr; a.h_init_seg = 0;
     a.h_out = p.seg_state; a.h_out_seg = seg_stride; a.seg_decay = p.seg_decay;
-    e = set_smem_attr(ssd_scan_tc_kernel<true>, kSmemAlloc, s);
+    auto kern = p.W > 0 ? ssd_scan_tc_kernel<true, true> : ssd_scan_tc_kernel<true, false>;
+    e = set_smem_attr(kern, kSmemAlloc, s);
     if (e != cudaSuccess) return e;
-    ssd_scan_tc_kernel<true><<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, a);
+    kern<<<grid, kThreadsTC, kSmemAlloc, s>>>(tm, tmx, a);
   } else {
     if (p.n_seg > 1) {
       a.h_init = p.seg_state; a.h_init_seg = seg_stride;
@@ -951,7 +954,8 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
     // adds what those chunks contribute
     a.h_out = p.h_final; a.h_out_seg = 0; a.seg_decay = nullptr;
     a.tail_chunks = p.tail_dh ? kTailChunks : 0;
-    e = set_smem_attr(ssd_scan_tc_kernel<false>, kSmemAlloc, s);
+    auto kern = p.W > 0 ? ssd_scan_tc_kernel<false, true> : ssd_scan_tc_kernel<false, false>;
+    e = set_smem_attr(kern, kSmemAlloc, s);
     if (e != cudaSuccess) return e;
     // Programmatic dependent launch when the front end directly precedes the scan: the scan's
     // set-up (TMEM, barriers, tensor maps, its first raw x loads) overlaps the front end's tail,
@@ -963,7 +967,7 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[0].val.programmaticStreamSerializationAllowed = p.n_seg == 1 ? 1 : 0;
     lc.attrs = at; lc.numAttrs = 1;
-    e = cudaLaunchKernelEx(&lc, ssd_scan_tc_kernel<false>, tm, tmx, a);
+    e = cudaLaunchKernelEx(&lc, kern, tm, tmx, a);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
