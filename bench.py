@@ -613,9 +613,15 @@ def bench_varlen(c: Ctx, nseq=128):
     h0 = ssd.to_device(datagen.random_state(seed, (nseq, H, P, N)))
     csi = ssd.to_device(datagen.random_conv_state(seed, (nseq, W, datagen.conv_dim(cfg))))
 
+    vws = ssd.alloc_workspace(ssd.varlen_workspace_size(cfg, cu), c.dev)
+
     def one_pass():
         ssd.prefill_varlen(cfg, cu, x, dtt, d["A"], d["D"], d["dt_bias"], d["conv_w"], None, None,
-                           None, h0, csi)
+                           None, h0, csi, workspace=vws)
+
+    def one_pass_no_state():
+        ssd.prefill_varlen(cfg, cu, x, dtt, d["A"], d["D"], d["dt_bias"], d["conv_w"], None, None,
+                           None, h0, csi, workspace=vws, want_state=False)
 
     ws = ssd.alloc_workspace(max(ssd.workspace_size(dict(cfg, seqlen=int(L))) for L in lens), c.dev)
 
@@ -627,7 +633,8 @@ def bench_varlen(c: Ctx, nseq=128):
                         workspace=ws)
 
     res = {}
-    for name, fn in (("one_pass", one_pass), ("per_sequence_calls", per_sequence)):
+    for name, fn in (("one_pass", one_pass), ("one_pass_without_final_states", one_pass_no_state),
+                     ("per_sequence_calls", per_sequence)):
         for _ in range(args.warmup):
             fn()
         ms, recs, _ = c.timed(fn, args.steps, flush=True, trace=(name == "one_pass"))

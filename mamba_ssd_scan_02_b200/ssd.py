@@ -207,6 +207,13 @@ def workspace_size(cfg: dict, seqlen: int | None = None, kernel: int | None = No
     return load().ssd_workspace_size(ctypes.byref(c))
 
 
+def varlen_workspace_size(cfg: dict, cu_seqlens, kernel: int | None = None) -> int:
+    """ssd_varlen_workspace_size for the packed batch with offsets cu_seqlens."""
+    cu = [int(v) for v in cu_seqlens]
+    c = make_config(dict(cfg, batch=1), seqlen=cu[-1], kernel=kernel)
+    return load().ssd_varlen_workspace_size(ctypes.byref(c), (c_int * len(cu))(*cu), len(cu) - 1)
+
+
 def alloc_workspace(nbytes: int, device="cuda"):
     import torch
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
@@ -274,10 +281,12 @@ def prefill_noalloc(cfg: dict, xBC, dt, A, D, dt_bias, conv_w=None, conv_b=None,
 
 
 def prefill_varlen(cfg: dict, cu_seqlens, xBC, dt, A, D, dt_bias, conv_w=None, conv_b=None, z=None,
-                   norm_w=None, h0=None, conv_state_in=None, *, stream=None, kernel: int | None = None):
+                   norm_w=None, h0=None, conv_state_in=None, *, workspace=None, stream=None,
+                   want_state: bool = True, kernel: int | None = None):
     """ssd_prefill_varlen: packed sequences xBC [T, conv_dim] (T = cu_seqlens[-1]) with
-    per-sequence carries [nseq, ...]; returns (y [T, d_inner], h_final [nseq, H, P, N],
-    conv_state_out [nseq, W, conv_dim] or None)."""
+    per-sequence carries [nseq, ...]; returns (y [T, d_inner], h_final [nseq, H, P, N] or None
+    when want_state is False, conv_state_out [nseq, W, conv_dim] or None).  Without the final
+    states the library skips the pass that computes their last chunks."""
     import torch
     lib = load()
     cu = [int(v) for v in cu_seqlens]
@@ -287,10 +296,11 @@ def prefill_varlen(cfg: dict, cu_seqlens, xBC, dt, A, D, dt_bias, conv_w=None, c
     d_inner, conv_dim = H * P, H * P + 2 * G * N
     dev = xBC.device
     y = torch.empty((T, d_inner), dtype=io_dtype(cfg), device=dev)
-    h_final = torch.empty((nseq, H, P, N), dtype=torch.float32, device=dev)
+    h_final = torch.empty((nseq, H, P, N), dtype=torch.float32, device=dev) if want_state else None
     cso = torch.empty((nseq, W, conv_dim), dtype=io_dtype(cfg), device=dev) if W > 0 else None
     cu_arr = (c_int * (nseq + 1))(*cu)
-    workspace = alloc_workspace(lib.ssd_varlen_workspace_size(ctypes.byref(c), cu_arr, nseq), dev)
+    if workspace is None:
+        workspace = alloc_workspace(lib.ssd_varlen_workspace_size(ctypes.byref(c), cu_arr, nseq), dev)
     a = PrefillArgs(
         xBC=_ptr(xBC), xBC_row_stride=xBC.stride(-2), dt=_ptr(dt), dt_row_stride=dt.stride(-2),
         z=_ptr(z), z_row_stride=z.stride(-2) if z is not None else 0, A=_ptr(A), D=_ptr(D),

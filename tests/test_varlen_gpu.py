@@ -27,11 +27,29 @@ def _case():
     return cfg, cu, inp
 
 
-def _gpu(cfg, cu, inp):
+def _gpu(cfg, cu, inp, **kw):
     from mamba_ssd_scan_02_b200 import ssd
     return ssd.prefill_varlen(cfg, cu, dev(inp["xBC"][0]), dev(inp["dt"][0]), dev(inp["A"]), dev(inp["D"]),
                               dev(inp["dt_bias"]), dev(inp["conv_w"]), None, dev(inp["z"][0]),
-                              dev(inp["norm_w"]), dev(inp["h0"]), dev(inp["conv_state_in"]))
+                              dev(inp["norm_w"]), dev(inp["h0"]), dev(inp["conv_state_in"]), **kw)
+
+
+def test_varlen_without_final_states(cuda_lib):
+    """Without final states the pass that computes their last chunks does not run (no
+    ssd_state_tail launch), and y and the conv caches are bit-identical to the full call's."""
+    import torch
+    from mamba_ssd_scan_02_b200 import ssd
+    cfg, cu, inp = _case()
+    y, hf, cso = _gpu(cfg, cu, inp)
+    ssd.trace_enable(True)
+    ssd.trace_read()
+    try:
+        y2, hf2, cso2 = _gpu(cfg, cu, inp, want_state=False)
+        names = [n for n, _ in ssd.trace_read()]
+    finally:
+        ssd.trace_enable(False)
+    assert hf2 is None and "ssd_state_tail" not in names, names
+    assert torch.equal(y, y2) and torch.equal(cso, cso2)
 
 
 def test_varlen_matches_oracle_per_sequence(cuda_lib, oracle):
