@@ -576,6 +576,9 @@ def bench_mixer(c: Ctx):
     per, table, dom = kernel_table(recs)
     fl = mixer_flops(cfg)
     pk, src = peaks()
+    sus, sus_src = pk.get("bf16_tflops_sustained"), src
+    if not sus:
+        sus, sus_src = FALLBACK_PEAKS["bf16_tflops_sustained"], "fallback"
     gemm_ms = statistics.mean(per["gemm_in_proj"])
     ach = fl["in_proj"] / (gemm_ms * 1e-3) / 1e12
     step_ms = total_ms / args.steps
@@ -585,12 +588,15 @@ def bench_mixer(c: Ctx):
             "layer_tflops": round(sum(fl.values()) / (step_ms * 1e-3) / 1e12, 1),
             "flops_per_step": fl, "gpu_launches": len(recs), "kernels": table, "clocks": clocks,
             "l2": "not flushed (hidden 671 MB per step)",
-            "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": pk["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": round(ach / pk["bf16_tflops"], 4),
+            # the GEMM runs inside a long step under the power cap: the sustained peak is its
+            # roof (the burst fraction is reported beside it)
+            "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": sus,
+                         "unit": "TFLOP/s", "frac": round(ach / sus, 4),
+                         "frac_of_burst": round(ach / pk["bf16_tflops"], 4),
                          "traffic": recorded_traffic("gemm_tc_kernel", "mixer_12b_in_proj"),
                          "kernel": "gemm_in_proj (gemm_tc_kernel)", "kernel_ms": round(gemm_ms, 4),
                          "algorithmic_flops": fl["in_proj"],
-                         "peak_source": f"{src} cuBLAS bf16 (burst)"},
+                         "peak_source": f"{sus_src} cuBLAS bf16 (sustained, seconds-long loop under the power cap)"},
             "dominant_kernel": dom}
 
 
