@@ -76,6 +76,26 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_b
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(g), "r"(src_bytes) : "memory");
 }
 
+// SiLU(a) = a / (1 + e^{-a}) = a / (1 + 2^{-a log2(e)}), two values at a time, from the
+// hardware base-2 exponential and reciprocal approximations (each within a few units in the
+// last place of fp32): about 2^-21 relative error, well inside the pass's fp32 accuracy (the
+// final state's error is dominated by the fp32 prefix sums of dt*A it shares with the scan)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float2 silu2(float2 a) {
+  const float2 t = __fmul2_rn(a, make_float2(-1.4426950408889634f, -1.4426950408889634f));
+  const float2 d = __fadd2_rn(make_float2(1.f, 1.f), make_float2(ex2_approx(t.x), ex2_approx(t.y)));
+  return __fmul2_rn(a, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+}
+
 __device__ __forceinline__ float2 ld_bf16x2(const __nv_bfloat16 *p) {
   const uint32_t u = *reinterpret_cast<const uint32_t *>(p);
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
@@ -256,9 +276,13 @@ __global__ void __launch_bounds__(kTailThreads, 1) state_tail_kernel(
         const __nv_bfloat16 *colp = raw + s_lo * kRawCh + rcol;  // raw row of time t-3 for s_lo
         const int nvalid = it.ntok - tok0 - s_lo;
         const float *wsr = ws + xhead * kTailMax + tok0 + s_lo;
-        // the strip's tokens, all present (kFull) or checked one by one
-        auto strip_tokens = [&](auto full_tag) {
-          constexpr bool kFull = decltype(full_tag)::value;
+        unsigned char *hrow = hi_tile + (uint32_t)s_lo * 128u;  // row s_lo of this thread's hi tile
+        // the strip's tokens, all present (kFull) or checked one by one; kX: x channels (times
+        // w_s); kConv: a causal conv (W > 0) -- compile-time, so the unrolled loop has no branch
+        auto strip_tokens = [&](auto full_tag, auto x_tag, auto conv_tag) {
+          constexpr bool kFull = decltype(full_tag)::value, kX = decltype(x_tag)::value,
+                         kConv = decltype(conv_tag)::value;
+          constexpr uint32_t kLo = kX ? OFF_XL - OFF_XH : OFF_AL - OFF_AH;  // lo tile after the hi one
           float2 xm3 = ld_bf16x2(colp), xm2 = ld_bf16x2(colp + kRawCh), xm1 = ld_bf16x2(colp + 2 * kRawCh);
 #pragma unroll 8
           for (int i = 0; i < kStripTok; ++i) {
@@ -266,11 +290,9 @@ __global__ void __launch_bounds__(kTailThreads, 1) state_tail_kernel(
             if (kFull || i < nvalid) {
               const float2 x0 = ld_bf16x2(colp + (i + 3) * kRawCh);
               float2 v = x0;
-              if (W > 0) {
-                const float2 a = __ffma2_rn(wt[3], x0, __ffma2_rn(wt[2], xm1, __ffma2_rn(wt[1], xm2, __ffma2_rn(wt[0], xm3, bias))));
-                v = make_float2(silu(a.x), silu(a.y));
-              }
-              if (is_x) {
+              if constexpr (kConv)
+                v = silu2(__ffma2_rn(wt[3], x0, __ffma2_rn(wt[2], xm1, __ffma2_rn(wt[1], xm2, __ffma2_rn(wt[0], xm3, bias)))));
+              if constexpr (kX) {
                 const float w = wsr[i];
                 v = __fmul2_rn(v, make_float2(w, w));
               }
@@ -281,13 +303,23 @@ __global__ void __launch_bounds__(kTailThreads, 1) state_tail_kernel(
               lw = *reinterpret_cast<const uint32_t *>(&lo);
               xm3 = xm2; xm2 = xm1; xm1 = x0;
             }
-            const uint32_t off = (uint32_t)(s_lo + i) * 128u + loff[i & 7];
-            *reinterpret_cast<uint32_t *>(hi_tile + off) = hw;
-            *reinterpret_cast<uint32_t *>(lo_tile + off) = lw;
+            unsigned char *q = hrow + (uint32_t)i * 128u + loff[i & 7];
+            *reinterpret_cast<uint32_t *>(q) = hw;
+            *reinterpret_cast<uint32_t *>(q + kLo) = lw;
           }
         };
-        if (nvalid >= kStripTok) strip_tokens(std::true_type{});
-        else strip_tokens(std::false_type{});
+        const bool full = nvalid >= kStripTok;
+        auto by_shape = [&](auto x_tag) {
+          if (W > 0) {
+            if (full) strip_tokens(std::true_type{}, x_tag, std::true_type{});
+            else strip_tokens(std::false_type{}, x_tag, std::true_type{});
+          } else {
+            if (full) strip_tokens(std::true_type{}, x_tag, std::false_type{});
+            else strip_tokens(std::false_type{}, x_tag, std::false_type{});
+          }
+        };
+        if (is_x) by_shape(std::true_type{});
+        else by_shape(std::false_type{});
       }
       fence_proxy_async();  // the tiles' generic writes, visible to the tensor cores
       if (__syncthreads_or(*abort_flag != 0)) {
