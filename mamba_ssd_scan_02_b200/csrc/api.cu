@@ -381,11 +381,13 @@ ssd_status_t run_prefill(const ssd_config_t *c_in, const ssd_prefill_args_t *a, 
                                   p.P * p.N, nullptr, span->state, span->decay, s);
       }));
     }
-    // The tail pass needs only the front end's outputs: it is forked onto a side stream right
-    // after the front end and launched after the scan, so that it takes the SMs the scan
-    // leaves free; it is joined before the fold.
+    // The tail pass needs only the front end's outputs.  When the scan leaves enough SMs free
+    // it is forked onto a side stream right after the front end and launched after the scan,
+    // so that it takes those SMs, and joined before the fold; otherwise it runs after the scan
+    // on this stream and folds into h_final itself.
     SideJoin side;
-    if (p.tail_dh) {
+    const bool tail_beside = p.tail_dh && tail_beside_scan(p);
+    if (tail_beside) {
       SSD_TRY(side_stream(&side.side));
       side.s = s;
       SSD_TRY(cudaEventRecord(side.side->fork, s));
@@ -397,11 +399,12 @@ ssd_status_t run_prefill(const ssd_config_t *c_in, const ssd_prefill_args_t *a, 
       SSD_TRY(traced("ssd_state_pass", s, [&] { return launch_state_pass(p, s); }));
     }
     SSD_TRY(traced("ssd_scan_tc", s, [&] { return launch_scan_tc(p, 0, s); }));
-    if (side.forked)
-      SSD_TRY(traced("ssd_state_tail", side.side->s, [&] { return launch_state_tail(p, side.side->s); }));
     if (side.forked) {
+      SSD_TRY(traced("ssd_state_tail", side.side->s, [&] { return launch_state_tail(p, false, side.side->s); }));
       SSD_TRY(side.join());
       SSD_TRY(traced("ssd_tail_fold", s, [&] { return launch_tail_fold(p, s); }));
+    } else if (p.tail_dh) {  // no room beside the scan: after it, folding into h_final itself
+      SSD_TRY(traced("ssd_state_tail", s, [&] { return launch_state_tail(p, true, s); }));
     }
     if (p.norm_groups > 0) {
       SSD_TRY(traced("ssd_gated_norm", s, [&] { return launch_gated_norm(p, s); }));

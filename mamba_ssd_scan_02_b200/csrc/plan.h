@@ -101,7 +101,11 @@ cudaError_t launch_span_prefix(const float *states, float *h_in, const float *de
 // beside the output scan, which leaves the state entering those chunks in h_final; the fold
 // then sets h_final = tail_dec * h_final + tail_dh.
 constexpr int kTailChunks = 2;
-cudaError_t launch_state_tail(const PrefillPlan &p, cudaStream_t s);
+// Where the tail pass runs: beside the output scan (on a side stream, on the SMs the scan
+// leaves free) when those SMs finish all its items within the scan's time; otherwise after the
+// scan on the same stream, where it folds into h_final itself (fold_in: no dH, no fold pass).
+bool tail_beside_scan(const PrefillPlan &p);
+cudaError_t launch_state_tail(const PrefillPlan &p, bool fold_in, cudaStream_t s);
 cudaError_t launch_tail_fold(const PrefillPlan &p, cudaStream_t s);
 // norms (norm.cu)
 cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s);  // yh (fp16) or yf (fp32) -> y

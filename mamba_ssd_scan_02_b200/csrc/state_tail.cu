@@ -14,7 +14,10 @@
 //
 // It needs only the front end's outputs, so it runs on a side stream beside the output scan,
 // on the SMs the scan leaves free: persistent CTAs (one per SM) work through items of up to
-// four heads of one group and batch row, which share the group's B channels.  Per item the CTA
+// four heads of one group and batch row, which share the group's B channels.  When the scan
+// leaves too few SMs free (many short sequences, large batches), it runs after the scan on
+// all SMs instead and folds its part into the state the scan left (h = e^{...} h + dH), with
+// no dH buffer and no fold pass.  Per item the CTA
 // computes every tail token's weight w_s per head; then, per 64 tokens (a round), it copies the
 // raw rows of the heads' x channels and the group's B channels (plus 3 history rows) into
 // shared memory with asynchronous 16-byte copies (the next round's copies, or the next item's
@@ -60,7 +63,8 @@ constexpr uint32_t OFF_XL = OFF_XH + 32768;          // w x low parts
 constexpr uint32_t OFF_WS = OFF_XL + 32768;          // token weights [4 heads][256] fp32
 constexpr uint32_t OFF_BAR = OFF_WS + kTailHeads * kTailMax * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + 8;           // [0] TMEM base, [1] abort flag, [2] drain flag
-constexpr uint32_t kTailSmem = OFF_MISC + 16 + 1024;  // + room to align the base
+constexpr uint32_t OFF_DEC = OFF_MISC + 16;          // the item's heads' tail decays [4] fp32
+constexpr uint32_t kTailSmem = OFF_DEC + 16 + 1024;  // + room to align the base
 constexpr uint32_t kTailCols = kTailHeads * kHeadDim;  // the accumulator: 64 columns per head
 static_assert(2 * kRawBuf <= OFF_AH && OFF_AH % 1024 == 0 && OFF_XH % 1024 == 0 && OFF_XL % 1024 == 0,
               "tile layout");
@@ -169,13 +173,14 @@ __global__ void __launch_bounds__(kTailThreads, 1) state_tail_kernel(
     const __nv_bfloat16 *__restrict__ conv_b, const __nv_bfloat16 *__restrict__ csi,
     const float *__restrict__ dte, const float *__restrict__ cs, float *__restrict__ dh_out,
     float *__restrict__ dec_out, int L, int B, int H, int G, int hpg, int conv_dim, int d_inner, int W,
-    int Lpad, int t_tail_uniform, const int *__restrict__ cu, int *err) {
+    int Lpad, int t_tail_uniform, const int *__restrict__ cu, int *err, float *h_fold) {
   extern __shared__ unsigned char tsm_raw[];
   // aligned by an offset from the shared array itself (not through an integer), so that the
   // compiler keeps every access derived from it in the shared address space
   unsigned char *tsm = tsm_raw + ((1024u - (smem_u32(tsm_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(tsm);
   float *ws = reinterpret_cast<float *>(tsm + OFF_WS);  // [4][256]
+  float *decs = reinterpret_cast<float *>(tsm + OFF_DEC);  // [4]
   uint32_t *misc = reinterpret_cast<uint32_t *>(tsm + OFF_MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
   volatile int *drain_flag = reinterpret_cast<volatile int *>(misc + 2);
@@ -356,11 +361,16 @@ __global__ void __launch_bounds__(kTailThreads, 1) state_tail_kernel(
       const float *csr = cs + ((long long)it.b * H + it.h0 + tid) * Lpad + it.t_tail;
       float sum = 0.f;
       for (int c0 = 0; c0 < it.ntok; c0 += 128) sum += csr[c0 + 127];
-      dec_out[(long long)it.b * H + it.h0 + tid] = __expf(sum);
+      decs[tid] = __expf(sum);
+      if (!h_fold) dec_out[(long long)it.b * H + it.h0 + tid] = decs[tid];
     }
-    if (warp < 4 * kTailHeads && (warp >> 2) < it.nh) {  // dH of head warp / 4, lanes 32 (warp % 4) ..
+    if (h_fold) __syncthreads();  // the decays, for the fold below
+    // dH of head warp / 4, lanes (state columns n) 32 (warp % 4) ..: into dh_out, or folded
+    // into the state the scan left in h_fold (h = dec h + dH)
+    if (warp < 4 * kTailHeads && (warp >> 2) < it.nh) {
       const int hh = warp >> 2, qd = warp & 3, nn = 32 * qd + lane;
-      float *dst = dh_out + ((long long)it.b * H + it.h0 + hh) * kHeadDim * kDState + nn;
+      float *dst = (h_fold ? h_fold : dh_out) + ((long long)it.b * H + it.h0 + hh) * kHeadDim * kDState + nn;
+      const float dec = decs[hh];
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {  // 16 columns (p) at a time
         float a[16];
@@ -368,8 +378,21 @@ __global__ void __launch_bounds__(kTailThreads, 1) state_tail_kernel(
           tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + (uint32_t)(kHeadDim * hh + 16 * c), a);
           tmem_ld_wait();
         }
+        if (nr == 0) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) dst[(16 * c + i) * kDState] = nr > 0 ? a[i] : 0.f;  // 32 consecutive n
+          for (int i = 0; i < 16; ++i) a[i] = 0.f;
+        }
+        float *q = dst + 16 * c * kDState;  // a warp stores 32 consecutive n
+        if (h_fold) {  // 16 loads in flight, then the stores
+          float hv[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) hv[i] = q[i * kDState];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) q[i * kDState] = fmaf(dec, hv[i], a[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) q[i * kDState] = a[i];
+        }
       }
     }
     tc_fence_before();
@@ -391,35 +414,57 @@ __global__ void __launch_bounds__(kTailThreads, 1) state_tail_kernel(
 
 }  // namespace
 
+namespace {
+
 // One tail item (four heads of a batch row) costs about as much as this many chunks of the scan.
 constexpr int kItemChunks = 4;
 
+struct TailGrid {
+  long long items, free_sms;
+  int sms;
+  bool beside;
+};
+
+// The output scan takes one SM per CTA (n_seg x H x B of them); the tail pass fits beside it
+// when the SMs it leaves free finish all tail items within the scan's time.
+TailGrid tail_grid(const PrefillPlan &p) {
+  TailGrid g{};
+  int dev = 0;
+  g.sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&g.sms, cudaDevAttrMultiProcessorCount, dev);
+  g.items = (long long)p.B * p.G * ((p.hpg + kTailHeads - 1) / kTailHeads);
+  const long long scan_ctas = (long long)p.n_seg * p.H * p.B;
+  const long long seg_chunks = (p.seg_len + 127) / 128;
+  g.free_sms = g.sms - scan_ctas;
+  const long long need = (g.items * kItemChunks + seg_chunks - 1) / seg_chunks;  // CTAs to keep pace
+  g.beside = g.free_sms >= need && g.free_sms >= 1;
+  return g;
+}
+
+}  // namespace
+
+bool tail_beside_scan(const PrefillPlan &p) { return tail_grid(p).beside; }
+
 // The tail starts at chunk nck-kTailChunks of the last segment (its first chunk when it has
-// fewer).  Grid: one CTA on each SM the output scan (one CTA per SM, n_seg x H x B of them)
-// leaves free, when they finish all items within the scan's time; otherwise one per SM of the
-// whole GPU, up to one CTA per item.
-cudaError_t launch_state_tail(const PrefillPlan &p, cudaStream_t s) {
+// fewer).  Grid: one CTA on each SM the scan leaves free when the pass runs beside it, else one
+// per SM of the whole GPU; at most one CTA per item.
+cudaError_t launch_state_tail(const PrefillPlan &p, bool fold_in, cudaStream_t s) {
   static_assert(kTailChunks * 128 <= kTailMax, "tail longer than the weight buffer");
   if (!p.tail_dh || p.L == 0) return cudaSuccess;
   if (p.xs % 8 || p.conv_dim % 8 || p.d_inner % 8) return cudaErrorInvalidValue;  // 16-byte copies
+  if (fold_in && !p.h_final) return cudaErrorInvalidValue;
   const int t_b = (p.n_seg - 1) * p.seg_len;
   const int nck = (p.L - t_b + 127) / 128;
   const int t_tail = t_b + 128 * (nck > kTailChunks ? nck - kTailChunks : 0);
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long items = (long long)p.B * p.G * ((p.hpg + kTailHeads - 1) / kTailHeads);
-  const long long scan_ctas = (long long)p.n_seg * p.H * p.B;
-  const long long seg_chunks = (p.seg_len + 127) / 128;
-  const long long free_sms = sms - scan_ctas;
-  const long long need = (items * kItemChunks + seg_chunks - 1) / seg_chunks;  // CTAs to keep pace
-  long long grid = free_sms >= need && free_sms >= 1 ? free_sms : sms;
-  if (grid > items) grid = items;
+  const TailGrid tg = tail_grid(p);
+  long long grid = tg.beside ? tg.free_sms : tg.sms;
+  if (grid > tg.items) grid = tg.items;
   cudaError_t e = set_smem_attr(state_tail_kernel, kTailSmem, s);
   if (e != cudaSuccess) return e;
   state_tail_kernel<<<(unsigned)grid, kTailThreads, kTailSmem, s>>>(
       (const __nv_bfloat16 *)p.xBC, p.xs, (const __nv_bfloat16 *)p.conv_w, (const __nv_bfloat16 *)p.conv_b,
       (const __nv_bfloat16 *)p.csi, p.dte_hm, p.cs_hm, p.tail_dh, p.tail_dec, p.L, p.B, p.H, p.G, p.hpg,
-      p.conv_dim, p.d_inner, p.W, p.Lpad, t_tail, p.cu, p.err);
+      p.conv_dim, p.d_inner, p.W, p.Lpad, t_tail, p.cu, p.err, fold_in ? p.h_final : nullptr);
   return cudaGetLastError();
 }
 
