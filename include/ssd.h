@@ -55,7 +55,7 @@ extern "C" {
 typedef enum {
   SSD_OK = 0,
   SSD_ERR_INVALID_ARG = 1,   /* missing/inconsistent argument or shape */
-  SSD_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement */
+  SSD_ERR_UNSUPPORTED = 2,   /* valid request the library does not implement */
   SSD_ERR_ALIGNMENT = 3,     /* pointer or row stride not aligned as required */
   SSD_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
   SSD_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up */
@@ -76,8 +76,8 @@ typedef struct {
   int batch;        /* B >= 1 */
   int seqlen;       /* L >= 0 tokens in this call (0: only the carries are copied) */
   int nheads;       /* H >= 1, multiple of ngroups */
-  int headdim;      /* P; this build supports 64 */
-  int dstate;       /* N; this build supports 128 */
+  int headdim;      /* P; the library supports 64 */
+  int dstate;       /* N; the library supports 128 */
   int ngroups;      /* G >= 1: B and C are shared by the H/G heads of a group */
   int chunk;        /* Q in {64, 128, 256}: tokens per chunk of the chunked scan */
   int conv_width;   /* W in 0..4; 0 = no conv and no activation (u = raw input) */
