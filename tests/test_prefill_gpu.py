@@ -90,6 +90,23 @@ def test_tail_covered_final_state_is_fp32_accurate(cuda_lib, oracle, L, W):
     assert r <= TOL_F32, f"L={L} W={W}: tail-only h_final max|err|/RMS = {r:.3e} > {TOL_F32:.1e}"
 
 
+def test_tail_after_the_scan_when_no_sms_are_free(cuda_lib, oracle):
+    """A uniform batch whose scan takes more CTAs than the GPU has SMs (3 rows x 64 heads): the
+    tail pass runs after the scan and folds into h_final itself (no fold pass).  y and h_final
+    meet the same bounds against the oracle as on the side-stream path."""
+    from mamba_ssd_scan_02_b200 import ssd
+    cfg = small_cfg(batch=3, nheads=64, ngroups=4, seqlen=300, norm_groups=4)
+    inp = make_case(cfg, seed_idx=11)
+    ssd.trace_enable(True)
+    ssd.trace_read()
+    try:
+        e1, e2 = _check(oracle, cfg, inp, 2, tag="tail after the scan")
+        names = [n for n, _ in ssd.trace_read()]
+    finally:
+        ssd.trace_enable(False)
+    assert "ssd_state_tail" in names and "ssd_tail_fold" not in names, names
+
+
 def test_tensor_kernel_rejects_fp32(cuda_lib):
     from mamba_ssd_scan_02_b200 import ssd
     cfg = small_cfg(dtype="f32", seqlen=64)
