@@ -194,7 +194,6 @@ __global__ void __launch_bounds__(kTailThreads, 1) state_tail_kernel(
   const int tcol = is_x ? 2 * (pair & 31) : (2 * (pair - 128)) & 63;  // column within its box
   unsigned char *hi_tile = tsm + (is_x ? OFF_XH + (uint32_t)xhead * 8192u
                                        : OFF_AH + (uint32_t)((2 * (pair - 128)) >> 6) * 8192u);
-  unsigned char *lo_tile = hi_tile + (is_x ? OFF_XL - OFF_XH : OFF_AL - OFF_AH);
   // byte offset of this thread's 4 bytes in a swizzled row r, by r mod 8 (16-byte chunk
   // c / 8 of row r sits at chunk (c / 8) ^ (r % 8))
   uint32_t loff[8];
