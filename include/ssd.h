@@ -256,6 +256,19 @@ int ssd_version(void);
  * to prefills running concurrently on other host threads. */
 void ssd_test_stall_scan(int chunk, unsigned long long wait_limit_ns);
 
+/* Debug build with device-side index checks (libssd_debug.so, compiled with
+ * -DSSD_DEBUG_BOUNDS): the kernels check the index of each store to y, the final and segment
+ * states, the tail pass's buffers, the fused front end's B/C and dt buffers and the gated
+ * norm's output against the buffer's extent.  An index outside it latches
+ * SSD_ERR_DEVICE_BOUNDS for ssd_get_device_error() and the store is skipped; nothing traps.
+ * Returns 1 in that build, 0 in the normal one (where the checks compile away). */
+int ssd_debug_bounds_build(void);
+
+/* Test hook of the debug build: the index checks allow 1/denom of each buffer's extent
+ * (denom <= 1 restores the full extents), so that a call with valid buffers trips them while
+ * every access stays inside its allocation.  Process-wide; no effect in the normal build. */
+void ssd_test_bounds_scale(int denom);
+
 /* Kernel tracing for measurement tools.  While enabled, every kernel the library launches
  * is bracketed by two CUDA events recorded on the stream it is launched on (so the timing
  * covers exactly that kernel).  Off by default; do not enable it while a stream is being

@@ -23,6 +23,9 @@ namespace {
 // and the wait limit its bounded waits then use; 0 = off.
 std::atomic<int> g_stall_chunk1{0};
 std::atomic<unsigned long long> g_stall_wait_ns{0};
+// Test hook (ssd_test_bounds_scale): the debug build's index checks allow 1/denom of each
+// buffer's extent; 1 = off.
+std::atomic<int> g_bounds_denom{1};
 
 constexpr int kMaxDevices = 64;
 constexpr long long kTargetCtas = 2 * 148;  // scan CTAs wanted in flight (2 per B200 SM)
@@ -311,6 +314,7 @@ ssd_status_t run_prefill(const ssd_config_t *c_in, const ssd_prefill_args_t *a, 
   p.rows = rows;
   p.stall_chunk1 = g_stall_chunk1.load();
   p.stall_wait_ns = g_stall_wait_ns.load();
+  p.bounds_denom = g_bounds_denom.load();
 
   if (span) {
     // the combine of internal segments (or of none) into the span's own state and decay
@@ -737,5 +741,15 @@ void ssd_test_stall_scan(int chunk, unsigned long long wait_limit_ns) {
   g_stall_wait_ns.store(wait_limit_ns);
   g_stall_chunk1.store(chunk >= 0 ? chunk + 1 : 0);
 }
+
+int ssd_debug_bounds_build(void) {
+#ifdef SSD_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+void ssd_test_bounds_scale(int denom) { g_bounds_denom.store(denom > 1 ? denom : 1); }
 
 }  // extern "C"

@@ -20,6 +20,21 @@ __device__ __forceinline__ void latch_error(int *err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
+// ---- index checks of the debug build ---------------------------------------------------------
+// Built with -DSSD_DEBUG_BOUNDS (libssd_debug.so), the kernels check the index of each global
+// store against the extent of the buffer it writes: an index outside [0, extent) latches
+// SSD_ERR_DEVICE_BOUNDS in the device error word and the store is skipped (no trap).  In the
+// normal build the check is the constant true and costs nothing.
+#ifdef SSD_DEBUG_BOUNDS
+__device__ __forceinline__ bool in_bounds(long long i, long long extent, int *err) {
+  if (i >= 0 && i < extent) return true;
+  latch_error(err, (int)SSD_ERR_DEVICE_BOUNDS);
+  return false;
+}
+#else
+__device__ __forceinline__ constexpr bool in_bounds(long long, long long, int *) { return true; }
+#endif
+
 // ---- row geometry of a batch -----------------------------------------------------------------
 // A uniform batch stores batch row b's token t at row b*L + t.  A variable-length batch packs
 // its sequences back to back: sequence b is rows cu[b] .. cu[b+1]-1 (cu: device offsets, B + 1

@@ -7,6 +7,7 @@
 // the Mamba-2 short convolution of window 4 in the Nemotron Nano 2 layers ("NVIDIA Nemotron
 // Nano 2" summary, section "Method").
 #include <algorithm>
+#include <climits>
 #include <type_traits>
 
 #include "common.cuh"
@@ -116,7 +117,8 @@ __device__ __forceinline__ void dt_cumsum_tile(const T *__restrict__ dt, long lo
                                                const float *__restrict__ A, float *__restrict__ dte,
                                                float *__restrict__ cs, int L, int H, int Lpad, int sp,
                                                float lo, float hi, int c0, int h0, int b, int tid,
-                                               float (*v)[9], bool active, const int *cu = nullptr) {
+                                               float (*v)[9], bool active, const int *cu = nullptr,
+                                               long long extent = LLONG_MAX, int *err = nullptr) {
   const int warp = tid / 32, lane = tid % 32;
   if (active) {
     const int tt = c0 + tid;
@@ -156,9 +158,11 @@ __device__ __forceinline__ void dt_cumsum_tile(const T *__restrict__ dt, long lo
     }
     const float excl = incl - run;
     const long long base = ((long long)b * H + h) * Lpad + c0 + 4 * lane;
-    *reinterpret_cast<float4 *>(dte + base) = make_float4(d[0], d[1], d[2], d[3]);
-    *reinterpret_cast<float4 *>(cs + base) =
-        make_float4(excl + c[0], excl + c[1], excl + c[2], excl + c[3]);
+    if (in_bounds(base + 3, extent, err)) {  // dte and cs have the same extent
+      *reinterpret_cast<float4 *>(dte + base) = make_float4(d[0], d[1], d[2], d[3]);
+      *reinterpret_cast<float4 *>(cs + base) =
+          make_float4(excl + c[0], excl + c[1], excl + c[2], excl + c[3]);
+    }
   }
 }
 
@@ -289,7 +293,8 @@ __device__ __forceinline__ void bc_conv_tile(const __nv_bfloat16 *__restrict__ x
                                              const __nv_bfloat16 *__restrict__ w,
                                              const __nv_bfloat16 *__restrict__ bias,
                                              __half *__restrict__ out, int L, int conv_dim, int c_begin,
-                                             int C_out, int bx, int by, int bz, const int *cu = nullptr) {
+                                             int C_out, int bx, int by, int bz, const int *cu = nullptr,
+                                             long long extent = LLONG_MAX, int *err = nullptr) {
   const int o4 = (bx * kBcThreads + threadIdx.x) * 4;
   if (o4 >= C_out) return;
   const int c4 = c_begin + o4;
@@ -355,8 +360,10 @@ __device__ __forceinline__ void bc_conv_tile(const __nv_bfloat16 *__restrict__ x
         x1[i] = x0[i];
       }
       const __half2 h01 = __floats2half2_rn(r[0], r[1]), h23 = __floats2half2_rn(r[2], r[3]);
-      *reinterpret_cast<uint2 *>(out + (rb + t) * C_out + o4) =
-          make_uint2(*reinterpret_cast<const uint32_t *>(&h01), *reinterpret_cast<const uint32_t *>(&h23));
+      const long long oi = (rb + t) * C_out + o4;
+      if (in_bounds(oi + 3, extent, err))
+        *reinterpret_cast<uint2 *>(out + oi) =
+            make_uint2(*reinterpret_cast<const uint32_t *>(&h01), *reinterpret_cast<const uint32_t *>(&h23));
     }
   };
   if (t1 - t0 == kBcTok) {
@@ -394,6 +401,8 @@ struct FrontArgs {
   float lo, hi;
   int n_dt, dt_tiles, dt_nch, dt_nhg, n_cso, gx, gy;
   const int *cu;  // packed variable-length batch offsets (device), or null
+  long long bc_extent, dt_extent;  // elements of bc and of dte (= cs): the debug build's checks
+  int *err;
 };
 
 template <int W>
@@ -407,7 +416,8 @@ __global__ void __launch_bounds__(kBcThreads, 4) front_tc_kernel(const FrontArgs
     const int qq = active ? q : 0;
     const int cx = qq % f.dt_nch, hy = (qq / f.dt_nch) % f.dt_nhg, b = qq / (f.dt_nch * f.dt_nhg);
     dt_cumsum_tile<__nv_bfloat16>(f.dt, f.ds, f.dt_bias, f.A, f.dte, f.cs, f.L, f.H, f.Lpad, f.sp, f.lo,
-                                  f.hi, cx * 128, hy * 8, b, threadIdx.x & 127, v[half], active, f.cu);
+                                  f.hi, cx * 128, hy * 8, b, threadIdx.x & 127, v[half], active, f.cu,
+                                  f.dt_extent, f.err);
     return;
   }
   j -= f.n_dt;
@@ -419,7 +429,7 @@ __global__ void __launch_bounds__(kBcThreads, 4) front_tc_kernel(const FrontArgs
   }
   j -= f.n_cso;
   bc_conv_tile<W>(f.xBC, f.xs, f.csi, f.conv_w, f.conv_b, f.bc, f.L, f.conv_dim, f.d_inner, f.C_out,
-                  j % f.gx, (j / f.gx) % f.gy, j / (f.gx * f.gy), f.cu);
+                  j % f.gx, (j / f.gx) % f.gy, j / (f.gx * f.gy), f.cu, f.bc_extent, f.err);
 }
 
 cudaError_t launch_bc_conv_f16(const PrefillPlan &p, cudaStream_t s) {
@@ -459,6 +469,9 @@ cudaError_t launch_front_tc(const PrefillPlan &p, bool with_cso, cudaStream_t s)
   f.B = p.B; f.L = p.L; f.H = p.H; f.Lpad = p.Lpad; f.conv_dim = p.conv_dim; f.d_inner = p.d_inner;
   f.C_out = 2 * p.G * p.N; f.W = p.W; f.sp = p.softplus; f.lo = p.dt_min; f.hi = p.dt_max;
   f.cu = p.cu;
+  f.bc_extent = checked_extent(p, p.rows * 2LL * p.G * p.N);
+  f.dt_extent = checked_extent(p, (long long)p.B * p.H * p.Lpad);
+  f.err = p.err;
   f.dt_nch = p.Lpad / 128; f.dt_nhg = (p.H + 7) / 8; f.dt_tiles = f.dt_nch * f.dt_nhg * p.B;
   f.n_dt = (f.dt_tiles + 1) / 2;
   const long long ncso = (with_cso && p.cso && p.W > 0) ? (long long)p.B * p.W * ((long long)p.conv_dim * 2 / 16) : 0;

@@ -39,7 +39,7 @@ __device__ __forceinline__ float ld_y(const __half *p) { return __half2float(*p)
 template <typename T, typename YT>
 __global__ void __launch_bounds__(kNormThreads) gated_norm_kernel(
     const YT *__restrict__ y, const T *__restrict__ z, long long zs, const T *__restrict__ w,
-    T *__restrict__ out, long long os, int d_inner, int gs, float eps, int nbg) {
+    T *__restrict__ out, long long os, int d_inner, int gs, float eps, int nbg, long long out_extent, int *err) {
   __shared__ float red[32];
   const long long row = blockIdx.x;
   const int c0 = blockIdx.y * gs;
@@ -58,7 +58,8 @@ __global__ void __launch_bounds__(kNormThreads) gated_norm_kernel(
     const float sz = silu(io<T>::ld(zr + i));
     const float yv = ld_y(yr + i);
     const float gv = nbg ? yv : yv * sz;
-    io<T>::st(orow + i, gv * r * (w ? io<T>::ld(w + c0 + i) : 1.f) * (nbg ? sz : 1.f));
+    if (in_bounds(row * os + c0 + i, out_extent, err))
+      io<T>::st(orow + i, gv * r * (w ? io<T>::ld(w + c0 + i) : 1.f) * (nbg ? sz : 1.f));
   }
 }
 
@@ -117,7 +118,7 @@ template <typename YT>
 __global__ void __launch_bounds__(1024) gated_norm_v8_kernel(
     const YT *__restrict__ y, const __nv_bfloat16 *__restrict__ z, long long zs,
     const __nv_bfloat16 *__restrict__ w, __nv_bfloat16 *__restrict__ out, long long os, int d_inner,
-    int gs, float eps, int nbg) {
+    int gs, float eps, int nbg, long long out_extent, int *err) {
   __shared__ float red[32];
   const long long row = blockIdx.x;
   const int c = blockIdx.y * gs + 8 * threadIdx.x;
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(1024) gated_norm_v8_kernel(
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) g[i] *= r * wv[i] * (nbg ? zv[i] : 1.f);
-  store8(out + row * os + c, g);
+  if (in_bounds(row * os + c + 7, out_extent, err)) store8(out + row * os + c, g);
 }
 
 cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s) {
@@ -153,22 +154,25 @@ cudaError_t launch_gated_norm(const PrefillPlan &p, cudaStream_t s) {
   const auto *z = (const __nv_bfloat16 *)p.z;
   const auto *w = (const __nv_bfloat16 *)p.norm_w;
   auto *o = (__nv_bfloat16 *)p.y;
+  const long long ext = checked_extent(p, (p.rows - 1) * p.ys + p.d_inner);
   if (p.yh) {  // tensor path: fp16 y, bf16 tensors
     if (!p.bf16) return cudaErrorInvalidValue;
     if (v8)
-      gated_norm_v8_kernel<__half><<<grid, gs / 8, 0, s>>>(p.yh, z, p.zs, w, o, p.ys, p.d_inner, gs, p.eps, p.nbg);
+      gated_norm_v8_kernel<__half><<<grid, gs / 8, 0, s>>>(p.yh, z, p.zs, w, o, p.ys, p.d_inner, gs, p.eps, p.nbg,
+                                                          ext, p.err);
     else
       gated_norm_kernel<__nv_bfloat16, __half><<<grid, kNormThreads, 0, s>>>(p.yh, z, p.zs, w, o, p.ys,
-                                                                             p.d_inner, gs, p.eps, p.nbg);
+                                                                             p.d_inner, gs, p.eps, p.nbg, ext, p.err);
   } else if (v8) {
-    gated_norm_v8_kernel<float><<<grid, gs / 8, 0, s>>>(p.yf, z, p.zs, w, o, p.ys, p.d_inner, gs, p.eps, p.nbg);
+    gated_norm_v8_kernel<float><<<grid, gs / 8, 0, s>>>(p.yf, z, p.zs, w, o, p.ys, p.d_inner, gs, p.eps, p.nbg, ext,
+                                                        p.err);
   } else if (p.bf16) {
     gated_norm_kernel<__nv_bfloat16, float><<<grid, kNormThreads, 0, s>>>(p.yf, z, p.zs, w, o, p.ys, p.d_inner,
-                                                                          gs, p.eps, p.nbg);
+                                                                          gs, p.eps, p.nbg, ext, p.err);
   } else {
     gated_norm_kernel<float, float><<<grid, kNormThreads, 0, s>>>(p.yf, (const float *)p.z, p.zs,
                                                                   (const float *)p.norm_w, (float *)p.y,
-                                                                  p.ys, p.d_inner, gs, p.eps, p.nbg);
+                                                                  p.ys, p.d_inner, gs, p.eps, p.nbg, ext, p.err);
   }
   return cudaGetLastError();
 }

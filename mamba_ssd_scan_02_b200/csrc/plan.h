@@ -55,7 +55,15 @@ struct PrefillPlan {
   // that the bounded waits run out after stall_wait_ns
   int stall_chunk1;
   unsigned long long stall_wait_ns;
+  // test hook of the debug build's index checks: the extents they allow are the buffers'
+  // divided by this (1 = the buffers' own)
+  int bounds_denom;
 };
+
+// The extent (elements) the index checks of the debug build allow for a buffer of n elements.
+inline long long checked_extent(const PrefillPlan &p, long long n) {
+  return p.bounds_denom > 1 ? n / p.bounds_denom : n;
+}
 
 struct DecodePlan {
   int B, H, P, N, G, W, norm_groups, hpg, d_inner, conv_dim;

@@ -47,7 +47,7 @@ __global__ void state_pass_kernel(const float4 *seg_state, float4 *h_in,
 // The final state's fold after the tail pass: h = dec h + dh per (batch row, head), where
 // dh and dec are what the last chunks contribute from a zero state and their total decay.
 __global__ void tail_fold_kernel(float4 *__restrict__ h, const float4 *__restrict__ dh,
-                                 const float *__restrict__ dec, long long n4) {
+                                 const float *__restrict__ dec, long long n4, long long h4_extent, int *err) {
   constexpr int kPer = kHeadDim * kDState / 4;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
        i += (long long)gridDim.x * blockDim.x) {
@@ -55,7 +55,7 @@ __global__ void tail_fold_kernel(float4 *__restrict__ h, const float4 *__restric
     float4 v = h[i];
     const float4 a = dh[i];
     v.x = fmaf(d, v.x, a.x); v.y = fmaf(d, v.y, a.y); v.z = fmaf(d, v.z, a.z); v.w = fmaf(d, v.w, a.w);
-    h[i] = v;
+    if (in_bounds(i, h4_extent, err)) h[i] = v;
   }
 }
 
@@ -67,7 +67,8 @@ cudaError_t launch_tail_fold(const PrefillPlan &p, cudaStream_t s) {
   long long blocks = (n4 + 255) / 256;
   if (blocks > 148 * 8) blocks = 148 * 8;
   tail_fold_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<float4 *>(p.h_final),
-                                                     reinterpret_cast<const float4 *>(p.tail_dh), p.tail_dec, n4);
+                                                     reinterpret_cast<const float4 *>(p.tail_dh), p.tail_dec, n4,
+                                                     checked_extent(p, n4), p.err);
   return cudaGetLastError();
 }
 

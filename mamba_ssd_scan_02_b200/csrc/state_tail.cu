@@ -173,7 +173,8 @@ __global__ void __launch_bounds__(kTailThreads, 1) state_tail_kernel(
     const __nv_bfloat16 *__restrict__ conv_b, const __nv_bfloat16 *__restrict__ csi,
     const float *__restrict__ dte, const float *__restrict__ cs, float *__restrict__ dh_out,
     float *__restrict__ dec_out, int L, int B, int H, int G, int hpg, int conv_dim, int d_inner, int W,
-    int Lpad, int t_tail_uniform, const int *__restrict__ cu, int *err, float *h_fold) {
+    int Lpad, int t_tail_uniform, const int *__restrict__ cu, int *err, float *h_fold,
+    long long dh_extent, long long dec_extent) {
   extern __shared__ unsigned char tsm_raw[];
   // aligned by an offset from the shared array itself (not through an integer), so that the
   // compiler keeps every access derived from it in the shared address space
@@ -361,14 +362,16 @@ __global__ void __launch_bounds__(kTailThreads, 1) state_tail_kernel(
       float sum = 0.f;
       for (int c0 = 0; c0 < it.ntok; c0 += 128) sum += csr[c0 + 127];
       decs[tid] = __expf(sum);
-      if (!h_fold) dec_out[(long long)it.b * H + it.h0 + tid] = decs[tid];
+      const long long di = (long long)it.b * H + it.h0 + tid;
+      if (!h_fold && in_bounds(di, dec_extent, err)) dec_out[di] = decs[tid];
     }
     if (h_fold) __syncthreads();  // the decays, for the fold below
     // dH of head warp / 4, lanes (state columns n) 32 (warp % 4) ..: into dh_out, or folded
     // into the state the scan left in h_fold (h = dec h + dH)
     if (warp < 4 * kTailHeads && (warp >> 2) < it.nh) {
       const int hh = warp >> 2, qd = warp & 3, nn = 32 * qd + lane;
-      float *dst = (h_fold ? h_fold : dh_out) + ((long long)it.b * H + it.h0 + hh) * kHeadDim * kDState + nn;
+      const long long d0 = ((long long)it.b * H + it.h0 + hh) * kHeadDim * kDState + nn;  // dst's index
+      float *dst = (h_fold ? h_fold : dh_out) + d0;
       const float dec = decs[hh];
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {  // 16 columns (p) at a time
@@ -382,15 +385,18 @@ __global__ void __launch_bounds__(kTailThreads, 1) state_tail_kernel(
           for (int i = 0; i < 16; ++i) a[i] = 0.f;
         }
         float *q = dst + 16 * c * kDState;  // a warp stores 32 consecutive n
+        const long long qi = d0 + 16 * c * kDState;  // q's index
         if (h_fold) {  // 16 loads in flight, then the stores
           float hv[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) hv[i] = q[i * kDState];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) q[i * kDState] = fmaf(dec, hv[i], a[i]);
+          for (int i = 0; i < 16; ++i)
+            if (in_bounds(qi + i * kDState, dh_extent, err)) q[i * kDState] = fmaf(dec, hv[i], a[i]);
         } else {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) q[i * kDState] = a[i];
+          for (int i = 0; i < 16; ++i)
+            if (in_bounds(qi + i * kDState, dh_extent, err)) q[i * kDState] = a[i];
         }
       }
     }
@@ -463,7 +469,8 @@ cudaError_t launch_state_tail(const PrefillPlan &p, bool fold_in, cudaStream_t s
   state_tail_kernel<<<(unsigned)grid, kTailThreads, kTailSmem, s>>>(
       (const __nv_bfloat16 *)p.xBC, p.xs, (const __nv_bfloat16 *)p.conv_w, (const __nv_bfloat16 *)p.conv_b,
       (const __nv_bfloat16 *)p.csi, p.dte_hm, p.cs_hm, p.tail_dh, p.tail_dec, p.L, p.B, p.H, p.G, p.hpg,
-      p.conv_dim, p.d_inner, p.W, p.Lpad, t_tail, p.cu, p.err, fold_in ? p.h_final : nullptr);
+      p.conv_dim, p.d_inner, p.W, p.Lpad, t_tail, p.cu, p.err, fold_in ? p.h_final : nullptr,
+      checked_extent(p, (long long)p.B * p.H * kHeadDim * kDState), checked_extent(p, (long long)p.B * p.H));
   return cudaGetLastError();
 }
 

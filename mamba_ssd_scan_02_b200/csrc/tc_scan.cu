@@ -155,6 +155,8 @@ struct TcArgs {
   unsigned long long wait_ns;  // limit of every bounded wait
   int debug_skip_chunk;        // test hook (-1 = off): the producer stops before loading this
                                // chunk's stage, so its consumers' bounded waits run out
+  long long y_extent, h_extent;  // elements of the y (or yh) and h_out buffers (index checks
+                               // of the debug build)
   const int *cu;               // packed variable-length batch: sequence b is token rows
                                // cu[b] .. cu[b+1]-1 (the tensor maps then have one batch row
                                // of all the tokens); null: row b*L + t
@@ -716,7 +718,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     const bool leader = (tid == 19 * 32);
     const uint32_t lane_off = (uint32_t)(32 * ew) << 16;
     const long long bh = (long long)b * a.H + h;
-    float *hout = a.h_out ? a.h_out + seg * a.h_out_seg + bh * 8192 : nullptr;
+    const long long hbase = seg * a.h_out_seg + bh * 8192;  // hout's offset in h_out
+    float *hout = a.h_out ? a.h_out + hbase : nullptr;
     // tail mode: only the last segment writes, the state entering its last tail_chunks chunks
     const bool tail = a.tail_chunks > 0 && seg == (int)gridDim.x - 1 && hout != nullptr;
     const int tail_k = nck - 1 - a.tail_chunks;  // state after this chunk (-1: the initial state)
@@ -735,7 +738,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         write_h_tile(smem, hr, n, half);
         if (tail && tail_k < 0) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) hout[(32 * half + i) * 128 + n] = hr[i];
+          for (int i = 0; i < 32; ++i)
+            if (in_bounds(hbase + (32 * half + i) * 128 + n, a.h_extent, a.err)) hout[(32 * half + i) * 128 + n] = hr[i];
         }
       }
       tmem_st_wait();
@@ -785,7 +789,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (htile) write_h_tile(smem, hr, n, half);
         if (tail && k == tail_k) {  // the state entering the tail, in fp32
 #pragma unroll
-          for (int i = 0; i < 32; ++i) hout[(32 * half + i) * 128 + n] = hr[i];
+          for (int i = 0; i < 32; ++i)
+            if (in_bounds(hbase + (32 * half + i) * 128 + n, a.h_extent, a.err)) hout[(32 * half + i) * 128 + n] = hr[i];
         }
       }
       tmem_st_wait();
@@ -830,17 +835,23 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           }
           if (tok < t_end) {
             if (a.yh) {
-              uint4 *dst = reinterpret_cast<uint4 *>(a.yh + row * a.d_inner + h * 64 + 32 * half);
+              const long long yo = row * a.d_inner + h * 64 + 32 * half;
+              uint4 *dst = reinterpret_cast<uint4 *>(a.yh + yo);
+              if (in_bounds(yo + 31, a.y_extent, a.err)) {
 #pragma unroll
-              for (int i = 0; i < 4; ++i)
-                dst[i] = make_uint4(pack_f16(yi[8 * i], yi[8 * i + 1]), pack_f16(yi[8 * i + 2], yi[8 * i + 3]),
-                                    pack_f16(yi[8 * i + 4], yi[8 * i + 5]), pack_f16(yi[8 * i + 6], yi[8 * i + 7]));
+                for (int i = 0; i < 4; ++i)
+                  dst[i] = make_uint4(pack_f16(yi[8 * i], yi[8 * i + 1]), pack_f16(yi[8 * i + 2], yi[8 * i + 3]),
+                                      pack_f16(yi[8 * i + 4], yi[8 * i + 5]), pack_f16(yi[8 * i + 6], yi[8 * i + 7]));
+              }
             } else {
-              uint4 *dst = reinterpret_cast<uint4 *>(a.y + row * a.ys + h * 64 + 32 * half);
+              const long long yo = row * a.ys + h * 64 + 32 * half;
+              uint4 *dst = reinterpret_cast<uint4 *>(a.y + yo);
+              if (in_bounds(yo + 31, a.y_extent, a.err)) {
 #pragma unroll
-              for (int i = 0; i < 4; ++i)
-                dst[i] = make_uint4(pack_bf16(yi[8 * i], yi[8 * i + 1]), pack_bf16(yi[8 * i + 2], yi[8 * i + 3]),
-                                    pack_bf16(yi[8 * i + 4], yi[8 * i + 5]), pack_bf16(yi[8 * i + 6], yi[8 * i + 7]));
+                for (int i = 0; i < 4; ++i)
+                  dst[i] = make_uint4(pack_bf16(yi[8 * i], yi[8 * i + 1]), pack_bf16(yi[8 * i + 2], yi[8 * i + 3]),
+                                      pack_bf16(yi[8 * i + 4], yi[8 * i + 5]), pack_bf16(yi[8 * i + 6], yi[8 * i + 7]));
+              }
             }
           }
         }
@@ -855,7 +866,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           tmem_ld32(tmem + TM_H + 32 * half + lane_off, hr);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) hout[(32 * half + i) * 128 + n] = hr[i];
+          for (int i = 0; i < 32; ++i)
+            if (in_bounds(hbase + (32 * half + i) * 128 + n, a.h_extent, a.err)) hout[(32 * half + i) * 128 + n] = hr[i];
         }
       }
       if (a.seg_decay && n == 0) a.seg_decay[(long long)seg * a.B * a.H + bh] = __expf(decay_sum);
@@ -934,12 +946,14 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
   a.debug_skip_chunk = p.stall_chunk1 - 1;
   a.d_inner = p.d_inner;
   a.cu = p.cu;
+  a.y_extent = checked_extent(p, p.yh ? p.rows * p.d_inner : (p.rows - 1) * p.ys + p.d_inner);
   const long long seg_stride = (long long)p.B * p.H * p.P * p.N;
   dim3 grid(p.n_seg, p.H, p.B);
   cudaError_t e;
   if (mode == 1) {
     a.h_init = nullptr; a.h_init_seg = 0;
     a.h_out = p.seg_state; a.h_out_seg = seg_stride; a.seg_decay = p.seg_decay;
+    a.h_extent = checked_extent(p, p.n_seg * seg_stride);
     auto kern = p.W > 0 ? ssd_scan_tc_kernel<true, true> : ssd_scan_tc_kernel<true, false>;
     e = set_smem_attr(kern, kSmemAlloc, s);
     if (e != cudaSuccess) return e;
@@ -953,6 +967,7 @@ cudaError_t launch_scan_tc(const PrefillPlan &p, int mode, cudaStream_t s) {
     // the last segment leaves the state before its last kTailChunks chunks; the fp32 tail pass
     // adds what those chunks contribute
     a.h_out = p.h_final; a.h_out_seg = 0; a.seg_decay = nullptr;
+    a.h_extent = checked_extent(p, seg_stride);
     a.tail_chunks = p.tail_dh ? kTailChunks : 0;
     auto kern = p.W > 0 ? ssd_scan_tc_kernel<false, true> : ssd_scan_tc_kernel<false, false>;
     e = set_smem_attr(kern, kSmemAlloc, s);

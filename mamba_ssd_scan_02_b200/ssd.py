@@ -21,6 +21,8 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libssd.so")
+# the same library with device-side index checks (-DSSD_DEBUG_BOUNDS), for tests
+DEBUG_LIB_PATH = os.path.join(_HERE, "libssd_debug.so")
 
 SSD_F32, SSD_BF16 = 0, 1
 KERNEL_AUTO, KERNEL_SIMT, KERNEL_TENSOR = 0, 1, 2
@@ -78,7 +80,21 @@ class TraceRecord(ctypes.Structure):
 EXPORTS = ("ssd_workspace_size", "ssd_prefill", "ssd_decode_step", "ssd_mixer_workspace_size",
            "mamba2_mixer_forward", "ssd_status_string", "ssd_get_device_error", "ssd_version",
            "ssd_trace_enable", "ssd_trace_read", "ssd_prefill_noalloc", "ssd_varlen_workspace_size",
-           "ssd_prefill_varlen", "ssd_test_stall_scan", "ssd_prefill_span_state", "ssd_span_prefix")
+           "ssd_prefill_varlen", "ssd_test_stall_scan", "ssd_prefill_span_state", "ssd_span_prefix",
+           "ssd_debug_bounds_build", "ssd_test_bounds_scale")
+
+def debug_bounds_build() -> bool:
+    """True for the library built with device-side index checks (libssd_debug.so)."""
+    return bool(load().ssd_debug_bounds_build())
+
+
+def test_bounds_scale(denom: int) -> None:
+    """Test hook of the debug build: its index checks allow 1/denom of each buffer's extent
+    (1 restores them), so a call with valid buffers trips them without any access leaving its
+    allocation."""
+    load().ssd_test_bounds_scale(int(denom))
+
+
 NOALLOC_WORKSPACE_BYTES = 64 << 20
 
 _lib = None
@@ -125,6 +141,10 @@ def load(path: str = LIB_PATH):
     lib.ssd_span_prefix.argtypes = [vp, vp, c_int, c_int, c_int, c_int, c_int, vp, vp, vp, vp]
     lib.ssd_test_stall_scan.restype = None
     lib.ssd_test_stall_scan.argtypes = [c_int, ctypes.c_ulonglong]
+    lib.ssd_debug_bounds_build.restype = c_int
+    lib.ssd_debug_bounds_build.argtypes = []
+    lib.ssd_test_bounds_scale.restype = None
+    lib.ssd_test_bounds_scale.argtypes = [c_int]
     lib.ssd_trace_enable.restype = c_int
     lib.ssd_trace_enable.argtypes = [c_int]
     lib.ssd_trace_read.restype = c_int

@@ -34,6 +34,19 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(ssd.EXPORTS) <= set(names)
 
 
+def test_debug_build_exports_the_same_symbols(lib):
+    """The normal build reports no index checks; the debug build (device-side index checks)
+    exports every declared symbol too and reports its checks."""
+    assert lib.ssd_debug_bounds_build() == 0
+    if not os.path.exists(ssd.DEBUG_LIB_PATH):
+        pytest.skip("libssd_debug.so not built")
+    dbg = ctypes.CDLL(ssd.DEBUG_LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(dbg, n), f"{n} not exported by the debug build"
+    dbg.ssd_debug_bounds_build.restype = ctypes.c_int
+    assert dbg.ssd_debug_bounds_build() == 1
+
+
 def test_c_struct_layout_matches_header(lib):
     # sizes the header implies on LP64: 16 four-byte fields; pointer/long long fields are 8 bytes
     assert ctypes.sizeof(ssd.SsdConfig) == 17 * 4
