@@ -17,21 +17,22 @@
 // four heads of one group and batch row, which share the group's B channels.  When the scan
 // leaves too few SMs free (many short sequences, large batches), it runs after the scan on
 // all SMs instead and folds its part into the state the scan left (h = e^{...} h + dH), with
-// no dH buffer and no fold pass.  Per item the CTA
-// computes every tail token's weight w_s per head; then, per 64 tokens (a round), it copies the
-// raw rows of the heads' x channels and the group's B channels (plus 3 history rows) into
-// shared memory with asynchronous 16-byte copies (the next round's copies, or the next item's
-// first, run during this round), and each thread runs the conv + SiLU in fp32 for two adjacent
-// channels over 16 tokens, multiplies the x channels by w_s, and splits each value v into fp16
-// parts, v = hi + lo + e with hi = fp16(v), lo = fp16(v - hi) and |e| <= 2^-22 |v| (plus an
-// absolute 2^-25 where lo falls below fp16's normal range), written into 128-byte-swizzled
-// operand tiles.  One thread then issues the round's update on the tensor cores, one MMA per
-// 16 tokens and product for all the item's heads (N = 64 per head), into a tensor-memory
-// accumulator (128 lanes = state column n, 64 columns per head), as three fp16 products with
-// fp32 accumulation:
+// no dH buffer and no fold pass.
+//
+// Per item the CTA computes every tail token's weight w_s per head; then, per 64 tokens (a
+// round), it copies the raw rows of the heads' x channels and the group's B channels (plus 3
+// history rows) into shared memory with asynchronous 16-byte copies (the next round's copies,
+// or the next item's first, run during this round), and each thread runs the conv + SiLU in
+// fp32 for two adjacent channels over 16 tokens, multiplies the x channels by w_s, and splits
+// each value v into fp16 parts, v = hi + lo + e with hi = fp16(v), lo = fp16(v - hi) and
+// |e| <= 2^-22 |v| (plus an absolute 2^-25 where lo falls below fp16's normal range), written
+// into 128-byte-swizzled operand tiles.  One thread then issues the round's update on the
+// tensor cores, one MMA per 16 tokens and product for all the item's heads (N = 64 per head),
+// into a tensor-memory accumulator (128 lanes = state column n, 64 columns per head), as three
+// fp16 products with fp32 accumulation:
 //   dH^T += B_hi^T X_hi + B_hi^T X_lo + B_lo^T X_hi
 // (the dropped lo*lo term is below 2^-22 of the product), which keeps the update at fp32
-// accuracy.  Sixteen warps finally read the accumulator and store dH.
+// accuracy.  Sixteen warps finally read the accumulator and store dH (or fold it).
 #include <algorithm>
 #include <type_traits>
 
