@@ -31,8 +31,9 @@ def _run(tmp_path, lib, denom, norm_groups):
 @pytest.mark.parametrize("norm_groups", [0, 2])
 def test_index_checks_of_the_debug_build(cuda_lib, tmp_path, norm_groups):
     from mamba_ssd_scan_02_b200 import ssd
-    if not os.path.exists(ssd.DEBUG_LIB_PATH):
-        pytest.fail("libssd_debug.so is not built (python -m mamba_ssd_scan_02_b200.build --debug-bounds)")
+    if not os.path.exists(ssd.DEBUG_LIB_PATH):  # normally built beside libssd.so by build()
+        from mamba_ssd_scan_02_b200 import build as _b
+        _b.build(debug_bounds=True)
     ref = _run(tmp_path, ssd.LIB_PATH, 1, norm_groups)
     assert ref["debug_build"] == 0 and ref["status"] == 0
     full = _run(tmp_path, ssd.DEBUG_LIB_PATH, 1, norm_groups)
