@@ -164,10 +164,13 @@ ssd_status_t ssd_prefill(const ssd_config_t *cfg, const ssd_prefill_args_t *args
  *    is packed tokens [cu_seqlens[i], cu_seqlens[i+1]) (an empty sequence copies its carries).
  *  cfg: batch = 1 and seqlen = cu_seqlens[nseq] (all tokens); the token tensors of args
  *    (xBC, dt, z, y) are the packed [seqlen, ...] rows; h0 / h_final are [nseq, H, P, N] and
- *    conv_state_in / conv_state_out [nseq, W, conv_dim] (NULL as in ssd_prefill).
+ *    conv_state_in / conv_state_out [nseq, W, conv_dim] (NULL as in ssd_prefill; with
+ *    h_final NULL the pass that computes the final states' last chunks is skipped).
  *  workspace: at least ssd_varlen_workspace_size(cfg, cu_seqlens, nseq) bytes.
- * Runs the prefill of each sequence in turn on `stream`; returns the first error (argument
- * errors, including inconsistent offsets, as SSD_ERR_INVALID_ARG). */
+ * On the tensor-core path (bf16 with the shapes its fused front end takes) the whole packed
+ * batch is one pass on `stream`, one launch of each kernel, bit-exact against one
+ * ssd_prefill per sequence; other paths run the prefill of each sequence in turn.  Returns the
+ * first error (argument errors, including inconsistent offsets, as SSD_ERR_INVALID_ARG). */
 size_t ssd_varlen_workspace_size(const ssd_config_t *cfg, const int *cu_seqlens, int nseq);
 ssd_status_t ssd_prefill_varlen(const ssd_config_t *cfg, const ssd_prefill_args_t *args,
                                 const int *cu_seqlens, int nseq, void *stream);
