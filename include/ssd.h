@@ -28,16 +28,17 @@
  *  - All pointers are DEVICE pointers owned by the caller.  The library never
  *    allocates device memory, frees or synchronises on these paths; it enqueues
  *    kernels on `stream` (a cudaStream_t, NULL = legacy default stream) and
- *    returns.  The tensor-core prefill runs its fp32 final-state pass on a
- *    library side stream, forked from `stream` after the front end and joined
- *    back into it within the same call, so every effect of the call is ordered
- *    on `stream` (stream capture included).  That side stream and its two
- *    events are created by the first such call on each host thread and device
- *    and kept for the life of the process.
+ *    returns.  When the scan leaves SMs free, the tensor-core prefill runs its
+ *    final-state pass (fp32 accuracy) on a library side stream, forked from
+ *    `stream` after the front end and joined back into it within the same call,
+ *    so every effect of the call is ordered on `stream` (stream capture
+ *    included); otherwise the pass runs on `stream` after the scan.  That side
+ *    stream and its two events are created by the first such call on each host
+ *    thread and device and kept for the life of the process.
  *  - Argument errors are reported synchronously before anything is launched.
  *    Launch failures come back as SSD_ERR_CUDA.  Errors raised inside kernels
- *    (a bounded wait that gave up) are latched in a device word read by
- *    ssd_get_device_error().
+ *    (a bounded wait that gave up, or, in the debug build, an index check) are
+ *    latched in a device word read by ssd_get_device_error().
  *  - Tensors read or written with 16-byte vectors (xBC, z, y, out, hidden, the
  *    weights, the conv caches, the states) must be 16-byte aligned, and their
  *    row strides must be multiples of 8 elements.
