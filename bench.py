@@ -18,7 +18,8 @@ events on the launching stream.  The same line carries:
     chunk 256, gated RMSNorm;
   - "mixer": the whole mixer layer at the 12B width (d_model 5120, 160 heads, B8 L8192),
     tensor-core roofline of its dominant GEMM;
-  - "cpu_baseline": the fp64 oracle timed on a bounded sample of the prefill workload.
+  - "cpu_baseline": the fp64 oracle timed on a bounded sample of the prefill workload;
+    "parity": the library's prefill on that sample against the oracle's result (max|err|/RMS).
 Multi-GPU (torchrun): one process per GPU, each an independent replica (weak scaling), time
 = max over ranks.  --impl reference times the fp64 CPU oracle on the same metric.
 """
@@ -686,9 +687,9 @@ def cpu_baseline(target_s: float = 10.0):
     while True:
         t0 = time.time()
         for _ in range(reps):
-            o.ssd_prefill(dict(cfg, seqlen=tok), inp["xBC"][:, :tok], inp["dt"][:, :tok],
-                          inp["A"], inp["D"], inp["dt_bias"], conv_w=inp["conv_w"],
-                          heads=(0, groups * hpg), threads=cores)
+            ref = o.ssd_prefill(dict(cfg, seqlen=tok), inp["xBC"][:, :tok], inp["dt"][:, :tok],
+                                inp["A"], inp["D"], inp["dt_bias"], conv_w=inp["conv_w"],
+                                heads=(0, groups * hpg), threads=cores)
         dt = time.time() - t0
         if dt >= target_s:
             break
@@ -706,7 +707,9 @@ def cpu_baseline(target_s: float = 10.0):
     o.ssd_prefill(dict(cfg, seqlen=tok1), inp["xBC"][:, :tok1], inp["dt"][:, :tok1], inp["A"], inp["D"],
                   inp["dt_bias"], conv_w=inp["conv_w"], heads=(0, hpg), threads=1)
     dt1 = time.time() - t0
+    parity = sample_parity(cfg, inp, tok, groups * hpg, ref)
     return {"value": round(reps * tok * frac / dt, 2), "unit": "tokens/s", "cores": cores,
+            "parity": parity,
             "kind": "oracle", "cpu_model": cpu_model(),
             "sample": f"prefill_8k inputs, first {tok} tokens x heads 0-{groups * hpg - 1} "
                       f"({groups}/{cfg['ngroups']} of the layer) x {reps} run(s), fp64, "
@@ -715,6 +718,31 @@ def cpu_baseline(target_s: float = 10.0):
                               "cores": 1,
                               "sample": f"first {tok1} tokens x heads 0-{hpg - 1} (1/{cfg['ngroups']} "
                                         f"of the layer), fp64, {dt1:.1f} s"}}
+
+
+def sample_parity(cfg, inp, tok, nh, ref):
+    """The library's prefill on the oracle's timing sample (the first `tok` tokens of the
+    prefill_8k inputs, all heads on the GPU) against the oracle's result for heads 0..nh-1:
+    max|err|/RMS of y and h_final, and of y's error beyond its bf16 storage rounding."""
+    import torch
+    from mamba_ssd_scan_02_b200 import ssd
+    c = dict(cfg, seqlen=tok)
+    d = {k: ssd.to_device(np.ascontiguousarray(inp[k][:, :tok])) for k in ("xBC", "dt")}
+    p = {k: ssd.to_device(inp[k]) for k in ("A", "D", "dt_bias", "conv_w")}
+    y, hf, _ = ssd.prefill(c, d["xBC"], d["dt"], p["A"], p["D"], p["dt_bias"], p["conv_w"])
+    torch.cuda.synchronize()
+    P = cfg["headdim"]
+    yg = y.float().cpu().numpy()[:, :, :nh * P].astype(np.float64)
+    yw = ref["y"].reshape(ref["y"].shape[0], ref["y"].shape[1], -1)
+    hg = ssd.to_numpy(hf)[:, :nh].astype(np.float64)
+    hw = ref["h_final"]
+    rms_y, rms_h = float(np.sqrt(np.mean(yw * yw))), float(np.sqrt(np.mean(hw * hw)))
+    return {"y_max_err_rms": float(np.max(np.abs(yg - yw)) / rms_y),
+            "y_excess_over_bf16_rounding": float(np.max(np.abs(yg - yw) - 2.0 ** -8 * np.abs(yw)) / rms_y),
+            "h_final_max_err_rms": float(np.max(np.abs(hg - hw)) / rms_h),
+            "bound": 2e-2, "oracle": "fp64",
+            "sample": f"prefill_8k inputs, first {tok} tokens x heads 0-{nh - 1}",
+            "device_status": int(ssd.get_device_error())}
 
 
 def cpu_model() -> str:
@@ -837,6 +865,7 @@ def main():
     if rank != 0:
         return
     cpu = None if (args.quick or world > 1) else cpu_baseline()
+    parity = cpu.pop("parity", None) if cpu else None  # the GPU path on the oracle's sample
     line = {
         "metric": METRIC, "value": round(res["value"], 1), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -845,7 +874,7 @@ def main():
         "config": dict(HEADLINE_CONFIG, parallelism=f"replicas x{world}"),
         "roofline": res["roofline"], "e2e": res["e2e"], "gpu_launches": res["gpu_launches"],
         "clocks": res["clocks"], "kernels": res["kernels"],
-        "path_bytes_per_step": res["path_bytes_per_step"], "cpu_baseline": cpu,
+        "path_bytes_per_step": res["path_bytes_per_step"], "cpu_baseline": cpu, "parity": parity,
         "device_status": status,
     }
     # The other workloads: their full records on stderr, a short summary of each at the end
